@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""DCU denoising-step throughput on one B200 (or N independent replicas).
+
+Workload (default): LLaDA-8B-shaped random-init bf16 model (32 layers,
+d = 4096, 32 x 128 MHA, SwiGLU 12288, vocab 126464), one sequence of
+N = 1024 = 768 prompt + 256 masked positions, B_layer = 32, B_window = 32,
+Fréchet commit with delta = 0.1.  A step is one DCU step (layer-0 refresh,
+per-layer dynamics / budget / selection / recompute / scatter) plus the commit
+(LM head on the masked rows, softmax-max, sort, Fréchet rule), i.e. every row
+of the hot path except the dense forward, which fills the caches once before
+timing and is reported separately.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle instead, on a bounded sample of the same step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "DCU denoise steps/s & gen tokens/s, LLaDA-8B shape, 1×B200; % of HBM roofline"
+
+WORKLOADS = {
+    "llada8b": dict(shape="LLADA_8B", n_prompt=768, n_gen=256, batch=1, B_layer=32, B_window=32, rule=0, param=0.1,
+                    desc="LLaDA-8B-shaped DCU step, N=1024 (768 prompt + 256 masked), B_layer=32, B_window=32, "
+                         "Frechet delta=0.1"),
+    "dream7b": dict(shape="DREAM_7B", n_prompt=768, n_gen=256, batch=1, B_layer=32, B_window=32, rule=2, param=0.9,
+                    desc="Dream-7B-shaped DCU step (GQA 28/4), N=1024, B_layer=32, B_window=32, factor f=0.9"),
+    "long8k": dict(shape="LLADA_8B", n_prompt=7680, n_gen=512, batch=1, B_layer=96, B_window=64, rule=0,
+                   param=0.05, desc="LLaDA-8B shape, N=8192 (7680 prompt + 512 masked), B_layer=96, B_window=64, "
+                                    "Frechet delta=0.05"),
+    "batch4": dict(shape="LLADA_8B", n_prompt=1536, n_gen=512, batch=4, B_layer=64, B_window=32, rule=1, param=0.9,
+                   desc="LLaDA-8B shape, 4 sequences x N=2048 (1536 prompt + 512 masked), B_layer=64, B_window=32, "
+                        "threshold tau=0.9"),
+}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks sampling
+
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def cpu_sample_step(shape, seed, N, n_prompt, B_layer, B_window, lm_rows=8, vocab_frac=8):
+    """Times the fp64 oracle on a bounded sample of one DCU step + commit and
+    extrapolates to a whole step: one layer's selection + recompute of
+    |W| + B_layer rows (x n_layers), and the LM head + softmax-max of `lm_rows`
+    masked rows over vocab / vocab_frac entries (scaled to all masked rows and
+    the full vocabulary), plus the commit over all masked positions."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle as O
+    from dynamic_layer_wise_b200 import inputs as I
+
+    cfg = O.Config(n_layers=shape.n_layers, d_model=shape.d_model, n_heads=shape.n_heads,
+                   n_kv_heads=shape.n_kv_heads, head_dim=shape.head_dim, d_ffn=shape.d_ffn, vocab=shape.vocab,
+                   dtype=shape.dtype)
+    D, Hkv, hd = shape.d_model, shape.n_kv_heads, shape.head_dim
+    ones = np.ones(D)
+    lw = {"attn_norm": ones, "ffn_norm": ones}
+    for n in I.LAYER_TENSORS:
+        lw[n] = I.as_f64(I.weight_values(shape, seed, n, 0), shape.dtype)
+    H = I.as_f64(I.normal_values(seed, 9001, 0, N * D, 0.5, shape.dtype), shape.dtype).reshape(N, D)
+    K = I.as_f64(I.normal_values(seed, 9002, 0, Hkv * N * hd, 1.0, shape.dtype), shape.dtype).reshape(Hkv, N, hd)
+    V = I.as_f64(I.normal_values(seed, 9003, 0, Hkv * N * hd, 0.05, shape.dtype), shape.dtype).reshape(Hkv, N, hd)
+    d = np.zeros(N, np.float32)
+    hot = I.uniform_ints(seed, 9004, 0, 3 * B_layer, N)
+    d[hot] = np.abs(I.normal_values(seed, 9005, 0, len(hot), 0.1, "f32")) + 1e-6
+    keys = [n_prompt]
+    nv = shape.vocab // vocab_frac
+    lm = I.as_f64(I.weight_values(shape, seed, "lm_head", rows=np.arange(nv)), shape.dtype)
+    n_masked = N - n_prompt
+    c_all = np.abs(I.normal_values(seed, 9006, 0, N, 0.001, "f32")) + 1e-5
+    masked = np.zeros(N, bool)
+    masked[n_prompt:] = True
+    t0 = time.perf_counter()
+    U = O.select_rows(d, keys, B_window, B_layer, 0)
+    O.layer_rows(lw, cfg, H[U], U, K.copy(), V.copy())
+    t1 = time.perf_counter()
+    O.confidence(H[:lm_rows], ones, lm, cfg.rms_eps)
+    t2 = time.perf_counter()
+    O.commit(c_all, np.zeros(N, np.int64), masked, np.zeros(N, np.int64), O.RULE_FRECHET, 0.1)
+    t3 = time.perf_counter()
+    step_s = shape.n_layers * (t1 - t0) + (t2 - t1) * vocab_frac * (n_masked / lm_rows) + (t3 - t2)
+    threads = max([x.get("num_threads", 1) for x in threadpool_info()] or [1])
+    sample = (f"1 of {shape.n_layers} layers ({len(U)} recomputed rows, N={N}) x {shape.n_layers}, "
+              f"LM head + softmax-max of {lm_rows} of {n_masked} masked rows over {nv} of {shape.vocab} vocab "
+              f"entries (scaled), commit over {n_masked}; measured {t3 - t0:.2f} s")
+    return step_s, t3 - t0, threads, sample
+
+
+# ---------------------------------------------------------------- roofline bookkeeping
+
+def gemm_algorithmic_bytes(shape, rows_per_layer):
+    """Weights + bf16 activation in/out bytes of the recompute GEMMs of one step."""
+    D, F, H, Hkv, hd = shape.d_model, shape.d_ffn, shape.n_heads, shape.n_kv_heads, shape.head_dim
+    es = 2 if shape.dtype == "bf16" else 4
+    gemms = [((H + 2 * Hkv) * hd, D), (D, H * hd), (2 * F, D), (D, F)]  # (n_out, K)
+    total = 0.0
+    for M in rows_per_layer:
+        for n_out, K in gemms:
+            total += es * (n_out * K + M * K + M * n_out)
+    return total, 4 * len(rows_per_layer)
+
+
+def step_algorithmic_bytes(shape, rows_per_layer, N, batch, n_masked):
+    """Roofline bytes of one step: all layer weights once, the LM head once,
+    the K/V stream over all N, and the recomputed rows' activations."""
+    es = 2 if shape.dtype == "bf16" else 4
+    w_layer = sum(o * i for o, i in shape.weight_shapes().values()) * es
+    kv = 2 * batch * shape.n_kv_heads * N * shape.head_dim * es
+    act = sum(M * shape.d_model * es * 2 for M in rows_per_layer)
+    return shape.n_layers * (w_layer + kv) + shape.vocab * shape.d_model * es + act + n_masked * shape.d_model * es
+
+
+def traffic_for(kernel_file: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        t = json.load(fh)
+    src = os.path.join(ROOT, "dynamic_layer_wise_b200", "csrc", kernel_file)
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    e = t.get(kernel_file)
+    if e and e.get("source_sha") == h:
+        return e.get("dram_bytes_per_launch")
+    return None
+
+
+# ---------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="dcu", choices=["dcu", "reference"])
+    ap.add_argument("--workload", default="llada8b", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = WORKLOADS[args.workload]
+
+    from dynamic_layer_wise_b200 import inputs as I
+    shape = getattr(I, wl["shape"])
+    N = wl["n_prompt"] + wl["n_gen"]
+    B = wl["batch"]
+    config = {"workload": wl["desc"], "batch": B, "seq_len": N, "B_layer": wl["B_layer"], "B_window": wl["B_window"],
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+              "l2": "inputs larger than L2: every step streams all layer weights (~15 GB) and the LM head"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        times = []
+        info = None
+        for i in range(args.warmup + args.steps):
+            step_s, measured, threads, sample = cpu_sample_step(shape, 0, N, wl["n_prompt"], wl["B_layer"],
+                                                                wl["B_window"])
+            if i >= args.warmup:
+                times.append(step_s)
+            info = (threads, sample)
+        ms = 1000.0 * statistics.mean(times)
+        v = 1000.0 / ms
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": config,
+                          "cpu_baseline": {"value": v, "unit": "steps/s", "cores": info[0], "kind": "oracle",
+                                           "sample": info[1]},
+                          "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from dynamic_layer_wise_b200 import dcu
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    stream = torch.cuda.current_stream()
+    W = I.device_weights(shape, 0)
+    ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
+    seq_seed = 1 + rank                                   # each replica decodes its own sequences
+    ids_h = torch.stack([torch.tensor(I.sequence_ids(seq_seed, b, wl["n_prompt"], wl["n_gen"], shape.vocab),
+                                      dtype=torch.int32) for b in range(B)])
+    ids = ids_h.cuda()
+    masked = (ids == shape.mask_id).to(torch.uint8)
+    pos = torch.zeros((B, N), dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
+
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    dcu.dcu_full_forward(ctx, ids)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    full_ms = e0.elapsed_time(e1)
+    dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
+
+    def step():
+        dcu.dcu_step(ctx, ids, pos, cnt, wl["B_layer"], wl["B_window"])
+        dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if dcu.dcu_status(ctx) != 0:
+        raise RuntimeError("device status word set during warm-up")
+    masked_before = int(masked.sum().item())
+
+    per_step_launches_guess = 2 + shape.n_layers * 11 + 6
+    dcu.dcu_profile_enable(ctx, args.steps * per_step_launches_guess)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = dcu.dcu_launch_count(ctx)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    launches = dcu.dcu_launch_count(ctx) - launches0
+    committed = masked_before - int(masked.sum().item())
+    ms_step = max_over_ranks(ms_total / args.steps)
+    steps_all = args.steps * world
+    value = steps_all / (ms_step * args.steps / 1000.0)
+    tokens_per_s = sum_over_ranks(committed) / (ms_step * args.steps / 1000.0)
+
+    per_kernel = {}
+    for k in range(dcu.DCU_K_COUNT):
+        ms_k, n_k = dcu.dcu_profile_read(ctx, k)
+        per_kernel[dcu.dcu_kernel_class_name(k)] = {"ms_per_step": ms_k / args.steps,
+                                                    "launches_per_step": n_k / args.steps,
+                                                    "share": ms_k / ms_total if ms_total > 0 else None}
+    rows = [int(dcu.dcu_get_tensor(ctx, dcu.DCU_T_SEL_COUNT, l).sum().item()) for l in range(shape.n_layers)]
+    gemm_bytes, gemm_launches = gemm_algorithmic_bytes(shape, rows)
+    gemm_ms_step = per_kernel["gemm"]["ms_per_step"]
+    hbm, tflops, peak_src = measured_peaks()
+    achieved = gemm_bytes / (gemm_ms_step / 1000.0) / 1e9 if gemm_ms_step > 0 else None
+    step_bytes = step_algorithmic_bytes(shape, rows, N, B, int(masked.sum().item()) + 1)
+    roofline = {"bound": "hbm", "kernel": "gemm (recompute projections + FFN)", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s", "frac": (achieved / hbm) if achieved else None,
+                "traffic": traffic_for("k_gemm_simt.cu"), "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": gemm_bytes / gemm_launches,
+                "step_bytes": step_bytes, "step_roofline_ms": step_bytes / (hbm * 1e9) * 1e3,
+                "step_frac_of_measured": (step_bytes / (hbm * 1e9) * 1e3) / ms_step,
+                "step_frac_of_8TBps": (step_bytes / 8e12 * 1e3) / ms_step}
+
+    e2e = None
+    if not args.no_e2e:
+        # through the C ABI with host buffers: ids/keys in from pinned memory, result out, every step
+        h_ids = ids.cpu().pin_memory()
+        h_pos = pos.cpu().pin_memory()
+        h_cnt = cnt.cpu().pin_memory()
+        h_out = torch.empty((B, N), dtype=torch.int32).pin_memory()
+        h_oc = torch.empty(B, dtype=torch.int32).pin_memory()
+        barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(args.steps):
+            ids.copy_(h_ids, non_blocking=True)
+            pos.copy_(h_pos, non_blocking=True)
+            cnt.copy_(h_cnt, non_blocking=True)
+            step()
+            h_out.copy_(pos, non_blocking=True)
+            h_oc.copy_(cnt, non_blocking=True)
+            h_ids.copy_(ids, non_blocking=True)
+            stream.synchronize()
+            h_pos.copy_(h_out)
+            h_cnt.copy_(h_oc)
+        a1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
+        e2e = {"value": steps_all / (e2e_ms * args.steps / 1000.0), "unit": "steps/s",
+               "h2d_bytes_per_step": 4 * (2 * B * N + B), "d2h_bytes_per_step": 4 * (2 * B * N + B),
+               "ms_per_step": e2e_ms}
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        step_s, measured, threads, sample = cpu_sample_step(shape, 0, N, wl["n_prompt"], wl["B_layer"],
+                                                            wl["B_window"])
+        cpu_base = {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        out = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32", "data": "synthetic",
+               "config": config, "gen_tokens_per_s": tokens_per_s, "full_forward_ms": full_ms,
+               "per_kernel": per_kernel, "rows_per_layer_last_step": rows, "roofline": roofline,
+               "cpu_baseline": cpu_base, "e2e": e2e, "clocks": clk, "gpu_launches": launches}
+        print(json.dumps(out))
+    ctx.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

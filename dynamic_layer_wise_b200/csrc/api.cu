@@ -1,0 +1,596 @@
+// C ABI of libdcu: context (caches + scratch arena), host orchestration of
+// the dense forward, the DCU step and the commit, stateless kernel entry
+// points, introspection and per-kernel event timing.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "../../include/dcu.h"
+#include "kernels.h"
+
+using namespace dcu;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+struct EventPair {
+  cudaEvent_t a = nullptr, b = nullptr;
+};
+
+struct ProfClass {
+  std::vector<EventPair> ev;
+  int64_t used = 0;
+  int64_t dropped = 0;
+};
+
+size_t esize(int dtype) { return dtype == DCU_BF16 ? 2 : 4; }
+
+}  // namespace
+
+struct dcu_ctx {
+  dcu_cfg cfg{};
+  int device = 0;
+  size_t esz = 2;
+  // weights (caller-owned)
+  const void *embed = nullptr, *lm_head = nullptr;
+  const float *final_norm = nullptr;
+  std::vector<const void *> wq, wk, wv, wo, wg, wu, wd;
+  std::vector<const float *> g1, g2;
+  // active shape
+  int B = 0, N = 0;
+  bool have_cache = false, first_step = true;
+  int64_t cap = 0;  // max_batch * max_seq rows
+  // caches
+  char *H = nullptr, *K = nullptr, *V = nullptr;
+  int32_t *prev_ids = nullptr;
+  float *d = nullptr, *s_cur = nullptr, *s_prev = nullptr;
+  int32_t *budgets = nullptr, *sel_idx = nullptr, *sel_cnt = nullptr;
+  int32_t *rowmap = nullptr, *ints = nullptr;  // ints: m_total, done, status, m_masked
+  float2 *rope_tab = nullptr;
+  // scratch
+  char *xs = nullptr, *Q = nullptr, *attn = nullptr, *act = nullptr;
+  float *hmid = nullptr, *C = nullptr, *conf = nullptr;
+  int32_t *amax = nullptr, *mrow = nullptr;
+  std::vector<void *> allocs;
+  std::string err;
+  // profiling
+  int32_t prof_max = 0;
+  int64_t launches = 0;
+  ProfClass prof[DCU_K_COUNT];
+
+  int32_t *m_total() { return ints + 0; }
+  int32_t *done() { return ints + 1; }
+  int32_t *status() { return ints + 2; }
+  int32_t *m_masked() { return ints + 3; }
+  size_t hslab() const { return (size_t)cap * cfg.d_model * esz; }
+  size_t kvslab() const { return (size_t)cap * cfg.n_kv_heads * cfg.head_dim * esz; }
+  void *Hl(int l) { return H + (size_t)l * hslab(); }
+  void *Kl(int l) { return K + (size_t)l * kvslab(); }
+  void *Vl(int l) { return V + (size_t)l * kvslab(); }
+  float *dl(int l) { return d + (size_t)l * cap; }
+};
+
+namespace {
+
+int fail(dcu_ctx *ctx, int code, const std::string &msg) {
+  if (ctx) ctx->err = msg;
+  g_last_error = msg;
+  return code;
+}
+
+#define CK(ctx, expr)                                                                       \
+  do {                                                                                      \
+    cudaError_t e_ = (expr);                                                                \
+    if (e_ != cudaSuccess)                                                                  \
+      return fail((ctx), DCU_ECUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+// A launch_* call enqueues exactly one kernel.
+#define LAUNCH(ctx, expr)            \
+  do {                               \
+    CK(ctx, expr);                   \
+    if (ctx) ++(ctx)->launches;      \
+  } while (0)
+
+struct Prof {
+  dcu_ctx *c;
+  int k;
+  cudaStream_t s;
+  EventPair *p = nullptr;
+  Prof(dcu_ctx *c_, int k_, cudaStream_t s_) : c(c_), k(k_), s(s_) {
+    if (!c || c->prof_max <= 0) return;
+    ProfClass &pc = c->prof[k];
+    if (pc.used >= (int64_t)pc.ev.size()) {
+      ++pc.dropped;
+      return;
+    }
+    p = &pc.ev[pc.used++];
+    cudaEventRecord(p->a, s);
+  }
+  ~Prof() {
+    if (p) cudaEventRecord(p->b, s);
+  }
+};
+
+template <class T>
+cudaError_t dalloc(dcu_ctx *c, T **p, size_t bytes) {
+  void *q = nullptr;
+  cudaError_t e = cudaMalloc(&q, bytes < 256 ? 256 : bytes);
+  if (e != cudaSuccess) return e;
+  c->allocs.push_back(q);
+  *p = reinterpret_cast<T *>(q);
+  return cudaSuccess;
+}
+
+void free_all(dcu_ctx *c) {
+  for (void *p : c->allocs) cudaFree(p);
+  c->allocs.clear();
+  for (auto &pc : c->prof)
+    for (auto &e : pc.ev) {
+      if (e.a) cudaEventDestroy(e.a);
+      if (e.b) cudaEventDestroy(e.b);
+    }
+}
+
+std::string check_cfg(const dcu_cfg *c) {
+  if (c->n_layers <= 0 || c->d_model <= 0 || c->n_heads <= 0 || c->n_kv_heads <= 0 || c->head_dim <= 0 ||
+      c->d_ffn <= 0 || c->vocab <= 0 || c->max_batch <= 0 || c->max_seq <= 0)
+    return "every size must be > 0";
+  if (c->dtype != DCU_F32 && c->dtype != DCU_BF16) return "dtype must be DCU_F32 or DCU_BF16";
+  if (c->d_model % 64) return "d_model must be a multiple of 64";
+  if (c->head_dim % 16 || c->head_dim > 256) return "head_dim must be a multiple of 16 and <= 256";
+  if (c->n_heads % c->n_kv_heads) return "n_heads must be a multiple of n_kv_heads";
+  if ((c->n_heads * c->head_dim) % 64 || (c->n_kv_heads * c->head_dim) % 64)
+    return "n_heads*head_dim and n_kv_heads*head_dim must be multiples of 64";
+  if (c->d_ffn % 64) return "d_ffn must be a multiple of 64";
+  if (c->max_seq > 16384) return "max_seq must be <= 16384";
+  if (c->mask_id < 0 || c->mask_id >= c->vocab) return "mask_id must be in [0, vocab)";
+  if (!(c->rms_eps > 0.0f)) return "rms_eps must be > 0";
+  if (c->rope_theta < 0.0f) return "rope_theta must be >= 0";
+  if (c->window_mode != DCU_WINDOW_INCLUSIVE && c->window_mode != DCU_WINDOW_HALFOPEN)
+    return "window_mode must be DCU_WINDOW_INCLUSIVE or DCU_WINDOW_HALFOPEN";
+  if ((long long)c->max_batch * c->max_seq > (1ll << 30)) return "max_batch * max_seq too large";
+  return "";
+}
+
+int run_gemm(dcu_ctx *c, const void *X, int ldx, const int32_t *m_total, const GemmSeg *segs, int nseg, int K,
+             int ldc, cudaStream_t s) {
+  Prof p(c, DCU_K_GEMM, s);
+  LAUNCH(c, launch_gemm_simt(c->cfg.dtype, X, ldx, m_total, (int)c->cap, segs, nseg, K, c->C, ldc, s));
+  return DCU_OK;
+}
+
+// One layer of recompute over the packed rows in ctx->rowmap / m_total.
+// dense: the rows are every position (full forward): no selection, no d.
+int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t *nkeys, int Bw, cudaStream_t s) {
+  const dcu_cfg &g = c->cfg;
+  const int L = g.n_layers, D = g.d_model, H = g.n_heads, Hkv = g.n_kv_heads, hd = g.head_dim, F = g.d_ffn;
+  const int dt = g.dtype, cap = (int)c->cap;
+  const bool last = (l + 1 == L);
+  if (!dense) {
+    Prof p(c, DCU_K_SELECT, s);
+    LAUNCH(c, launch_select(c->dl(l), keys, nkeys, c->budgets + l, L, c->B, c->N, Bw, g.window_mode,
+                        c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
+                        last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->status(), s));
+  }
+  {
+    Prof p(c, DCU_K_GATHER, s);
+    LAUNCH(c, launch_gather_norm(dt, c->rowmap, c->m_total(), cap, c->Hl(l), c->g1[l], g.rms_eps, D, c->xs, s));
+  }
+  const int nqkv = (H + 2 * Hkv) * hd;
+  GemmSeg qkv[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
+  if (int rc = run_gemm(c, c->xs, D, c->m_total(), qkv, 3, D, nqkv, s)) return rc;
+  {
+    Prof p(c, DCU_K_EPILOGUE, s);
+    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->rope_tab,
+                         g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
+  }
+  {
+    Prof p(c, DCU_K_ATTN, s);
+    LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l), c->attn,
+                           s));
+  }
+  GemmSeg o[1] = {{c->wo[l], D}};
+  if (int rc = run_gemm(c, c->attn, H * hd, c->m_total(), o, 1, H * hd, D, s)) return rc;
+  {
+    Prof p(c, DCU_K_EPILOGUE, s);
+    LAUNCH(c, launch_epi_o(dt, c->C, D, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l], g.rms_eps, D, c->hmid, c->xs,
+                       s));
+  }
+  GemmSeg gu[2] = {{c->wg[l], F}, {c->wu[l], F}};
+  if (int rc = run_gemm(c, c->xs, D, c->m_total(), gu, 2, D, 2 * F, s)) return rc;
+  {
+    Prof p(c, DCU_K_EPILOGUE, s);
+    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, c->m_total(), cap, F, c->act, s));
+  }
+  GemmSeg dn[1] = {{c->wd[l], D}};
+  if (int rc = run_gemm(c, c->act, F, c->m_total(), dn, 1, F, D, s)) return rc;
+  {
+    Prof p(c, DCU_K_SCATTER, s);
+    const bool want_d = !dense && !last;
+    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, c->rowmap, c->m_total(), cap, c->hmid, c->Hl(l + 1),
+                                  want_d ? c->g1[l + 1] : nullptr, want_d ? c->dl(l + 1) : nullptr, D, s));
+  }
+  return DCU_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dcu_last_error(const dcu_ctx *ctx) { return ctx ? ctx->err.c_str() : g_last_error.c_str(); }
+
+int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
+  if (!out) return fail(nullptr, DCU_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (!w || !cfg) return fail(nullptr, DCU_EINVAL, "weights or cfg is NULL");
+  std::string why = check_cfg(cfg);
+  if (!why.empty()) return fail(nullptr, DCU_EINVAL, "bad cfg: " + why);
+  if (!w->embed || !w->final_norm || !w->lm_head || !w->attn_norm || !w->wq || !w->wk || !w->wv || !w->wo ||
+      !w->ffn_norm || !w->w_gate || !w->w_up || !w->w_down)
+    return fail(nullptr, DCU_EINVAL, "a weight pointer is NULL");
+  for (int l = 0; l < cfg->n_layers; ++l)
+    if (!w->attn_norm[l] || !w->wq[l] || !w->wk[l] || !w->wv[l] || !w->wo[l] || !w->ffn_norm[l] ||
+        !w->w_gate[l] || !w->w_up[l] || !w->w_down[l])
+      return fail(nullptr, DCU_EINVAL, "layer " + std::to_string(l) + ": a weight pointer is NULL");
+
+  dcu_ctx *c = new (std::nothrow) dcu_ctx();
+  if (!c) return fail(nullptr, DCU_ENOMEM, "host allocation failed");
+  c->cfg = *cfg;
+  c->esz = esize(cfg->dtype);
+  cudaGetDevice(&c->device);
+  c->embed = w->embed;
+  c->lm_head = w->lm_head;
+  c->final_norm = (const float *)w->final_norm;
+  const int L = cfg->n_layers;
+  for (int l = 0; l < L; ++l) {
+    c->wq.push_back(w->wq[l]);
+    c->wk.push_back(w->wk[l]);
+    c->wv.push_back(w->wv[l]);
+    c->wo.push_back(w->wo[l]);
+    c->wg.push_back(w->w_gate[l]);
+    c->wu.push_back(w->w_up[l]);
+    c->wd.push_back(w->w_down[l]);
+    c->g1.push_back((const float *)w->attn_norm[l]);
+    c->g2.push_back((const float *)w->ffn_norm[l]);
+  }
+  c->cap = (int64_t)cfg->max_batch * cfg->max_seq;
+  const size_t cap = (size_t)c->cap, D = cfg->d_model, F = cfg->d_ffn, Hhd = (size_t)cfg->n_heads * cfg->head_dim;
+  const size_t nqkv = (size_t)(cfg->n_heads + 2 * cfg->n_kv_heads) * cfg->head_dim;
+  size_t cw = nqkv;
+  if (D > cw) cw = D;
+  if (2 * F > cw) cw = 2 * F;
+  if ((size_t)cfg->vocab > cw) cw = cfg->vocab;
+  size_t xw = D > F ? D : F;
+  cudaError_t e = cudaSuccess;
+#define AL(ptr, bytes)                                                                  \
+  if (e == cudaSuccess) {                                                               \
+    e = dalloc(c, &(ptr), (bytes));                                                     \
+  }
+  AL(c->H, (size_t)(L + 1) * c->hslab());
+  AL(c->K, (size_t)L * c->kvslab());
+  AL(c->V, (size_t)L * c->kvslab());
+  AL(c->prev_ids, cap * 4);
+  AL(c->d, (size_t)L * cap * 4);
+  AL(c->s_cur, (size_t)cfg->max_batch * L * 4);
+  AL(c->s_prev, (size_t)cfg->max_batch * L * 4);
+  AL(c->budgets, (size_t)cfg->max_batch * L * 4);
+  AL(c->sel_idx, (size_t)L * cap * 4);
+  AL(c->sel_cnt, (size_t)L * cfg->max_batch * 4);
+  AL(c->rowmap, cap * 4);
+  AL(c->mrow, cap * 4);
+  AL(c->ints, 64);
+  AL(c->rope_tab, (size_t)cfg->max_seq * (cfg->head_dim / 2) * sizeof(float2));
+  AL(c->xs, cap * xw * c->esz);
+  AL(c->Q, cap * Hhd * c->esz);
+  AL(c->attn, cap * Hhd * c->esz);
+  AL(c->act, cap * F * c->esz);
+  AL(c->hmid, cap * D * 4);
+  AL(c->C, cap * cw * 4);
+  AL(c->conf, cap * 4);
+  AL(c->amax, cap * 4);
+#undef AL
+  if (e != cudaSuccess) {
+    std::string m = std::string("device allocation failed: ") + cudaGetErrorString(e);
+    cudaGetLastError();
+    free_all(c);
+    delete c;
+    return fail(nullptr, DCU_ENOMEM, m);
+  }
+  e = cudaMemset(c->ints, 0, 64);
+  if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
+  if (e == cudaSuccess && cfg->rope_theta > 0.0f)
+    e = launch_rope_table(c->rope_tab, cfg->max_seq, cfg->head_dim, cfg->rope_theta, 0);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    std::string m = std::string("context setup failed: ") + cudaGetErrorString(e);
+    free_all(c);
+    delete c;
+    return fail(nullptr, DCU_ECUDA, m);
+  }
+  *out = c;
+  return DCU_OK;
+}
+
+void dcu_destroy(dcu_ctx *ctx) {
+  if (!ctx) return;
+  cudaDeviceSynchronize();
+  free_all(ctx);
+  delete ctx;
+}
+
+int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_stream_t stream) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (!ids) return fail(c, DCU_EINVAL, "token_ids is NULL");
+  if (B <= 0 || N <= 0) return fail(c, DCU_EINVAL, "B and N must be > 0");
+  if (B > c->cfg.max_batch || N > c->cfg.max_seq)
+    return fail(c, DCU_ECAPACITY, "B or N above the context's max_batch / max_seq");
+  cudaStream_t s = (cudaStream_t)stream;
+  c->B = B;
+  c->N = N;
+  const int BN = B * N;
+  {
+    Prof p(c, DCU_K_REFRESH, s);
+    LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
+                               c->cfg.d_model, c->cfg.vocab, 1, c->status(), s));
+  }
+  LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), s));
+  for (int l = 0; l < c->cfg.n_layers; ++l)
+    if (int rc = run_layer(c, l, true, nullptr, nullptr, 0, s)) return rc;
+  CK(c, cudaMemsetAsync(c->s_prev, 0, (size_t)c->cfg.max_batch * c->cfg.n_layers * 4, s));
+  c->first_step = true;
+  c->have_cache = true;
+  return DCU_OK;
+}
+
+int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t *nkeys, int32_t B_layer,
+             int32_t B_window, dcu_stream_t stream) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (!c->have_cache) return fail(c, DCU_ESTATE, "dcu_step before dcu_full_forward");
+  if (!ids || !keys || !nkeys) return fail(c, DCU_EINVAL, "token_ids, key_positions or n_keys is NULL");
+  if (B_layer < 0 || B_window < 0) return fail(c, DCU_EINVAL, "B_layer and B_window must be >= 0");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int L = c->cfg.n_layers, BN = c->B * c->N;
+  {
+    Prof p(c, DCU_K_BUDGET, s);
+    LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, c->first_step ? 1 : 0, c->budgets, s));
+  }
+  {
+    Prof p(c, DCU_K_REFRESH, s);
+    LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
+                               c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
+  }
+  for (int l = 0; l < L; ++l)
+    if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) return rc;
+  CK(c, cudaMemcpyAsync(c->s_prev, c->s_cur, (size_t)c->B * L * 4, cudaMemcpyDeviceToDevice, s));
+  c->first_step = false;
+  return DCU_OK;
+}
+
+int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
+                  int32_t *out_count, dcu_stream_t stream) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (!c->have_cache) return fail(c, DCU_ESTATE, "commit_select before dcu_full_forward");
+  if (rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR)
+    return fail(c, DCU_EINVAL, "rule must be DCU_FRECHET, DCU_THRESHOLD or DCU_FACTOR");
+  if (!masked || !ids || !out_pos || !out_count) return fail(c, DCU_EINVAL, "a buffer is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  const dcu_cfg &g = c->cfg;
+  const int cap = (int)c->cap;
+  {
+    Prof p(c, DCU_K_LMHEAD, s);
+    LAUNCH(c, launch_plan_masked(masked, c->B, c->N, c->mrow, c->m_masked(), s));
+    LAUNCH(c, launch_gather_norm(g.dtype, c->mrow, c->m_masked(), cap, c->Hl(g.n_layers), c->final_norm, g.rms_eps,
+                             g.d_model, c->xs, s));
+    GemmSeg lm[1] = {{c->lm_head, g.vocab}};
+    LAUNCH(c, launch_gemm_simt(g.dtype, c->xs, g.d_model, c->m_masked(), cap, lm, 1, g.d_model, c->C, g.vocab, s));
+    LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));
+  }
+  {
+    Prof p(c, DCU_K_COMMIT, s);
+    LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, out_pos, out_count, s));
+  }
+  return DCU_OK;
+}
+
+int dcu_status(dcu_ctx *c, dcu_stream_t stream, int32_t *bits) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  CK(c, cudaStreamSynchronize((cudaStream_t)stream));
+  int32_t v = 0;
+  CK(c, cudaMemcpy(&v, c->status(), 4, cudaMemcpyDeviceToHost));
+  if (bits) *bits = v;
+  if (v != 0) {
+    CK(c, cudaMemset(c->status(), 0, 4));
+    return fail(c, DCU_EDEVICE, "device status word " + std::to_string(v));
+  }
+  return DCU_OK;
+}
+
+// ---------------------------------------------------------------- stateless kernels
+
+int dcu_budget_split(const float *s_prev, int32_t B, int32_t L, int32_t B_layer, int32_t uniform, int32_t *budgets,
+                     dcu_stream_t stream) {
+  if (!s_prev || !budgets || B <= 0 || L <= 0 || B_layer < 0)
+    return fail(nullptr, DCU_EINVAL, "dcu_budget_split: bad argument");
+  CK(nullptr, launch_budget_split(s_prev, B, L, B_layer, uniform, budgets, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+int dcu_select_tokens(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets, int32_t B,
+                      int32_t N, int32_t B_window, int32_t window_mode, int32_t *idx, int32_t *count, float *s,
+                      int32_t *status, dcu_stream_t stream) {
+  if (!d || !keys || !nkeys || !budgets || !idx || !count || !s || B <= 0 || N <= 0 || N > 16384 ||
+      B_window < 0 || (window_mode != 0 && window_mode != 1))
+    return fail(nullptr, DCU_EINVAL, "dcu_select_tokens: bad argument");
+  CK(nullptr, launch_select(d, keys, nkeys, budgets, 1, B, N, B_window, window_mode, idx, count, s, 1, nullptr,
+                            nullptr, nullptr, nullptr, status, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+int dcu_cosine_distance(const void *x, const void *y, const float *gain, int64_t rows, int32_t D, int32_t dtype,
+                        float *d, dcu_stream_t stream) {
+  if (!x || !y || !gain || !d || rows < 0 || D <= 0 || D % 8 || (dtype != DCU_F32 && dtype != DCU_BF16))
+    return fail(nullptr, DCU_EINVAL, "dcu_cosine_distance: bad argument");
+  CK(nullptr, launch_cosine_distance(dtype, x, y, gain, rows, D, d, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t *argmax, uint8_t *masked,
+                    int32_t *ids, int32_t B, int32_t N, int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {
+  if ((rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR) || !conf || !argmax || !masked || !ids ||
+      !out_pos || !out_count || B <= 0 || N <= 0 || N > 16384)
+    return fail(nullptr, DCU_EINVAL, "dcu_commit_rule: bad argument");
+  CK(nullptr, launch_commit_rule(rule, param, conf, argmax, masked, ids, B, N, out_pos, out_count,
+                                 (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+// ---------------------------------------------------------------- introspection
+
+static int tensor_ptr(dcu_ctx *c, int kind, int layer, char **p, int64_t *bytes) {
+  if (!c->have_cache) return fail(c, DCU_ESTATE, "no active shape (run dcu_full_forward first)");
+  const dcu_cfg &g = c->cfg;
+  const int L = g.n_layers;
+  const int64_t BN = (int64_t)c->B * c->N;
+  auto need = [&](int lo, int hi) { return layer >= lo && layer <= hi; };
+  switch (kind) {
+    case DCU_T_H:
+      if (!need(0, L)) break;
+      *p = (char *)c->Hl(layer);
+      *bytes = BN * g.d_model * (int64_t)c->esz;
+      return DCU_OK;
+    case DCU_T_K:
+    case DCU_T_V:
+      if (!need(0, L - 1)) break;
+      *p = (char *)(kind == DCU_T_K ? c->Kl(layer) : c->Vl(layer));
+      *bytes = BN * g.n_kv_heads * g.head_dim * (int64_t)c->esz;
+      return DCU_OK;
+    case DCU_T_D:
+      if (!need(0, L - 1)) break;
+      *p = (char *)c->dl(layer);
+      *bytes = BN * 4;
+      return DCU_OK;
+    case DCU_T_S:
+      *p = (char *)c->s_cur;
+      *bytes = (int64_t)c->B * L * 4;
+      return DCU_OK;
+    case DCU_T_S_PREV:
+      *p = (char *)c->s_prev;
+      *bytes = (int64_t)c->B * L * 4;
+      return DCU_OK;
+    case DCU_T_BUDGET:
+      *p = (char *)c->budgets;
+      *bytes = (int64_t)c->B * L * 4;
+      return DCU_OK;
+    case DCU_T_SEL:
+      if (!need(0, L - 1)) break;
+      *p = (char *)(c->sel_idx + (size_t)layer * c->cap);
+      *bytes = BN * 4;
+      return DCU_OK;
+    case DCU_T_SEL_COUNT:
+      if (!need(0, L - 1)) break;
+      *p = (char *)(c->sel_cnt + (size_t)layer * g.max_batch);
+      *bytes = (int64_t)c->B * 4;
+      return DCU_OK;
+    case DCU_T_CONF:
+      *p = (char *)c->conf;
+      *bytes = BN * 4;
+      return DCU_OK;
+    case DCU_T_ARGMAX:
+      *p = (char *)c->amax;
+      *bytes = BN * 4;
+      return DCU_OK;
+    default:
+      return fail(c, DCU_EINVAL, "unknown tensor kind");
+  }
+  return fail(c, DCU_EINVAL, "layer out of range for this tensor kind");
+}
+
+int dcu_tensor_bytes(const dcu_ctx *cc, int32_t kind, int64_t *bytes) {
+  dcu_ctx *c = const_cast<dcu_ctx *>(cc);
+  if (!c || !bytes) return fail(nullptr, DCU_EINVAL, "ctx or bytes is NULL");
+  char *p;
+  int layer = (kind == DCU_T_S || kind == DCU_T_S_PREV || kind == DCU_T_BUDGET || kind == DCU_T_CONF ||
+               kind == DCU_T_ARGMAX)
+                  ? 0
+                  : 0;
+  return tensor_ptr(c, kind, layer, &p, bytes);
+}
+
+int dcu_get_tensor(dcu_ctx *c, int32_t kind, int32_t layer, void *dst, int64_t bytes, dcu_stream_t stream) {
+  if (!c || !dst) return fail(c, DCU_EINVAL, "ctx or dst is NULL");
+  char *p;
+  int64_t n;
+  if (int rc = tensor_ptr(c, kind, layer, &p, &n)) return rc;
+  if (bytes != n) return fail(c, DCU_EINVAL, "size mismatch: expected " + std::to_string(n) + " bytes");
+  CK(c, cudaMemcpyAsync(dst, p, n, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+int dcu_set_tensor(dcu_ctx *c, int32_t kind, int32_t layer, const void *src, int64_t bytes, dcu_stream_t stream) {
+  if (!c || !src) return fail(c, DCU_EINVAL, "ctx or src is NULL");
+  if (kind != DCU_T_H && kind != DCU_T_K && kind != DCU_T_V && kind != DCU_T_S_PREV)
+    return fail(c, DCU_EINVAL, "only H, K, V and S_PREV can be set");
+  char *p;
+  int64_t n;
+  if (int rc = tensor_ptr(c, kind, layer, &p, &n)) return rc;
+  if (bytes != n) return fail(c, DCU_EINVAL, "size mismatch: expected " + std::to_string(n) + " bytes");
+  CK(c, cudaMemcpyAsync(p, src, n, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
+  if (kind == DCU_T_S_PREV) c->first_step = false;
+  return DCU_OK;
+}
+
+// ---------------------------------------------------------------- profiling
+
+int dcu_profile_enable(dcu_ctx *c, int32_t max_launches) {
+  if (!c || max_launches < 0) return fail(c, DCU_EINVAL, "bad argument");
+  for (auto &pc : c->prof) {
+    for (auto &e : pc.ev) {
+      cudaEventDestroy(e.a);
+      cudaEventDestroy(e.b);
+    }
+    pc.ev.clear();
+    pc.used = pc.dropped = 0;
+    for (int i = 0; i < max_launches; ++i) {
+      EventPair e;
+      CK(c, cudaEventCreate(&e.a));
+      CK(c, cudaEventCreate(&e.b));
+      pc.ev.push_back(e);
+    }
+  }
+  c->prof_max = max_launches;
+  return DCU_OK;
+}
+
+int dcu_profile_read(dcu_ctx *c, int32_t k, double *total_ms, int64_t *launches, int32_t reset) {
+  if (!c || k < 0 || k >= DCU_K_COUNT || !total_ms || !launches) return fail(c, DCU_EINVAL, "bad argument");
+  ProfClass &pc = c->prof[k];
+  double t = 0.0;
+  for (int64_t i = 0; i < pc.used; ++i) {
+    CK(c, cudaEventSynchronize(pc.ev[i].b));
+    float ms = 0.f;
+    CK(c, cudaEventElapsedTime(&ms, pc.ev[i].a, pc.ev[i].b));
+    t += ms;
+  }
+  *total_ms = t;
+  *launches = pc.used;
+  if (pc.dropped) return fail(c, DCU_ECAPACITY, "more launches than profile slots");
+  if (reset) pc.used = pc.dropped = 0;
+  return DCU_OK;
+}
+
+int64_t dcu_launch_count(const dcu_ctx *c) { return c ? c->launches : 0; }
+
+const char *dcu_kernel_class_name(int32_t k) {
+  static const char *names[DCU_K_COUNT] = {"refresh", "budget",   "select", "gather", "gemm",
+                                           "epilogue", "attention", "scatter", "lmhead", "commit"};
+  return (k >= 0 && k < DCU_K_COUNT) ? names[k] : "?";
+}
+
+}  // extern "C"

@@ -1,0 +1,140 @@
+// Shared device helpers of libdcu (sm_100a).
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/dcu.h"
+
+namespace dcu {
+
+typedef __nv_bfloat16 bf16;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+
+template <class T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+template <class T> __device__ __forceinline__ uint32_t bits_of(T x);
+template <> __device__ __forceinline__ uint32_t bits_of<float>(float x) { return __float_as_uint(x); }
+template <> __device__ __forceinline__ uint32_t bits_of<bf16>(bf16 x) { return (uint32_t)__bfloat16_as_ushort(x); }
+
+// 16-byte vector of T: 4 floats or 8 bf16.
+template <class T> struct Vec;
+template <> struct Vec<float> { static constexpr int n = 4; };
+template <> struct Vec<bf16> { static constexpr int n = 8; };
+
+template <class T>
+__device__ __forceinline__ void load_vec(const T *p, float (&v)[Vec<T>::n], uint32_t (&b)[Vec<T>::n]) {
+  uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const T *e = reinterpret_cast<const T *>(&u);
+#pragma unroll
+  for (int i = 0; i < Vec<T>::n; ++i) { v[i] = to_f(e[i]); b[i] = bits_of<T>(e[i]); }
+}
+
+template <class T>
+__device__ __forceinline__ void load_vec(const T *p, float (&v)[Vec<T>::n]) {
+  uint4 u = *reinterpret_cast<const uint4 *>(p);
+  const T *e = reinterpret_cast<const T *>(&u);
+#pragma unroll
+  for (int i = 0; i < Vec<T>::n; ++i) v[i] = to_f(e[i]);
+}
+
+template <class T>
+__device__ __forceinline__ void store_vec(T *p, const float (&v)[Vec<T>::n]) {
+  uint4 u;
+  T *e = reinterpret_cast<T *>(&u);
+#pragma unroll
+  for (int i = 0; i < Vec<T>::n; ++i) e[i] = from_f<T>(v[i]);
+  *reinterpret_cast<uint4 *>(p) = u;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Block-wide sum with a fixed reduction tree (deterministic).  `red` must
+// hold blockDim.x / 32 elements; every thread gets the result.
+template <class T>
+__device__ __forceinline__ T block_sum(T v, T *red) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  T t = (threadIdx.x < nw) ? red[threadIdx.x] : T(0);
+  if (w == 0) t = warp_sum(t);
+  if (threadIdx.x == 0) red[0] = t;
+  __syncthreads();
+  T r = red[0];
+  __syncthreads();
+  return r;
+}
+
+// Exclusive prefix sum over the block of one int per thread (thread order);
+// returns the exclusive prefix, total in *total.  `red` holds 32 ints.
+__device__ __forceinline__ int block_exclusive_scan(int v, int *red, int *total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) red[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = (lane < nw) ? red[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    red[lane] = t;  // inclusive scan of warp totals
+  }
+  __syncthreads();
+  int base = (w > 0) ? red[w - 1] : 0;
+  *total = red[nw - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+// Cosine distance of [DLLM] "关键设计 1" from fp64 partial sums, with the
+// equal-rows / zero-norm rules; clamped to [0, 2].
+__device__ __forceinline__ float finish_cosine_distance(double dot, double nx, double ny, bool same) {
+  if (same) return 0.0f;
+  if (nx == 0.0 && ny == 0.0) return 0.0f;
+  if (nx == 0.0 || ny == 0.0) return 1.0f;
+  double d = 1.0 - dot / (sqrt(nx) * sqrt(ny));
+  d = d < 0.0 ? 0.0 : (d > 2.0 ? 2.0 : d);
+  return (float)d;
+}
+
+// Row r of the packed recompute set -> global row b*N + i (written by the
+// select / plan kernels).
+struct RowPlan {
+  const int32_t *rowmap;   // [cap] global row index b*N + i
+  const int32_t *m_total;  // device scalar
+};
+
+}  // namespace dcu

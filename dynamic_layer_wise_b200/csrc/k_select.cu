@@ -1,0 +1,411 @@
+// Integer-deciding kernels of the DCU step and the commit:
+//   * layer budget split (one thread per sequence, fp64),
+//   * per-layer token selection: forced window + top-B radix select outside
+//     it + index-ordered compaction, plus s = mean d (one CTA per sequence),
+//   * row plans (which packed row is which sequence position),
+//   * the commit rule: bitonic sort of confidences, fp64 prefix scan,
+//     Fréchet / threshold / factor count, commit (one CTA per sequence).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcu {
+
+static constexpr int kSelThreads = 1024;
+static constexpr int kMaxSeq = 16384;
+
+// ------------------------------------------------------------------ budget split
+// [DLLM] "关键设计 1", the budget equation B^l = (B_layer * L) s^l / sum_k s^k,
+// rounded by floor + largest remainder (ties -> lower layer) so that each row
+// sums to B_layer * L; uniform when asked or when the row sums to 0.  If the
+// floors overshoot (q rounded up to an integer), one is taken back from the
+// layers with the smallest fractional parts (ties -> higher layer) above 0.
+__global__ void k_budget_split(const float *__restrict__ s_prev, int B, int L, int B_layer, int uniform,
+                               int32_t *__restrict__ budgets) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const float *s = s_prev + (size_t)b * L;
+  int32_t *out = budgets + (size_t)b * L;
+  double total = 0.0;
+  for (int l = 0; l < L; ++l) total = __dadd_rn(total, (double)s[l]);
+  if (uniform || total == 0.0) {
+    for (int l = 0; l < L; ++l) out[l] = B_layer;
+    return;
+  }
+  const double T = (double)B_layer * (double)L;
+  long long sum_fl = 0;
+  for (int l = 0; l < L; ++l) {
+    double q = __ddiv_rn(__dmul_rn(T, (double)s[l]), total);
+    long long f = (long long)floor(q);
+    out[l] = (int32_t)f;
+    sum_fl += f;
+  }
+  long long R = (long long)B_layer * L - sum_fl;
+  if (R == 0) return;
+  // ranks are computed against the untouched floors, then applied
+  for (int l = 0; l < L; ++l) {
+    double ql = __ddiv_rn(__dmul_rn(T, (double)s[l]), total);
+    double fl = floor(ql), frl = ql - fl;
+    int rank = 0;
+    for (int k = 0; k < L; ++k) {
+      double qk = __ddiv_rn(__dmul_rn(T, (double)s[k]), total);
+      double fk = floor(qk), frk = qk - fk;
+      if (R > 0) {
+        if (frk > frl || (frk == frl && k < l)) ++rank;
+      } else {
+        if (fk > 0.0 && (frk < frl || (frk == frl && k > l))) ++rank;
+      }
+    }
+    if (R > 0 && rank < R) out[l] = (int32_t)fl + 1;
+    if (R < 0 && fl > 0.0 && rank < -R) out[l] = (int32_t)fl - 1;
+  }
+}
+
+cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform, int32_t *budgets,
+                                cudaStream_t s) {
+  k_budget_split<<<(B + 63) / 64, 64, 0, s>>>(s_prev, B, L, B_layer, uniform, budgets);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ selection
+// One CTA per sequence.  s = mean(d) (fp64, fixed tree); W = union of the key
+// windows ([DLLM] "关键设计 2"); k = min(budget, N - |W|); the k-th largest d
+// outside W is found by a 4-pass MSB radix select on the float bits (d >= 0,
+// so the bits order like the values); ties at the threshold go to the lower
+// indices; U = W + selected, compacted in index order.
+__global__ void __launch_bounds__(kSelThreads)
+    k_select(const float *__restrict__ d, const int32_t *__restrict__ keys, const int32_t *__restrict__ nkeys,
+             const int32_t *__restrict__ budgets, int budget_stride, int B, int N, int Bw, int mode,
+             int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
+             float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
+             int32_t *__restrict__ done, int32_t *__restrict__ status) {
+  extern __shared__ uint8_t smem[];
+  uint32_t *sd = reinterpret_cast<uint32_t *>(smem);     // [N] d bits
+  uint8_t *flag = smem + (size_t)N * sizeof(uint32_t);   // [N] 0 none, 1 window, 2 top-B
+  __shared__ int hist[256];
+  __shared__ int red_i[32];
+  __shared__ double red_d[32];
+  __shared__ int s_bin, s_rem;
+  __shared__ bool s_last;
+
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const float *db = d + (size_t)b * N;
+
+  double acc = 0.0;
+  for (int i = tid; i < N; i += nthr) {
+    float v = db[i];
+    sd[i] = __float_as_uint(v);
+    flag[i] = 0;
+    acc += (double)v;
+  }
+  if (d_next_zero)
+    for (int i = tid; i < N; i += nthr) d_next_zero[(size_t)b * N + i] = 0.f;
+  acc = block_sum(acc, red_d);
+  if (tid == 0) s_out[(size_t)b * s_stride] = (float)(acc / (double)N);
+
+  // forced window
+  int nk = nkeys[b];
+  if (nk < 0 || nk > N) {
+    if (tid == 0 && status) atomicOr(status, DCU_ST_BAD_KEY);
+    nk = nk < 0 ? 0 : N;
+  }
+  if (Bw > 0 && nk > 0) {
+    const int h = Bw / 2;
+    const int width = (mode == 0) ? (2 * h + 1) : Bw;
+    const long long total = (long long)nk * width;
+    for (long long t = tid; t < total; t += nthr) {
+      const int k = (int)(t / width), off = (int)(t - (long long)k * width);
+      const int p = keys[(size_t)b * N + k];
+      if (p < 0 || p >= N) {
+        if (off == 0 && status) atomicOr(status, DCU_ST_BAD_KEY);
+        continue;
+      }
+      const int i = p - h + off;
+      if (i >= 0 && i < N) flag[i] = 1;
+    }
+  }
+  __syncthreads();
+  int inW = 0;
+  for (int i = tid; i < N; i += nthr) inW += (flag[i] == 1);
+  inW = block_sum(inW, red_i);
+  const int avail = N - inW;
+  int k = budgets[(size_t)b * budget_stride];
+  k = k < 0 ? 0 : (k > avail ? avail : k);
+
+  uint32_t thr = 0xffffffffu;  // select d > thr, plus `need` ties at thr
+  int need = 0;
+  bool take_all = (k == avail);
+  if (k > 0 && !take_all) {
+    uint32_t prefix = 0, mask = 0;
+    int rem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int t = tid; t < 256; t += nthr) hist[t] = 0;
+      __syncthreads();
+      for (int i = tid; i < N; i += nthr) {
+        const uint32_t u = sd[i];
+        if (flag[i] == 0 && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        int cum = 0, bin = 0;
+        for (bin = 255; bin >= 0; --bin) {
+          if (cum + hist[bin] >= rem) break;
+          cum += hist[bin];
+        }
+        s_bin = bin;
+        s_rem = rem - cum;
+      }
+      __syncthreads();
+      prefix |= (uint32_t)s_bin << shift;
+      mask |= 255u << shift;
+      rem = s_rem;
+      __syncthreads();
+    }
+    thr = prefix;
+    need = rem;
+  }
+
+  // mark the top-B: strictly above thr, then the first `need` ties in index order
+  const int chunk = (N + nthr - 1) / nthr;
+  const int i0 = tid * chunk, i1 = min(N, i0 + chunk);
+  int nt = 0;
+  if (k > 0) {
+    for (int i = i0; i < i1; ++i) {
+      if (flag[i] != 0) continue;
+      if (take_all || sd[i] > thr) flag[i] = 2;
+      else if (sd[i] == thr) ++nt;
+    }
+  }
+  int tot;
+  int before = block_exclusive_scan(nt, red_i, &tot);
+  if (k > 0 && !take_all && need > 0) {
+    for (int i = i0; i < i1; ++i) {
+      if (flag[i] == 0 && sd[i] == thr) {
+        if (before < need) flag[i] = 2;
+        ++before;
+      }
+    }
+  }
+  __syncthreads();
+  // compaction in index order
+  int ns = 0;
+  for (int i = i0; i < i1; ++i) ns += (flag[i] != 0);
+  int pos = block_exclusive_scan(ns, red_i, &tot);
+  int32_t *ib = idx + (size_t)b * N;
+  for (int i = i0; i < i1; ++i)
+    if (flag[i] != 0) ib[pos++] = i;
+  if (tid == 0) count[b] = tot;
+
+  // the last CTA to finish builds the packed row plan of all sequences
+  if (rowmap == nullptr) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(done, 1) == B - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  int off = 0;
+  for (int bb = 0; bb < B; ++bb) {
+    const int c = *((volatile int32_t *)count + bb);
+    const volatile int32_t *src = idx + (size_t)bb * N;
+    for (int j = tid; j < c; j += nthr) rowmap[off + j] = bb * N + src[j];
+    off += c;
+  }
+  if (tid == 0) {
+    *m_total = off;
+    *done = 0;
+  }
+}
+
+cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
+                          int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
+                          float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
+                          int32_t *done, int32_t *status, cudaStream_t s) {
+  if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
+  size_t smem = (size_t)N * 5;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSeq * 5);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  k_select<<<B, kSelThreads, smem, s>>>(d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
+                                        s_stride, d_next_zero, rowmap, m_total, done, status);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ row plans
+__global__ void k_plan_all(int BN, int32_t *rowmap, int32_t *m_total) {
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < BN; r += gridDim.x * blockDim.x) rowmap[r] = r;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *m_total = BN;
+}
+
+cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, cudaStream_t s) {
+  const int BN = B * N;
+  int grid = (BN + 255) / 256;
+  if (grid > 1024) grid = 1024;
+  k_plan_all<<<grid, 256, 0, s>>>(BN, rowmap, m_total);
+  return cudaGetLastError();
+}
+
+// Masked positions of all sequences, in (b, i) order, as packed rows.
+__global__ void __launch_bounds__(1024) k_plan_masked(const uint8_t *__restrict__ masked, int B, int N,
+                                                      int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total) {
+  __shared__ int red[32];
+  const int BN = B * N, nthr = blockDim.x, tid = threadIdx.x;
+  const int chunk = (BN + nthr - 1) / nthr;
+  const int i0 = tid * chunk, i1 = min(BN, i0 + chunk);
+  int c = 0;
+  for (int i = i0; i < i1; ++i) c += masked[i] != 0;
+  int tot;
+  int pos = block_exclusive_scan(c, red, &tot);
+  for (int i = i0; i < i1; ++i)
+    if (masked[i]) rowmap[pos++] = i;
+  if (tid == 0) *m_total = tot;
+}
+
+cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
+                               cudaStream_t s) {
+  k_plan_masked<<<1, 1024, 0, s>>>(masked, B, N, rowmap, m_total);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ commit rule
+// [FRECHET] "整体框架": sort the masked positions by confidence (descending;
+// ties -> lower position: key = c bits << 32 | ~position), then
+//   Fréchet ("关键设计 1/2"): S_n = sum_{j<=n} c_(j) (fp64), L_n = max(0, S_n - (n-1)),
+//     U_n = 1 - c_(n), n* = max{n : L_n - U_n > delta}, else 1;
+//   threshold ("研究背景与动机"): n* = #{c >= tau}, else 1;
+//   factor (same): n* = max{n : (n+1)(1 - c_(n)) < f}, else 1;
+// commit the first n*: ids <- argmax, masked <- 0, out_positions, out_count.
+__global__ void __launch_bounds__(1024)
+    k_commit_rule(int rule, float param, const float *__restrict__ conf, const int32_t *__restrict__ amax,
+                  uint8_t *__restrict__ masked, int32_t *__restrict__ ids, int N, int32_t *__restrict__ out_pos,
+                  int32_t *__restrict__ out_count) {
+  extern __shared__ uint64_t keys[];  // [P]
+  __shared__ int red[32];
+  __shared__ double redd[32];
+  __shared__ int s_best;
+  const int b = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
+  const uint8_t *mb = masked + (size_t)b * N;
+  const float *cb = conf + (size_t)b * N;
+
+  // compact the masked positions (index order) into keys
+  const int chunk = (N + nthr - 1) / nthr;
+  const int i0 = tid * chunk, i1 = min(N, i0 + chunk);
+  int c = 0;
+  for (int i = i0; i < i1; ++i) c += mb[i] != 0;
+  int m;
+  int pos = block_exclusive_scan(c, red, &m);
+  for (int i = i0; i < i1; ++i)
+    if (mb[i]) keys[pos++] = ((uint64_t)__float_as_uint(cb[i]) << 32) | (uint64_t)(~(uint32_t)i);
+  int P = 1;
+  while (P < m) P <<= 1;
+  for (int t = m + tid; t < P; t += nthr) keys[t] = 0ull;
+  __syncthreads();
+  // bitonic sort, descending
+  for (int size = 2; size <= P; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = tid; t < P; t += nthr) {
+        const int partner = t ^ stride;
+        if (partner > t) {
+          const bool desc = ((t & size) == 0);
+          const uint64_t a = keys[t], bk = keys[partner];
+          if (desc ? (a < bk) : (a > bk)) { keys[t] = bk; keys[partner] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // n*: each thread takes a contiguous run of sorted entries; fp64 prefix sums
+  const int run = (m + nthr - 1) / nthr;
+  const int j0 = tid * run, j1 = min(m, j0 + run);
+  double local = 0.0;
+  for (int j = j0; j < j1; ++j) local += (double)__uint_as_float((uint32_t)(keys[j] >> 32));
+  // exclusive scan of the per-thread fp64 sums (thread order)
+  {
+    const int lane = tid & 31, w = tid >> 5, nw = nthr >> 5;
+    double x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      double y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) redd[w] = x;
+    __syncthreads();
+    if (w == 0) {
+      double t = (lane < nw) ? redd[lane] : 0.0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        double y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      redd[lane] = t;
+    }
+    __syncthreads();
+    local = ((w > 0) ? redd[w - 1] : 0.0) + x - local;  // exclusive prefix of this thread's run
+    __syncthreads();
+  }
+  if (tid == 0) s_best = 0;
+  __syncthreads();
+  int best = 0;
+  const double prm = (double)param;
+  double S = local;
+  for (int j = j0; j < j1; ++j) {
+    const int n = j + 1;
+    const float cj = __uint_as_float((uint32_t)(keys[j] >> 32));
+    const double c64 = (double)cj;
+    S = __dadd_rn(S, c64);
+    bool pass;
+    if (rule == DCU_FRECHET) {
+      double Ln = __dsub_rn(S, (double)(n - 1));
+      Ln = Ln > 0.0 ? Ln : 0.0;
+      const double Un = __dsub_rn(1.0, c64);
+      pass = __dsub_rn(Ln, Un) > prm;
+    } else if (rule == DCU_THRESHOLD) {
+      pass = cj >= param;
+    } else {
+      pass = __dmul_rn((double)(n + 1), __dsub_rn(1.0, c64)) < prm;
+    }
+    if (pass && n > best) best = n;
+  }
+  if (rule == DCU_THRESHOLD) {
+    int cnt = 0;
+    for (int j = j0; j < j1; ++j) cnt += (__uint_as_float((uint32_t)(keys[j] >> 32)) >= param);
+    cnt = block_sum(cnt, red);
+    best = cnt;
+    if (tid == 0) s_best = best;
+  } else {
+    atomicMax(&s_best, best);
+  }
+  __syncthreads();
+  int nstar = s_best;
+  if (m == 0) nstar = 0;
+  else if (nstar == 0) nstar = 1;
+  for (int j = tid; j < nstar; j += nthr) {
+    const int p = (int)(~(uint32_t)(keys[j] & 0xffffffffull));
+    out_pos[(size_t)b * N + j] = p;
+    ids[(size_t)b * N + p] = amax[(size_t)b * N + p];
+    masked[(size_t)b * N + p] = 0;
+  }
+  if (tid == 0) out_count[b] = nstar;
+}
+
+cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
+                               int32_t *ids, int B, int N, int32_t *out_pos, int32_t *out_count, cudaStream_t s) {
+  if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
+  int P = 1;
+  while (P < N) P <<= 1;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e =
+        cudaFuncSetAttribute(k_commit_rule, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSeq * sizeof(uint64_t));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  k_commit_rule<<<B, 1024, (size_t)P * sizeof(uint64_t), s>>>(rule, param, conf, amax, masked, ids, N, out_pos,
+                                                               out_count);
+  return cudaGetLastError();
+}
+
+}  // namespace dcu

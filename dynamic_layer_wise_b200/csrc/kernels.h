@@ -1,0 +1,62 @@
+// Host-side launchers of the libdcu kernels (internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dcu {
+
+// One weight matrix of a concatenated GEMM output: rows [row0, row0 + rows) of
+// the output come from W ([rows][K], row-major).
+struct GemmSeg {
+  const void *W;
+  int rows;
+};
+
+// ---- row kernels (k_rows.cu)
+cudaError_t launch_rope_table(float2 *tab, int max_seq, int head_dim, float theta, cudaStream_t s);
+cudaError_t launch_embed_refresh(int dtype, const int32_t *ids, int32_t *prev_ids, const void *embed, void *H0,
+                                 float *d0, const float *g0, int BN, int D, int V, int full, int32_t *status,
+                                 cudaStream_t s);
+cudaError_t launch_cosine_distance(int dtype, const void *x, const void *y, const float *g, int64_t rows, int D,
+                                   float *d, cudaStream_t s);
+cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *m_total, int cap, const void *H,
+                               const float *g, float eps, int D, void *xs, cudaStream_t s);
+cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total,
+                           int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab, int use_rope, void *Q,
+                           void *Kc, void *Vc, cudaStream_t s);
+cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
+                         const void *Hl, const float *g2, float eps, int D, float *hmid, void *xs, cudaStream_t s);
+cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const int32_t *m_total, int cap, int F, void *act,
+                              cudaStream_t s);
+cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const int32_t *rowmap,
+                                    const int32_t *m_total, int cap, const float *hmid, void *Hnext,
+                                    const float *g_next, float *d_next, int D, cudaStream_t s);
+cudaError_t launch_softmax_max(const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
+                               int V, float *conf, int32_t *amax, cudaStream_t s);
+
+// ---- selection, budgets and commit (k_select.cu)
+cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform, int32_t *budgets,
+                                cudaStream_t s);
+// budgets: pointer to element [0] of the layer's column; budget_stride = L.
+// s_out: pointer to the layer's column of s [B][L]; s_stride = L.
+// rowmap / m_total / done may be null (stateless use).
+cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
+                          int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
+                          float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
+                          int32_t *done, int32_t *status, cudaStream_t s);
+cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, cudaStream_t s);
+cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
+                               cudaStream_t s);
+cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
+                               int32_t *ids, int B, int N, int32_t *out_pos, int32_t *out_count, cudaStream_t s);
+
+// ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total
+cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,
+                             const GemmSeg *segs, int nseg, int K, float *C, int ldc, cudaStream_t s);
+
+// ---- attention (k_attn.cu): out[r][h] = softmax(q K^T / sqrt(hd)) V over all N keys of row r's sequence
+cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,
+                             int N, int H, int Hkv, int hd, const void *Kc, const void *Vc, void *out,
+                             cudaStream_t s);
+
+}  // namespace dcu

@@ -237,3 +237,35 @@ def device_fill_(t, value: float, stream=None):
     if rc != 0:
         raise RuntimeError(f"dcugen_fill failed ({rc})")
     return t
+
+
+def device_weights(shape: ModelShape, seed: int, device: str = "cuda") -> dict:
+    """The seeded synthetic model on the device, in the layout of include/dcu.h
+    (norm gains float32 ones), filled by the device generator."""
+    import torch
+    dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
+
+    def rnd(tid, rows, cols):
+        t = torch.empty((rows, cols), dtype=dt, device=device)
+        return device_normal_(t, seed, tid, shape.init_std)
+
+    def ones():
+        return torch.ones(shape.d_model, dtype=torch.float32, device=device)
+
+    ws = shape.weight_shapes()
+    layers = []
+    for l in range(shape.n_layers):
+        lw = {"attn_norm": ones(), "ffn_norm": ones()}
+        for name in LAYER_TENSORS:
+            lw[name] = rnd(layer_tid(l, name), *ws[name])
+        layers.append(lw)
+    return {"embed": rnd(TID_EMBED, shape.vocab, shape.d_model),
+            "lm_head": rnd(TID_LM_HEAD, shape.vocab, shape.d_model),
+            "final_norm": ones(), "layers": layers}
+
+
+def cfg_dict(shape: ModelShape, max_batch: int, max_seq: int, window_mode: int = 0) -> dict:
+    return dict(n_layers=shape.n_layers, d_model=shape.d_model, n_heads=shape.n_heads, n_kv_heads=shape.n_kv_heads,
+                head_dim=shape.head_dim, d_ffn=shape.d_ffn, vocab=shape.vocab, mask_id=shape.mask_id,
+                max_batch=max_batch, max_seq=max_seq, dtype=shape.dtype, rms_eps=shape.rms_eps,
+                rope_theta=shape.rope_theta, window_mode=window_mode)

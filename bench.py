@@ -110,7 +110,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- CPU oracle sample
 
-def cpu_sample_step(shape, seed, N, n_prompt, B_layer, B_window, lm_rows=8, vocab_frac=8):
+def cpu_sample_step(shape, seed, N, n_prompt, B_layer, B_window, lm_rows=32, vocab_frac=4, target_s=8.0):
     """Times the fp64 oracle on a bounded sample of one DCU step + commit and
     extrapolates to a whole step: one layer's selection + recompute of
     |W| + B_layer rows (x n_layers), and the LM head + softmax-max of `lm_rows`
@@ -143,20 +143,25 @@ def cpu_sample_step(shape, seed, N, n_prompt, B_layer, B_window, lm_rows=8, voca
     c_all = np.abs(I.normal_values(seed, 9006, 0, N, 0.001, "f32")) + 1e-5
     masked = np.zeros(N, bool)
     masked[n_prompt:] = True
-    t0 = time.perf_counter()
-    U = O.select_rows(d, keys, B_window, B_layer, 0)
-    O.layer_rows(lw, cfg, H[U], U, K.copy(), V.copy())
+    t_start = time.perf_counter()
+    reps, t_layer = 0, 0.0
+    while reps < 32 and (reps == 0 or t_layer < target_s):
+        t0 = time.perf_counter()
+        U = O.select_rows(d, keys, B_window, B_layer, 0)
+        O.layer_rows(lw, cfg, H[U], U, K.copy(), V.copy())
+        t_layer += time.perf_counter() - t0
+        reps += 1
     t1 = time.perf_counter()
     O.confidence(H[:lm_rows], ones, lm, cfg.rms_eps)
     t2 = time.perf_counter()
     O.commit(c_all, np.zeros(N, np.int64), masked, np.zeros(N, np.int64), O.RULE_FRECHET, 0.1)
     t3 = time.perf_counter()
-    step_s = shape.n_layers * (t1 - t0) + (t2 - t1) * vocab_frac * (n_masked / lm_rows) + (t3 - t2)
+    step_s = shape.n_layers * (t_layer / reps) + (t2 - t1) * vocab_frac * (n_masked / lm_rows) + (t3 - t2)
     threads = max([x.get("num_threads", 1) for x in threadpool_info()] or [1])
-    sample = (f"1 of {shape.n_layers} layers ({len(U)} recomputed rows, N={N}) x {shape.n_layers}, "
+    sample = (f"layer 0 of {shape.n_layers} ({len(U)} recomputed rows, N={N}) timed {reps}x, scaled x{shape.n_layers}; "
               f"LM head + softmax-max of {lm_rows} of {n_masked} masked rows over {nv} of {shape.vocab} vocab "
-              f"entries (scaled), commit over {n_masked}; measured {t3 - t0:.2f} s")
-    return step_s, t3 - t0, threads, sample
+              f"entries (scaled), commit over {n_masked}; measured {t3 - t_start:.2f} s")
+    return step_s, t3 - t_start, threads, sample
 
 
 # ---------------------------------------------------------------- roofline bookkeeping

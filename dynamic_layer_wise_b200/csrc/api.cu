@@ -221,6 +221,10 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
 
 }  // namespace
 
+namespace dcu {
+void set_global_error(const char *msg) { g_last_error = msg; }
+}  // namespace dcu
+
 extern "C" {
 
 const char *dcu_last_error(const dcu_ctx *ctx) { return ctx ? ctx->err.c_str() : g_last_error.c_str(); }

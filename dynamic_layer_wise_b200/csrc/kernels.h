@@ -5,6 +5,9 @@
 
 namespace dcu {
 
+// Sets the text dcu_last_error(NULL) returns (calls that have no context).
+void set_global_error(const char *msg);
+
 // One weight matrix of a concatenated GEMM output: rows [row0, row0 + rows) of
 // the output come from W ([rows][K], row-major).
 struct GemmSeg {

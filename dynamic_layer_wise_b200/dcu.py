@@ -73,6 +73,7 @@ _SIGS = {
     "dcu_profile_read": (_i32, [_vp, _i32, ctypes.POINTER(_f64), ctypes.POINTER(_i64), _i32]),
     "dcu_kernel_class_name": (ctypes.c_char_p, [_i32]),
     "dcu_launch_count": (_i64, [_vp]),
+    "dcu_lm_confidence_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
 }
 
 
@@ -279,3 +280,16 @@ def dcu_kernel_class_name(k: int) -> str:
 
 def dcu_launch_count(ctx: Context) -> int:
     return int(lib().dcu_launch_count(ctx.handle))
+
+
+def dcu_lm_confidence_noalloc(h_rows, final_norm, lm_head, rms_eps: float = 1e-5, stream=None):
+    """Confidence and argmax of final-layer rows with no device allocation by the
+    library (the outputs are allocated here, by the caller side)."""
+    m, D = h_rows.shape
+    V = lm_head.shape[0]
+    dt = {torch.bfloat16: DCU_BF16, torch.float32: DCU_F32}[h_rows.dtype]
+    conf = torch.empty(m, dtype=torch.float32, device=h_rows.device)
+    amax = torch.empty(m, dtype=torch.int32, device=h_rows.device)
+    _check(lib().dcu_lm_confidence_noalloc(_ptr(h_rows), _ptr(final_norm), _ptr(lm_head), m, D, V, dt,
+                                           float(rms_eps), _ptr(conf), _ptr(amax), _stream(stream)))
+    return conf, amax

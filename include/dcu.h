@@ -179,6 +179,26 @@ int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t 
                     int32_t *token_ids, int32_t B, int32_t N, int32_t *out_positions, int32_t *out_count,
                     dcu_stream_t stream);
 
+/* LM-head confidence and argmax of m final-layer rows without any device
+ * allocation, for callers that cannot call cudaMalloc (a host framework that
+ * owns every device allocation through its own pool, or a serving process
+ * whose allocator is frozen).  The pages have no counterpart to this call: it
+ * is the LM-head stage of commit_select (final RMSNorm, logits, max softmax
+ * probability, lowest-id argmax) as a stateless function.
+ * h_rows: dev [m][D] in dtype; final_norm: dev float [D]; lm_head: dev
+ * [V][D] in dtype; conf: dev float [m]; argmax: dev int32 [m].
+ * Scratch is one static device array of about 12 MB inside libdcu, held by
+ * every GPU that loads the library until the process exits; the call
+ * allocates nothing.  The first call on a device takes the array's address
+ * (cudaGetSymbolAddress) with that device current, so make that first call
+ * before any stream capture.  Calls share the array: calls that overlap on
+ * the GPU (other streams, other host threads) race and must be serialised by
+ * the caller.  Limits: m <= 256 and D <= 8192 (DCU_ECAPACITY beyond),
+ * D % 64 == 0 (DCU_EINVAL). */
+int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_norm, const void *lm_head, int32_t m,
+                              int32_t D, int32_t V, int32_t dtype, float rms_eps, float *conf, int32_t *argmax,
+                              dcu_stream_t stream);
+
 /* ---- introspection (tests, teacher forcing) ---- */
 
 #define DCU_T_H         0  /* layer 0..L   : [B][N][d_model] dtype        */

@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "../../include/dcu.h"
+#include "gemm_tc.h"
 #include "kernels.h"
 
 using namespace dcu;
@@ -31,6 +32,10 @@ struct ProfClass {
 size_t esize(int dtype) { return dtype == DCU_BF16 ? 2 : 4; }
 
 }  // namespace
+
+struct LayerMaps {
+  CUtensorMap wq, wk, wv, wo, wg, wu, wd;
+};
 
 struct dcu_ctx {
   dcu_cfg cfg{};
@@ -58,6 +63,14 @@ struct dcu_ctx {
   int32_t *amax = nullptr, *mrow = nullptr;
   std::vector<void *> allocs;
   std::string err;
+  // tcgen05 GEMM state (bf16 models)
+  int num_sms = 148;
+  int gemm_bn = 128;          // token tile of the current call
+  int gemm_rows_hint = 128;   // expected rows per layer of the current call
+  size_t ws_elems = 0;        // capacity of C in floats
+  std::vector<LayerMaps> lmaps;
+  CUtensorMap lm_map;
+  CUtensorMap xs_map[2], attn_map[2], act_map[2];  // token tiles 128, 256
   // profiling
   int32_t prof_max = 0;
   int64_t launches = 0;
@@ -158,10 +171,57 @@ std::string check_cfg(const dcu_cfg *c) {
   return "";
 }
 
-int run_gemm(dcu_ctx *c, const void *X, int ldx, const int32_t *m_total, const GemmSeg *segs, int nseg, int K,
-             int ldc, cudaStream_t s) {
+// Activation operand of a GEMM: the packed rows X [cap][K] (row pitch ldx)
+// and, for the tcgen05 path, its tensor maps for token tiles of 128 and 256.
+struct ActOperand {
+  const void *X;
+  int ldx, K;
+  const CUtensorMap *map128, *map256;
+};
+
+// ws[split][m][n] = sum_k X[m][k] W[n][k] over the concatenated segments;
+// returns the number of split-K partials written in *splits.
+int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
+             const CUtensorMap *const *amaps, int nseg, int ldc, cudaStream_t s, int *splits, int max_splits = 16) {
   Prof p(c, DCU_K_GEMM, s);
-  LAUNCH(c, launch_gemm_simt(c->cfg.dtype, X, ldx, m_total, (int)c->cap, segs, nseg, K, c->C, ldc, s));
+  const int cap = (int)c->cap;
+  if (c->cfg.dtype != DCU_BF16) {
+    *splits = 1;
+    LAUNCH(c, launch_gemm_simt(c->cfg.dtype, x.X, x.ldx, m_total, cap, segs, nseg, x.K, c->C, ldc, s));
+    return DCU_OK;
+  }
+  TcParams tp;
+  memset(&tp, 0, sizeof(tp));
+  int tile = 0, col = 0;
+  for (int i = 0; i < nseg; ++i) {
+    tp.a[i] = *amaps[i];
+    tp.seg_tile0[i] = tile;
+    tp.seg_col0[i] = col;
+    tp.seg_rows[i] = segs[i].rows;
+    tile += (segs[i].rows + 127) / 128;
+    col += segs[i].rows;
+  }
+  tp.seg_tile0[nseg] = tile;
+  tp.nseg = nseg;
+  tp.n_tiles = tile;
+  tp.kblocks = x.K / 64;
+  const int bn = c->gemm_bn;
+  tp.b = bn == 256 ? *x.map256 : *x.map128;
+  const int passes_hint = (c->gemm_rows_hint + bn - 1) / bn;
+  int sp = choose_splits(tile, tp.kblocks, passes_hint < 1 ? 1 : passes_hint, c->num_sms);
+  const size_t per_split = (size_t)cap * ldc;
+  while (sp > 1 && ((size_t)sp * per_split > c->ws_elems || sp > max_splits)) --sp;
+  tp.splits = sp;
+  tp.ldc = ldc;
+  tp.m_total = m_total;
+  tp.m_host = 0;
+  tp.ws = c->C;
+  tp.split_stride = (long long)per_split;
+  tp.status = c->status();
+  const long long units_max = (long long)tile * sp * ((cap + bn - 1) / bn);
+  const int grid = (int)(units_max < c->num_sms ? units_max : c->num_sms);
+  *splits = sp;
+  LAUNCH(c, launch_gemm_tc(tp, bn, grid, s));
   return DCU_OK;
 }
 
@@ -175,46 +235,64 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   if (!dense) {
     Prof p(c, DCU_K_SELECT, s);
     LAUNCH(c, launch_select(c->dl(l), keys, nkeys, c->budgets + l, L, c->B, c->N, Bw, g.window_mode,
-                        c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
-                        last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->status(), s));
+                            c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
+                            last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->status(), s));
   }
   {
     Prof p(c, DCU_K_GATHER, s);
     LAUNCH(c, launch_gather_norm(dt, c->rowmap, c->m_total(), cap, c->Hl(l), c->g1[l], g.rms_eps, D, c->xs, s));
   }
+  const LayerMaps *lm = c->lmaps.empty() ? nullptr : &c->lmaps[l];
+  const ActOperand xs{c->xs, D, D, &c->xs_map[0], &c->xs_map[1]};
+  const ActOperand at{c->attn, H * hd, H * hd, &c->attn_map[0], &c->attn_map[1]};
+  const ActOperand ac{c->act, F, F, &c->act_map[0], &c->act_map[1]};
+  int sp = 1;
   const int nqkv = (H + 2 * Hkv) * hd;
-  GemmSeg qkv[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
-  if (int rc = run_gemm(c, c->xs, D, c->m_total(), qkv, 3, D, nqkv, s)) return rc;
+  {
+    GemmSeg seg[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
+    const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &sp)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->rope_tab,
-                         g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
+    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, sp, (size_t)cap * nqkv, c->rowmap, c->m_total(), cap, c->N, H, Hkv,
+                             hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
   }
   {
     Prof p(c, DCU_K_ATTN, s);
-    LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l), c->attn,
-                           s));
+    LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
+                               c->attn, s));
   }
-  GemmSeg o[1] = {{c->wo[l], D}};
-  if (int rc = run_gemm(c, c->attn, H * hd, c->m_total(), o, 1, H * hd, D, s)) return rc;
+  {
+    GemmSeg seg[1] = {{c->wo[l], D}};
+    const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
+    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &sp)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_o(dt, c->C, D, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l], g.rms_eps, D, c->hmid, c->xs,
-                       s));
+    LAUNCH(c, launch_epi_o(dt, c->C, D, sp, (size_t)cap * D, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l],
+                           g.rms_eps, D, c->hmid, c->xs, s));
   }
-  GemmSeg gu[2] = {{c->wg[l], F}, {c->wu[l], F}};
-  if (int rc = run_gemm(c, c->xs, D, c->m_total(), gu, 2, D, 2 * F, s)) return rc;
+  {
+    GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
+    const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &sp)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, c->m_total(), cap, F, c->act, s));
+    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, sp, (size_t)cap * 2 * F, c->m_total(), cap, F, c->act, s));
   }
-  GemmSeg dn[1] = {{c->wd[l], D}};
-  if (int rc = run_gemm(c, c->act, F, c->m_total(), dn, 1, F, D, s)) return rc;
+  {
+    GemmSeg seg[1] = {{c->wd[l], D}};
+    const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
+    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &sp)) return rc;
+  }
   {
     Prof p(c, DCU_K_SCATTER, s);
     const bool want_d = !dense && !last;
-    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, c->rowmap, c->m_total(), cap, c->hmid, c->Hl(l + 1),
-                                  want_d ? c->g1[l + 1] : nullptr, want_d ? c->dl(l + 1) : nullptr, D, s));
+    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, sp, (size_t)cap * D, c->rowmap, c->m_total(), cap, c->hmid,
+                                      c->Hl(l + 1), want_d ? c->g1[l + 1] : nullptr,
+                                      want_d ? c->dl(l + 1) : nullptr, D, s));
   }
   return DCU_OK;
 }
@@ -243,6 +321,14 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
         !w->w_gate[l] || !w->w_up[l] || !w->w_down[l])
       return fail(nullptr, DCU_EINVAL, "layer " + std::to_string(l) + ": a weight pointer is NULL");
 
+  {
+    auto mis = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    bool bad = mis(w->embed) || mis(w->lm_head) || mis(w->final_norm);
+    for (int l = 0; l < cfg->n_layers && !bad; ++l)
+      bad = mis(w->wq[l]) || mis(w->wk[l]) || mis(w->wv[l]) || mis(w->wo[l]) || mis(w->w_gate[l]) ||
+            mis(w->w_up[l]) || mis(w->w_down[l]) || mis(w->attn_norm[l]) || mis(w->ffn_norm[l]);
+    if (bad) return fail(nullptr, DCU_EINVAL, "weight pointers must be 16-byte aligned");
+  }
   dcu_ctx *c = new (std::nothrow) dcu_ctx();
   if (!c) return fail(nullptr, DCU_ENOMEM, "host allocation failed");
   c->cfg = *cfg;
@@ -266,10 +352,27 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   c->cap = (int64_t)cfg->max_batch * cfg->max_seq;
   const size_t cap = (size_t)c->cap, D = cfg->d_model, F = cfg->d_ffn, Hhd = (size_t)cfg->n_heads * cfg->head_dim;
   const size_t nqkv = (size_t)(cfg->n_heads + 2 * cfg->n_kv_heads) * cfg->head_dim;
-  size_t cw = nqkv;
-  if (D > cw) cw = D;
-  if (2 * F > cw) cw = 2 * F;
-  if ((size_t)cfg->vocab > cw) cw = cfg->vocab;
+  {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) == cudaSuccess && sms > 0)
+      c->num_sms = sms;
+  }
+  // C holds the GEMM outputs as split-K partials: per row, max over the GEMMs
+  // of splits x output width (the LM head runs unsplit).
+  size_t cw = (size_t)cfg->vocab;
+  if (cfg->dtype == DCU_BF16) {
+    const size_t widths[4] = {nqkv, D, 2 * F, D};
+    const size_t ks[4] = {D, Hhd, D, F};
+    for (int i = 0; i < 4; ++i) {
+      const int tiles = (int)((widths[i] + 127) / 128);
+      const int sp = choose_splits(tiles, (int)(ks[i] / 64), 1, c->num_sms);
+      if ((size_t)sp * widths[i] > cw) cw = (size_t)sp * widths[i];
+    }
+  } else {
+    if (nqkv > cw) cw = nqkv;
+    if (2 * F > cw) cw = 2 * F;
+  }
+  c->ws_elems = cap * cw;
   size_t xw = D > F ? D : F;
   cudaError_t e = cudaSuccess;
 #define AL(ptr, bytes)                                                                  \
@@ -312,6 +415,36 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   if (e == cudaSuccess && cfg->rope_theta > 0.0f)
     e = launch_rope_table(c->rope_tab, cfg->max_seq, cfg->head_dim, cfg->rope_theta, 0);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e == cudaSuccess && cfg->dtype == DCU_BF16) {
+    // tensor maps of every weight matrix (box 64 x 128) and of the packed activation buffers (box 64 x 128|256)
+    bool ok = true;
+    auto wmap = [&](CUtensorMap *m, const void *w, size_t rows, size_t k) {
+      ok = ok && encode_tmap_bf16(m, w, k, rows, k * 2, 64, 128);
+    };
+    c->lmaps.resize(L);
+    for (int l = 0; l < L; ++l) {
+      LayerMaps &m = c->lmaps[l];
+      wmap(&m.wq, c->wq[l], Hhd, D);
+      wmap(&m.wk, c->wk[l], (size_t)cfg->n_kv_heads * cfg->head_dim, D);
+      wmap(&m.wv, c->wv[l], (size_t)cfg->n_kv_heads * cfg->head_dim, D);
+      wmap(&m.wo, c->wo[l], D, Hhd);
+      wmap(&m.wg, c->wg[l], F, D);
+      wmap(&m.wu, c->wu[l], F, D);
+      wmap(&m.wd, c->wd[l], D, F);
+    }
+    wmap(&c->lm_map, c->lm_head, (size_t)cfg->vocab, D);
+    const uint32_t bns[2] = {128, 256};
+    for (int i = 0; i < 2; ++i) {
+      ok = ok && encode_tmap_bf16(&c->xs_map[i], c->xs, D, cap, D * 2, 64, bns[i]);
+      ok = ok && encode_tmap_bf16(&c->attn_map[i], c->attn, Hhd, cap, Hhd * 2, 64, bns[i]);
+      ok = ok && encode_tmap_bf16(&c->act_map[i], c->act, F, cap, F * 2, 64, bns[i]);
+    }
+    if (!ok) {
+      free_all(c);
+      delete c;
+      return fail(nullptr, DCU_ECUDA, "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
+    }
+  }
   if (e != cudaSuccess) {
     std::string m = std::string("context setup failed: ") + cudaGetErrorString(e);
     free_all(c);
@@ -345,6 +478,8 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
                                c->cfg.d_model, c->cfg.vocab, 1, c->status(), s));
   }
   LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), s));
+  c->gemm_bn = 256;
+  c->gemm_rows_hint = BN;
   for (int l = 0; l < c->cfg.n_layers; ++l)
     if (int rc = run_layer(c, l, true, nullptr, nullptr, 0, s)) return rc;
   CK(c, cudaMemsetAsync(c->s_prev, 0, (size_t)c->cfg.max_batch * c->cfg.n_layers * 4, s));
@@ -361,6 +496,12 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
   if (B_layer < 0 || B_window < 0) return fail(c, DCU_EINVAL, "B_layer and B_window must be >= 0");
   cudaStream_t s = (cudaStream_t)stream;
   const int L = c->cfg.n_layers, BN = c->B * c->N;
+  {
+    // expected rows per layer: twice the mean budget plus a few windows per sequence
+    const long long est = (long long)c->B * (2LL * B_layer + 2LL * (B_window + 1));
+    c->gemm_rows_hint = (int)(est < BN ? est : BN);
+    c->gemm_bn = c->gemm_rows_hint <= 128 ? 128 : 256;
+  }
   {
     Prof p(c, DCU_K_BUDGET, s);
     LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, c->first_step ? 1 : 0, c->budgets, s));
@@ -393,7 +534,12 @@ int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_
     LAUNCH(c, launch_gather_norm(g.dtype, c->mrow, c->m_masked(), cap, c->Hl(g.n_layers), c->final_norm, g.rms_eps,
                              g.d_model, c->xs, s));
     GemmSeg lm[1] = {{c->lm_head, g.vocab}};
-    LAUNCH(c, launch_gemm_simt(g.dtype, c->xs, g.d_model, c->m_masked(), cap, lm, 1, g.d_model, c->C, g.vocab, s));
+    const CUtensorMap *am[1] = {&c->lm_map};
+    const ActOperand xs{c->xs, g.d_model, g.d_model, &c->xs_map[0], &c->xs_map[1]};
+    c->gemm_bn = 256;
+    c->gemm_rows_hint = 256;
+    int sp = 1;
+    if (int rc = run_gemm(c, xs, c->m_masked(), lm, am, 1, g.vocab, s, &sp, 1)) return rc;
     LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));
   }
   {
@@ -452,6 +598,48 @@ int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t 
     return fail(nullptr, DCU_EINVAL, "dcu_commit_rule: bad argument");
   CK(nullptr, launch_commit_rule(rule, param, conf, argmax, masked, ids, B, N, out_pos, out_count,
                                  (cudaStream_t)stream));
+  return DCU_OK;
+}
+
+int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout, int32_t dtype, float *Y,
+               dcu_stream_t stream) {
+  auto mis = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+  if (!X || !W || !Y || M < 0 || K <= 0 || Nout <= 0 || (dtype != DCU_F32 && dtype != DCU_BF16) || mis(X) ||
+      mis(W) || mis(Y) || (dtype == DCU_BF16 ? (K % 64) : (K % 16)))
+    return fail(nullptr, DCU_EINVAL, "dcu_linear: bad argument");
+  if (M == 0) return DCU_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (dtype == DCU_F32) {
+    GemmSeg seg{W, Nout};
+    CK(nullptr, launch_gemm_simt(dtype, X, K, nullptr, M, &seg, 1, K, Y, Nout, s));
+    return DCU_OK;
+  }
+  TcParams tp;
+  memset(&tp, 0, sizeof(tp));
+  const int bn = M <= 128 ? 128 : 256;
+  if (!encode_tmap_bf16(&tp.a[0], W, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, 64, 128) ||
+      !encode_tmap_bf16(&tp.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)bn))
+    return fail(nullptr, DCU_ECUDA, "dcu_linear: cuTensorMapEncodeTiled failed");
+  const int tiles = (Nout + 127) / 128;
+  tp.seg_tile0[0] = 0;
+  tp.seg_tile0[1] = tiles;
+  tp.seg_col0[0] = 0;
+  tp.seg_rows[0] = Nout;
+  tp.nseg = 1;
+  tp.n_tiles = tiles;
+  tp.kblocks = K / 64;
+  tp.splits = 1;
+  tp.ldc = Nout;
+  tp.m_total = nullptr;
+  tp.m_host = M;
+  tp.ws = Y;
+  tp.split_stride = 0;
+  tp.status = nullptr;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long units = (long long)tiles * ((M + bn - 1) / bn);
+  CK(nullptr, launch_gemm_tc(tp, bn, (int)(units < sms ? units : sms), s));
   return DCU_OK;
 }
 

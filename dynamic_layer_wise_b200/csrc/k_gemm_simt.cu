@@ -33,10 +33,11 @@ __device__ __forceinline__ void load4<bf16>(const bf16 *p, float (&v)[4]) {
 
 template <class T>
 __global__ void __launch_bounds__(256) k_gemm_simt(const T *__restrict__ X, int ldx, const int32_t *__restrict__ m_total,
-                                                   SegTable segs, int ntot, int K, float *__restrict__ C, int ldc) {
+                                                   int m_host, SegTable segs, int ntot, int K, float *__restrict__ C,
+                                                   int ldc) {
   __shared__ __align__(16) float As[BK][BM + 4];
   __shared__ __align__(16) float Bs[BK][BN + 4];
-  const int M = *m_total;
+  const int M = m_total ? *m_total : m_host;
   const int m_tiles = (M + BM - 1) / BM;
   const int n_tiles = (ntot + BN - 1) / BN;
   const int tid = threadIdx.x;
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(const T *__restrict__ X, int 
 
 cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,
                              const GemmSeg *segs, int nseg, int K, float *C, int ldc, cudaStream_t s) {
+  if (m_cap <= 0) return cudaSuccess;
   if (nseg < 1 || nseg > 4 || (K % BK) != 0) return cudaErrorInvalidValue;
   SegTable t{};
   t.nseg = nseg;
@@ -114,9 +116,9 @@ cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m
   int grid = (int)(cap_tiles < 148 * 8 ? cap_tiles : 148 * 8);
   if (grid < 1) grid = 1;
   if (dtype == DCU_BF16)
-    k_gemm_simt<bf16><<<grid, 256, 0, s>>>((const bf16 *)X, ldx, m_total, t, r, K, C, ldc);
+    k_gemm_simt<bf16><<<grid, 256, 0, s>>>((const bf16 *)X, ldx, m_total, m_cap, t, r, K, C, ldc);
   else
-    k_gemm_simt<float><<<grid, 256, 0, s>>>((const float *)X, ldx, m_total, t, r, K, C, ldc);
+    k_gemm_simt<float><<<grid, 256, 0, s>>>((const float *)X, ldx, m_total, m_cap, t, r, K, C, ldc);
   return cudaGetLastError();
 }
 

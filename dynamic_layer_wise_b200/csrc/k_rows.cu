@@ -8,6 +8,13 @@
 
 namespace dcu {
 
+// Split-K partials of a GEMM output element, summed in split order.
+__device__ __forceinline__ float csum(const float *c, size_t sstride, int splits, size_t j) {
+  float v = c[j];
+  for (int sp = 1; sp < splits; ++sp) v += c[sp * sstride + j];
+  return v;
+}
+
 static inline int row_grid(int rows_cap) {
   int g = rows_cap < 148 * 16 ? rows_cap : 148 * 16;
   return g > 0 ? g : 1;
@@ -186,7 +193,8 @@ cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *
 // k at the row's position; q -> Q[r]; k, v -> the layer's K/V cache at
 // (b, kv head, i).
 template <class T>
-__global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const int32_t *__restrict__ rowmap,
+__global__ void k_epi_qkv(const float *__restrict__ C, int ldc, int splits, size_t sstride,
+                          const int32_t *__restrict__ rowmap,
                           const int32_t *__restrict__ m_total, int N, int H, int Hkv, int hd,
                           const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q, T *__restrict__ Kc,
                           T *__restrict__ Vc) {
@@ -199,7 +207,7 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const int32_t *_
     for (int t = threadIdx.x; t < (H + Hkv) * half; t += blockDim.x) {
       const int head = t / half, j = t - head * half;
       const int base = head * hd;  // q heads first, then k heads (contiguous in C)
-      float a = c[base + j], bb = c[base + j + half];
+      float a = csum(c, sstride, splits, base + j), bb = csum(c, sstride, splits, base + j + half);
       if (use_rope) {
         float2 cs = rope_tab[(size_t)i * half + j];
         float a2 = a * cs.x - bb * cs.y;
@@ -220,19 +228,19 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const int32_t *_
     const float *cv = c + (size_t)(H + Hkv) * hd;
     for (int t = threadIdx.x; t < Hkv * hd; t += blockDim.x) {
       const int kvh = t / hd, j = t - kvh * hd;
-      Vc[(((size_t)b * Hkv + kvh) * N + i) * hd + j] = from_f<T>(cv[t]);
+      Vc[(((size_t)b * Hkv + kvh) * N + i) * hd + j] = from_f<T>(csum(cv, sstride, splits, t));
     }
   }
 }
 
-cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total,
-                           int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab, int use_rope, void *Q,
-                           void *Kc, void *Vc, cudaStream_t s) {
+cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+                           const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
+                           int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_qkv<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
+    k_epi_qkv<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
                                                    (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc);
   else
-    k_epi_qkv<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
+    k_epi_qkv<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
                                                     (float *)Q, (float *)Kc, (float *)Vc);
   return cudaGetLastError();
 }
@@ -240,7 +248,8 @@ cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const int32_t *ro
 // ------------------------------------------------------------------ O epilogue
 // hmid[r] = H_l[row] + C[r] (fp32); xs[r] = T(RMSNorm(hmid[r]) * g2).
 template <class T>
-__global__ void k_epi_o(const float *__restrict__ C, int ldc, const int32_t *__restrict__ rowmap,
+__global__ void k_epi_o(const float *__restrict__ C, int ldc, int splits, size_t sstride,
+                        const int32_t *__restrict__ rowmap,
                         const int32_t *__restrict__ m_total, const T *__restrict__ Hl, const float *__restrict__ g2,
                         float eps, int D, float *__restrict__ hmid, T *__restrict__ xs) {
   __shared__ double red[32];
@@ -256,7 +265,7 @@ __global__ void k_epi_o(const float *__restrict__ C, int ldc, const int32_t *__r
       load_vec(x + j, v);
 #pragma unroll
       for (int i = 0; i < VN; ++i) {
-        v[i] += c[j + i];
+        v[i] += csum(c, sstride, splits, j + i);
         hm[j + i] = v[i];
         ss += (double)v[i] * (double)v[i];
       }
@@ -273,13 +282,14 @@ __global__ void k_epi_o(const float *__restrict__ C, int ldc, const int32_t *__r
   }
 }
 
-cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
-                         const void *Hl, const float *g2, float eps, int D, float *hmid, void *xs, cudaStream_t s) {
+cudaError_t launch_epi_o(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+                         const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
+                         float *hmid, void *xs, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_o<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, (const bf16 *)Hl, g2, eps, D, hmid,
+    k_epi_o<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, (const bf16 *)Hl, g2, eps, D, hmid,
                                                  (bf16 *)xs);
   else
-    k_epi_o<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, (const float *)Hl, g2, eps, D, hmid,
+    k_epi_o<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, (const float *)Hl, g2, eps, D, hmid,
                                                   (float *)xs);
   return cudaGetLastError();
 }
@@ -287,24 +297,25 @@ cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const int32_t *rowm
 // ------------------------------------------------------------------ SwiGLU epilogue
 // C row r = [gate (F) | up (F)];  act[r] = T(silu(gate) * up).
 template <class T>
-__global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, const int32_t *__restrict__ m_total, int F,
+__global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, int splits, size_t sstride,
+                             const int32_t *__restrict__ m_total, int F,
                              T *__restrict__ act) {
   const int M = *m_total;
   for (int r = blockIdx.x; r < M; r += gridDim.x) {
     const float *c = C + (size_t)r * ldc;
     for (int j = threadIdx.x; j < F; j += blockDim.x) {
-      const float gt = c[j], up = c[F + j];
+      const float gt = csum(c, sstride, splits, j), up = csum(c, sstride, splits, F + j);
       act[(size_t)r * F + j] = from_f<T>(gt / (1.0f + expf(-gt)) * up);
     }
   }
 }
 
-cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const int32_t *m_total, int cap, int F, void *act,
-                              cudaStream_t s) {
+cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *m_total,
+                              int cap, int F, void *act, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_swiglu<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, m_total, F, (bf16 *)act);
+    k_epi_swiglu<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, m_total, F, (bf16 *)act);
   else
-    k_epi_swiglu<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, m_total, F, (float *)act);
+    k_epi_swiglu<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, m_total, F, (float *)act);
   return cudaGetLastError();
 }
 
@@ -313,7 +324,8 @@ cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const int32_t 
 // ([DLLM] "关键设计 1", computed against the cached row before it is
 // overwritten); H_{l+1}[row] = new.
 template <class T>
-__global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, const int32_t *__restrict__ rowmap,
+__global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, int splits, size_t sstride,
+                                   const int32_t *__restrict__ rowmap,
                                    const int32_t *__restrict__ m_total, const float *__restrict__ hmid,
                                    T *__restrict__ Hn, const float *__restrict__ g_next, float *__restrict__ d_next,
                                    int D) {
@@ -330,7 +342,7 @@ __global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, const i
     for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
       float v[VN];
 #pragma unroll
-      for (int i = 0; i < VN; ++i) v[i] = hm[j + i] + c[j + i];
+      for (int i = 0; i < VN; ++i) v[i] = hm[j + i] + csum(c, sstride, splits, j + i);
       if (d_next) {
         float ov[VN];
         uint32_t ob[VN];
@@ -359,14 +371,14 @@ __global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, const i
   }
 }
 
-cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const int32_t *rowmap,
-                                    const int32_t *m_total, int cap, const float *hmid, void *Hnext,
-                                    const float *g_next, float *d_next, int D, cudaStream_t s) {
+cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, int splits, size_t sstride,
+                                    const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
+                                    void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_down_scatter<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, hmid, (bf16 *)Hnext, g_next,
+    k_epi_down_scatter<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, hmid, (bf16 *)Hnext, g_next,
                                                             d_next, D);
   else
-    k_epi_down_scatter<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, rowmap, m_total, hmid, (float *)Hnext, g_next,
+    k_epi_down_scatter<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, hmid, (float *)Hnext, g_next,
                                                              d_next, D);
   return cudaGetLastError();
 }

@@ -24,16 +24,18 @@ cudaError_t launch_cosine_distance(int dtype, const void *x, const void *y, cons
                                    float *d, cudaStream_t s);
 cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *m_total, int cap, const void *H,
                                const float *g, float eps, int D, void *xs, cudaStream_t s);
-cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total,
-                           int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab, int use_rope, void *Q,
-                           void *Kc, void *Vc, cudaStream_t s);
-cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
-                         const void *Hl, const float *g2, float eps, int D, float *hmid, void *xs, cudaStream_t s);
-cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const int32_t *m_total, int cap, int F, void *act,
-                              cudaStream_t s);
-cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const int32_t *rowmap,
-                                    const int32_t *m_total, int cap, const float *hmid, void *Hnext,
-                                    const float *g_next, float *d_next, int D, cudaStream_t s);
+// C: GEMM output as `splits` partials [splits][cap][ldc] (sstride elements apart), summed in split order.
+cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+                           const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
+                           int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s);
+cudaError_t launch_epi_o(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+                         const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
+                         float *hmid, void *xs, cudaStream_t s);
+cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *m_total,
+                              int cap, int F, void *act, cudaStream_t s);
+cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, int splits, size_t sstride,
+                                    const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
+                                    void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s);
 cudaError_t launch_softmax_max(const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
                                int V, float *conf, int32_t *amax, cudaStream_t s);
 
@@ -53,7 +55,7 @@ cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *row
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
                                int32_t *ids, int B, int N, int32_t *out_pos, int32_t *out_count, cudaStream_t s);
 
-// ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total
+// ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total (m < m_cap when m_total is null)
 cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,
                              const GemmSeg *segs, int nseg, int K, float *C, int ldc, cudaStream_t s);
 

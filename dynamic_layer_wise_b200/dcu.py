@@ -73,6 +73,7 @@ _SIGS = {
     "dcu_profile_read": (_i32, [_vp, _i32, ctypes.POINTER(_f64), ctypes.POINTER(_i64), _i32]),
     "dcu_kernel_class_name": (ctypes.c_char_p, [_i32]),
     "dcu_launch_count": (_i64, [_vp]),
+    "dcu_linear": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]),
     "dcu_lm_confidence_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
 }
 
@@ -293,3 +294,13 @@ def dcu_lm_confidence_noalloc(h_rows, final_norm, lm_head, rms_eps: float = 1e-5
     _check(lib().dcu_lm_confidence_noalloc(_ptr(h_rows), _ptr(final_norm), _ptr(lm_head), m, D, V, dt,
                                            float(rms_eps), _ptr(conf), _ptr(amax), _stream(stream)))
     return conf, amax
+
+
+def dcu_linear(X, W, stream=None):
+    """Y = X W^T in fp32 (X [M][K], W [Nout][K], bf16 or float32)."""
+    M, K = X.shape
+    Nout = W.shape[0]
+    dt = {torch.bfloat16: DCU_BF16, torch.float32: DCU_F32}[X.dtype]
+    Y = torch.empty((M, Nout), dtype=torch.float32, device=X.device)
+    _check(lib().dcu_linear(_ptr(X), _ptr(W), M, K, Nout, dt, _ptr(Y), _stream(stream)))
+    return Y

@@ -179,6 +179,13 @@ int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t 
                     int32_t *token_ids, int32_t B, int32_t N, int32_t *out_positions, int32_t *out_count,
                     dcu_stream_t stream);
 
+/* Y[m][n] = sum_k X[m][k] W[n][k] in fp32: the recompute GEMM (tcgen05 with
+ * TMA-staged operands for bf16, CUDA cores for float32) as a stateless call.
+ * X: dev [M][K] dtype; W: dev [Nout][K] dtype; Y: dev float [M][Nout]; all
+ * 16-byte aligned; K % 64 == 0 (bf16) or K % 16 == 0 (float32). */
+int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout, int32_t dtype, float *Y,
+               dcu_stream_t stream);
+
 /* LM-head confidence and argmax of m final-layer rows without any device
  * allocation, for callers that cannot call cudaMalloc (a host framework that
  * owns every device allocation through its own pool, or a serving process

@@ -11,6 +11,22 @@ from dynamic_layer_wise_b200 import inputs as I
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("M,K,Nout", [(1, 64, 128), (17, 256, 1000), (65, 4096, 384), (128, 512, 256),
+                                      (130, 1024, 640), (300, 128, 200), (1024, 256, 128)])
+def test_linear_parity(dtype, M, K, Nout):
+    """The recompute GEMM (tcgen05 for bf16) against an fp64 product of the same
+    stored values; fp32 accumulation bounds the error by ~K * 2^-24 * sum|x||w|."""
+    rng = np.random.default_rng(M * 7 + K)
+    x = O.store(rng.standard_normal((M, K)), dtype)
+    w = O.store(rng.standard_normal((Nout, K)) * 0.02, dtype)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    y = dcu.dcu_linear(torch.tensor(x).to(tdt).cuda(), torch.tensor(w).to(tdt).cuda()).cpu().numpy()
+    ref = x @ w.T
+    bound = np.abs(x) @ np.abs(w).T * (K * 2.0 ** -23 + 1e-7)
+    assert np.all(np.abs(y - ref) <= bound), float(np.max(np.abs(y - ref) / bound))
+
+
 def test_device_generator_matches_host_bits():
     for dtype, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
         for seed, tid, start, n in ((0, 1, 0, 100003), (7, 123, 5_000_000, 4099), (2**31 + 5, 77, 2**33, 1000)):

@@ -42,7 +42,33 @@ WORKLOADS = {
     "batch4": dict(shape="LLADA_8B", n_prompt=1536, n_gen=512, batch=4, B_layer=64, B_window=32, rule=1, param=0.9,
                    desc="LLaDA-8B shape, 4 sequences x N=2048 (1536 prompt + 512 masked), B_layer=64, B_window=32, "
                         "threshold tau=0.9"),
+    "toy": dict(shape="TOY", n_prompt=192, n_gen=64, batch=1, B_layer=16, B_window=16, rule=0, param=0.1,
+                desc="toy fp32 DCU step (4 layers, d=256), N=256 (192 prompt + 64 masked), B_layer=16, B_window=16, "
+                     "Frechet delta=0.1"),
 }
+
+
+# ---------------------------------------------------------------- replicas (one per rank, no collective on the data path)
+
+def replica_seed(rank: int) -> int:
+    """Seed of the sequences rank `rank` decodes (the model weights are shared)."""
+    return 1 + rank
+
+
+def reduce_over_ranks(x: float, world: int, op: str, device) -> float:
+    """max / sum of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank: int, world: int, ms_step_max: float, steps: int) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (ms_step_max * steps / 1000.0)
 
 
 def measured_peaks():
@@ -204,6 +230,24 @@ def traffic_for(kernel_file: str):
     return None
 
 
+# ---------------------------------------------------------------- profiling cases
+
+def profile_case_gemm(shape, reps):
+    """The QKV recompute GEMM alone (M = 65 selected rows, K = d_model,
+    N = (H + 2 H_kv) hd): for ncu captures of the tcgen05 kernel."""
+    import torch
+    from dynamic_layer_wise_b200 import dcu
+    from dynamic_layer_wise_b200 import inputs as I
+    n_out = (shape.n_heads + 2 * shape.n_kv_heads) * shape.head_dim
+    W = I.device_normal_(torch.empty((n_out, shape.d_model), dtype=torch.bfloat16, device="cuda"), 0, 1, 0.02)
+    X = I.device_normal_(torch.empty((65, shape.d_model), dtype=torch.bfloat16, device="cuda"), 0, 2, 1.0)
+    for _ in range(max(1, reps)):
+        dcu.dcu_linear(X, W)
+    torch.cuda.synchronize()
+    print(json.dumps({"case": "gemm", "M": 65, "K": shape.d_model, "N": n_out, "reps": reps}))
+    return 0
+
+
 # ---------------------------------------------------------------- main
 
 def main():
@@ -215,6 +259,12 @@ def main():
     ap.add_argument("--workload", default="llada8b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graphs", action="store_true", help="launch every kernel directly (no CUDA graphs)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="profiling only: override the number of layers (the JSON line is then not a bench value)")
+    ap.add_argument("--case", default="", choices=["", "gemm"],
+                    help="profiling only: run one kernel on a small case instead of the step (gemm: QKV shape, "
+                         "M = 65 rows, 100 MB of weights)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -224,6 +274,11 @@ def main():
 
     from dynamic_layer_wise_b200 import inputs as I
     shape = getattr(I, wl["shape"])
+    if args.layers:
+        import dataclasses
+        shape = dataclasses.replace(shape, n_layers=args.layers)
+    if args.case == "gemm":
+        return profile_case_gemm(shape, args.steps)
     N = wl["n_prompt"] + wl["n_gen"]
     B = wl["batch"]
     config = {"workload": wl["desc"], "batch": B, "seq_len": N, "B_layer": wl["B_layer"], "B_window": wl["B_window"],
@@ -265,23 +320,16 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_over_ranks(x, world, "max", "cuda")
 
     def sum_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
+        return reduce_over_ranks(x, world, "sum", "cuda")
 
     stream = torch.cuda.current_stream()
     W = I.device_weights(shape, 0)
     ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
-    seq_seed = 1 + rank                                   # each replica decodes its own sequences
+    dcu.dcu_set_graphs(ctx, not args.no_graphs)
+    seq_seed = replica_seed(rank)                         # each replica decodes its own sequences
     ids_h = torch.stack([torch.tensor(I.sequence_ids(seq_seed, b, wl["n_prompt"], wl["n_gen"], shape.vocab),
                                       dtype=torch.int32) for b in range(B)])
     ids = ids_h.cuda()
@@ -302,15 +350,18 @@ def main():
         dcu.dcu_step(ctx, ids, pos, cnt, wl["B_layer"], wl["B_window"])
         dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
 
+    # event timing of every kernel class; graphs are captured (with their
+    # event-record nodes) during warm-up, so no capture happens while timing
+    per_step_launches_guess = 2 + shape.n_layers * 11 + 6
+    dcu.dcu_profile_enable(ctx, (args.steps + args.warmup) * per_step_launches_guess)
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if dcu.dcu_status(ctx) != 0:
         raise RuntimeError("device status word set during warm-up")
+    for k in range(dcu.DCU_K_COUNT):
+        dcu.dcu_profile_read(ctx, k, reset=True)
     masked_before = int(masked.sum().item())
-
-    per_step_launches_guess = 2 + shape.n_layers * 11 + 6
-    dcu.dcu_profile_enable(ctx, args.steps * per_step_launches_guess)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -330,7 +381,7 @@ def main():
     committed = masked_before - int(masked.sum().item())
     ms_step = max_over_ranks(ms_total / args.steps)
     steps_all = args.steps * world
-    value = steps_all / (ms_step * args.steps / 1000.0)
+    value = aggregate_rate(args.steps, world, ms_step, args.steps)
     tokens_per_s = sum_over_ranks(committed) / (ms_step * args.steps / 1000.0)
 
     per_kernel = {}
@@ -396,7 +447,10 @@ def main():
                "vs_baseline": None, "dtype": "bf16" if shape.dtype == "bf16" else "f32", "data": "synthetic",
                "config": config, "gen_tokens_per_s": tokens_per_s, "full_forward_ms": full_ms,
                "per_kernel": per_kernel, "rows_per_layer_last_step": rows, "roofline": roofline,
-               "cpu_baseline": cpu_base, "e2e": e2e, "clocks": clk, "gpu_launches": launches}
+               "cpu_baseline": cpu_base, "e2e": e2e, "clocks": clk, "gpu_launches": launches,
+               "graphs": not args.no_graphs}
+        if args.layers:
+            out["profiling_only"] = f"n_layers overridden to {args.layers}: not a bench value"
         print(json.dumps(out))
     ctx.close()
     if world > 1:

@@ -29,7 +29,21 @@ struct ProfClass {
   int64_t dropped = 0;
 };
 
+// A captured dcu_step or commit_select: instantiated graph, the kernels it
+// launches and (when captured with profiling on) its event-record nodes.
+struct GraphEntry {
+  uint64_t key[10] = {};
+  cudaGraphExec_t exec = nullptr;
+  int64_t kernels = 0;
+  std::vector<std::pair<int, EventPair>> ev;
+  int64_t replays = 0;  // since the last profile reset
+  uint64_t last_use = 0;
+};
+constexpr size_t kMaxGraphs = 16;
+
 size_t esize(int dtype) { return dtype == DCU_BF16 ? 2 : 4; }
+
+constexpr int kAttnMaxSplits = 8;
 
 }  // namespace
 
@@ -60,6 +74,10 @@ struct dcu_ctx {
   // scratch
   char *xs = nullptr, *Q = nullptr, *attn = nullptr, *act = nullptr;
   float *hmid = nullptr, *C = nullptr, *conf = nullptr;
+  int32_t *seq_off = nullptr, *attn_ctr = nullptr;
+  float *attn_po = nullptr;
+  float2 *attn_ml = nullptr;
+  int attn_qt_cap = 1;
   int32_t *amax = nullptr, *mrow = nullptr;
   std::vector<void *> allocs;
   std::string err;
@@ -68,9 +86,18 @@ struct dcu_ctx {
   int gemm_bn = 128;          // token tile of the current call
   int gemm_rows_hint = 128;   // expected rows per layer of the current call
   size_t ws_elems = 0;        // capacity of C in floats
+  float2 *smx = nullptr;      // LM-head softmax statistics per (vocab tile, row)
+  int32_t *smx_arg = nullptr;
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
-  CUtensorMap xs_map[2], attn_map[2], act_map[2];  // token tiles 128, 256
+  CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of 16 and 64 rows
+  // CUDA graphs of dcu_step / commit_select
+  bool use_graphs = true;
+  bool capturing = false;
+  cudaStream_t cap_stream = nullptr;
+  std::vector<GraphEntry> graphs;
+  GraphEntry *cur_graph = nullptr;
+  uint64_t use_clock = 0;
   // profiling
   int32_t prof_max = 0;
   int64_t launches = 0;
@@ -80,6 +107,7 @@ struct dcu_ctx {
   int32_t *done() { return ints + 1; }
   int32_t *status() { return ints + 2; }
   int32_t *m_masked() { return ints + 3; }
+  int32_t *uniform_flag() { return ints + 4; }  // 1: the next step splits its budget uniformly
   size_t hslab() const { return (size_t)cap * cfg.d_model * esz; }
   size_t kvslab() const { return (size_t)cap * cfg.n_kv_heads * cfg.head_dim * esz; }
   void *Hl(int l) { return H + (size_t)l * hslab(); }
@@ -115,8 +143,18 @@ struct Prof {
   int k;
   cudaStream_t s;
   EventPair *p = nullptr;
+  bool ext = false;
   Prof(dcu_ctx *c_, int k_, cudaStream_t s_) : c(c_), k(k_), s(s_) {
     if (!c || c->prof_max <= 0) return;
+    if (c->capturing && c->cur_graph) {  // event-record nodes inside the graph
+      EventPair e;
+      if (cudaEventCreate(&e.a) != cudaSuccess || cudaEventCreate(&e.b) != cudaSuccess) return;
+      c->cur_graph->ev.push_back({k, e});
+      p = &c->cur_graph->ev.back().second;
+      ext = true;
+      cudaEventRecordWithFlags(p->a, s, cudaEventRecordExternal);
+      return;
+    }
     ProfClass &pc = c->prof[k];
     if (pc.used >= (int64_t)pc.ev.size()) {
       ++pc.dropped;
@@ -126,7 +164,12 @@ struct Prof {
     cudaEventRecord(p->a, s);
   }
   ~Prof() {
-    if (p) cudaEventRecord(p->b, s);
+    if (p) {
+      if (ext)
+        cudaEventRecordWithFlags(p->b, s, cudaEventRecordExternal);
+      else
+        cudaEventRecord(p->b, s);
+    }
   }
 };
 
@@ -140,7 +183,21 @@ cudaError_t dalloc(dcu_ctx *c, T **p, size_t bytes) {
   return cudaSuccess;
 }
 
+void free_graph(GraphEntry &g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  g.exec = nullptr;
+  for (auto &e : g.ev) {
+    if (e.second.a) cudaEventDestroy(e.second.a);
+    if (e.second.b) cudaEventDestroy(e.second.b);
+  }
+  g.ev.clear();
+}
+
 void free_all(dcu_ctx *c) {
+  for (auto &g : c->graphs) free_graph(g);
+  c->graphs.clear();
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
+  c->cap_stream = nullptr;
   for (void *p : c->allocs) cudaFree(p);
   c->allocs.clear();
   for (auto &pc : c->prof)
@@ -161,7 +218,12 @@ std::string check_cfg(const dcu_cfg *c) {
   if ((c->n_heads * c->head_dim) % 64 || (c->n_kv_heads * c->head_dim) % 64)
     return "n_heads*head_dim and n_kv_heads*head_dim must be multiples of 64";
   if (c->d_ffn % 64) return "d_ffn must be a multiple of 64";
+  if (c->dtype == DCU_BF16 && (c->d_model % 128 || c->d_ffn % 128 || (c->n_heads * c->head_dim) % 128 ||
+                               (c->n_kv_heads * c->head_dim) % 128))
+    return "bf16 models need d_model, d_ffn, n_heads*head_dim and n_kv_heads*head_dim to be multiples of 128";
   if (c->max_seq > 16384) return "max_seq must be <= 16384";
+  if (c->n_layers > 1024) return "n_layers must be <= 1024";
+  if (c->max_batch > 255) return "max_batch must be <= 255";
   if (c->mask_id < 0 || c->mask_id >= c->vocab) return "mask_id must be in [0, vocab)";
   if (!(c->rms_eps > 0.0f)) return "rms_eps must be > 0";
   if (c->rope_theta < 0.0f) return "rope_theta must be >= 0";
@@ -172,21 +234,22 @@ std::string check_cfg(const dcu_cfg *c) {
 }
 
 // Activation operand of a GEMM: the packed rows X [cap][K] (row pitch ldx)
-// and, for the tcgen05 path, its tensor maps for token tiles of 128 and 256.
+// and, for the tcgen05 path, its tensor map (16-row boxes).
 struct ActOperand {
   const void *X;
   int ldx, K;
-  const CUtensorMap *map128, *map256;
+  const CUtensorMap *map16, *map64;
 };
 
-// ws[split][m][n] = sum_k X[m][k] W[n][k] over the concatenated segments;
-// returns the number of split-K partials written in *splits.
+// C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
+// stream-K slots described by *geo (geo->grid == 0: a single slot).
 int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
-             const CUtensorMap *const *amaps, int nseg, int ldc, cudaStream_t s, int *splits, int max_splits = 16) {
-  Prof p(c, DCU_K_GEMM, s);
+             const CUtensorMap *const *amaps, int nseg, int ldc, cudaStream_t s, SlotGeo *geo,
+             bool tile_aligned = false, int prof_class = DCU_K_GEMM) {
+  Prof p(c, prof_class, s);
   const int cap = (int)c->cap;
+  memset(geo, 0, sizeof(*geo));
   if (c->cfg.dtype != DCU_BF16) {
-    *splits = 1;
     LAUNCH(c, launch_gemm_simt(c->cfg.dtype, x.X, x.ldx, m_total, cap, segs, nseg, x.K, c->C, ldc, s));
     return DCU_OK;
   }
@@ -203,25 +266,24 @@ int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const Gemm
   }
   tp.seg_tile0[nseg] = tile;
   tp.nseg = nseg;
-  tp.n_tiles = tile;
-  tp.kblocks = x.K / 64;
-  const int bn = c->gemm_bn;
-  tp.b = bn == 256 ? *x.map256 : *x.map128;
-  const int passes_hint = (c->gemm_rows_hint + bn - 1) / bn;
-  int sp = choose_splits(tile, tp.kblocks, passes_hint < 1 ? 1 : passes_hint, c->num_sms);
-  const size_t per_split = (size_t)cap * ldc;
-  while (sp > 1 && ((size_t)sp * per_split > c->ws_elems || sp > max_splits)) --sp;
-  tp.splits = sp;
+  tp.b16 = *x.map16;
+  tp.b64 = *x.map64;
   tp.ldc = ldc;
   tp.m_total = m_total;
-  tp.m_host = 0;
-  tp.ws = c->C;
-  tp.split_stride = (long long)per_split;
+  tp.out = c->C;
   tp.status = c->status();
-  const long long units_max = (long long)tile * sp * ((cap + bn - 1) / bn);
-  const int grid = (int)(units_max < c->num_sms ? units_max : c->num_sms);
-  *splits = sp;
-  LAUNCH(c, launch_gemm_tc(tp, bn, grid, s));
+  SlotGeo g;
+  g.n_tiles = tile;
+  g.kblocks = x.K / 64;
+  g.tile_aligned = tile_aligned ? 1 : 0;
+  const long long T = (long long)tile * g.kblocks;
+  g.grid = tile_aligned ? (tile < c->num_sms ? tile : c->num_sms) : (int)(T < c->num_sms ? T : c->num_sms);
+  g.slot_stride = (long long)cap * ldc;
+  if ((size_t)tc_max_slots(tile, g.grid) * cap * ldc > c->ws_elems)
+    return fail(c, DCU_ECUDA, "GEMM workspace too small for the stream-K slots");
+  tp.geo = g;
+  *geo = g;
+  LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
   return DCU_OK;
 }
 
@@ -236,7 +298,8 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     Prof p(c, DCU_K_SELECT, s);
     LAUNCH(c, launch_select(c->dl(l), keys, nkeys, c->budgets + l, L, c->B, c->N, Bw, g.window_mode,
                             c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
-                            last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->status(), s));
+                            last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->seq_off,
+                            c->status(), s));
   }
   {
     Prof p(c, DCU_K_GATHER, s);
@@ -246,51 +309,68 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   const ActOperand xs{c->xs, D, D, &c->xs_map[0], &c->xs_map[1]};
   const ActOperand at{c->attn, H * hd, H * hd, &c->attn_map[0], &c->attn_map[1]};
   const ActOperand ac{c->act, F, F, &c->act_map[0], &c->act_map[1]};
-  int sp = 1;
+  SlotGeo geo;
   const int nqkv = (H + 2 * Hkv) * hd;
   {
     GemmSeg seg[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
     const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &sp)) return rc;
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo)) return rc;
   }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, sp, (size_t)cap * nqkv, c->rowmap, c->m_total(), cap, c->N, H, Hkv,
+    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), cap, c->N, H, Hkv,
                              hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
   }
   {
     Prof p(c, DCU_K_ATTN, s);
-    LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
-                               c->attn, s));
+    if (c->attn_po) {
+      const int G = H / Hkv;
+      const int rows_seq = dense ? c->N : (c->gemm_rows_hint + c->B - 1) / c->B;
+      int qt_grid = (rows_seq * G + 127) / 128;
+      qt_grid = qt_grid < 1 ? 1 : (qt_grid > c->attn_qt_cap ? c->attn_qt_cap : qt_grid);
+      // one wave: (sequence, kv head, query tile) items x key splits <= SM count (one CTA per SM)
+      const long long items = (long long)c->B * Hkv * qt_grid;
+      int splits = (int)(c->num_sms / items);
+      const int max_sp = (c->N + 63) / 64;
+      splits = splits < 1 ? 1 : (splits > kAttnMaxSplits ? kAttnMaxSplits : splits);
+      if (splits > max_sp) splits = max_sp;
+      const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
+      splits = (c->N + kc - 1) / kc;
+      LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l), c->attn,
+                                     c->attn_po, c->attn_ml, c->attn_ctr, splits, qt_grid, c->attn_qt_cap, s));
+    } else {
+      LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
+                                 c->attn, s));
+    }
   }
   {
     GemmSeg seg[1] = {{c->wo[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
-    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &sp)) return rc;
+    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
   }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_o(dt, c->C, D, sp, (size_t)cap * D, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l],
+    LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l],
                            g.rms_eps, D, c->hmid, c->xs, s));
   }
   {
     GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
     const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &sp)) return rc;
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo)) return rc;
   }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, sp, (size_t)cap * 2 * F, c->m_total(), cap, F, c->act, s));
+    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), cap, F, c->act, s));
   }
   {
     GemmSeg seg[1] = {{c->wd[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
-    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &sp)) return rc;
+    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
   }
   {
     Prof p(c, DCU_K_SCATTER, s);
     const bool want_d = !dense && !last;
-    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, sp, (size_t)cap * D, c->rowmap, c->m_total(), cap, c->hmid,
+    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, geo, c->rowmap, c->m_total(), cap, c->hmid,
                                       c->Hl(l + 1), want_d ? c->g1[l + 1] : nullptr,
                                       want_d ? c->dl(l + 1) : nullptr, D, s));
   }
@@ -357,20 +437,21 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, c->device) == cudaSuccess && sms > 0)
       c->num_sms = sms;
   }
-  // C holds the GEMM outputs as split-K partials: per row, max over the GEMMs
-  // of splits x output width (the LM head runs unsplit).
-  size_t cw = (size_t)cfg->vocab;
+  // C holds a GEMM output as its stream-K slots (bf16) or one result (float32)
+  size_t cw = cfg->dtype == DCU_BF16 ? 0 : (size_t)cfg->vocab;  // bf16: the LM head stores no logits
+  if (nqkv > cw) cw = nqkv;
+  if (2 * F > cw) cw = 2 * F;
+  if (D > cw) cw = D;
   if (cfg->dtype == DCU_BF16) {
     const size_t widths[4] = {nqkv, D, 2 * F, D};
     const size_t ks[4] = {D, Hhd, D, F};
     for (int i = 0; i < 4; ++i) {
-      const int tiles = (int)((widths[i] + 127) / 128);
-      const int sp = choose_splits(tiles, (int)(ks[i] / 64), 1, c->num_sms);
-      if ((size_t)sp * widths[i] > cw) cw = (size_t)sp * widths[i];
+      const size_t tiles = (widths[i] + 127) / 128;
+      const long long T = (long long)tiles * (long long)(ks[i] / 64);
+      const int grid = (int)(T < c->num_sms ? T : c->num_sms);
+      const size_t w = (size_t)tc_max_slots((int)tiles, grid) * widths[i];
+      if (w > cw) cw = w;
     }
-  } else {
-    if (nqkv > cw) cw = nqkv;
-    if (2 * F > cw) cw = 2 * F;
   }
   c->ws_elems = cap * cw;
   size_t xw = D > F ? D : F;
@@ -399,8 +480,21 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   AL(c->act, cap * F * c->esz);
   AL(c->hmid, cap * D * 4);
   AL(c->C, cap * cw * 4);
+  if (cfg->dtype == DCU_BF16) {
+    const size_t vt = ((size_t)cfg->vocab + 127) / 128;
+    AL(c->smx, vt * cap * sizeof(float2));
+    AL(c->smx_arg, vt * cap * 4);
+  }
   AL(c->conf, cap * 4);
   AL(c->amax, cap * 4);
+  AL(c->seq_off, ((size_t)cfg->max_batch + 1) * 4);
+  if (cfg->dtype == DCU_BF16 && (cfg->head_dim == 64 || cfg->head_dim == 128)) {
+    const int G = cfg->n_heads / cfg->n_kv_heads;
+    c->attn_qt_cap = (int)(((size_t)cfg->max_seq * G + 127) / 128);
+    AL(c->attn_po, (size_t)kAttnMaxSplits * cap * Hhd * 4);
+    AL(c->attn_ml, (size_t)kAttnMaxSplits * cap * cfg->n_heads * sizeof(float2));
+    AL(c->attn_ctr, (size_t)cfg->max_batch * cfg->n_kv_heads * c->attn_qt_cap * 4);
+  }
 #undef AL
   if (e != cudaSuccess) {
     std::string m = std::string("device allocation failed: ") + cudaGetErrorString(e);
@@ -409,7 +503,10 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     delete c;
     return fail(nullptr, DCU_ENOMEM, m);
   }
-  e = cudaMemset(c->ints, 0, 64);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
+  if (e == cudaSuccess && c->attn_ctr)
+    e = cudaMemset(c->attn_ctr, 0, (size_t)cfg->max_batch * cfg->n_kv_heads * c->attn_qt_cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
   if (e == cudaSuccess && cfg->rope_theta > 0.0f)
@@ -433,11 +530,11 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
       wmap(&m.wd, c->wd[l], D, F);
     }
     wmap(&c->lm_map, c->lm_head, (size_t)cfg->vocab, D);
-    const uint32_t bns[2] = {128, 256};
+    const uint32_t boxes[2] = {16, 64};
     for (int i = 0; i < 2; ++i) {
-      ok = ok && encode_tmap_bf16(&c->xs_map[i], c->xs, D, cap, D * 2, 64, bns[i]);
-      ok = ok && encode_tmap_bf16(&c->attn_map[i], c->attn, Hhd, cap, Hhd * 2, 64, bns[i]);
-      ok = ok && encode_tmap_bf16(&c->act_map[i], c->act, F, cap, F * 2, 64, bns[i]);
+      ok = ok && encode_tmap_bf16(&c->xs_map[i], c->xs, D, cap, D * 2, 64, boxes[i]);
+      ok = ok && encode_tmap_bf16(&c->attn_map[i], c->attn, Hhd, cap, Hhd * 2, 64, boxes[i]);
+      ok = ok && encode_tmap_bf16(&c->act_map[i], c->act, F, cap, F * 2, 64, boxes[i]);
     }
     if (!ok) {
       free_all(c);
@@ -477,24 +574,29 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
     LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
                                c->cfg.d_model, c->cfg.vocab, 1, c->status(), s));
   }
-  LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), s));
+  LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), c->seq_off, s));
   c->gemm_bn = 256;
   c->gemm_rows_hint = BN;
   for (int l = 0; l < c->cfg.n_layers; ++l)
     if (int rc = run_layer(c, l, true, nullptr, nullptr, 0, s)) return rc;
   CK(c, cudaMemsetAsync(c->s_prev, 0, (size_t)c->cfg.max_batch * c->cfg.n_layers * 4, s));
+  {
+    static const int32_t one = 1;
+    CK(c, cudaMemcpyAsync(c->uniform_flag(), &one, 4, cudaMemcpyHostToDevice, s));
+  }
   c->first_step = true;
   c->have_cache = true;
   return DCU_OK;
 }
 
-int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t *nkeys, int32_t B_layer,
-             int32_t B_window, dcu_stream_t stream) {
-  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
-  if (!c->have_cache) return fail(c, DCU_ESTATE, "dcu_step before dcu_full_forward");
-  if (!ids || !keys || !nkeys) return fail(c, DCU_EINVAL, "token_ids, key_positions or n_keys is NULL");
-  if (B_layer < 0 || B_window < 0) return fail(c, DCU_EINVAL, "B_layer and B_window must be >= 0");
-  cudaStream_t s = (cudaStream_t)stream;
+}  // extern "C"
+
+namespace {
+
+// Every launch of one DCU step on stream s (uses only state that is fixed for
+// a given (pointers, B_layer, B_window, B, N), so it can be captured once).
+int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t *nkeys, int B_layer,
+                 int B_window, cudaStream_t s) {
   const int L = c->cfg.n_layers, BN = c->B * c->N;
   {
     // expected rows per layer: twice the mean budget plus a few windows per sequence
@@ -504,18 +606,156 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
   }
   {
     Prof p(c, DCU_K_BUDGET, s);
-    LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, c->first_step ? 1 : 0, c->budgets, s));
+    LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, 0, c->uniform_flag(), c->budgets, s));
   }
   {
     Prof p(c, DCU_K_REFRESH, s);
     LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
-                               c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
+                                   c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
   }
   for (int l = 0; l < L; ++l)
     if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) return rc;
   CK(c, cudaMemcpyAsync(c->s_prev, c->s_cur, (size_t)c->B * L * 4, cudaMemcpyDeviceToDevice, s));
-  c->first_step = false;
+  CK(c, cudaMemsetAsync(c->uniform_flag(), 0, 4, s));
   return DCU_OK;
+}
+
+int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
+                   int32_t *out_count, cudaStream_t s) {
+  const dcu_cfg &g = c->cfg;
+  const int cap = (int)c->cap;
+  {
+    {
+      Prof p(c, DCU_K_LMHEAD, s);
+      LAUNCH(c, launch_plan_masked(masked, c->B, c->N, c->mrow, c->m_masked(), s));
+    }
+    {
+      Prof p(c, DCU_K_LMHEAD, s);
+      LAUNCH(c, launch_gather_norm(g.dtype, c->mrow, c->m_masked(), cap, c->Hl(g.n_layers), c->final_norm,
+                                   g.rms_eps, g.d_model, c->xs, s));
+    }
+    GemmSeg lm[1] = {{c->lm_head, g.vocab}};
+    c->gemm_bn = 256;
+    c->gemm_rows_hint = 256;
+    if (g.dtype == DCU_BF16) {
+      // tcgen05 LM head with the softmax statistics fused into its epilogue
+      Prof p(c, DCU_K_LMHEAD, s);
+      TcParams tp;
+      memset(&tp, 0, sizeof(tp));
+      tp.a[0] = c->lm_map;
+      tp.b16 = c->xs_map[0];
+      tp.b64 = c->xs_map[1];
+      const int tiles = (g.vocab + 127) / 128;
+      tp.seg_tile0[0] = 0;
+      tp.seg_tile0[1] = tiles;
+      tp.seg_rows[0] = g.vocab;
+      tp.nseg = 1;
+      tp.geo.n_tiles = tiles;
+      tp.geo.kblocks = g.d_model / 64;
+      tp.geo.grid = tiles < c->num_sms ? tiles : c->num_sms;
+      tp.geo.tile_aligned = 1;
+      tp.ldc = g.vocab;
+      tp.m_total = c->m_masked();
+      tp.status = c->status();
+      tp.epi_mode = 1;
+      tp.smx = c->smx;
+      tp.smx_arg = c->smx_arg;
+      tp.ldm = cap;
+      LAUNCH(c, launch_gemm_tc(tp, 256, s));
+    } else {
+      SlotGeo geo;
+      const ActOperand xs{c->xs, g.d_model, g.d_model, nullptr, nullptr};
+      if (int rc = run_gemm(c, xs, c->m_masked(), lm, nullptr, 1, g.vocab, s, &geo, true, DCU_K_LMHEAD)) return rc;
+    }
+    Prof p(c, DCU_K_LMHEAD, s);
+    if (g.dtype == DCU_BF16)
+      LAUNCH(c, launch_lm_combine(c->smx, c->smx_arg, (g.vocab + 127) / 128, cap, c->mrow, c->m_masked(), cap,
+                                  c->conf, c->amax, s));
+    else
+      LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));
+  }
+  {
+    Prof p(c, DCU_K_COMMIT, s);
+    LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, out_pos, out_count, s));
+  }
+  return DCU_OK;
+}
+
+// Runs `body` directly, or through a cached CUDA graph keyed by `key` (captured
+// on the context's private stream, launched on s).
+template <class F>
+int run_graphed(dcu_ctx *c, const uint64_t (&key)[10], cudaStream_t s, F &&body) {
+  if (!c->use_graphs) return body(s);
+  GraphEntry *g = nullptr;
+  for (auto &e : c->graphs)
+    if (memcmp(e.key, key, sizeof(key)) == 0) g = &e;
+  if (!g) {
+    if (c->graphs.size() >= kMaxGraphs) {  // evict the least recently used
+      size_t victim = 0;
+      for (size_t i = 1; i < c->graphs.size(); ++i)
+        if (c->graphs[i].last_use < c->graphs[victim].last_use) victim = i;
+      CK(c, cudaStreamSynchronize(c->cap_stream));
+      CK(c, cudaDeviceSynchronize());
+      free_graph(c->graphs[victim]);
+      c->graphs.erase(c->graphs.begin() + (long)victim);
+    }
+    c->graphs.emplace_back();
+    g = &c->graphs.back();
+    memcpy(g->key, key, sizeof(key));
+    CK(c, cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+    const int64_t l0 = c->launches;
+    c->capturing = true;
+    c->cur_graph = g;
+    const int rc = body(c->cap_stream);
+    c->capturing = false;
+    c->cur_graph = nullptr;
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(c->cap_stream, &graph);
+    g->kernels = c->launches - l0;
+    c->launches = l0;
+    cudaError_t ei = cudaSuccess;
+    if (rc == DCU_OK && e == cudaSuccess) ei = cudaGraphInstantiate(&g->exec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    if (rc != DCU_OK || e != cudaSuccess || ei != cudaSuccess) {
+      free_graph(*g);
+      c->graphs.pop_back();
+      cudaGetLastError();
+      if (rc != DCU_OK) return rc;
+      return fail(c, DCU_ECUDA, std::string("graph capture failed: ") +
+                                    cudaGetErrorString(e != cudaSuccess ? e : ei));
+    }
+  }
+  g->last_use = ++c->use_clock;
+  CK(c, cudaGraphLaunch(g->exec, s));
+  ++g->replays;
+  c->launches += g->kernels;
+  return DCU_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t *nkeys, int32_t B_layer,
+             int32_t B_window, dcu_stream_t stream) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (!c->have_cache) return fail(c, DCU_ESTATE, "dcu_step before dcu_full_forward");
+  if (!ids || !keys || !nkeys) return fail(c, DCU_EINVAL, "token_ids, key_positions or n_keys is NULL");
+  if (B_layer < 0 || B_window < 0) return fail(c, DCU_EINVAL, "B_layer and B_window must be >= 0");
+  const uint64_t key[10] = {1,
+                            (uint64_t)(uintptr_t)ids,
+                            (uint64_t)(uintptr_t)keys,
+                            (uint64_t)(uintptr_t)nkeys,
+                            (uint64_t)B_layer,
+                            (uint64_t)B_window,
+                            ((uint64_t)c->B << 32) | (uint64_t)c->N,
+                            (uint64_t)(c->prof_max > 0),
+                            0,
+                            0};
+  int rc = run_graphed(c, key, (cudaStream_t)stream,
+                       [&](cudaStream_t s) { return enqueue_step(c, ids, keys, nkeys, B_layer, B_window, s); });
+  if (rc == DCU_OK) c->first_step = false;
+  return rc;
 }
 
 int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
@@ -525,27 +765,26 @@ int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_
   if (rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR)
     return fail(c, DCU_EINVAL, "rule must be DCU_FRECHET, DCU_THRESHOLD or DCU_FACTOR");
   if (!masked || !ids || !out_pos || !out_count) return fail(c, DCU_EINVAL, "a buffer is NULL");
-  cudaStream_t s = (cudaStream_t)stream;
-  const dcu_cfg &g = c->cfg;
-  const int cap = (int)c->cap;
-  {
-    Prof p(c, DCU_K_LMHEAD, s);
-    LAUNCH(c, launch_plan_masked(masked, c->B, c->N, c->mrow, c->m_masked(), s));
-    LAUNCH(c, launch_gather_norm(g.dtype, c->mrow, c->m_masked(), cap, c->Hl(g.n_layers), c->final_norm, g.rms_eps,
-                             g.d_model, c->xs, s));
-    GemmSeg lm[1] = {{c->lm_head, g.vocab}};
-    const CUtensorMap *am[1] = {&c->lm_map};
-    const ActOperand xs{c->xs, g.d_model, g.d_model, &c->xs_map[0], &c->xs_map[1]};
-    c->gemm_bn = 256;
-    c->gemm_rows_hint = 256;
-    int sp = 1;
-    if (int rc = run_gemm(c, xs, c->m_masked(), lm, am, 1, g.vocab, s, &sp, 1)) return rc;
-    LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));
-  }
-  {
-    Prof p(c, DCU_K_COMMIT, s);
-    LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, out_pos, out_count, s));
-  }
+  uint32_t pbits;
+  memcpy(&pbits, &param, 4);
+  const uint64_t key[10] = {2,
+                            (uint64_t)rule,
+                            (uint64_t)pbits,
+                            (uint64_t)(uintptr_t)masked,
+                            (uint64_t)(uintptr_t)ids,
+                            (uint64_t)(uintptr_t)out_pos,
+                            (uint64_t)(uintptr_t)out_count,
+                            ((uint64_t)c->B << 32) | (uint64_t)c->N,
+                            (uint64_t)(c->prof_max > 0),
+                            0};
+  return run_graphed(c, key, (cudaStream_t)stream, [&](cudaStream_t s) {
+    return enqueue_commit(c, rule, param, masked, ids, out_pos, out_count, s);
+  });
+}
+
+int dcu_set_graphs(dcu_ctx *c, int32_t on) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  c->use_graphs = on != 0;
   return DCU_OK;
 }
 
@@ -566,9 +805,9 @@ int dcu_status(dcu_ctx *c, dcu_stream_t stream, int32_t *bits) {
 
 int dcu_budget_split(const float *s_prev, int32_t B, int32_t L, int32_t B_layer, int32_t uniform, int32_t *budgets,
                      dcu_stream_t stream) {
-  if (!s_prev || !budgets || B <= 0 || L <= 0 || B_layer < 0)
+  if (!s_prev || !budgets || B <= 0 || L <= 0 || L > 1024 || B_layer < 0)
     return fail(nullptr, DCU_EINVAL, "dcu_budget_split: bad argument");
-  CK(nullptr, launch_budget_split(s_prev, B, L, B_layer, uniform, budgets, (cudaStream_t)stream));
+  CK(nullptr, launch_budget_split(s_prev, B, L, B_layer, uniform, nullptr, budgets, (cudaStream_t)stream));
   return DCU_OK;
 }
 
@@ -579,7 +818,7 @@ int dcu_select_tokens(const float *d, const int32_t *keys, const int32_t *nkeys,
       B_window < 0 || (window_mode != 0 && window_mode != 1))
     return fail(nullptr, DCU_EINVAL, "dcu_select_tokens: bad argument");
   CK(nullptr, launch_select(d, keys, nkeys, budgets, 1, B, N, B_window, window_mode, idx, count, s, 1, nullptr,
-                            nullptr, nullptr, nullptr, status, (cudaStream_t)stream));
+                            nullptr, nullptr, nullptr, nullptr, status, (cudaStream_t)stream));
   return DCU_OK;
 }
 
@@ -618,7 +857,8 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
   memset(&tp, 0, sizeof(tp));
   const int bn = M <= 128 ? 128 : 256;
   if (!encode_tmap_bf16(&tp.a[0], W, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, 64, 128) ||
-      !encode_tmap_bf16(&tp.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)bn))
+      !encode_tmap_bf16(&tp.b16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 16) ||
+      !encode_tmap_bf16(&tp.b64, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 64))
     return fail(nullptr, DCU_ECUDA, "dcu_linear: cuTensorMapEncodeTiled failed");
   const int tiles = (Nout + 127) / 128;
   tp.seg_tile0[0] = 0;
@@ -626,20 +866,19 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
   tp.seg_col0[0] = 0;
   tp.seg_rows[0] = Nout;
   tp.nseg = 1;
-  tp.n_tiles = tiles;
-  tp.kblocks = K / 64;
-  tp.splits = 1;
   tp.ldc = Nout;
   tp.m_total = nullptr;
   tp.m_host = M;
-  tp.ws = Y;
-  tp.split_stride = 0;
+  tp.out = Y;
   tp.status = nullptr;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long units = (long long)tiles * ((M + bn - 1) / bn);
-  CK(nullptr, launch_gemm_tc(tp, bn, (int)(units < sms ? units : sms), s));
+  tp.geo.n_tiles = tiles;
+  tp.geo.kblocks = K / 64;
+  tp.geo.tile_aligned = 1;
+  tp.geo.grid = tiles < sms ? tiles : sms;
+  CK(nullptr, launch_gemm_tc(tp, bn, s));
   return DCU_OK;
 }
 
@@ -734,7 +973,10 @@ int dcu_set_tensor(dcu_ctx *c, int32_t kind, int32_t layer, const void *src, int
   if (int rc = tensor_ptr(c, kind, layer, &p, &n)) return rc;
   if (bytes != n) return fail(c, DCU_EINVAL, "size mismatch: expected " + std::to_string(n) + " bytes");
   CK(c, cudaMemcpyAsync(p, src, n, cudaMemcpyDeviceToDevice, (cudaStream_t)stream));
-  if (kind == DCU_T_S_PREV) c->first_step = false;
+  if (kind == DCU_T_S_PREV) {
+    c->first_step = false;
+    CK(c, cudaMemsetAsync(c->uniform_flag(), 0, 4, (cudaStream_t)stream));
+  }
   return DCU_OK;
 }
 
@@ -770,10 +1012,34 @@ int dcu_profile_read(dcu_ctx *c, int32_t k, double *total_ms, int64_t *launches,
     CK(c, cudaEventElapsedTime(&ms, pc.ev[i].a, pc.ev[i].b));
     t += ms;
   }
+  int64_t n = pc.used;
+  // graphs: event-record nodes hold the times of the graph's most recent
+  // replay; they stand for each of its replays since the last reset
+  for (auto &g : c->graphs) {
+    if (g.replays == 0) continue;
+    double tg = 0.0;
+    int64_t ng = 0;
+    for (auto &e : g.ev) {
+      if (e.first != k) continue;
+      CK(c, cudaEventSynchronize(e.second.b));
+      float ms = 0.f;
+      CK(c, cudaEventElapsedTime(&ms, e.second.a, e.second.b));
+      tg += ms;
+      ++ng;
+    }
+    t += tg * (double)g.replays;
+    n += ng * g.replays;
+  }
   *total_ms = t;
-  *launches = pc.used;
+  *launches = n;
   if (pc.dropped) return fail(c, DCU_ECAPACITY, "more launches than profile slots");
-  if (reset) pc.used = pc.dropped = 0;
+  if (reset) {
+    pc.used = pc.dropped = 0;
+    bool all_read = true;
+    for (int kk = 0; kk < DCU_K_COUNT; ++kk) all_read = all_read && (kk <= k);
+    if (all_read)
+      for (auto &g : c->graphs) g.replays = 0;
+  }
   return DCU_OK;
 }
 

@@ -6,28 +6,65 @@
 
 namespace dcu {
 
+constexpr int kTcMaxStages = 12;             // deepest smem ring
+constexpr uint32_t kTcABytes = 128u * 128u;  // weight tile: 128 rows x 64 bf16
+constexpr uint32_t kTcBBoxBytes = 16u * 128u;  // activation box: 16 rows x 64 bf16
+constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (one CTA per SM)
+
+// Stream-K schedule: the flattened (tile, k block) space of one token pass,
+// T = n_tiles * kblocks, is cut into G contiguous ranges [c*T/G, (c+1)*T/G)
+// (with tile_aligned the cut points are rounded down to whole tiles).  A tile
+// is computed in nslots pieces, one per CTA whose range meets it; piece j is
+// stored in slot j, so a consumer sums slots 0..nslots-1 of the tile in slot
+// order and the result does not depend on CTA scheduling.
+struct SlotGeo {
+  int n_tiles, kblocks, grid, tile_aligned;
+  long long slot_stride;  // elements between two slots (cap * ldc)
+};
+
+__host__ __device__ inline long long sk_begin(const SlotGeo &g, int c) {
+  if (g.tile_aligned) return (long long)g.n_tiles * c / g.grid * g.kblocks;
+  return (long long)g.n_tiles * g.kblocks * c / g.grid;
+}
+// CTA whose range holds flattened index x
+__host__ __device__ inline int sk_owner(const SlotGeo &g, long long x) {
+  const long long T = (long long)g.n_tiles * g.kblocks;
+  int c = (int)((x * (long long)g.grid) / T);
+  if (c >= g.grid) c = g.grid - 1;
+  while (c + 1 < g.grid && sk_begin(g, c + 1) <= x) ++c;
+  while (c > 0 && sk_begin(g, c) > x) --c;
+  return c;
+}
+__host__ __device__ inline int sk_first(const SlotGeo &g, int tile) { return sk_owner(g, (long long)tile * g.kblocks); }
+__host__ __device__ inline int sk_nslots(const SlotGeo &g, int tile) {
+  return sk_owner(g, (long long)(tile + 1) * g.kblocks - 1) - sk_first(g, tile) + 1;
+}
+
 // Kernel parameters (passed as a __grid_constant__ so the tensor maps can be
-// addressed by TMA).  Output column of segment s, row r: seg_col0[s] + r.
+// addressed by TMA).  Output column of segment s, row r: seg_col0[s] + r;
+// every segment but the last has rows % 128 == 0, so column n lies in tile n / 128.
+// out[slot][m][n] = the piece `slot` of sum_k X[m][k] * W[n][k] for m < M.
 struct TcParams {
   CUtensorMap a[3];        // weight segments, bf16 [rows][K], box 64 x 128, 128-byte swizzle
-  CUtensorMap b;           // packed activations, bf16 [cap][K], box 64 x BN, 128-byte swizzle
+  CUtensorMap b16, b64;    // packed activations, bf16 [cap][K], boxes 64 x 16 and 64 x 64, 128-byte swizzle
   int seg_tile0[4];        // first 128-row tile of segment s; seg_tile0[nseg] = n_tiles
   int seg_col0[3];         // first output column of segment s
   int seg_rows[3];         // rows of segment s
-  int nseg, n_tiles, kblocks, splits, ldc;
+  int nseg, ldc;
+  SlotGeo geo;             // n_tiles, kblocks, grid (= gridDim.x), tile_aligned, slot stride
   const int32_t *m_total;  // device row count M (or null: m_host)
   int m_host;
-  float *ws;               // partials [splits][cap][ldc]
-  long long split_stride;  // elements between two splits' partials
-  int32_t *status;         // device status word (DCU_ST_TIMEOUT)
-};
-
-template <int BN>
-struct TcCfg {
-  static constexpr int STAGES = BN <= 64 ? 8 : (BN <= 128 ? 6 : 4);
-  static constexpr uint32_t A_BYTES = 128u * 64u * 2u;
-  static constexpr uint32_t B_BYTES = (uint32_t)BN * 64u * 2u;
-  static constexpr size_t SMEM = (size_t)STAGES * (A_BYTES + B_BYTES) + 1024;
+  float *out;              // [slots][cap][ldc]
+  int32_t *status;         // device status word (DCU_ST_TIMEOUT) or null
+  uint32_t smem_bytes;
+  // epi_mode 1 (LM head, tile_aligned): instead of storing logits, every tile
+  // writes per token m its softmax statistics over the tile's 128 vocabulary
+  // entries: smx[tile][m] = (max, sum of exp(z - max)), smx_arg[tile][m] =
+  // lowest id reaching the max; row pitch ldm.
+  int epi_mode;
+  float2 *smx;
+  int32_t *smx_arg;
+  int ldm;
 };
 
 // Row-major bf16 matrix [outer][inner] with row pitch row_bytes, box
@@ -35,7 +72,15 @@ struct TcCfg {
 // missing or the encoding is rejected.
 bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                       uint32_t box_inner, uint32_t box_outer);
-int choose_splits(int n_tiles, int kblocks, int passes, int num_sms);
-cudaError_t launch_gemm_tc(const TcParams &p, int bn, int grid, cudaStream_t s);
+// bn: token rows per pass (128 or 256); the grid is p.geo.grid CTAs.
+cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s);
+// Most pieces a tile can be cut into under the stream-K split over `grid` CTAs.
+int tc_max_slots(int n_tiles, int grid);
+// Merges the per-tile softmax statistics of the LM head (epi_mode 1): for packed
+// row r (position rowmap[r]), conf = 1 / sum_t s_t exp(m_t - M), argmax = the
+// lowest id reaching M = max_t m_t.
+cudaError_t launch_lm_combine(const float2 *smx, const int32_t *smx_arg, int n_tiles, int ldm,
+                              const int32_t *rowmap, const int32_t *m_total, int cap, float *conf, int32_t *amax,
+                              cudaStream_t s);
 
 }  // namespace dcu

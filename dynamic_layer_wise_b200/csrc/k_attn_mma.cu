@@ -1,0 +1,359 @@
+// Tensor-core attention of the recomputed queries over all N cached keys of
+// their sequence (bidirectional, unmasked; [DLLM] "研究背景与动机").
+//
+// One CTA per (sequence b, kv head, key split, tile of 128 queries); a query is
+// a (packed row, query head) pair of the kv head's GQA group, so the CTA reads
+// its K/V chunk from HBM once for every query of the group.  8 warps x 16
+// queries; K/V are staged in shared memory in 64-key sub-chunks with cp.async
+// (double buffer, zero-filled past N); S = Q K^T and O += P V run on
+// mma.sync m16n8k16 bf16 (fp32 accumulate) with an online softmax in
+// registers.  With several key splits, each CTA writes (O, max, sum) partials
+// and the last CTA of the tile (atomic counter, reset after use) merges them
+// in split order, so the result does not depend on CTA scheduling.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcu {
+namespace {
+
+constexpr int QT = 128;  // queries per CTA
+constexpr int KS = 64;   // keys per sub-chunk
+
+__device__ __forceinline__ uint32_t smem_u32a(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool valid) {
+  const int n = valid ? 16 : 0;  // zero-fill when invalid
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+struct AttnArgs {
+  const bf16 *Q;            // [cap][H][hd]
+  const bf16 *Kc, *Vc;      // [B][Hkv][N][hd]
+  bf16 *out;                // [cap][H][hd]
+  const int32_t *seq_off;   // [B + 1] packed-row offsets of the sequences
+  float *part_o;            // [splits][cap * H][hd] partial outputs
+  float2 *part_ml;          // [splits][cap * H] (max, sum) in log2 units
+  int32_t *counters;        // [B][Hkv][qt_cap] arrival counters (zero between launches)
+  int B, N, H, Hkv, splits, kc, qt_grid, qt_cap;
+  float scale_log2;         // log2(e) / sqrt(hd)
+};
+
+template <int HD>
+__device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int *s_last, int b, int kvh, int ks, int qt,
+                                          int row0, int nq) {
+  constexpr int LD = HD + 8;  // padded row (elements): 16-byte shift per row, conflict-free ldmatrix
+  constexpr int CPR = HD / 8;  // 16-byte chunks per row
+  bf16 *Qs = reinterpret_cast<bf16 *>(sm);  // [QT][LD]
+  bf16 *Ks = Qs + QT * LD;                   // [2][KS][LD]
+  bf16 *Vs = Ks + 2 * KS * LD;               // [2][KS][LD]
+  const int G = a.H / a.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int k_begin = ks * a.kc;
+  const int k_end = min(a.N, k_begin + a.kc);
+  const bf16 *Kb = a.Kc + ((size_t)b * a.Hkv + kvh) * (size_t)a.N * HD;
+  const bf16 *Vb = a.Vc + ((size_t)b * a.Hkv + kvh) * (size_t)a.N * HD;
+
+  // Q tile -> shared (query q -> packed row row0 + q / G, head kvh * G + q % G)
+  for (int c = tid; c < QT * CPR; c += blockDim.x) {
+    const int qi = c / CPR, ch = c - qi * CPR;
+    const int q = qt * QT + qi;
+    const bool ok = q < nq;
+    const int r = row0 + (ok ? q / G : 0), h = kvh * G + (ok ? q % G : 0);
+    cp_async16(smem_u32a(Qs + qi * LD + ch * 8), a.Q + ((size_t)r * a.H + h) * HD + ch * 8, ok);
+  }
+  auto load_kv = [&](int buf, int key0) {
+    for (int c = tid; c < KS * CPR; c += blockDim.x) {
+      const int ki = c / CPR, ch = c - ki * CPR;
+      const int key = key0 + ki;
+      const bool ok = key < k_end;
+      const size_t off = (size_t)(ok ? key : k_begin) * HD + ch * 8;
+      cp_async16(smem_u32a(Ks + (buf * KS + ki) * LD + ch * 8), Kb + off, ok);
+      cp_async16(smem_u32a(Vs + (buf * KS + ki) * LD + ch * 8), Vb + off, ok);
+    }
+  };
+  load_kv(0, k_begin);
+  cp_async_commit();
+
+  float o[HD / 8][4];
+#pragma unroll
+  for (int i = 0; i < HD / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  uint32_t qf[HD / 16][4];
+  const bool warp_active = (qt * QT + warp * 16) < nq;
+
+  const int n_sub = (k_end - k_begin + KS - 1) / KS;
+  for (int sc = 0; sc < n_sub; ++sc) {
+    const int buf = sc & 1;
+    if (sc + 1 < n_sub) load_kv(buf ^ 1, k_begin + (sc + 1) * KS);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    if (sc == 0 && warp_active) {
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+        const int rr = warp * 16 + (lane & 15), cc = kk * 16 + (lane >> 4) * 8;
+        ldsm_x4(smem_u32a(Qs + rr * LD + cc), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
+      }
+    }
+    if (warp_active) {
+      const bf16 *Kt = Ks + buf * KS * LD;
+      const bf16 *Vt = Vs + buf * KS * LD;
+      float s[KS / 8][4];
+#pragma unroll
+      for (int j = 0; j < KS / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk) {
+#pragma unroll
+        for (int j = 0; j < KS / 16; ++j) {
+          // keys 16j .. 16j+15, d 16kk .. 16kk+15
+          const int key = j * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int d = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(smem_u32a(Kt + key * LD + d), b0, b1, b2, b3);
+          mma_bf16(s[2 * j], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
+          mma_bf16(s[2 * j + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
+        }
+      }
+      // online softmax (log2 domain); keys past k_end are masked
+      const int key_base = k_begin + sc * KS;
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < KS / 8; ++j) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = key_base + j * 8 + t * 2 + (e & 1);
+          const float v = key < k_end ? s[j][e] * a.scale_log2 : -INFINITY;
+          s[j][e] = v;
+          mx[e >> 1] = fmaxf(mx[e >> 1], v);
+        }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
+        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+      }
+      float corr[2], mnew[2], psum[2] = {0.f, 0.f};
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        mnew[h2] = fmaxf(m_run[h2], mx[h2]);
+        corr[h2] = (m_run[h2] == -INFINITY) ? 0.f : exp2f(m_run[h2] - mnew[h2]);
+        m_run[h2] = mnew[h2];
+      }
+      uint32_t pf[KS / 16][4];
+#pragma unroll
+      for (int j = 0; j < KS / 8; ++j) {
+        const float p0 = exp2f(s[j][0] - mnew[0]), p1 = exp2f(s[j][1] - mnew[0]);
+        const float p2 = exp2f(s[j][2] - mnew[1]), p3 = exp2f(s[j][3] - mnew[1]);
+        psum[0] += p0 + p1;
+        psum[1] += p2 + p3;
+        const int kk = j >> 1;
+        if ((j & 1) == 0) {
+          pf[kk][0] = pack_bf16(p0, p1);
+          pf[kk][1] = pack_bf16(p2, p3);
+        } else {
+          pf[kk][2] = pack_bf16(p0, p1);
+          pf[kk][3] = pack_bf16(p2, p3);
+        }
+      }
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 1);
+        psum[h2] += __shfl_xor_sync(0xffffffffu, psum[h2], 2);
+        l_run[h2] = l_run[h2] * corr[h2] + psum[h2];
+      }
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i) {
+        o[i][0] *= corr[0];
+        o[i][1] *= corr[0];
+        o[i][2] *= corr[1];
+        o[i][3] *= corr[1];
+      }
+      // O += P V: k = keys (KS / 16 steps), n = d (HD / 8 tiles)
+#pragma unroll
+      for (int kk = 0; kk < KS / 16; ++kk) {
+#pragma unroll
+        for (int i = 0; i < HD / 16; ++i) {
+          const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int d = i * 16 + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(smem_u32a(Vt + key * LD + d), b0, b1, b2, b3);
+          mma_bf16(o[2 * i], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b0, b1);
+          mma_bf16(o[2 * i + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b2, b3);
+        }
+      }
+    }
+    __syncthreads();  // the buffer is refilled in the next iteration
+  }
+
+  if (a.splits == 1) {  // single split: normalise and store
+    if (warp_active) {
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int q = qt * QT + warp * 16 + g + h2 * 8;
+        if (q >= nq) continue;
+        const int r = row0 + q / G, h = kvh * G + q % G;
+        const float inv = 1.f / l_run[h2];
+        bf16 *dst = a.out + ((size_t)r * a.H + h) * HD;
+#pragma unroll
+        for (int i = 0; i < HD / 8; ++i)
+          *reinterpret_cast<__nv_bfloat162 *>(dst + i * 8 + t * 2) =
+              __floats2bfloat162_rn(o[i][2 * h2] * inv, o[i][2 * h2 + 1] * inv);
+      }
+    }
+    return;
+  }
+  // partials of this split: plane = packed (row, head) pairs of all sequences
+  const size_t plane = (size_t)a.seq_off[a.B] * a.H;
+  if (warp_active) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int q = qt * QT + warp * 16 + g + h2 * 8;
+      if (q >= nq) continue;
+      const int r = row0 + q / G, h = kvh * G + q % G;
+      const size_t qidx = (size_t)r * a.H + h;
+      float *dst = a.part_o + ((size_t)ks * plane + qidx) * HD;
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i)
+        *reinterpret_cast<float2 *>(dst + i * 8 + t * 2) = make_float2(o[i][2 * h2], o[i][2 * h2 + 1]);
+      if (t == 0) a.part_ml[(size_t)ks * plane + qidx] = make_float2(m_run[h2], l_run[h2]);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  int32_t *ctr = a.counters + ((size_t)b * a.Hkv + kvh) * a.qt_cap + qt;
+  if (tid == 0) *s_last = (atomicAdd(ctr, 1) == a.splits - 1);
+  __syncthreads();
+  if (!*s_last) return;
+  __threadfence();
+  // merge the splits of this tile's queries in split order
+  const int nq_tile = min(QT, nq - qt * QT);
+  for (int c = tid; c < nq_tile * (HD / 4); c += blockDim.x) {
+    const int qi = c / (HD / 4), d4 = (c - qi * (HD / 4)) * 4;
+    const int q = qt * QT + qi;
+    const int r = row0 + q / G, h = kvh * G + q % G;
+    const size_t qidx = (size_t)r * a.H + h;
+    float M = -INFINITY;
+    for (int sp = 0; sp < a.splits; ++sp) M = fmaxf(M, __ldcg(a.part_ml + sp * plane + qidx).x);
+    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < a.splits; ++sp) {
+      const float2 ml = __ldcg(a.part_ml + sp * plane + qidx);
+      if (ml.x == -INFINITY) continue;
+      const float w = exp2f(ml.x - M);
+      L += ml.y * w;
+      const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sp * plane + qidx) * HD + d4));
+      acc[0] += v.x * w;
+      acc[1] += v.y * w;
+      acc[2] += v.z * w;
+      acc[3] += v.w * w;
+    }
+    const float inv = 1.f / L;
+    bf16 *dst = a.out + qidx * HD + d4;
+    *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    *reinterpret_cast<__nv_bfloat162 *>(dst + 2) = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+  }
+  __syncthreads();
+  if (tid == 0) *ctr = 0;
+}
+
+// grid = B x Hkv x splits x qt_grid; the CTA walks query tiles qt, qt + qt_grid, ...
+template <int HD>
+__global__ void __launch_bounds__(256, 1) k_attn_mma(const AttnArgs a) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int s_last;
+  int item = blockIdx.x;
+  const int per_b = a.Hkv * a.splits * a.qt_grid;
+  const int b = item / per_b;
+  if (b >= a.B) return;
+  item -= b * per_b;
+  const int qt0 = item / (a.Hkv * a.splits);
+  item -= qt0 * a.Hkv * a.splits;
+  const int kvh = item / a.splits, ks = item - kvh * a.splits;
+  const int row0 = a.seq_off[b], nq = (a.seq_off[b + 1] - row0) * (a.H / a.Hkv);
+  if (ks * a.kc >= a.N) return;
+  for (int qt = qt0; qt * QT < nq; qt += a.qt_grid) {
+    attn_tile<HD>(a, sm, &s_last, b, kvh, ks, qt, row0, nq);
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t attn_mma_smem(int hd) { return (size_t)(QT + 4 * KS) * (hd + 8) * sizeof(bf16); }
+
+cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
+                                 const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
+                                 int32_t *counters, int splits, int qt_grid, int qt_cap, cudaStream_t s) {
+  if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
+  AttnArgs a;
+  a.Q = (const bf16 *)Q;
+  a.Kc = (const bf16 *)Kc;
+  a.Vc = (const bf16 *)Vc;
+  a.out = (bf16 *)out;
+  a.seq_off = seq_off;
+  a.part_o = part_o;
+  a.part_ml = part_ml;
+  a.counters = counters;
+  a.B = B;
+  a.N = N;
+  a.H = H;
+  a.Hkv = Hkv;
+  a.splits = splits;
+  a.kc = ((N + splits - 1) / splits + KS - 1) / KS * KS;
+  a.qt_grid = qt_grid;
+  a.qt_cap = qt_cap;
+  a.scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
+  const size_t smem = attn_mma_smem(hd);
+  const int grid = B * Hkv * splits * qt_grid;
+  if (grid <= 0) return cudaSuccess;
+  if (hd == 128) {
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_attn_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    k_attn_mma<128><<<grid, 256, smem, s>>>(a);
+  } else {
+    static bool attr = false;
+    if (!attr) {
+      cudaError_t e = cudaFuncSetAttribute(k_attn_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    k_attn_mma<64><<<grid, 256, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace dcu

@@ -158,60 +158,87 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return;
 }
 
-struct Unit {
-  int tile, split, pass, seg, arow, kb0, kb1, m0;
+struct Frag {
+  int tile, kb0, kb1, seg, arow, slot;
 };
 
-__device__ __forceinline__ Unit decode_unit(const TcParams &p, int u, int passes) {
-  Unit w;
-  w.pass = u % passes;
-  const int ts = u / passes;
-  w.split = ts % p.splits;
-  w.tile = ts / p.splits;
-  w.kb0 = (int)((long long)w.split * p.kblocks / p.splits);
-  w.kb1 = (int)((long long)(w.split + 1) * p.kblocks / p.splits);
+// Fragment iterator over this CTA's stream-K range, pass by pass.
+struct FragIter {
+  long long pos, end;
+  int pass;
+};
+
+__device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIter &it, Frag &f) {
+  while (it.pos >= it.end) {
+    if (++it.pass >= passes) return false;
+    it.pos = sk_begin(p.geo, blockIdx.x);
+  }
+  const int KB = p.geo.kblocks;
+  const int t = (int)(it.pos / KB);
+  const int kb0 = (int)(it.pos - (long long)t * KB);
+  const long long left = it.end - it.pos;
+  const int kb1 = (int)((long long)kb0 + left < KB ? kb0 + left : KB);
+  it.pos += kb1 - kb0;
+  f.tile = t;
+  f.kb0 = kb0;
+  f.kb1 = kb1;
   int seg = 0;
-  while (seg + 1 < p.nseg && w.tile >= p.seg_tile0[seg + 1]) ++seg;
-  w.seg = seg;
-  w.arow = (w.tile - p.seg_tile0[seg]) * 128;
-  return w;
+  while (seg + 1 < p.nseg && t >= p.seg_tile0[seg + 1]) ++seg;
+  f.seg = seg;
+  f.arow = (t - p.seg_tile0[seg]) * 128;
+  f.slot = (int)blockIdx.x - sk_first(p.geo, t);
+  return true;
 }
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 template <int BN>
 __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
-  using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * C::STAGES + 3];
+  __shared__ __align__(8) uint64_t bars[2 * kTcMaxStages + 5];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ float2 smx_w[4][16];
+  __shared__ int smx_i[4][16];
 
   const int M = p.m_total ? *p.m_total : p.m_host;
   if (M <= 0) return;
   const int passes = (M + BN - 1) / BN;
-  const int n_units = p.n_tiles * p.splits * passes;
-  if ((int)blockIdx.x >= n_units) return;
+  const long long my_begin = sk_begin(p.geo, blockIdx.x), my_end = sk_begin(p.geo, blockIdx.x + 1);
+  if (my_begin >= my_end) return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // ring depth from the activation rows actually loaded (16-row boxes)
+  const int nb_max = (min(BN, M) + 15) / 16;
+  const uint32_t stage_bytes = kTcABytes + (uint32_t)nb_max * kTcBBoxBytes;
+  int stages = (int)((p.smem_bytes - 1024u) / stage_bytes);
+  stages = stages > kTcMaxStages ? kTcMaxStages : stages;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sA = sbase, sB = sbase + C::STAGES * C::A_BYTES;
   const uint32_t bar0 = smem_u32(bars);
-  const uint32_t tfull = bar0 + 8u * (2 * C::STAGES), tempty = tfull + 8u, drain = tfull + 16u;
+  // two TMEM accumulators (columns [0, BN) and [BN, 2 BN)) alternate between fragments
+  const uint32_t tfull0 = bar0 + 8u * (2 * kTcMaxStages), tempty0 = tfull0 + 16u, drain = tfull0 + 32u;
+#define TFULL(a) (tfull0 + 8u * (uint32_t)(a))
+#define TEMPTY(a) (tempty0 + 8u * (uint32_t)(a))
 #define FULL(s) (bar0 + 8u * (uint32_t)(s))
-#define EMPTY(s) (bar0 + 8u * (uint32_t)(C::STAGES + (s)))
+#define EMPTY(s) (bar0 + 8u * (uint32_t)(kTcMaxStages + (s)))
+#define STAGE_A(s) (sbase + (uint32_t)(s) * stage_bytes)
+#define STAGE_B(s) (sbase + (uint32_t)(s) * stage_bytes + kTcABytes)
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < stages; ++s) {
       mbar_init(FULL(s), 1);
       mbar_init(EMPTY(s), 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 4);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(TFULL(a), 1);
+      mbar_init(TEMPTY(a), 4);
+    }
     mbar_init(drain, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_slot), BN);
+    tmem_alloc(smem_u32(&tmem_slot), 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -224,70 +251,81 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();  // weights stream through once
       const uint64_t pol_x = policy_evict_last();   // activations are re-read by every tile
-      uint32_t fill_parity[C::STAGES];
-      bool used[C::STAGES];
-      for (int s = 0; s < C::STAGES; ++s) used[s] = false;
+      uint32_t fill_parity[kTcMaxStages];
+      bool used[kTcMaxStages];
+      for (int s = 0; s < kTcMaxStages; ++s) used[s] = false;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u, passes);
-        const int m0 = w.pass * BN;
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+      FragIter it{my_begin, my_end, 0};
+      Frag f;
+      while (ok && next_frag(p, passes, it, f)) {
+        const int m0 = it.pass * BN;
+        const int nb = (min(BN, M - m0) + 15) / 16;  // 16-row boxes: 64-row boxes first, then the rest
+        const int n64 = nb / 4, n16 = nb - 4 * n64;
+        for (int kb = f.kb0; kb < f.kb1; ++kb) {
           if (!wait_bounded(EMPTY(stage), phase ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(FULL(stage), C::A_BYTES + C::B_BYTES);
-          tma_load_2d(sA + stage * C::A_BYTES, &p.a[w.seg], kb * 64, w.arow, FULL(stage), pol_w);
-          tma_load_2d(sB + stage * C::B_BYTES, &p.b, kb * 64, m0, FULL(stage), pol_x);
+          mbar_expect_tx(FULL(stage), kTcABytes + (uint32_t)nb * kTcBBoxBytes);
+          tma_load_2d(STAGE_A(stage), &p.a[f.seg], kb * 64, f.arow, FULL(stage), pol_w);
+          for (int j = 0; j < n64; ++j)
+            tma_load_2d(STAGE_B(stage) + (uint32_t)j * 4u * kTcBBoxBytes, &p.b64, kb * 64, m0 + 64 * j, FULL(stage),
+                        pol_x);
+          for (int j = 0; j < n16; ++j)
+            tma_load_2d(STAGE_B(stage) + (uint32_t)(4 * n64 + j) * kTcBBoxBytes, &p.b16, kb * 64,
+                        m0 + 64 * n64 + 16 * j, FULL(stage), pol_x);
           used[stage] = true;
           fill_parity[stage] = phase;
-          if (++stage == C::STAGES) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
       if (!ok)
-        for (int s = 0; s < C::STAGES; ++s)
+        for (int s = 0; s < stages; ++s)
           if (used[s]) wait_drain(FULL(s), fill_parity[s]);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, tphase = 0;
+      uint32_t phase = 0, nfrag = 0;
       bool ok = true, issued = false;
-      for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(p, u, passes);
-        const int mrows = min(BN, M - w.pass * BN);
+      FragIter it{my_begin, my_end, 0};
+      Frag f;
+      while (ok && next_frag(p, passes, it, f)) {
+        const int mrows = min(BN, M - it.pass * BN);
         const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
-        if (!wait_bounded(tempty, tphase ^ 1u, abort_v, p.status)) {
+        const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
+        const uint32_t dtm = tmem + acc * (uint32_t)BN;
+        if (!wait_bounded(TEMPTY(acc), (use & 1u) ^ 1u, abort_v, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        for (int kb = f.kb0; kb < f.kb1; ++kb) {
           if (!wait_bounded(FULL(stage), phase, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sw128_desc(sA + stage * C::A_BYTES);
-          const uint64_t bd = sw128_desc(sB + stage * C::B_BYTES);
+          const uint64_t ad = sw128_desc(STAGE_A(stage));
+          const uint64_t bd = sw128_desc(STAGE_B(stage));
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
-            tc_mma(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+            tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
           issued = true;
           tc_commit(EMPTY(stage));
-          if (++stage == C::STAGES) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        tc_commit(tfull);
-        tphase ^= 1u;
+        tc_commit(TFULL(acc));
+        ++nfrag;
       }
       if (!ok && issued) {
         tc_commit(drain);
@@ -296,19 +334,73 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    uint32_t tphase = 0;
-    for (int u = blockIdx.x; u < n_units; u += gridDim.x) {
-      const Unit w = decode_unit(p, u, passes);
-      const int m0 = w.pass * BN;
+    uint32_t nfrag = 0;
+    FragIter it{my_begin, my_end, 0};
+    Frag f;
+    while (next_frag(p, passes, it, f)) {
+      const int m0 = it.pass * BN;
       const int mrows = min(BN, M - m0);
-      if (!wait_bounded(tfull, tphase, abort_v, p.status)) break;
+      const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
+      const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q * 32) << 16);
+      if (!wait_bounded(TFULL(acc), use & 1u, abort_v, p.status)) break;
       tc_fence_after();
-      const int rin = w.arow + q * 32 + lane;  // row within the weight segment
-      const bool col_ok = rin < p.seg_rows[w.seg];
-      float *dst = p.ws + (size_t)w.split * (size_t)p.split_stride + (size_t)(p.seg_col0[w.seg] + rin);
+      const int rin = f.arow + q * 32 + lane;  // row within the weight segment
+      const bool col_ok = rin < p.seg_rows[f.seg];
+      const size_t col = (size_t)(p.seg_col0[f.seg] + rin);
+      if (p.epi_mode == 1) {
+        // softmax statistics of this tile's 128 vocabulary entries per token
+        for (int c = 0; c < mrows; c += 16) {
+          float v[16];
+          tmem_ld16(tacc + (uint32_t)c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float mx = col_ok ? v[j] : -INFINITY;
+            int ix = col_ok ? (int)col : 0x7fffffff;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+              const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
+              if (om > mx || (om == mx && oi < ix)) { mx = om; ix = oi; }
+            }
+            float e = col_ok ? expf(v[j] - mx) : 0.f;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
+            if (lane == j) {  // lane j keeps column c + j of this warp
+              smx_w[q][j] = make_float2(mx, e);
+              smx_i[q][j] = ix;
+            }
+          }
+          epi_bar();
+          if (warp == 2 && lane < 16 && c + lane < mrows) {  // merge the 4 lane quarters of column c + lane
+            float M4 = -INFINITY;
+            int I4 = 0x7fffffff;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float2 t = smx_w[w][lane];
+              if (t.x > M4 || (t.x == M4 && smx_i[w][lane] < I4)) { M4 = t.x; I4 = smx_i[w][lane]; }
+            }
+            float S4 = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float2 t = smx_w[w][lane];
+              if (t.x != -INFINITY) S4 += t.y * expf(t.x - M4);
+            }
+            const size_t o = (size_t)f.tile * p.ldm + (size_t)(m0 + c + lane);
+            p.smx[o] = make_float2(M4, S4);
+            p.smx_arg[o] = I4;
+          }
+          epi_bar();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(TEMPTY(acc));
+        ++nfrag;
+        continue;
+      }
+      float *dst = p.out + (size_t)f.slot * (size_t)p.geo.slot_stride + col;
       for (int c = 0; c < mrows; c += 16) {
         float v[16];
-        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+        tmem_ld16(tacc + (uint32_t)c, v);
         if (col_ok) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -317,16 +409,20 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);
-      tphase ^= 1u;
+      if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
+      ++nfrag;
     }
   }
 #undef FULL
 #undef EMPTY
+#undef TFULL
+#undef TEMPTY
+#undef STAGE_A
+#undef STAGE_B
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -363,40 +459,81 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int choose_splits(int n_tiles, int kblocks, int passes, int num_sms) {
-  // minimise (waves x k blocks per unit + per-unit epilogue cost), ties to fewer splits
-  double best = 1e30;
-  int best_s = 1;
-  for (int s = 1; s <= 16 && s <= kblocks; ++s) {
-    const long long units = (long long)n_tiles * s * passes;
-    const long long waves = (units + num_sms - 1) / num_sms;
-    const double cost = (double)waves * ((double)((kblocks + s - 1) / s) + 2.0);
-    if (cost < best - 1e-9) {
-      best = cost;
-      best_s = s;
-    }
-  }
-  return best_s;
-}
-
 template <int BN>
 static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)TcCfg<BN>::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  k_gemm_tc<BN><<<grid, 192, TcCfg<BN>::SMEM, s>>>(p);
+  k_gemm_tc<BN><<<grid, 192, kTcSmem, s>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_tc(const TcParams &p, int bn, int grid, cudaStream_t s) {
-  if (bn == 64) return launch_bn<64>(p, grid, s);
+cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
+  const int grid = p.geo.grid;
+  if (grid <= 0) return cudaSuccess;
+  p.smem_bytes = (uint32_t)kTcSmem;
   if (bn == 128) return launch_bn<128>(p, grid, s);
   if (bn == 256) return launch_bn<256>(p, grid, s);
   return cudaErrorInvalidValue;
+}
+
+int tc_max_slots(int n_tiles, int grid) { return (grid + n_tiles - 1) / n_tiles + 1; }
+
+namespace {
+__global__ void __launch_bounds__(512) k_lm_combine(const float2 *__restrict__ smx, const int32_t *__restrict__ arg,
+                                                    int n_tiles, int ldm, const int32_t *__restrict__ rowmap,
+                                                    const int32_t *__restrict__ m_total, float *__restrict__ conf,
+                                                    int32_t *__restrict__ amax) {
+  __shared__ float sm[32];
+  __shared__ int si[32];
+  __shared__ double sd[32];
+  const int M = *m_total;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    float mx = -INFINITY;
+    int ix = 0x7fffffff;
+    for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+      const float2 v = smx[(size_t)t * ldm + r];
+      const int i = arg[(size_t)t * ldm + r];
+      if (v.x > mx || (v.x == mx && i < ix)) { mx = v.x; ix = i; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
+      if (om > mx || (om == mx && oi < ix)) { mx = om; ix = oi; }
+    }
+    __syncthreads();
+    if (lane == 0) { sm[w] = mx; si[w] = ix; }
+    __syncthreads();
+    mx = -INFINITY;
+    ix = 0x7fffffff;
+    for (int i = 0; i < nw; ++i)
+      if (sm[i] > mx || (sm[i] == mx && si[i] < ix)) { mx = sm[i]; ix = si[i]; }
+    double sum = 0.0;
+    for (int t = threadIdx.x; t < n_tiles; t += blockDim.x) {
+      const float2 v = smx[(size_t)t * ldm + r];
+      if (v.x != -INFINITY) sum += (double)v.y * exp((double)v.x - (double)mx);
+    }
+    sum = block_sum(sum, sd);
+    if (threadIdx.x == 0) {
+      const int row = rowmap[r];
+      conf[row] = (float)(1.0 / sum);
+      amax[row] = ix;
+    }
+  }
+}
+}  // namespace
+
+cudaError_t launch_lm_combine(const float2 *smx, const int32_t *smx_arg, int n_tiles, int ldm,
+                              const int32_t *rowmap, const int32_t *m_total, int cap, float *conf, int32_t *amax,
+                              cudaStream_t s) {
+  const int grid = cap < 148 * 8 ? cap : 148 * 8;
+  k_lm_combine<<<grid > 0 ? grid : 1, 512, 0, s>>>(smx, smx_arg, n_tiles, ldm, rowmap, m_total, conf, amax);
+  return cudaGetLastError();
 }
 
 }  // namespace dcu

@@ -4,16 +4,10 @@
 // LM head.  One CTA per row (grid-stride), 16-byte vector accesses along the
 // row; HBM-bound.
 #include "common.cuh"
+#include "gemm_tc.h"
 #include "kernels.h"
 
 namespace dcu {
-
-// Split-K partials of a GEMM output element, summed in split order.
-__device__ __forceinline__ float csum(const float *c, size_t sstride, int splits, size_t j) {
-  float v = c[j];
-  for (int sp = 1; sp < splits; ++sp) v += c[sp * sstride + j];
-  return v;
-}
 
 static inline int row_grid(int rows_cap) {
   int g = rows_cap < 148 * 16 ? rows_cap : 148 * 16;
@@ -188,147 +182,196 @@ cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *
   return cudaGetLastError();
 }
 
+// 4 consecutive GEMM outputs (j % 4 == 0): the pieces of column j's 128-wide
+// tile summed in slot order (one piece when geo.grid == 0).
+__device__ __forceinline__ float4 csum4(const float *c, const SlotGeo &geo, size_t j) {
+  float4 v = *reinterpret_cast<const float4 *>(c + j);
+  const int ns = geo.grid <= 0 ? 1 : sk_nslots(geo, (int)(j >> 7));
+  for (int sp = 1; sp < ns; ++sp) {
+    const float4 w = *reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)geo.slot_stride + j);
+    v.x += w.x;
+    v.y += w.y;
+    v.z += w.z;
+    v.w += w.w;
+  }
+  return v;
+}
+
+template <class T>
+__device__ __forceinline__ void store4(T *p, float a, float b, float c, float d);
+template <>
+__device__ __forceinline__ void store4<float>(float *p, float a, float b, float c, float d) {
+  *reinterpret_cast<float4 *>(p) = make_float4(a, b, c, d);
+}
+template <>
+__device__ __forceinline__ void store4<bf16>(bf16 *p, float a, float b, float c, float d) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t *>(&lo);
+  u.y = *reinterpret_cast<uint32_t *>(&hi);
+  *reinterpret_cast<uint2 *>(p) = u;
+}
+
+static inline int flat_grid(long long items_cap) {
+  long long g = (items_cap + 255) / 256;
+  if (g > 148 * 16) g = 148 * 16;
+  return g > 0 ? (int)g : 1;
+}
+
 // ------------------------------------------------------------------ QKV epilogue
 // C row r = [q (H*hd) | k (Hkv*hd) | v (Hkv*hd)].  RoPE (rotate-half) on q and
 // k at the row's position; q -> Q[r]; k, v -> the layer's K/V cache at
-// (b, kv head, i).
+// (b, kv head, i).  Work items of 4 consecutive pairs (RoPE) or 4 consecutive
+// v values, flattened over all rows so every SM has loads in flight.
 template <class T>
-__global__ void k_epi_qkv(const float *__restrict__ C, int ldc, int splits, size_t sstride,
-                          const int32_t *__restrict__ rowmap,
-                          const int32_t *__restrict__ m_total, int N, int H, int Hkv, int hd,
-                          const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q, T *__restrict__ Kc,
-                          T *__restrict__ Vc) {
+__global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo geo,
+                          const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total, int N, int H,
+                          int Hkv, int hd, const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q,
+                          T *__restrict__ Kc, T *__restrict__ Vc) {
   const int M = *m_total;
   const int half = hd / 2;
-  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+  const int n_rope = (H + Hkv) * half / 4, n_v = Hkv * hd / 4;
+  const int per_row = n_rope + n_v;
+  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < (long long)M * per_row;
+       it += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(it / per_row), u = (int)(it - (long long)r * per_row);
     const int row = rowmap[r];
     const int b = row / N, i = row - b * N;
     const float *c = C + (size_t)r * ldc;
-    for (int t = threadIdx.x; t < (H + Hkv) * half; t += blockDim.x) {
+    if (u < n_rope) {
+      const int t = u * 4;
       const int head = t / half, j = t - head * half;
       const int base = head * hd;  // q heads first, then k heads (contiguous in C)
-      float a = csum(c, sstride, splits, base + j), bb = csum(c, sstride, splits, base + j + half);
+      const float4 a = csum4(c, geo, base + j), bb = csum4(c, geo, base + j + half);
+      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
       if (use_rope) {
-        float2 cs = rope_tab[(size_t)i * half + j];
-        float a2 = a * cs.x - bb * cs.y;
-        float b2 = bb * cs.x + a * cs.y;
-        a = a2;
-        bb = b2;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 cs = rope_tab[(size_t)i * half + j + e];
+          const float a2 = av[e] * cs.x - bv[e] * cs.y;
+          const float b2 = bv[e] * cs.x + av[e] * cs.y;
+          av[e] = a2;
+          bv[e] = b2;
+        }
       }
-      T *dst;
-      if (head < H) {
-        dst = Q + (size_t)r * H * hd + (size_t)head * hd;
-      } else {
-        const int kvh = head - H;
-        dst = Kc + (((size_t)b * Hkv + kvh) * N + i) * hd;
-      }
-      dst[j] = from_f<T>(a);
-      dst[j + half] = from_f<T>(bb);
-    }
-    const float *cv = c + (size_t)(H + Hkv) * hd;
-    for (int t = threadIdx.x; t < Hkv * hd; t += blockDim.x) {
+      T *dst = head < H ? Q + (size_t)r * H * hd + (size_t)head * hd
+                        : Kc + (((size_t)b * Hkv + (head - H)) * N + i) * hd;
+      store4<T>(dst + j, av[0], av[1], av[2], av[3]);
+      store4<T>(dst + j + half, bv[0], bv[1], bv[2], bv[3]);
+    } else {
+      const int t = (u - n_rope) * 4;
       const int kvh = t / hd, j = t - kvh * hd;
-      Vc[(((size_t)b * Hkv + kvh) * N + i) * hd + j] = from_f<T>(csum(cv, sstride, splits, t));
+      const float4 v = csum4(c, geo, (size_t)(H + Hkv) * hd + t);
+      store4<T>(Vc + (((size_t)b * Hkv + kvh) * N + i) * hd + j, v.x, v.y, v.z, v.w);
     }
   }
 }
 
-cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                            const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
                            int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s) {
+  const long long items = (long long)cap * ((H + Hkv) * (hd / 2) / 4 + Hkv * hd / 4);
   if (dtype == DCU_BF16)
-    k_epi_qkv<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
-                                                   (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc);
+    k_epi_qkv<bf16><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
+                                                      rope_tab, use_rope, (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc);
   else
-    k_epi_qkv<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, N, H, Hkv, hd, rope_tab, use_rope,
-                                                    (float *)Q, (float *)Kc, (float *)Vc);
+    k_epi_qkv<float><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
+                                                       rope_tab, use_rope, (float *)Q, (float *)Kc, (float *)Vc);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ O epilogue
-// hmid[r] = H_l[row] + C[r] (fp32); xs[r] = T(RMSNorm(hmid[r]) * g2).
+// hmid[r] = H_l[row] + C[r] (fp32); xs[r] = T(RMSNorm(hmid[r]) * g2).  One CTA
+// of 512 threads per row, 8 consecutive elements per thread per pass.
 template <class T>
-__global__ void k_epi_o(const float *__restrict__ C, int ldc, int splits, size_t sstride,
-                        const int32_t *__restrict__ rowmap,
-                        const int32_t *__restrict__ m_total, const T *__restrict__ Hl, const float *__restrict__ g2,
-                        float eps, int D, float *__restrict__ hmid, T *__restrict__ xs) {
+__global__ void __launch_bounds__(512)
+    k_epi_o(const float *__restrict__ C, int ldc, const SlotGeo geo, const int32_t *__restrict__ rowmap,
+            const int32_t *__restrict__ m_total, const T *__restrict__ Hl, const float *__restrict__ g2, float eps,
+            int D, float *__restrict__ hmid, T *__restrict__ xs) {
   __shared__ double red[32];
-  constexpr int VN = Vec<T>::n;
   const int M = *m_total;
   for (int r = blockIdx.x; r < M; r += gridDim.x) {
     const T *x = Hl + (size_t)rowmap[r] * D;
     const float *c = C + (size_t)r * ldc;
     float *hm = hmid + (size_t)r * D;
     double ss = 0;
-    for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
-      float v[VN];
-      load_vec(x + j, v);
-#pragma unroll
-      for (int i = 0; i < VN; ++i) {
-        v[i] += csum(c, sstride, splits, j + i);
-        hm[j + i] = v[i];
-        ss += (double)v[i] * (double)v[i];
+    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
+      float v[8];
+      if (Vec<T>::n == 8) {
+        load_vec(x + j, *reinterpret_cast<float(*)[Vec<T>::n]>(v));
+      } else {
+        load_vec(x + j, *reinterpret_cast<float(*)[Vec<T>::n]>(v));
+        load_vec(x + j + 4, *reinterpret_cast<float(*)[Vec<T>::n]>(v + 4));
       }
+      const float4 c0 = csum4(c, geo, j), c1 = csum4(c, geo, j + 4);
+      v[0] += c0.x; v[1] += c0.y; v[2] += c0.z; v[3] += c0.w;
+      v[4] += c1.x; v[5] += c1.y; v[6] += c1.z; v[7] += c1.w;
+      *reinterpret_cast<float4 *>(hm + j) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4 *>(hm + j + 4) = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss += (double)v[e] * (double)v[e];
     }
     ss = block_sum(ss, red);
     const float inv = (float)(1.0 / sqrt(ss / (double)D + (double)eps));
     T *o = xs + (size_t)r * D;
-    for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
-      float v[VN];
-#pragma unroll
-      for (int i = 0; i < VN; ++i) v[i] = hm[j + i] * inv * g2[j + i];
-      store_vec(o + j, v);
+    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
+      const float4 h0 = *reinterpret_cast<const float4 *>(hm + j), h1 = *reinterpret_cast<const float4 *>(hm + j + 4);
+      store4<T>(o + j, h0.x * inv * g2[j], h0.y * inv * g2[j + 1], h0.z * inv * g2[j + 2], h0.w * inv * g2[j + 3]);
+      store4<T>(o + j + 4, h1.x * inv * g2[j + 4], h1.y * inv * g2[j + 5], h1.z * inv * g2[j + 6],
+                h1.w * inv * g2[j + 7]);
     }
   }
 }
 
-cudaError_t launch_epi_o(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                          const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
                          float *hmid, void *xs, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_o<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, (const bf16 *)Hl, g2, eps, D, hmid,
-                                                 (bf16 *)xs);
+    k_epi_o<bf16><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, (const bf16 *)Hl, g2, eps, D,
+                                                hmid, (bf16 *)xs);
   else
-    k_epi_o<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, (const float *)Hl, g2, eps, D, hmid,
-                                                  (float *)xs);
+    k_epi_o<float><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, (const float *)Hl, g2, eps,
+                                                 D, hmid, (float *)xs);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ SwiGLU epilogue
-// C row r = [gate (F) | up (F)];  act[r] = T(silu(gate) * up).
+// C row r = [gate (F) | up (F)];  act[r] = T(silu(gate) * up), 4 values per work item.
 template <class T>
-__global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, int splits, size_t sstride,
-                             const int32_t *__restrict__ m_total, int F,
-                             T *__restrict__ act) {
+__global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, const SlotGeo geo,
+                             const int32_t *__restrict__ m_total, int F, T *__restrict__ act) {
   const int M = *m_total;
-  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+  const int per_row = F / 4;
+  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < (long long)M * per_row;
+       it += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(it / per_row), j = (int)(it - (long long)r * per_row) * 4;
     const float *c = C + (size_t)r * ldc;
-    for (int j = threadIdx.x; j < F; j += blockDim.x) {
-      const float gt = csum(c, sstride, splits, j), up = csum(c, sstride, splits, F + j);
-      act[(size_t)r * F + j] = from_f<T>(gt / (1.0f + expf(-gt)) * up);
-    }
+    const float4 gt = csum4(c, geo, j), up = csum4(c, geo, (size_t)F + j);
+    store4<T>(act + (size_t)r * F + j, gt.x / (1.0f + expf(-gt.x)) * up.x, gt.y / (1.0f + expf(-gt.y)) * up.y,
+              gt.z / (1.0f + expf(-gt.z)) * up.z, gt.w / (1.0f + expf(-gt.w)) * up.w);
   }
 }
 
-cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *m_total,
+cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *m_total,
                               int cap, int F, void *act, cudaStream_t s) {
+  const long long items = (long long)cap * (F / 4);
   if (dtype == DCU_BF16)
-    k_epi_swiglu<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, m_total, F, (bf16 *)act);
+    k_epi_swiglu<bf16><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, m_total, F, (bf16 *)act);
   else
-    k_epi_swiglu<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, m_total, F, (float *)act);
+    k_epi_swiglu<float><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, m_total, F, (float *)act);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ down epilogue + scatter
 // new = T(hmid[r] + C[r]); if d_next: d_next[row] = distance(new, H_{l+1}[row])
 // ([DLLM] "关键设计 1", computed against the cached row before it is
-// overwritten); H_{l+1}[row] = new.
+// overwritten); H_{l+1}[row] = new.  512 threads per row, 8 elements each.
 template <class T>
-__global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, int splits, size_t sstride,
-                                   const int32_t *__restrict__ rowmap,
-                                   const int32_t *__restrict__ m_total, const float *__restrict__ hmid,
-                                   T *__restrict__ Hn, const float *__restrict__ g_next, float *__restrict__ d_next,
-                                   int D) {
+__global__ void __launch_bounds__(512)
+    k_epi_down_scatter(const float *__restrict__ C, int ldc, const SlotGeo geo,
+                       const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
+                       const float *__restrict__ hmid, T *__restrict__ Hn, const float *__restrict__ g_next,
+                       float *__restrict__ d_next, int D) {
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
   const int M = *m_total;
@@ -339,27 +382,31 @@ __global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, int spl
     T *dst = Hn + (size_t)row * D;
     double dot = 0, nx = 0, ny = 0;
     bool same = true;
-    for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
-      float v[VN];
-#pragma unroll
-      for (int i = 0; i < VN; ++i) v[i] = hm[j + i] + csum(c, sstride, splits, j + i);
+    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
+      const float4 c0 = csum4(c, geo, j), c1 = csum4(c, geo, j + 4);
+      const float4 h0 = *reinterpret_cast<const float4 *>(hm + j), h1 = *reinterpret_cast<const float4 *>(hm + j + 4);
+      float v[8] = {h0.x + c0.x, h0.y + c0.y, h0.z + c0.z, h0.w + c0.w,
+                    h1.x + c1.x, h1.y + c1.y, h1.z + c1.z, h1.w + c1.w};
       if (d_next) {
-        float ov[VN];
-        uint32_t ob[VN];
-        load_vec(dst + j, ov, ob);
+        float ov[8];
+        uint32_t ob[8];
 #pragma unroll
-        for (int i = 0; i < VN; ++i) {
-          T nt = from_f<T>(v[i]);
-          float nv = to_f(nt);
-          same = same && (bits_of<T>(nt) == ob[i]);
-          double gg = (double)g_next[j + i];
-          double a = gg * (double)nv, b = gg * (double)ov[i];
+        for (int q = 0; q < 8; q += VN)
+          load_vec(dst + j + q, *reinterpret_cast<float(*)[VN]>(ov + q), *reinterpret_cast<uint32_t(*)[VN]>(ob + q));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const T nt = from_f<T>(v[e]);
+          const float nv = to_f(nt);
+          same = same && (bits_of<T>(nt) == ob[e]);
+          const double gg = (double)g_next[j + e];
+          const double a = gg * (double)nv, b = gg * (double)ov[e];
           dot += a * b;
           nx += a * a;
           ny += b * b;
         }
       }
-      store_vec(dst + j, v);
+#pragma unroll
+      for (int q = 0; q < 8; q += VN) store_vec(dst + j + q, *reinterpret_cast<float(*)[VN]>(v + q));
     }
     if (d_next) {
       same = __syncthreads_and(same);
@@ -371,15 +418,15 @@ __global__ void k_epi_down_scatter(const float *__restrict__ C, int ldc, int spl
   }
 }
 
-cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, int splits, size_t sstride,
+cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const SlotGeo geo,
                                     const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
                                     void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_down_scatter<bf16><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, hmid, (bf16 *)Hnext, g_next,
-                                                            d_next, D);
+    k_epi_down_scatter<bf16><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, hmid,
+                                                            (bf16 *)Hnext, g_next, d_next, D);
   else
-    k_epi_down_scatter<float><<<row_grid(cap), 256, 0, s>>>(C, ldc, splits, sstride, rowmap, m_total, hmid, (float *)Hnext, g_next,
-                                                             d_next, D);
+    k_epi_down_scatter<float><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, hmid,
+                                                             (float *)Hnext, g_next, d_next, D);
   return cudaGetLastError();
 }
 

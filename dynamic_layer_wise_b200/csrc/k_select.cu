@@ -19,50 +19,68 @@ static constexpr int kMaxSeq = 16384;
 // sums to B_layer * L; uniform when asked or when the row sums to 0.  If the
 // floors overshoot (q rounded up to an integer), one is taken back from the
 // layers with the smallest fractional parts (ties -> higher layer) above 0.
-__global__ void k_budget_split(const float *__restrict__ s_prev, int B, int L, int B_layer, int uniform,
-                               int32_t *__restrict__ budgets) {
-  const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b >= B) return;
+// One CTA per sequence, one thread per layer; the sum of s is taken in layer
+// order by one thread so it matches a sequential fp64 sum bit for bit.
+__global__ void k_budget_split(const float *__restrict__ s_prev, int L, int B_layer, int uniform_arg,
+                               const int32_t *__restrict__ uniform_flag, int32_t *__restrict__ budgets) {
+  const int uniform = uniform_arg || (uniform_flag && *uniform_flag);
+  extern __shared__ double sh[];  // [L] fractional parts, then [L] floors
+  double *frac = sh, *flr = sh + L;
+  __shared__ double s_total;
+  __shared__ long long s_sumfl;
+  const int b = blockIdx.x;
   const float *s = s_prev + (size_t)b * L;
   int32_t *out = budgets + (size_t)b * L;
-  double total = 0.0;
-  for (int l = 0; l < L; ++l) total = __dadd_rn(total, (double)s[l]);
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int l = 0; l < L; ++l) t = __dadd_rn(t, (double)s[l]);
+    s_total = t;
+  }
+  __syncthreads();
+  const double total = s_total;
   if (uniform || total == 0.0) {
-    for (int l = 0; l < L; ++l) out[l] = B_layer;
+    for (int l = threadIdx.x; l < L; l += blockDim.x) out[l] = B_layer;
     return;
   }
   const double T = (double)B_layer * (double)L;
-  long long sum_fl = 0;
-  for (int l = 0; l < L; ++l) {
-    double q = __ddiv_rn(__dmul_rn(T, (double)s[l]), total);
-    long long f = (long long)floor(q);
-    out[l] = (int32_t)f;
-    sum_fl += f;
+  for (int l = threadIdx.x; l < L; l += blockDim.x) {
+    const double q = __ddiv_rn(__dmul_rn(T, (double)s[l]), total);
+    const double f = floor(q);
+    flr[l] = f;
+    frac[l] = q - f;  // exact (Sterbenz)
   }
-  long long R = (long long)B_layer * L - sum_fl;
-  if (R == 0) return;
-  // ranks are computed against the untouched floors, then applied
-  for (int l = 0; l < L; ++l) {
-    double ql = __ddiv_rn(__dmul_rn(T, (double)s[l]), total);
-    double fl = floor(ql), frl = ql - fl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long t = 0;
+    for (int l = 0; l < L; ++l) t += (long long)flr[l];
+    s_sumfl = t;
+  }
+  __syncthreads();
+  const long long R = (long long)B_layer * L - s_sumfl;
+  for (int l = threadIdx.x; l < L; l += blockDim.x) {
+    const double frl = frac[l], fl = flr[l];
     int rank = 0;
     for (int k = 0; k < L; ++k) {
-      double qk = __ddiv_rn(__dmul_rn(T, (double)s[k]), total);
-      double fk = floor(qk), frk = qk - fk;
+      const double frk = frac[k];
       if (R > 0) {
         if (frk > frl || (frk == frl && k < l)) ++rank;
-      } else {
-        if (fk > 0.0 && (frk < frl || (frk == frl && k > l))) ++rank;
+      } else if (R < 0) {
+        if (flr[k] > 0.0 && (frk < frl || (frk == frl && k > l))) ++rank;
       }
     }
-    if (R > 0 && rank < R) out[l] = (int32_t)fl + 1;
-    if (R < 0 && fl > 0.0 && rank < -R) out[l] = (int32_t)fl - 1;
+    int v = (int)fl;
+    if (R > 0 && rank < R) v += 1;
+    if (R < 0 && fl > 0.0 && rank < -R) v -= 1;
+    out[l] = v;
   }
 }
 
-cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform, int32_t *budgets,
-                                cudaStream_t s) {
-  k_budget_split<<<(B + 63) / 64, 64, 0, s>>>(s_prev, B, L, B_layer, uniform, budgets);
+cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform,
+                                const int32_t *uniform_flag, int32_t *budgets, cudaStream_t s) {
+  if (B <= 0 || L <= 0) return cudaSuccess;
+  const int threads = L < 256 ? ((L + 31) / 32) * 32 : 256;
+  k_budget_split<<<B, threads, (size_t)2 * L * sizeof(double), s>>>(s_prev, L, B_layer, uniform, uniform_flag,
+                                                                      budgets);
   return cudaGetLastError();
 }
 
@@ -77,7 +95,7 @@ __global__ void __launch_bounds__(kSelThreads)
              const int32_t *__restrict__ budgets, int budget_stride, int B, int N, int Bw, int mode,
              int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
              float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
-             int32_t *__restrict__ done, int32_t *__restrict__ status) {
+             int32_t *__restrict__ done, int32_t *__restrict__ seq_off, int32_t *__restrict__ status) {
   extern __shared__ uint8_t smem[];
   uint32_t *sd = reinterpret_cast<uint32_t *>(smem);     // [N] d bits
   uint8_t *flag = smem + (size_t)N * sizeof(uint32_t);   // [N] 0 none, 1 window, 2 top-B
@@ -146,14 +164,32 @@ __global__ void __launch_bounds__(kSelThreads)
         if (flag[i] == 0 && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
       }
       __syncthreads();
-      if (tid == 0) {
-        int cum = 0, bin = 0;
-        for (bin = 255; bin >= 0; --bin) {
-          if (cum + hist[bin] >= rem) break;
-          cum += hist[bin];
+      if (tid < 32) {
+        // warp 0: lane j owns bins 255-8j .. 248-8j (descending); find the bin where
+        // the count of candidates from the top reaches rem
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          cnt[e] = hist[255 - 8 * tid - e];
+          tot += cnt[e];
         }
-        s_bin = bin;
-        s_rem = rem - cum;
+        int incl = tot;  // inclusive prefix over lanes (higher bins first)
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += y;
+        }
+        const int excl = incl - tot;
+        const unsigned hit = __ballot_sync(0xffffffffu, excl < rem && incl >= rem);
+        if (hit && tid == __ffs(hit) - 1) {
+          int cum = excl, e = 0;
+          for (; e < 8; ++e) {
+            if (cum + cnt[e] >= rem) break;
+            cum += cnt[e];
+          }
+          s_bin = 255 - 8 * tid - e;
+          s_rem = rem - cum;
+        }
       }
       __syncthreads();
       prefix |= (uint32_t)s_bin << shift;
@@ -209,9 +245,11 @@ __global__ void __launch_bounds__(kSelThreads)
     const int c = *((volatile int32_t *)count + bb);
     const volatile int32_t *src = idx + (size_t)bb * N;
     for (int j = tid; j < c; j += nthr) rowmap[off + j] = bb * N + src[j];
+    if (tid == 0 && seq_off) seq_off[bb] = off;
     off += c;
   }
   if (tid == 0) {
+    if (seq_off) seq_off[B] = off;
     *m_total = off;
     *done = 0;
   }
@@ -220,7 +258,7 @@ __global__ void __launch_bounds__(kSelThreads)
 cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
                           int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
                           float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
-                          int32_t *done, int32_t *status, cudaStream_t s) {
+                          int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s) {
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   size_t smem = (size_t)N * 5;
   static bool attr_set = false;
@@ -230,21 +268,23 @@ cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nk
     attr_set = true;
   }
   k_select<<<B, kSelThreads, smem, s>>>(d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
-                                        s_stride, d_next_zero, rowmap, m_total, done, status);
+                                        s_stride, d_next_zero, rowmap, m_total, done, seq_off, status);
   return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ row plans
-__global__ void k_plan_all(int BN, int32_t *rowmap, int32_t *m_total) {
+__global__ void k_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off) {
+  const int BN = B * N;
   for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < BN; r += gridDim.x * blockDim.x) rowmap[r] = r;
+  if (blockIdx.x == 0 && threadIdx.x <= B) seq_off[threadIdx.x] = threadIdx.x * N;
   if (blockIdx.x == 0 && threadIdx.x == 0) *m_total = BN;
 }
 
-cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, cudaStream_t s) {
+cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off, cudaStream_t s) {
   const int BN = B * N;
   int grid = (BN + 255) / 256;
   if (grid > 1024) grid = 1024;
-  k_plan_all<<<grid, 256, 0, s>>>(BN, rowmap, m_total);
+  k_plan_all<<<grid, 256, 0, s>>>(B, N, rowmap, m_total, seq_off);
   return cudaGetLastError();
 }
 

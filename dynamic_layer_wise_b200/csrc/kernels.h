@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gemm_tc.h"
+
 namespace dcu {
 
 // Sets the text dcu_last_error(NULL) returns (calls that have no context).
@@ -24,32 +26,34 @@ cudaError_t launch_cosine_distance(int dtype, const void *x, const void *y, cons
                                    float *d, cudaStream_t s);
 cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *m_total, int cap, const void *H,
                                const float *g, float eps, int D, void *xs, cudaStream_t s);
-// C: GEMM output as `splits` partials [splits][cap][ldc] (sstride elements apart), summed in split order.
-cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+// C: GEMM output as slots [slot][cap][ldc] under the slot geometry `geo` (geo.grid == 0: one slot).
+cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                            const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
                            int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s);
-cudaError_t launch_epi_o(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *rowmap,
+cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                          const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
                          float *hmid, void *xs, cudaStream_t s);
-cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, int splits, size_t sstride, const int32_t *m_total,
+cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *m_total,
                               int cap, int F, void *act, cudaStream_t s);
-cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, int splits, size_t sstride,
+cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const SlotGeo geo,
                                     const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
                                     void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s);
 cudaError_t launch_softmax_max(const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
                                int V, float *conf, int32_t *amax, cudaStream_t s);
 
 // ---- selection, budgets and commit (k_select.cu)
-cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform, int32_t *budgets,
-                                cudaStream_t s);
+// uniform split when `uniform` != 0 or *uniform_flag != 0 (uniform_flag may be null)
+cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, int uniform,
+                                const int32_t *uniform_flag, int32_t *budgets, cudaStream_t s);
 // budgets: pointer to element [0] of the layer's column; budget_stride = L.
 // s_out: pointer to the layer's column of s [B][L]; s_stride = L.
 // rowmap / m_total / done may be null (stateless use).
 cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
                           int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
                           float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
-                          int32_t *done, int32_t *status, cudaStream_t s);
-cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, cudaStream_t s);
+                          int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s);
+// rowmap = identity over B * N rows; seq_off[b] = b * N (B <= 255)
+cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off, cudaStream_t s);
 cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
                                cudaStream_t s);
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
@@ -58,6 +62,15 @@ cudaError_t launch_commit_rule(int rule, float param, const float *conf, const i
 // ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total (m < m_cap when m_total is null)
 cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,
                              const GemmSeg *segs, int nseg, int K, float *C, int ldc, cudaStream_t s);
+
+// ---- tensor-core attention (k_attn_mma.cu), bf16, head_dim 64 or 128.  Rows of
+// sequence b are packed rows [seq_off[b], seq_off[b + 1]).  part_o / part_ml hold
+// `splits` partial results ([splits][rows * H][hd] / [splits][rows * H]); counters
+// ([B][Hkv][qt_cap], zero) are reset by the kernel after use.
+size_t attn_mma_smem(int hd);
+cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
+                                 const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
+                                 int32_t *counters, int splits, int qt_grid, int qt_cap, cudaStream_t s);
 
 // ---- attention (k_attn.cu): out[r][h] = softmax(q K^T / sqrt(hd)) V over all N keys of row r's sequence
 cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,

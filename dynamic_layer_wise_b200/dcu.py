@@ -73,6 +73,7 @@ _SIGS = {
     "dcu_profile_read": (_i32, [_vp, _i32, ctypes.POINTER(_f64), ctypes.POINTER(_i64), _i32]),
     "dcu_kernel_class_name": (ctypes.c_char_p, [_i32]),
     "dcu_launch_count": (_i64, [_vp]),
+    "dcu_set_graphs": (_i32, [_vp, _i32]),
     "dcu_linear": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]),
     "dcu_lm_confidence_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
 }
@@ -304,3 +305,7 @@ def dcu_linear(X, W, stream=None):
     Y = torch.empty((M, Nout), dtype=torch.float32, device=X.device)
     _check(lib().dcu_linear(_ptr(X), _ptr(W), M, K, Nout, dt, _ptr(Y), _stream(stream)))
     return Y
+
+
+def dcu_set_graphs(ctx: Context, on: bool):
+    _check(lib().dcu_set_graphs(ctx.handle, int(bool(on))), ctx.handle)

@@ -165,6 +165,25 @@ def weight_values(shape: ModelShape, seed: int, name: str, layer: int | None = N
     return np.stack(out) if out else np.zeros((0, n_cols), dtype=np.uint16 if shape.dtype == "bf16" else np.float32)
 
 
+def weight_rows(shape: ModelShape, seed: int, name: str, row0: int, row1: int, layer: int | None = None,
+                threads: int = 8) -> np.ndarray:
+    """Rows [row0, row1) of a weight tensor in its storage dtype (generated in
+    parallel chunks)."""
+    from concurrent.futures import ThreadPoolExecutor
+    if name in ("embed", "lm_head"):
+        tid = TID_EMBED if name == "embed" else TID_LM_HEAD
+        n_cols = shape.d_model
+    else:
+        tid = layer_tid(layer, name)
+        n_cols = shape.weight_shapes()[name][1]
+    step = max(1, (row1 - row0 + threads - 1) // threads)
+    parts = [(r, min(row1, r + step)) for r in range(row0, row1, step)]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        out = list(ex.map(lambda ab: normal_values(seed, tid, ab[0] * n_cols, (ab[1] - ab[0]) * n_cols,
+                                                    shape.init_std, shape.dtype), parts))
+    return np.concatenate(out).reshape(row1 - row0, n_cols) if out else np.zeros((0, n_cols))
+
+
 def as_f64(values: np.ndarray, dtype: str) -> np.ndarray:
     """Exact conversion of stored values (bf16 bits or float32) to float64."""
     if dtype == "bf16":

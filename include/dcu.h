@@ -139,6 +139,12 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
 int commit_select(dcu_ctx *ctx, int32_t rule, float param, uint8_t *masked, int32_t *token_ids,
                   int32_t *out_positions, int32_t *out_count, dcu_stream_t stream);
 
+/* dcu_step and commit_select are captured into CUDA graphs (once per distinct
+ * set of pointers, budgets and active shape; at most 16 kept, least recently
+ * used evicted) and replayed on the caller's stream.  on = 0 launches every
+ * kernel directly instead.  Default: on. */
+int dcu_set_graphs(dcu_ctx *ctx, int32_t on);
+
 /* Synchronises the stream, returns DCU_EDEVICE if the device status word is
  * non-zero (its bits in *bits when bits is not NULL) and clears it. */
 int dcu_status(dcu_ctx *ctx, dcu_stream_t stream, int32_t *bits);
@@ -245,7 +251,10 @@ int dcu_set_tensor(dcu_ctx *ctx, int32_t kind, int32_t layer, const void *src, i
  * between resets) or off (0). */
 int dcu_profile_enable(dcu_ctx *ctx, int32_t max_launches);
 /* Synchronises and returns the summed event time (ms) and launch count of a
- * kernel class since the last reset; reset != 0 clears the class afterwards. */
+ * kernel class since the last reset; reset != 0 clears the class afterwards.
+ * Launches inside a graph are timed by event-record nodes of the graph's most
+ * recent replay, counted once per replay; the replay counts are cleared when
+ * the last class (DCU_K_COUNT - 1) is read with reset. */
 int dcu_profile_read(dcu_ctx *ctx, int32_t kernel_class, double *total_ms, int64_t *launches, int32_t reset);
 const char *dcu_kernel_class_name(int32_t kernel_class);
 /* Number of kernels the context has launched since it was created. */

@@ -33,6 +33,19 @@ class LazyRows:
         return out
 
 
+class LazyMatrix:
+    """Row-slice access to a seeded [rows][cols] weight matrix, generated on
+    demand (for the LM head of the 8B shapes)."""
+
+    def __init__(self, shape, seed, name, rows):
+        self.spec, self.seed, self.name = shape, seed, name
+        self.shape = (rows, shape.d_model)
+
+    def __getitem__(self, sl):
+        r0, r1, _ = sl.indices(self.shape[0])
+        return I.as_f64(I.weight_rows(self.spec, self.seed, self.name, r0, r1), self.spec.dtype)
+
+
 def oracle_weights(shape: I.ModelShape, seed: int, lazy_vocab: bool = False, layers=None) -> O.Weights:
     dt = shape.dtype
 

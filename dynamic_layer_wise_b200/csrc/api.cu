@@ -74,7 +74,7 @@ struct dcu_ctx {
   // scratch
   char *xs = nullptr, *Q = nullptr, *attn = nullptr, *act = nullptr;
   float *hmid = nullptr, *C = nullptr, *conf = nullptr;
-  int32_t *seq_off = nullptr, *attn_ctr = nullptr;
+  int32_t *seq_off = nullptr;
   float *attn_po = nullptr;
   float2 *attn_ml = nullptr;
   int attn_qt_cap = 1;
@@ -91,10 +91,37 @@ struct dcu_ctx {
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
   CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of 16 and 64 rows
+  // per-tile piece counts of each stream-K geometry used so far (device tables)
+  struct SlotTable {
+    int n_tiles, kblocks, grid, tile_aligned;
+    int32_t *dev;
+  };
+  std::vector<SlotTable> slot_tables;
+  const int32_t *slot_table(const SlotGeo &g) {
+    for (auto &t : slot_tables)
+      if (t.n_tiles == g.n_tiles && t.kblocks == g.kblocks && t.grid == g.grid && t.tile_aligned == g.tile_aligned)
+        return t.dev;
+    std::vector<int32_t> h(g.n_tiles);
+    for (int i = 0; i < g.n_tiles; ++i) h[i] = sk_nslots(g, i);
+    int32_t *d = nullptr;
+    if (cudaMalloc(&d, h.size() * 4) != cudaSuccess) return nullptr;
+    if (cudaMemcpy(d, h.data(), h.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaFree(d);
+      return nullptr;
+    }
+    allocs.push_back(d);
+    slot_tables.push_back({g.n_tiles, g.kblocks, g.grid, g.tile_aligned, d});
+    return d;
+  }
   // CUDA graphs of dcu_step / commit_select
   bool use_graphs = true;
   bool capturing = false;
   cudaStream_t cap_stream = nullptr;
+  // side stream of the weight L2 prefetches (forked from and joined back into
+  // the step's stream; inside a capture the fork / join become graph edges)
+  cudaStream_t pf_stream = nullptr;
+  cudaEvent_t pf_fork = nullptr, pf_join = nullptr;
+  bool pf_pending = false;
   std::vector<GraphEntry> graphs;
   GraphEntry *cur_graph = nullptr;
   uint64_t use_clock = 0;
@@ -198,6 +225,11 @@ void free_all(dcu_ctx *c) {
   c->graphs.clear();
   if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   c->cap_stream = nullptr;
+  if (c->pf_stream) cudaStreamDestroy(c->pf_stream);
+  c->pf_stream = nullptr;
+  if (c->pf_fork) cudaEventDestroy(c->pf_fork);
+  if (c->pf_join) cudaEventDestroy(c->pf_join);
+  c->pf_fork = c->pf_join = nullptr;
   for (void *p : c->allocs) cudaFree(p);
   c->allocs.clear();
   for (auto &pc : c->prof)
@@ -241,6 +273,43 @@ struct ActOperand {
   const CUtensorMap *map16, *map64;
 };
 
+// tcgen05 GEMM parameters of C[m][n] = sum_k X[m][k] W[n][k] over the
+// concatenated weight segments (stream-K over all SMs unless tile_aligned).
+int gemm_params(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
+                const CUtensorMap *const *amaps, int nseg, int ldc, bool tile_aligned, TcParams *tp) {
+  const int cap = (int)c->cap;
+  memset(tp, 0, sizeof(*tp));
+  int tile = 0, col = 0;
+  for (int i = 0; i < nseg; ++i) {
+    tp->a[i] = *amaps[i];
+    tp->seg_tile0[i] = tile;
+    tp->seg_col0[i] = col;
+    tp->seg_rows[i] = segs[i].rows;
+    tile += (segs[i].rows + 127) / 128;
+    col += segs[i].rows;
+  }
+  tp->seg_tile0[nseg] = tile;
+  tp->nseg = nseg;
+  tp->b16 = *x.map16;
+  tp->b64 = *x.map64;
+  tp->ldc = ldc;
+  tp->m_total = m_total;
+  tp->out = c->C;
+  tp->status = c->status();
+  SlotGeo g;
+  g.n_tiles = tile;
+  g.kblocks = x.K / 64;
+  g.tile_aligned = tile_aligned ? 1 : 0;
+  const long long T = (long long)tile * g.kblocks;
+  g.grid = tile_aligned ? (tile < c->num_sms ? tile : c->num_sms) : (int)(T < c->num_sms ? T : c->num_sms);
+  g.slot_stride = (long long)cap * ldc;
+  if ((size_t)tc_max_slots(tile, g.grid) * cap * ldc > c->ws_elems)
+    return fail(c, DCU_ECUDA, "GEMM workspace too small for the stream-K slots");
+  g.nslots = c->slot_table(g);
+  tp->geo = g;
+  return DCU_OK;
+}
+
 // C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
 // stream-K slots described by *geo (geo->grid == 0: a single slot).
 int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
@@ -254,46 +323,65 @@ int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const Gemm
     return DCU_OK;
   }
   TcParams tp;
-  memset(&tp, 0, sizeof(tp));
-  int tile = 0, col = 0;
-  for (int i = 0; i < nseg; ++i) {
-    tp.a[i] = *amaps[i];
-    tp.seg_tile0[i] = tile;
-    tp.seg_col0[i] = col;
-    tp.seg_rows[i] = segs[i].rows;
-    tile += (segs[i].rows + 127) / 128;
-    col += segs[i].rows;
-  }
-  tp.seg_tile0[nseg] = tile;
-  tp.nseg = nseg;
-  tp.b16 = *x.map16;
-  tp.b64 = *x.map64;
-  tp.ldc = ldc;
-  tp.m_total = m_total;
-  tp.out = c->C;
-  tp.status = c->status();
-  SlotGeo g;
-  g.n_tiles = tile;
-  g.kblocks = x.K / 64;
-  g.tile_aligned = tile_aligned ? 1 : 0;
-  const long long T = (long long)tile * g.kblocks;
-  g.grid = tile_aligned ? (tile < c->num_sms ? tile : c->num_sms) : (int)(T < c->num_sms ? T : c->num_sms);
-  g.slot_stride = (long long)cap * ldc;
-  if ((size_t)tc_max_slots(tile, g.grid) * cap * ldc > c->ws_elems)
-    return fail(c, DCU_ECUDA, "GEMM workspace too small for the stream-K slots");
-  tp.geo = g;
-  *geo = g;
+  if (int rc = gemm_params(c, x, m_total, segs, amaps, nseg, ldc, tile_aligned, &tp)) return rc;
+  *geo = tp.geo;
   LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
+  return DCU_OK;
+}
+
+// Forks onto the prefetch stream an L2 prefetch of the first `frac` of every
+// CTA range of a later GEMM over these weight segments (K columns): the
+// weights are read-only, so the prefetch overlaps whatever the step's stream
+// runs until that GEMM starts.  Joined back at the end of the step.
+int prefetch_gemm(dcu_ctx *c, const ActOperand &x, const GemmSeg *segs, const CUtensorMap *const *amaps, int nseg,
+                  int ldc, double frac, cudaStream_t s) {
+  if (c->cfg.dtype != DCU_BF16 || frac <= 0.0 || !amaps[0] || !c->pf_stream) return DCU_OK;
+  TcParams tp;
+  if (int rc = gemm_params(c, x, c->m_total(), segs, amaps, nseg, ldc, false, &tp)) return rc;
+  const double per_cta = (double)tp.geo.n_tiles * tp.geo.kblocks / tp.geo.grid;
+  const int kb = (int)(frac * per_cta + 0.999);
+  CK(c, cudaEventRecord(c->pf_fork, s));
+  CK(c, cudaStreamWaitEvent(c->pf_stream, c->pf_fork, 0));
+  LAUNCH(c, launch_prefetch_w(tp, kb, c->pf_stream));
+  c->pf_pending = true;
+  return DCU_OK;
+}
+
+// Joins the prefetch stream back into s (required before a capture ends).
+int prefetch_join(dcu_ctx *c, cudaStream_t s) {
+  if (!c->pf_pending) return DCU_OK;
+  CK(c, cudaEventRecord(c->pf_join, c->pf_stream));
+  CK(c, cudaStreamWaitEvent(s, c->pf_join, 0));
+  c->pf_pending = false;
   return DCU_OK;
 }
 
 // One layer of recompute over the packed rows in ctx->rowmap / m_total.
 // dense: the rows are every position (full forward): no selection, no d.
+// Fractions of each GEMM's per-CTA weight range prefetched into L2 ahead of
+// it (the window before it: scatter + select + gather for QKV, RoPE +
+// attention for O, the O and SwiGLU epilogues for gate|up and down).
+constexpr double kPrefetchQKV = 0.5, kPrefetchO = 1.0, kPrefetchGateUp = 0.25, kPrefetchDown = 0.35;
+
+int prefetch_qkv(dcu_ctx *c, int l, cudaStream_t s) {
+  if (c->lmaps.empty()) return DCU_OK;
+  const dcu_cfg &g = c->cfg;
+  const LayerMaps &lm = c->lmaps[l];
+  const ActOperand xs{c->xs, g.d_model, g.d_model, &c->xs_map[0], &c->xs_map[1]};
+  GemmSeg seg[3] = {{c->wq[l], g.n_heads * g.head_dim}, {c->wk[l], g.n_kv_heads * g.head_dim},
+                    {c->wv[l], g.n_kv_heads * g.head_dim}};
+  const CUtensorMap *am[3] = {&lm.wq, &lm.wk, &lm.wv};
+  return prefetch_gemm(c, xs, seg, am, 3, (g.n_heads + 2 * g.n_kv_heads) * g.head_dim, kPrefetchQKV, s);
+}
+
 int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t *nkeys, int Bw, cudaStream_t s) {
   const dcu_cfg &g = c->cfg;
   const int L = g.n_layers, D = g.d_model, H = g.n_heads, Hkv = g.n_kv_heads, hd = g.head_dim, F = g.d_ffn;
   const int dt = g.dtype, cap = (int)c->cap;
   const bool last = (l + 1 == L);
+  // grid size of the row kernels: the expected recompute-set size (their loops
+  // stride over the device row count, so any count is covered)
+  const int gcap = dense ? cap : std::min(cap, std::max(1, c->gemm_rows_hint));
   if (!dense) {
     Prof p(c, DCU_K_SELECT, s);
     LAUNCH(c, launch_select(c->dl(l), keys, nkeys, c->budgets + l, L, c->B, c->N, Bw, g.window_mode,
@@ -303,7 +391,7 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   }
   {
     Prof p(c, DCU_K_GATHER, s);
-    LAUNCH(c, launch_gather_norm(dt, c->rowmap, c->m_total(), cap, c->Hl(l), c->g1[l], g.rms_eps, D, c->xs, s));
+    LAUNCH(c, launch_gather_norm(dt, c->rowmap, c->m_total(), gcap, c->Hl(l), c->g1[l], g.rms_eps, D, c->xs, s));
   }
   const LayerMaps *lm = c->lmaps.empty() ? nullptr : &c->lmaps[l];
   const ActOperand xs{c->xs, D, D, &c->xs_map[0], &c->xs_map[1]};
@@ -316,9 +404,14 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
     if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo)) return rc;
   }
+  if (!dense) {  // the O projection's weights stream into L2 during RoPE / attention
+    GemmSeg seg[1] = {{c->wo[l], D}};
+    const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
+    if (int rc = prefetch_gemm(c, at, seg, am, 1, D, kPrefetchO, s)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), cap, c->N, H, Hkv,
+    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), gcap, c->N, H, Hkv,
                              hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
   }
   {
@@ -337,9 +430,10 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
       const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
       splits = (c->N + kc - 1) / kc;
       LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l), c->attn,
-                                     c->attn_po, c->attn_ml, c->attn_ctr, splits, qt_grid, c->attn_qt_cap, s));
+                                     c->attn_po, c->attn_ml, splits, qt_grid, gcap, s));
+      if (splits > 1) ++c->launches;  // the merge kernel
     } else {
-      LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), cap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
+      LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), gcap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
                                  c->attn, s));
     }
   }
@@ -348,9 +442,14 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
     if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
   }
+  if (!dense) {
+    GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
+    const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
+    if (int rc = prefetch_gemm(c, xs, seg, am, 2, 2 * F, kPrefetchGateUp, s)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), cap, c->Hl(l), c->g2[l],
+    LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->Hl(l), c->g2[l],
                            g.rms_eps, D, c->hmid, c->xs, s));
   }
   {
@@ -358,19 +457,27 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
     if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo)) return rc;
   }
+  if (!dense) {
+    GemmSeg seg[1] = {{c->wd[l], D}};
+    const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
+    if (int rc = prefetch_gemm(c, ac, seg, am, 1, D, kPrefetchDown, s)) return rc;
+  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), cap, F, c->act, s));
+    LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), gcap, F, c->act, s));
   }
   {
     GemmSeg seg[1] = {{c->wd[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
     if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
   }
+  if (!dense && !last) {  // the next layer's QKV weights, during scatter / select / gather
+    if (int rc = prefetch_qkv(c, l + 1, s)) return rc;
+  }
   {
     Prof p(c, DCU_K_SCATTER, s);
     const bool want_d = !dense && !last;
-    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, geo, c->rowmap, c->m_total(), cap, c->hmid,
+    LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->hmid,
                                       c->Hl(l + 1), want_d ? c->g1[l + 1] : nullptr,
                                       want_d ? c->dl(l + 1) : nullptr, D, s));
   }
@@ -493,7 +600,6 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     c->attn_qt_cap = (int)(((size_t)cfg->max_seq * G + 127) / 128);
     AL(c->attn_po, (size_t)kAttnMaxSplits * cap * Hhd * 4);
     AL(c->attn_ml, (size_t)kAttnMaxSplits * cap * cfg->n_heads * sizeof(float2));
-    AL(c->attn_ctr, (size_t)cfg->max_batch * cfg->n_kv_heads * c->attn_qt_cap * 4);
   }
 #undef AL
   if (e != cudaSuccess) {
@@ -504,9 +610,10 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     return fail(nullptr, DCU_ENOMEM, m);
   }
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->pf_stream, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->pf_fork, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->pf_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
-  if (e == cudaSuccess && c->attn_ctr)
-    e = cudaMemset(c->attn_ctr, 0, (size_t)cfg->max_batch * cfg->n_kv_heads * c->attn_qt_cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
   if (e == cudaSuccess && cfg->rope_theta > 0.0f)
@@ -540,6 +647,24 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
       free_all(c);
       delete c;
       return fail(nullptr, DCU_ECUDA, "cuTensorMapEncodeTiled failed (driver entry point missing or bad layout)");
+    }
+    // piece-count tables of the four layer GEMMs' stream-K geometries (built
+    // here so that no allocation happens while a step is captured)
+    const size_t widths[4] = {nqkv, D, 2 * F, D};
+    const size_t ks[4] = {D, Hhd, D, F};
+    for (int i = 0; i < 4; ++i) {
+      SlotGeo g;
+      g.n_tiles = (int)((widths[i] + 127) / 128);
+      g.kblocks = (int)(ks[i] / 64);
+      g.tile_aligned = 0;
+      const long long T = (long long)g.n_tiles * g.kblocks;
+      g.grid = (int)(T < c->num_sms ? T : c->num_sms);
+      g.slot_stride = 0;
+      if (!c->slot_table(g)) {
+        free_all(c);
+        delete c;
+        return fail(nullptr, DCU_ENOMEM, "slot table allocation failed");
+      }
     }
   }
   if (e != cudaSuccess) {
@@ -604,6 +729,7 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
     c->gemm_rows_hint = (int)(est < BN ? est : BN);
     c->gemm_bn = c->gemm_rows_hint <= 128 ? 128 : 256;
   }
+  if (int rc = prefetch_qkv(c, 0, s)) return rc;  // layer 0's QKV weights, during budget / refresh / select
   {
     Prof p(c, DCU_K_BUDGET, s);
     LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, 0, c->uniform_flag(), c->budgets, s));
@@ -614,7 +740,11 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
                                    c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
   }
   for (int l = 0; l < L; ++l)
-    if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) return rc;
+    if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) {
+      prefetch_join(c, s);  // a capture must not end with the side stream forked
+      return rc;
+    }
+  if (int rc = prefetch_join(c, s)) return rc;
   CK(c, cudaMemcpyAsync(c->s_prev, c->s_cur, (size_t)c->B * L * 4, cudaMemcpyDeviceToDevice, s));
   CK(c, cudaMemsetAsync(c->uniform_flag(), 0, 4, s));
   return DCU_OK;

@@ -130,6 +130,42 @@ __device__ __forceinline__ float finish_cosine_distance(double dot, double nx, d
   return (float)d;
 }
 
+// Lets the next kernel of the stream, when launched with programmatic stream
+// serialization, start its independent prologue now.
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Programmatic dependent launch: waits until the previous kernel of the stream
+// has completed and its writes are visible (a no-op without a programmatic edge).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// First statement of every kernel launched by launch_pdl: wait for the
+// predecessor, then let the successor be scheduled (so at most one kernel of
+// the stream waits ahead of the running one).
+__device__ __forceinline__ void pdl_enter() {
+  griddep_wait();
+  allow_dependents();
+}
+
+// Launch with programmatic stream serialization: the kernel's CTAs may be
+// scheduled while its predecessor finishes, hiding the launch latency; the
+// kernel must call pdl_enter() (or griddep_wait()) before touching anything
+// the predecessor reads or writes.
+template <class... Exp, class... Act>
+inline cudaError_t launch_pdl(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Act &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Act &&>(args)...);
+}
+
 // Row r of the packed recompute set -> global row b*N + i (written by the
 // select / plan kernels).
 struct RowPlan {

@@ -6,7 +6,9 @@
 
 namespace dcu {
 
-constexpr int kTcMaxStages = 12;             // deepest smem ring
+constexpr int kTcMaxA = 16;                 // deepest weight-tile ring
+constexpr int kTcMaxB = 4;                  // deepest activation-tile ring
+constexpr int kTcThreads = 224;             // 7 warps: W producer, MMA, 4 epilogue, X producer
 constexpr uint32_t kTcABytes = 128u * 128u;  // weight tile: 128 rows x 64 bf16
 constexpr uint32_t kTcBBoxBytes = 16u * 128u;  // activation box: 16 rows x 64 bf16
 constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (one CTA per SM)
@@ -19,7 +21,8 @@ constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (o
 // order and the result does not depend on CTA scheduling.
 struct SlotGeo {
   int n_tiles, kblocks, grid, tile_aligned;
-  long long slot_stride;  // elements between two slots (cap * ldc)
+  long long slot_stride;        // elements between two slots (cap * ldc)
+  const int32_t *nslots = nullptr;  // device table [n_tiles] of sk_nslots (consumers), or null
 };
 
 __host__ __device__ inline long long sk_begin(const SlotGeo &g, int c) {
@@ -74,6 +77,9 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
                       uint32_t box_inner, uint32_t box_outer);
 // bn: token rows per pass (128 or 256); the grid is p.geo.grid CTAs.
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s);
+// L2 prefetch of the first kb_count k blocks of every CTA's range of the GEMM
+// described by p (weights only; see k_prefetch_w).
+cudaError_t launch_prefetch_w(const TcParams &p, int kb_count, cudaStream_t s);
 // Most pieces a tile can be cut into under the stream-K split over `grid` CTAs.
 int tc_max_slots(int n_tiles, int grid);
 // Merges the per-tile softmax statistics of the LM head (epi_mode 1): for packed

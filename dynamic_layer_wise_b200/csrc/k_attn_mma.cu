@@ -5,11 +5,12 @@
 // a (packed row, query head) pair of the kv head's GQA group, so the CTA reads
 // its K/V chunk from HBM once for every query of the group.  8 warps x 16
 // queries; K/V are staged in shared memory in 64-key sub-chunks with cp.async
-// (double buffer, zero-filled past N); S = Q K^T and O += P V run on
+// (a ring of 4, three sub-chunks in flight ahead of the one in use,
+// zero-filled past N); S = Q K^T and O += P V run on
 // mma.sync m16n8k16 bf16 (fp32 accumulate) with an online softmax in
 // registers.  With several key splits, each CTA writes (O, max, sum) partials
-// and the last CTA of the tile (atomic counter, reset after use) merges them
-// in split order, so the result does not depend on CTA scheduling.
+// and k_attn_merge combines them in split order (one thread per query head and
+// 4 output dims), so the result does not depend on CTA scheduling.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,6 +19,7 @@ namespace {
 
 constexpr int QT = 128;  // queries per CTA
 constexpr int KS = 64;   // keys per sub-chunk
+constexpr int NST = 4;   // K/V sub-chunk buffers: NST - 1 loads in flight ahead of the one in use
 
 __device__ __forceinline__ uint32_t smem_u32a(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -63,19 +65,18 @@ struct AttnArgs {
   const int32_t *seq_off;   // [B + 1] packed-row offsets of the sequences
   float *part_o;            // [splits][cap * H][hd] partial outputs
   float2 *part_ml;          // [splits][cap * H] (max, sum) in log2 units
-  int32_t *counters;        // [B][Hkv][qt_cap] arrival counters (zero between launches)
-  int B, N, H, Hkv, splits, kc, qt_grid, qt_cap;
+  int B, N, H, Hkv, splits, kc, qt_grid;
   float scale_log2;         // log2(e) / sqrt(hd)
 };
 
 template <int HD>
-__device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int *s_last, int b, int kvh, int ks, int qt,
-                                          int row0, int nq) {
+__device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b, int kvh, int ks, int qt, int row0,
+                                          int nq) {
   constexpr int LD = HD + 8;  // padded row (elements): 16-byte shift per row, conflict-free ldmatrix
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
   bf16 *Qs = reinterpret_cast<bf16 *>(sm);  // [QT][LD]
-  bf16 *Ks = Qs + QT * LD;                   // [2][KS][LD]
-  bf16 *Vs = Ks + 2 * KS * LD;               // [2][KS][LD]
+  bf16 *Ks = Qs + QT * LD;                   // [NST][KS][LD]
+  bf16 *Vs = Ks + NST * KS * LD;             // [NST][KS][LD]
   const int G = a.H / a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -102,8 +103,14 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int *s
       cp_async16(smem_u32a(Vs + (buf * KS + ki) * LD + ch * 8), Vb + off, ok);
     }
   };
-  load_kv(0, k_begin);
-  cp_async_commit();
+  const int n_sub = (k_end - k_begin + KS - 1) / KS;
+  // prologue: sub-chunks 0 .. NST-2 (one commit group each, empty past the end,
+  // so group g always holds sub-chunk g; the Q tile rides in group 0)
+#pragma unroll
+  for (int st = 0; st < NST - 1; ++st) {
+    if (st < n_sub) load_kv(st, k_begin + st * KS);
+    cp_async_commit();
+  }
 
   float o[HD / 8][4];
 #pragma unroll
@@ -112,12 +119,12 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int *s
   uint32_t qf[HD / 16][4];
   const bool warp_active = (qt * QT + warp * 16) < nq;
 
-  const int n_sub = (k_end - k_begin + KS - 1) / KS;
   for (int sc = 0; sc < n_sub; ++sc) {
-    const int buf = sc & 1;
-    if (sc + 1 < n_sub) load_kv(buf ^ 1, k_begin + (sc + 1) * KS);
+    const int buf = sc % NST;
+    const int nxt = sc + NST - 1;  // refills the buffer consumed in iteration sc - 1
+    if (nxt < n_sub) load_kv(nxt % NST, k_begin + nxt * KS);
     cp_async_commit();
-    cp_async_wait<1>();
+    cp_async_wait<NST - 1>();  // group sc (sub-chunk sc) has landed
     __syncthreads();
     if (sc == 0 && warp_active) {
 #pragma unroll
@@ -249,48 +256,13 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int *s
       if (t == 0) a.part_ml[(size_t)ks * plane + qidx] = make_float2(m_run[h2], l_run[h2]);
     }
   }
-  __threadfence();
-  __syncthreads();
-  int32_t *ctr = a.counters + ((size_t)b * a.Hkv + kvh) * a.qt_cap + qt;
-  if (tid == 0) *s_last = (atomicAdd(ctr, 1) == a.splits - 1);
-  __syncthreads();
-  if (!*s_last) return;
-  __threadfence();
-  // merge the splits of this tile's queries in split order
-  const int nq_tile = min(QT, nq - qt * QT);
-  for (int c = tid; c < nq_tile * (HD / 4); c += blockDim.x) {
-    const int qi = c / (HD / 4), d4 = (c - qi * (HD / 4)) * 4;
-    const int q = qt * QT + qi;
-    const int r = row0 + q / G, h = kvh * G + q % G;
-    const size_t qidx = (size_t)r * a.H + h;
-    float M = -INFINITY;
-    for (int sp = 0; sp < a.splits; ++sp) M = fmaxf(M, __ldcg(a.part_ml + sp * plane + qidx).x);
-    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int sp = 0; sp < a.splits; ++sp) {
-      const float2 ml = __ldcg(a.part_ml + sp * plane + qidx);
-      if (ml.x == -INFINITY) continue;
-      const float w = exp2f(ml.x - M);
-      L += ml.y * w;
-      const float4 v = __ldcg(reinterpret_cast<const float4 *>(a.part_o + (sp * plane + qidx) * HD + d4));
-      acc[0] += v.x * w;
-      acc[1] += v.y * w;
-      acc[2] += v.z * w;
-      acc[3] += v.w * w;
-    }
-    const float inv = 1.f / L;
-    bf16 *dst = a.out + qidx * HD + d4;
-    *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-    *reinterpret_cast<__nv_bfloat162 *>(dst + 2) = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-  }
-  __syncthreads();
-  if (tid == 0) *ctr = 0;
 }
 
 // grid = B x Hkv x splits x qt_grid; the CTA walks query tiles qt, qt + qt_grid, ...
 template <int HD>
 __global__ void __launch_bounds__(256, 1) k_attn_mma(const AttnArgs a) {
+  pdl_enter();
   extern __shared__ __align__(16) uint8_t sm[];
-  __shared__ int s_last;
   int item = blockIdx.x;
   const int per_b = a.Hkv * a.splits * a.qt_grid;
   const int b = item / per_b;
@@ -302,19 +274,63 @@ __global__ void __launch_bounds__(256, 1) k_attn_mma(const AttnArgs a) {
   const int row0 = a.seq_off[b], nq = (a.seq_off[b + 1] - row0) * (a.H / a.Hkv);
   if (ks * a.kc >= a.N) return;
   for (int qt = qt0; qt * QT < nq; qt += a.qt_grid) {
-    attn_tile<HD>(a, sm, &s_last, b, kvh, ks, qt, row0, nq);
+    attn_tile<HD>(a, sm, b, kvh, ks, qt, row0, nq);
     __syncthreads();
+  }
+}
+
+// out[q][d..d+3] = sum_s exp2(m_s - M) O_s / sum_s exp2(m_s - M) l_s over the
+// key splits s, for every packed (row, head) pair q.
+template <int HD>
+__global__ void k_attn_merge(const float *__restrict__ part_o, const float2 *__restrict__ part_ml,
+                             const int32_t *__restrict__ seq_off, int B, int H, int splits, bf16 *__restrict__ out) {
+  pdl_enter();
+  const size_t plane = (size_t)seq_off[B] * H;
+  const long long items = (long long)plane * (HD / 4);
+  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < items;
+       it += (long long)gridDim.x * blockDim.x) {
+    const size_t q = (size_t)(it / (HD / 4));
+    const int d4 = (int)(it - (long long)q * (HD / 4)) * 4;
+    float2 ml[8];
+    float4 ov[8];
+#pragma unroll
+    for (int sp = 0; sp < 8; ++sp) {
+      if (sp < splits) {
+        ml[sp] = __ldcg(part_ml + sp * plane + q);
+        ov[sp] = __ldcg(reinterpret_cast<const float4 *>(part_o + (sp * plane + q) * HD + d4));
+      }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < 8; ++sp)
+      if (sp < splits) M = fmaxf(M, ml[sp].x);
+    float L = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int sp = 0; sp < 8; ++sp) {
+      if (sp < splits && ml[sp].x != -INFINITY) {
+        const float w = exp2f(ml[sp].x - M);
+        L += ml[sp].y * w;
+        acc[0] += ov[sp].x * w;
+        acc[1] += ov[sp].y * w;
+        acc[2] += ov[sp].z * w;
+        acc[3] += ov[sp].w * w;
+      }
+    }
+    const float inv = 1.f / L;
+    bf16 *dst = out + q * HD + d4;
+    *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+    *reinterpret_cast<__nv_bfloat162 *>(dst + 2) = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
   }
 }
 
 }  // namespace
 
-size_t attn_mma_smem(int hd) { return (size_t)(QT + 4 * KS) * (hd + 8) * sizeof(bf16); }
+size_t attn_mma_smem(int hd) { return (size_t)(QT + 2 * NST * KS) * (hd + 8) * sizeof(bf16); }
 
 cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
                                  const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
-                                 int32_t *counters, int splits, int qt_grid, int qt_cap, cudaStream_t s) {
-  if (hd != 64 && hd != 128) return cudaErrorInvalidValue;
+                                 int splits, int qt_grid, int cap_rows, cudaStream_t s) {
+  if ((hd != 64 && hd != 128) || splits < 1 || splits > 8) return cudaErrorInvalidValue;
   AttnArgs a;
   a.Q = (const bf16 *)Q;
   a.Kc = (const bf16 *)Kc;
@@ -323,7 +339,6 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
   a.seq_off = seq_off;
   a.part_o = part_o;
   a.part_ml = part_ml;
-  a.counters = counters;
   a.B = B;
   a.N = N;
   a.H = H;
@@ -331,7 +346,6 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
   a.splits = splits;
   a.kc = ((N + splits - 1) / splits + KS - 1) / KS * KS;
   a.qt_grid = qt_grid;
-  a.qt_cap = qt_cap;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
   const size_t smem = attn_mma_smem(hd);
   const int grid = B * Hkv * splits * qt_grid;
@@ -343,7 +357,7 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
       if (e != cudaSuccess) return e;
       attr = true;
     }
-    k_attn_mma<128><<<grid, 256, smem, s>>>(a);
+    launch_pdl(k_attn_mma<128>, grid, 256, smem, s, a);
   } else {
     static bool attr = false;
     if (!attr) {
@@ -351,8 +365,17 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
       if (e != cudaSuccess) return e;
       attr = true;
     }
-    k_attn_mma<64><<<grid, 256, smem, s>>>(a);
+    launch_pdl(k_attn_mma<64>, grid, 256, smem, s, a);
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  const long long items = (long long)cap_rows * H * (hd / 4);
+  long long mg = (items + 255) / 256;
+  const int mgrid = (int)(mg < 148 * 8 ? mg : 148 * 8);
+  if (hd == 128)
+    launch_pdl(k_attn_merge<128>, mgrid, 256, 0, s, part_o, part_ml, seq_off, B, H, splits, (bf16 *)out);
+  else
+    launch_pdl(k_attn_merge<64>, mgrid, 256, 0, s, part_o, part_ml, seq_off, B, H, splits, (bf16 *)out);
   return cudaGetLastError();
 }
 

@@ -7,10 +7,14 @@
 // set of ~65 rows still drives full 128-row tensor-core instructions while
 // every weight byte is read from HBM once.  Accumulators live in TMEM.
 //
-// Warp roles (192 threads, one CTA per SM, persistent over work units):
-//   warp 0      TMA producer (one lane): STAGES-deep ring of (W tile, X tile)
+// Warp roles (224 threads, one CTA per SM, persistent over work units):
+//   warp 0      weight producer (one lane): deep ring of 16 KB W tiles; it
+//               starts before the previous launch has finished (weights are
+//               never written by a kernel)
+//   warp 6      activation producer (one lane): shallow ring of X tiles (from
+//               L2), after the programmatic-dependency wait
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma (K=16)
-//               per 64-wide k block, tcgen05.commit frees the smem stage
+//               per 64-wide k block, tcgen05.commit frees both smem stages
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 tile, coalesced
 //               stores of the split-K partial (32 lanes = 32 consecutive n)
 // A work unit is (weight tile, k split, token pass); the row count M is read
@@ -192,15 +196,41 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+
+// Position in this CTA's (fragment, k block) sequence.
+struct KCursor {
+  FragIter it;
+  Frag f;
+  int kb, m0, nb;
+  bool valid;
+  __device__ __forceinline__ void load_frag(int BN, int M) {
+    kb = f.kb0;
+    m0 = it.pass * BN;
+    nb = (min(BN, M - m0) + 15) / 16;
+  }
+  __device__ __forceinline__ void start(const TcParams &p, int passes, long long b, long long e, int BN, int M) {
+    it = FragIter{b, e, 0};
+    valid = next_frag(p, passes, it, f);
+    if (valid) load_frag(BN, M);
+  }
+  __device__ __forceinline__ void advance(const TcParams &p, int passes, int BN, int M) {
+    if (++kb < f.kb1) return;
+    valid = next_frag(p, passes, it, f);
+    if (valid) load_frag(BN, M);
+  }
+};
+
 template <int BN>
-__global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * kTcMaxStages + 5];
+  __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ float2 smx_w[4][16];
   __shared__ int smx_i[4][16];
 
+  // The row count is written by the select / plan kernel two launches before
+  // this one, so it is final even while the previous launch still runs.
   const int M = p.m_total ? *p.m_total : p.m_host;
   if (M <= 0) return;
   const int passes = (M + BN - 1) / BN;
@@ -208,26 +238,38 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
   if (my_begin >= my_end) return;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // ring depth from the activation rows actually loaded (16-row boxes)
+  // Two rings: weight tiles (16 KB, from HBM) and activation tiles (16-row
+  // boxes of the rows actually loaded, from L2).  The activation ring only has
+  // to cover the L2 latency, so most of shared memory holds weight tiles in
+  // flight.
   const int nb_max = (min(BN, M) + 15) / 16;
-  const uint32_t stage_bytes = kTcABytes + (uint32_t)nb_max * kTcBBoxBytes;
-  int stages = (int)((p.smem_bytes - 1024u) / stage_bytes);
-  stages = stages > kTcMaxStages ? kTcMaxStages : stages;
+  const uint32_t b_stage = (uint32_t)nb_max * kTcBBoxBytes;
+  const int SB = nb_max >= 12 ? 3 : 4;
+  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage) / kTcABytes);
+  SA = SA > kTcMaxA ? kTcMaxA : SA;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t bbase = sbase + (uint32_t)SA * kTcABytes;
   const uint32_t bar0 = smem_u32(bars);
   // two TMEM accumulators (columns [0, BN) and [BN, 2 BN)) alternate between fragments
-  const uint32_t tfull0 = bar0 + 8u * (2 * kTcMaxStages), tempty0 = tfull0 + 16u, drain = tfull0 + 32u;
+#define FULL_A(s) (bar0 + 8u * (uint32_t)(s))
+#define EMPTY_A(s) (bar0 + 8u * (uint32_t)(kTcMaxA + (s)))
+#define FULL_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + (s)))
+#define EMPTY_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + kTcMaxB + (s)))
+  const uint32_t tfull0 = bar0 + 8u * (uint32_t)(2 * kTcMaxA + 2 * kTcMaxB), tempty0 = tfull0 + 16u,
+                 drain = tfull0 + 32u;
 #define TFULL(a) (tfull0 + 8u * (uint32_t)(a))
 #define TEMPTY(a) (tempty0 + 8u * (uint32_t)(a))
-#define FULL(s) (bar0 + 8u * (uint32_t)(s))
-#define EMPTY(s) (bar0 + 8u * (uint32_t)(kTcMaxStages + (s)))
-#define STAGE_A(s) (sbase + (uint32_t)(s) * stage_bytes)
-#define STAGE_B(s) (sbase + (uint32_t)(s) * stage_bytes + kTcABytes)
+#define STAGE_A(s) (sbase + (uint32_t)(s) * kTcABytes)
+#define STAGE_B(s) (bbase + (uint32_t)(s) * b_stage)
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(FULL(s), 1);
-      mbar_init(EMPTY(s), 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(FULL_A(s), 1);
+      mbar_init(EMPTY_A(s), 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(FULL_B(s), 1);
+      mbar_init(EMPTY_B(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(TFULL(a), 1);
@@ -248,50 +290,80 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
   volatile int *abort_v = &abort_flag;
 
   if (warp == 0) {
+    // weight producer: the weights are never written by a kernel, so the ring
+    // fills before (and while) the previous launch finishes
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();  // weights stream through once
-      const uint64_t pol_x = policy_evict_last();   // activations are re-read by every tile
-      uint32_t fill_parity[kTcMaxStages];
-      bool used[kTcMaxStages];
-      for (int s = 0; s < kTcMaxStages; ++s) used[s] = false;
+      uint32_t fill_parity[kTcMaxA];
+      bool used[kTcMaxA];
+      for (int s = 0; s < kTcMaxA; ++s) used[s] = false;
+      KCursor ca;
+      ca.start(p, passes, my_begin, my_end, BN, M);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      FragIter it{my_begin, my_end, 0};
-      Frag f;
-      while (ok && next_frag(p, passes, it, f)) {
-        const int m0 = it.pass * BN;
-        const int nb = (min(BN, M - m0) + 15) / 16;  // 16-row boxes: 64-row boxes first, then the rest
-        const int n64 = nb / 4, n16 = nb - 4 * n64;
-        for (int kb = f.kb0; kb < f.kb1; ++kb) {
-          if (!wait_bounded(EMPTY(stage), phase ^ 1u, abort_v, p.status)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(FULL(stage), kTcABytes + (uint32_t)nb * kTcBBoxBytes);
-          tma_load_2d(STAGE_A(stage), &p.a[f.seg], kb * 64, f.arow, FULL(stage), pol_w);
-          for (int j = 0; j < n64; ++j)
-            tma_load_2d(STAGE_B(stage) + (uint32_t)j * 4u * kTcBBoxBytes, &p.b64, kb * 64, m0 + 64 * j, FULL(stage),
-                        pol_x);
-          for (int j = 0; j < n16; ++j)
-            tma_load_2d(STAGE_B(stage) + (uint32_t)(4 * n64 + j) * kTcBBoxBytes, &p.b16, kb * 64,
-                        m0 + 64 * n64 + 16 * j, FULL(stage), pol_x);
-          used[stage] = true;
-          fill_parity[stage] = phase;
-          if (++stage == stages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+      while (ca.valid) {
+        if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(FULL_A(stage), kTcABytes);
+        tma_load_2d(STAGE_A(stage), &p.a[ca.f.seg], ca.kb * 64, ca.f.arow, FULL_A(stage), pol_w);
+        used[stage] = true;
+        fill_parity[stage] = phase;
+        ca.advance(p, passes, BN, M);
+        if (++stage == SA) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
       if (!ok)
-        for (int s = 0; s < stages; ++s)
-          if (used[s]) wait_drain(FULL(s), fill_parity[s]);
+        for (int s = 0; s < SA; ++s)
+          if (used[s]) wait_drain(FULL_A(s), fill_parity[s]);
+    }
+  } else if (warp == 6) {
+    // activation producer: the packed rows are written by the previous launch
+    if (lane == 0) {
+      griddep_wait();
+      allow_dependents();  // the next kernel may be scheduled (it waits for this grid)
+      const uint64_t pol_x = policy_evict_last();  // activations are re-read by every tile
+      uint32_t fill_parity[kTcMaxB];
+      bool used[kTcMaxB];
+      for (int s = 0; s < kTcMaxB; ++s) used[s] = false;
+      KCursor cb;
+      cb.start(p, passes, my_begin, my_end, BN, M);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      while (cb.valid) {
+        if (!wait_bounded(EMPTY_B(stage), phase ^ 1u, abort_v, p.status)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(FULL_B(stage), (uint32_t)cb.nb * kTcBBoxBytes);
+        const int n64 = cb.nb / 4, n16 = cb.nb - 4 * n64;
+        for (int j = 0; j < n64; ++j)
+          tma_load_2d(STAGE_B(stage) + (uint32_t)j * 4u * kTcBBoxBytes, &p.b64, cb.kb * 64, cb.m0 + 64 * j,
+                      FULL_B(stage), pol_x);
+        for (int j = 0; j < n16; ++j)
+          tma_load_2d(STAGE_B(stage) + (uint32_t)(4 * n64 + j) * kTcBBoxBytes, &p.b16, cb.kb * 64,
+                      cb.m0 + 64 * n64 + 16 * j, FULL_B(stage), pol_x);
+        used[stage] = true;
+        fill_parity[stage] = phase;
+        cb.advance(p, passes, BN, M);
+        if (++stage == SB) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok)
+        for (int s = 0; s < SB; ++s)
+          if (used[s]) wait_drain(FULL_B(s), fill_parity[s]);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0, nfrag = 0;
+      int sa = 0, sb = 0;
+      uint32_t pa = 0, pb = 0, nfrag = 0;
       bool ok = true, issued = false;
       FragIter it{my_begin, my_end, 0};
       Frag f;
@@ -306,21 +378,26 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
         }
         tc_fence_after();
         for (int kb = f.kb0; kb < f.kb1; ++kb) {
-          if (!wait_bounded(FULL(stage), phase, abort_v, p.status)) {
+          if (!wait_bounded(FULL_A(sa), pa, abort_v, p.status) || !wait_bounded(FULL_B(sb), pb, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sw128_desc(STAGE_A(stage));
-          const uint64_t bd = sw128_desc(STAGE_B(stage));
+          const uint64_t ad = sw128_desc(STAGE_A(sa));
+          const uint64_t bd = sw128_desc(STAGE_B(sb));
 #pragma unroll
           for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
             tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
           issued = true;
-          tc_commit(EMPTY(stage));
-          if (++stage == stages) {
-            stage = 0;
-            phase ^= 1u;
+          tc_commit(EMPTY_A(sa));  // both stages are free once these MMAs have read them
+          tc_commit(EMPTY_B(sb));
+          if (++sa == SA) {
+            sa = 0;
+            pa ^= 1u;
+          }
+          if (++sb == SB) {
+            sb = 0;
+            pb ^= 1u;
           }
         }
         if (!ok) break;
@@ -332,7 +409,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
         wait_drain(drain, 0);
       }
     }
-  } else {
+  } else if (warp >= 2 && warp <= 5) {
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     uint32_t nfrag = 0;
     FragIter it{my_begin, my_end, 0};
@@ -413,8 +490,10 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
       ++nfrag;
     }
   }
-#undef FULL
-#undef EMPTY
+#undef FULL_A
+#undef EMPTY_A
+#undef FULL_B
+#undef EMPTY_B
 #undef TFULL
 #undef TEMPTY
 #undef STAGE_A
@@ -424,6 +503,25 @@ __global__ void __launch_bounds__(192, 1) k_gemm_tc(const __grid_constant__ TcPa
     tc_fence_after();
     tmem_dealloc(tmem, 2 * BN);
   }
+}
+
+// L2 prefetch of the weight tiles a later launch of k_gemm_tc with the same
+// parameters will read first: CTA c issues, in order, the first `kb_count` k
+// blocks of GEMM CTA c's stream-K range (first token pass) as bulk tensor
+// prefetches.  It only moves weights (never written by a kernel) into L2, so it
+// may run on a side stream concurrently with anything.
+__global__ void __launch_bounds__(32) k_prefetch_w(const __grid_constant__ TcParams p, int kb_count) {
+  if (threadIdx.x != 0) return;
+  const long long b = sk_begin(p.geo, blockIdx.x), e0 = sk_begin(p.geo, blockIdx.x + 1);
+  const long long e = (b + kb_count < e0) ? b + kb_count : e0;
+  FragIter it{b, e, 0};
+  Frag f;
+  while (next_frag(p, 1, it, f))
+    for (int kb = f.kb0; kb < f.kb1; ++kb)
+      asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                       reinterpret_cast<uint64_t>(&p.a[f.seg])),
+                   "r"(kb * 64), "r"(f.arow)
+                   : "memory");
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -461,14 +559,25 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
 
 template <int BN>
 static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
+  static bool attr_set = false;
+  if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
     if (e != cudaSuccess) return e;
-    attr = true;
+    attr_set = true;
   }
-  k_gemm_tc<BN><<<grid, 192, kTcSmem, s>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the CTAs may start while the previous kernel
+  // finishes; they wait (griddepcontrol.wait) before reading its outputs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = kTcSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN>, p);
 }
 
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
@@ -480,6 +589,12 @@ cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
   return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_prefetch_w(const TcParams &p, int kb_count, cudaStream_t s) {
+  if (p.geo.grid <= 0 || kb_count <= 0) return cudaSuccess;
+  k_prefetch_w<<<p.geo.grid, 32, 0, s>>>(p, kb_count);
+  return cudaGetLastError();
+}
+
 int tc_max_slots(int n_tiles, int grid) { return (grid + n_tiles - 1) / n_tiles + 1; }
 
 namespace {
@@ -487,6 +602,7 @@ __global__ void __launch_bounds__(512) k_lm_combine(const float2 *__restrict__ s
                                                     int n_tiles, int ldm, const int32_t *__restrict__ rowmap,
                                                     const int32_t *__restrict__ m_total, float *__restrict__ conf,
                                                     int32_t *__restrict__ amax) {
+  pdl_enter();
   __shared__ float sm[32];
   __shared__ int si[32];
   __shared__ double sd[32];
@@ -532,7 +648,7 @@ cudaError_t launch_lm_combine(const float2 *smx, const int32_t *smx_arg, int n_t
                               const int32_t *rowmap, const int32_t *m_total, int cap, float *conf, int32_t *amax,
                               cudaStream_t s) {
   const int grid = cap < 148 * 8 ? cap : 148 * 8;
-  k_lm_combine<<<grid > 0 ? grid : 1, 512, 0, s>>>(smx, smx_arg, n_tiles, ldm, rowmap, m_total, conf, amax);
+  launch_pdl(k_lm_combine, grid > 0 ? grid : 1, 512, 0, s, smx, smx_arg, n_tiles, ldm, rowmap, m_total, conf, amax);
   return cudaGetLastError();
 }
 

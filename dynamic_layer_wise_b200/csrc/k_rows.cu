@@ -64,6 +64,7 @@ template <class T>
 __global__ void k_embed_refresh(const int32_t *__restrict__ ids, int32_t *__restrict__ prev_ids,
                                 const T *__restrict__ embed, T *__restrict__ H0, float *__restrict__ d0,
                                 const float *__restrict__ g0, int BN, int D, int V, int full, int32_t *status) {
+  pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
   for (int r = blockIdx.x; r < BN; r += gridDim.x) {
@@ -106,10 +107,10 @@ cudaError_t launch_embed_refresh(int dtype, const int32_t *ids, int32_t *prev_id
                                  cudaStream_t s) {
   if (BN <= 0) return cudaSuccess;
   if (dtype == DCU_BF16)
-    k_embed_refresh<bf16><<<row_grid(BN), 256, 0, s>>>(ids, prev_ids, (const bf16 *)embed, (bf16 *)H0, d0, g0, BN,
+    launch_pdl(k_embed_refresh<bf16>, row_grid(BN), 256, 0, s, ids, prev_ids, (const bf16 *)embed, (bf16 *)H0, d0, g0, BN,
                                                         D, V, full, status);
   else
-    k_embed_refresh<float><<<row_grid(BN), 256, 0, s>>>(ids, prev_ids, (const float *)embed, (float *)H0, d0, g0,
+    launch_pdl(k_embed_refresh<float>, row_grid(BN), 256, 0, s, ids, prev_ids, (const float *)embed, (float *)H0, d0, g0,
                                                          BN, D, V, full, status);
   return cudaGetLastError();
 }
@@ -148,6 +149,7 @@ template <class T>
 __global__ void k_gather_norm(const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
                               const T *__restrict__ H, const float *__restrict__ g, float eps, int D,
                               T *__restrict__ xs) {
+  pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
   const int M = *m_total;
@@ -176,9 +178,9 @@ __global__ void k_gather_norm(const int32_t *__restrict__ rowmap, const int32_t 
 cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *m_total, int cap, const void *H,
                                const float *g, float eps, int D, void *xs, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_gather_norm<bf16><<<row_grid(cap), 256, 0, s>>>(rowmap, m_total, (const bf16 *)H, g, eps, D, (bf16 *)xs);
+    launch_pdl(k_gather_norm<bf16>, row_grid(cap), 256, 0, s, rowmap, m_total, (const bf16 *)H, g, eps, D, (bf16 *)xs);
   else
-    k_gather_norm<float><<<row_grid(cap), 256, 0, s>>>(rowmap, m_total, (const float *)H, g, eps, D, (float *)xs);
+    launch_pdl(k_gather_norm<float>, row_grid(cap), 256, 0, s, rowmap, m_total, (const float *)H, g, eps, D, (float *)xs);
   return cudaGetLastError();
 }
 
@@ -186,7 +188,7 @@ cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *
 // tile summed in slot order (one piece when geo.grid == 0).
 __device__ __forceinline__ float4 csum4(const float *c, const SlotGeo &geo, size_t j) {
   float4 v = *reinterpret_cast<const float4 *>(c + j);
-  const int ns = geo.grid <= 0 ? 1 : sk_nslots(geo, (int)(j >> 7));
+  const int ns = geo.grid <= 0 ? 1 : (geo.nslots ? __ldg(geo.nslots + (j >> 7)) : sk_nslots(geo, (int)(j >> 7)));
   for (int sp = 1; sp < ns; ++sp) {
     const float4 w = *reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)geo.slot_stride + j);
     v.x += w.x;
@@ -228,6 +230,7 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
                           const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total, int N, int H,
                           int Hkv, int hd, const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q,
                           T *__restrict__ Kc, T *__restrict__ Vc) {
+  pdl_enter();
   const int M = *m_total;
   const int half = hd / 2;
   const int n_rope = (H + Hkv) * half / 4, n_v = Hkv * hd / 4;
@@ -272,10 +275,10 @@ cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const SlotGeo geo
                            int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s) {
   const long long items = (long long)cap * ((H + Hkv) * (hd / 2) / 4 + Hkv * hd / 4);
   if (dtype == DCU_BF16)
-    k_epi_qkv<bf16><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
+    launch_pdl(k_epi_qkv<bf16>, flat_grid(items), 256, 0, s, C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
                                                       rope_tab, use_rope, (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc);
   else
-    k_epi_qkv<float><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
+    launch_pdl(k_epi_qkv<float>, flat_grid(items), 256, 0, s, C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
                                                        rope_tab, use_rope, (float *)Q, (float *)Kc, (float *)Vc);
   return cudaGetLastError();
 }
@@ -288,6 +291,7 @@ __global__ void __launch_bounds__(512)
     k_epi_o(const float *__restrict__ C, int ldc, const SlotGeo geo, const int32_t *__restrict__ rowmap,
             const int32_t *__restrict__ m_total, const T *__restrict__ Hl, const float *__restrict__ g2, float eps,
             int D, float *__restrict__ hmid, T *__restrict__ xs) {
+  pdl_enter();
   __shared__ double red[32];
   const int M = *m_total;
   for (int r = blockIdx.x; r < M; r += gridDim.x) {
@@ -327,10 +331,10 @@ cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const SlotGeo geo, 
                          const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
                          float *hmid, void *xs, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_o<bf16><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, (const bf16 *)Hl, g2, eps, D,
+    launch_pdl(k_epi_o<bf16>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, (const bf16 *)Hl, g2, eps, D,
                                                 hmid, (bf16 *)xs);
   else
-    k_epi_o<float><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, (const float *)Hl, g2, eps,
+    launch_pdl(k_epi_o<float>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, (const float *)Hl, g2, eps,
                                                  D, hmid, (float *)xs);
   return cudaGetLastError();
 }
@@ -340,6 +344,7 @@ cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const SlotGeo geo, 
 template <class T>
 __global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, const SlotGeo geo,
                              const int32_t *__restrict__ m_total, int F, T *__restrict__ act) {
+  pdl_enter();
   const int M = *m_total;
   const int per_row = F / 4;
   for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < (long long)M * per_row;
@@ -356,9 +361,9 @@ cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const SlotGeo 
                               int cap, int F, void *act, cudaStream_t s) {
   const long long items = (long long)cap * (F / 4);
   if (dtype == DCU_BF16)
-    k_epi_swiglu<bf16><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, m_total, F, (bf16 *)act);
+    launch_pdl(k_epi_swiglu<bf16>, flat_grid(items), 256, 0, s, C, ldc, geo, m_total, F, (bf16 *)act);
   else
-    k_epi_swiglu<float><<<flat_grid(items), 256, 0, s>>>(C, ldc, geo, m_total, F, (float *)act);
+    launch_pdl(k_epi_swiglu<float>, flat_grid(items), 256, 0, s, C, ldc, geo, m_total, F, (float *)act);
   return cudaGetLastError();
 }
 
@@ -372,6 +377,7 @@ __global__ void __launch_bounds__(512)
                        const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
                        const float *__restrict__ hmid, T *__restrict__ Hn, const float *__restrict__ g_next,
                        float *__restrict__ d_next, int D) {
+  pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
   const int M = *m_total;
@@ -422,10 +428,10 @@ cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const Sl
                                     const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
                                     void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s) {
   if (dtype == DCU_BF16)
-    k_epi_down_scatter<bf16><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, hmid,
+    launch_pdl(k_epi_down_scatter<bf16>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, hmid,
                                                             (bf16 *)Hnext, g_next, d_next, D);
   else
-    k_epi_down_scatter<float><<<row_grid(cap), 512, 0, s>>>(C, ldc, geo, rowmap, m_total, hmid,
+    launch_pdl(k_epi_down_scatter<float>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, hmid,
                                                              (float *)Hnext, g_next, d_next, D);
   return cudaGetLastError();
 }

@@ -23,6 +23,7 @@ static constexpr int kMaxSeq = 16384;
 // order by one thread so it matches a sequential fp64 sum bit for bit.
 __global__ void k_budget_split(const float *__restrict__ s_prev, int L, int B_layer, int uniform_arg,
                                const int32_t *__restrict__ uniform_flag, int32_t *__restrict__ budgets) {
+  pdl_enter();
   const int uniform = uniform_arg || (uniform_flag && *uniform_flag);
   extern __shared__ double sh[];  // [L] fractional parts, then [L] floors
   double *frac = sh, *flr = sh + L;
@@ -79,7 +80,7 @@ cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, 
                                 const int32_t *uniform_flag, int32_t *budgets, cudaStream_t s) {
   if (B <= 0 || L <= 0) return cudaSuccess;
   const int threads = L < 256 ? ((L + 31) / 32) * 32 : 256;
-  k_budget_split<<<B, threads, (size_t)2 * L * sizeof(double), s>>>(s_prev, L, B_layer, uniform, uniform_flag,
+  launch_pdl(k_budget_split, B, threads, (size_t)2 * L * sizeof(double), s, s_prev, L, B_layer, uniform, uniform_flag,
                                                                       budgets);
   return cudaGetLastError();
 }
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kSelThreads)
              int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
              float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
              int32_t *__restrict__ done, int32_t *__restrict__ seq_off, int32_t *__restrict__ status) {
+  pdl_enter();
   extern __shared__ uint8_t smem[];
   uint32_t *sd = reinterpret_cast<uint32_t *>(smem);     // [N] d bits
   uint8_t *flag = smem + (size_t)N * sizeof(uint32_t);   // [N] 0 none, 1 window, 2 top-B
@@ -153,15 +155,31 @@ __global__ void __launch_bounds__(kSelThreads)
   uint32_t thr = 0xffffffffu;  // select d > thr, plus `need` ties at thr
   int need = 0;
   bool take_all = (k == avail);
+  int nz = 0;  // candidates with d > 0: when they all fit, the threshold is 0
   if (k > 0 && !take_all) {
+    for (int i = tid; i < N; i += nthr) nz += (flag[i] == 0 && sd[i] != 0u);
+    nz = block_sum(nz, red_i);
+  }
+  if (k > 0 && !take_all && nz <= k) {
+    thr = 0u;
+    need = k - nz;
+  } else if (k > 0 && !take_all) {
     uint32_t prefix = 0, mask = 0;
     int rem = k;
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int t = tid; t < 256; t += nthr) hist[t] = 0;
       __syncthreads();
-      for (int i = tid; i < N; i += nthr) {
-        const uint32_t u = sd[i];
-        if (flag[i] == 0 && (u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+      // warp-aggregated: one shared atomic per distinct bin per warp (most d
+      // share a few bins, e.g. the stuck-in-mud zeros)
+      for (int base = 0; base < N; base += nthr) {
+        const int i = base + tid;
+        int bin = -1;
+        if (i < N) {
+          const uint32_t u = sd[i];
+          if (flag[i] == 0 && (u & mask) == prefix) bin = (int)((u >> shift) & 255u);
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
       }
       __syncthreads();
       if (tid < 32) {
@@ -267,7 +285,9 @@ cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nk
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_select<<<B, kSelThreads, smem, s>>>(d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
+  // short sequences: fewer threads make the ~25 block barriers cheaper
+  const int threads = N <= 2048 ? 256 : kSelThreads;
+  launch_pdl(k_select, B, threads, smem, s, d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
                                         s_stride, d_next_zero, rowmap, m_total, done, seq_off, status);
   return cudaGetLastError();
 }
@@ -291,6 +311,7 @@ cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int
 // Masked positions of all sequences, in (b, i) order, as packed rows.
 __global__ void __launch_bounds__(1024) k_plan_masked(const uint8_t *__restrict__ masked, int B, int N,
                                                       int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total) {
+  pdl_enter();
   __shared__ int red[32];
   const int BN = B * N, nthr = blockDim.x, tid = threadIdx.x;
   const int chunk = (BN + nthr - 1) / nthr;
@@ -306,7 +327,7 @@ __global__ void __launch_bounds__(1024) k_plan_masked(const uint8_t *__restrict_
 
 cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
                                cudaStream_t s) {
-  k_plan_masked<<<1, 1024, 0, s>>>(masked, B, N, rowmap, m_total);
+  launch_pdl(k_plan_masked, 1, 1024, 0, s, masked, B, N, rowmap, m_total);
   return cudaGetLastError();
 }
 
@@ -322,6 +343,7 @@ __global__ void __launch_bounds__(1024)
     k_commit_rule(int rule, float param, const float *__restrict__ conf, const int32_t *__restrict__ amax,
                   uint8_t *__restrict__ masked, int32_t *__restrict__ ids, int N, int32_t *__restrict__ out_pos,
                   int32_t *__restrict__ out_count) {
+  pdl_enter();
   extern __shared__ uint64_t keys[];  // [P]
   __shared__ int red[32];
   __shared__ double redd[32];
@@ -443,7 +465,7 @@ cudaError_t launch_commit_rule(int rule, float param, const float *conf, const i
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  k_commit_rule<<<B, 1024, (size_t)P * sizeof(uint64_t), s>>>(rule, param, conf, amax, masked, ids, N, out_pos,
+  launch_pdl(k_commit_rule, B, 1024, (size_t)P * sizeof(uint64_t), s, rule, param, conf, amax, masked, ids, N, out_pos,
                                                                out_count);
   return cudaGetLastError();
 }

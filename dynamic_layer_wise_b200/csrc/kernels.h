@@ -64,13 +64,14 @@ cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m
                              const GemmSeg *segs, int nseg, int K, float *C, int ldc, cudaStream_t s);
 
 // ---- tensor-core attention (k_attn_mma.cu), bf16, head_dim 64 or 128.  Rows of
-// sequence b are packed rows [seq_off[b], seq_off[b + 1]).  part_o / part_ml hold
-// `splits` partial results ([splits][rows * H][hd] / [splits][rows * H]); counters
-// ([B][Hkv][qt_cap], zero) are reset by the kernel after use.
+// sequence b are packed rows [seq_off[b], seq_off[b + 1]).  With splits > 1 (<= 8)
+// part_o / part_ml hold the key splits' partial results ([splits][rows * H][hd] /
+// [splits][rows * H]) and a merge kernel follows (two launches); cap_rows bounds
+// the packed rows.
 size_t attn_mma_smem(int hd);
 cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
                                  const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
-                                 int32_t *counters, int splits, int qt_grid, int qt_cap, cudaStream_t s);
+                                 int splits, int qt_grid, int cap_rows, cudaStream_t s);
 
 // ---- attention (k_attn.cu): out[r][h] = softmax(q K^T / sqrt(hd)) V over all N keys of row r's sequence
 cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,

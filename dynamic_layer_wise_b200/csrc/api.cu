@@ -90,7 +90,10 @@ struct dcu_ctx {
   int32_t *smx_arg = nullptr;
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
-  CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of 16 and 64 rows
+  CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of min(128, cap) and min(256, cap) rows
+  uint32_t act_box[2] = {128, 256};
+  // per layer: K and V of the active shape as [B*Hkv*N rows][hd], box 64 x 64 (attention)
+  std::vector<CUtensorMap> kv_maps;
   // per-tile piece counts of each stream-K geometry used so far (device tables)
   struct SlotTable {
     int n_tiles, kblocks, grid, tile_aligned;
@@ -117,11 +120,6 @@ struct dcu_ctx {
   bool use_graphs = true;
   bool capturing = false;
   cudaStream_t cap_stream = nullptr;
-  // side stream of the weight L2 prefetches (forked from and joined back into
-  // the step's stream; inside a capture the fork / join become graph edges)
-  cudaStream_t pf_stream = nullptr;
-  cudaEvent_t pf_fork = nullptr, pf_join = nullptr;
-  bool pf_pending = false;
   std::vector<GraphEntry> graphs;
   GraphEntry *cur_graph = nullptr;
   uint64_t use_clock = 0;
@@ -225,11 +223,6 @@ void free_all(dcu_ctx *c) {
   c->graphs.clear();
   if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   c->cap_stream = nullptr;
-  if (c->pf_stream) cudaStreamDestroy(c->pf_stream);
-  c->pf_stream = nullptr;
-  if (c->pf_fork) cudaEventDestroy(c->pf_fork);
-  if (c->pf_join) cudaEventDestroy(c->pf_join);
-  c->pf_fork = c->pf_join = nullptr;
   for (void *p : c->allocs) cudaFree(p);
   c->allocs.clear();
   for (auto &pc : c->prof)
@@ -270,7 +263,7 @@ std::string check_cfg(const dcu_cfg *c) {
 struct ActOperand {
   const void *X;
   int ldx, K;
-  const CUtensorMap *map16, *map64;
+  const CUtensorMap *map128, *map256;  // activation boxes for 128- and 256-token passes
 };
 
 // tcgen05 GEMM parameters of C[m][n] = sum_k X[m][k] W[n][k] over the
@@ -290,8 +283,8 @@ int gemm_params(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const G
   }
   tp->seg_tile0[nseg] = tile;
   tp->nseg = nseg;
-  tp->b16 = *x.map16;
-  tp->b64 = *x.map64;
+  tp->b = c->gemm_bn == 128 ? *x.map128 : *x.map256;
+  tp->b_rows = (int)c->act_box[c->gemm_bn == 128 ? 0 : 1];
   tp->ldc = ldc;
   tp->m_total = m_total;
   tp->out = c->C;
@@ -329,51 +322,9 @@ int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const Gemm
   return DCU_OK;
 }
 
-// Forks onto the prefetch stream an L2 prefetch of the first `frac` of every
-// CTA range of a later GEMM over these weight segments (K columns): the
-// weights are read-only, so the prefetch overlaps whatever the step's stream
-// runs until that GEMM starts.  Joined back at the end of the step.
-int prefetch_gemm(dcu_ctx *c, const ActOperand &x, const GemmSeg *segs, const CUtensorMap *const *amaps, int nseg,
-                  int ldc, double frac, cudaStream_t s) {
-  if (c->cfg.dtype != DCU_BF16 || frac <= 0.0 || !amaps[0] || !c->pf_stream) return DCU_OK;
-  TcParams tp;
-  if (int rc = gemm_params(c, x, c->m_total(), segs, amaps, nseg, ldc, false, &tp)) return rc;
-  const double per_cta = (double)tp.geo.n_tiles * tp.geo.kblocks / tp.geo.grid;
-  const int kb = (int)(frac * per_cta + 0.999);
-  CK(c, cudaEventRecord(c->pf_fork, s));
-  CK(c, cudaStreamWaitEvent(c->pf_stream, c->pf_fork, 0));
-  LAUNCH(c, launch_prefetch_w(tp, kb, c->pf_stream));
-  c->pf_pending = true;
-  return DCU_OK;
-}
-
-// Joins the prefetch stream back into s (required before a capture ends).
-int prefetch_join(dcu_ctx *c, cudaStream_t s) {
-  if (!c->pf_pending) return DCU_OK;
-  CK(c, cudaEventRecord(c->pf_join, c->pf_stream));
-  CK(c, cudaStreamWaitEvent(s, c->pf_join, 0));
-  c->pf_pending = false;
-  return DCU_OK;
-}
 
 // One layer of recompute over the packed rows in ctx->rowmap / m_total.
 // dense: the rows are every position (full forward): no selection, no d.
-// Fractions of each GEMM's per-CTA weight range prefetched into L2 ahead of
-// it (the window before it: scatter + select + gather for QKV, RoPE +
-// attention for O, the O and SwiGLU epilogues for gate|up and down).
-constexpr double kPrefetchQKV = 0.5, kPrefetchO = 1.0, kPrefetchGateUp = 0.25, kPrefetchDown = 0.35;
-
-int prefetch_qkv(dcu_ctx *c, int l, cudaStream_t s) {
-  if (c->lmaps.empty()) return DCU_OK;
-  const dcu_cfg &g = c->cfg;
-  const LayerMaps &lm = c->lmaps[l];
-  const ActOperand xs{c->xs, g.d_model, g.d_model, &c->xs_map[0], &c->xs_map[1]};
-  GemmSeg seg[3] = {{c->wq[l], g.n_heads * g.head_dim}, {c->wk[l], g.n_kv_heads * g.head_dim},
-                    {c->wv[l], g.n_kv_heads * g.head_dim}};
-  const CUtensorMap *am[3] = {&lm.wq, &lm.wk, &lm.wv};
-  return prefetch_gemm(c, xs, seg, am, 3, (g.n_heads + 2 * g.n_kv_heads) * g.head_dim, kPrefetchQKV, s);
-}
-
 int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t *nkeys, int Bw, cudaStream_t s) {
   const dcu_cfg &g = c->cfg;
   const int L = g.n_layers, D = g.d_model, H = g.n_heads, Hkv = g.n_kv_heads, hd = g.head_dim, F = g.d_ffn;
@@ -404,11 +355,6 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
     if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo)) return rc;
   }
-  if (!dense) {  // the O projection's weights stream into L2 during RoPE / attention
-    GemmSeg seg[1] = {{c->wo[l], D}};
-    const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
-    if (int rc = prefetch_gemm(c, at, seg, am, 1, D, kPrefetchO, s)) return rc;
-  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), gcap, c->N, H, Hkv,
@@ -429,8 +375,9 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
       if (splits > max_sp) splits = max_sp;
       const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
       splits = (c->N + kc - 1) / kc;
-      LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l), c->attn,
-                                     c->attn_po, c->attn_ml, splits, qt_grid, gcap, s));
+      LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
+                                     &c->kv_maps[2 * l], &c->kv_maps[2 * l + 1], c->attn, c->attn_po, c->attn_ml,
+                                     splits, qt_grid, gcap, c->status(), s));
       if (splits > 1) ++c->launches;  // the merge kernel
     } else {
       LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), gcap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
@@ -442,11 +389,6 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
     if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
   }
-  if (!dense) {
-    GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
-    const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
-    if (int rc = prefetch_gemm(c, xs, seg, am, 2, 2 * F, kPrefetchGateUp, s)) return rc;
-  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->Hl(l), c->g2[l],
@@ -457,11 +399,6 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
     if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo)) return rc;
   }
-  if (!dense) {
-    GemmSeg seg[1] = {{c->wd[l], D}};
-    const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
-    if (int rc = prefetch_gemm(c, ac, seg, am, 1, D, kPrefetchDown, s)) return rc;
-  }
   {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), gcap, F, c->act, s));
@@ -470,9 +407,6 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     GemmSeg seg[1] = {{c->wd[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
     if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
-  }
-  if (!dense && !last) {  // the next layer's QKV weights, during scatter / select / gather
-    if (int rc = prefetch_qkv(c, l + 1, s)) return rc;
   }
   {
     Prof p(c, DCU_K_SCATTER, s);
@@ -610,9 +544,6 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     return fail(nullptr, DCU_ENOMEM, m);
   }
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->pf_stream, cudaStreamNonBlocking);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->pf_fork, cudaEventDisableTiming);
-  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->pf_join, cudaEventDisableTiming);
   if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
@@ -637,7 +568,13 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
       wmap(&m.wd, c->wd[l], D, F);
     }
     wmap(&c->lm_map, c->lm_head, (size_t)cfg->vocab, D);
-    const uint32_t boxes[2] = {16, 64};
+    // box rows: the token pass, or the buffer rounded up to 16 when it is shorter
+    // (rows past the buffer are zero-filled; a box height that is not a multiple
+    // of 16 is never used)
+    const uint32_t cap16 = (uint32_t)((cap + 15) / 16 * 16);
+    c->act_box[0] = cap16 < 128u ? cap16 : 128u;
+    c->act_box[1] = cap16 < 256u ? cap16 : 256u;
+    const uint32_t boxes[2] = {c->act_box[0], c->act_box[1]};
     for (int i = 0; i < 2; ++i) {
       ok = ok && encode_tmap_bf16(&c->xs_map[i], c->xs, D, cap, D * 2, 64, boxes[i]);
       ok = ok && encode_tmap_bf16(&c->attn_map[i], c->attn, Hhd, cap, Hhd * 2, 64, boxes[i]);
@@ -694,6 +631,15 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
   c->B = B;
   c->N = N;
   const int BN = B * N;
+  if (c->attn_po) {  // K / V tensor maps of the tensor-core attention for this shape
+    const dcu_cfg &g = c->cfg;
+    c->kv_maps.resize(2 * (size_t)g.n_layers);
+    const uint64_t rows = (uint64_t)B * g.n_kv_heads * N, hd = (uint64_t)g.head_dim;
+    for (int l = 0; l < g.n_layers; ++l)
+      if (!encode_tmap_bf16(&c->kv_maps[2 * l], c->Kl(l), hd, rows, hd * 2, 64, 64) ||
+          !encode_tmap_bf16(&c->kv_maps[2 * l + 1], c->Vl(l), hd, rows, hd * 2, 64, 64))
+        return fail(c, DCU_ECUDA, "cuTensorMapEncodeTiled failed for the K / V cache");
+  }
   {
     Prof p(c, DCU_K_REFRESH, s);
     LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
@@ -729,7 +675,6 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
     c->gemm_rows_hint = (int)(est < BN ? est : BN);
     c->gemm_bn = c->gemm_rows_hint <= 128 ? 128 : 256;
   }
-  if (int rc = prefetch_qkv(c, 0, s)) return rc;  // layer 0's QKV weights, during budget / refresh / select
   {
     Prof p(c, DCU_K_BUDGET, s);
     LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, 0, c->uniform_flag(), c->budgets, s));
@@ -740,11 +685,7 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
                                    c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
   }
   for (int l = 0; l < L; ++l)
-    if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) {
-      prefetch_join(c, s);  // a capture must not end with the side stream forked
-      return rc;
-    }
-  if (int rc = prefetch_join(c, s)) return rc;
+    if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) return rc;
   CK(c, cudaMemcpyAsync(c->s_prev, c->s_cur, (size_t)c->B * L * 4, cudaMemcpyDeviceToDevice, s));
   CK(c, cudaMemsetAsync(c->uniform_flag(), 0, 4, s));
   return DCU_OK;
@@ -773,8 +714,8 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *
       TcParams tp;
       memset(&tp, 0, sizeof(tp));
       tp.a[0] = c->lm_map;
-      tp.b16 = c->xs_map[0];
-      tp.b64 = c->xs_map[1];
+      tp.b = c->xs_map[1];
+      tp.b_rows = (int)c->act_box[1];
       const int tiles = (g.vocab + 127) / 128;
       tp.seg_tile0[0] = 0;
       tp.seg_tile0[1] = tiles;
@@ -986,10 +927,11 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
   TcParams tp;
   memset(&tp, 0, sizeof(tp));
   const int bn = M <= 128 ? 128 : 256;
+  const int m16 = (M + 15) / 16 * 16, b_rows = m16 < bn ? m16 : bn;  // activation box rows (multiple of 16)
   if (!encode_tmap_bf16(&tp.a[0], W, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, 64, 128) ||
-      !encode_tmap_bf16(&tp.b16, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 16) ||
-      !encode_tmap_bf16(&tp.b64, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 64))
+      !encode_tmap_bf16(&tp.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)b_rows))
     return fail(nullptr, DCU_ECUDA, "dcu_linear: cuTensorMapEncodeTiled failed");
+  tp.b_rows = b_rows;
   const int tiles = (Nout + 127) / 128;
   tp.seg_tile0[0] = 0;
   tp.seg_tile0[1] = tiles;

@@ -10,7 +10,6 @@ constexpr int kTcMaxA = 16;                 // deepest weight-tile ring
 constexpr int kTcMaxB = 4;                  // deepest activation-tile ring
 constexpr int kTcThreads = 224;             // 7 warps: W producer, MMA, 4 epilogue, X producer
 constexpr uint32_t kTcABytes = 128u * 128u;  // weight tile: 128 rows x 64 bf16
-constexpr uint32_t kTcBBoxBytes = 16u * 128u;  // activation box: 16 rows x 64 bf16
 constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (one CTA per SM)
 
 // Stream-K schedule: the flattened (tile, k block) space of one token pass,
@@ -49,7 +48,8 @@ __host__ __device__ inline int sk_nslots(const SlotGeo &g, int tile) {
 // out[slot][m][n] = the piece `slot` of sum_k X[m][k] * W[n][k] for m < M.
 struct TcParams {
   CUtensorMap a[3];        // weight segments, bf16 [rows][K], box 64 x 128, 128-byte swizzle
-  CUtensorMap b16, b64;    // packed activations, bf16 [cap][K], boxes 64 x 16 and 64 x 64, 128-byte swizzle
+  CUtensorMap b;           // packed activations, bf16 [cap][K], box 64 x b_rows, 128-byte swizzle
+  int b_rows;              // rows of the activation box: the token pass (BN) or fewer when cap < BN
   int seg_tile0[4];        // first 128-row tile of segment s; seg_tile0[nseg] = n_tiles
   int seg_col0[3];         // first output column of segment s
   int seg_rows[3];         // rows of segment s
@@ -77,9 +77,6 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
                       uint32_t box_inner, uint32_t box_outer);
 // bn: token rows per pass (128 or 256); the grid is p.geo.grid CTAs.
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s);
-// L2 prefetch of the first kb_count k blocks of every CTA's range of the GEMM
-// described by p (weights only; see k_prefetch_w).
-cudaError_t launch_prefetch_w(const TcParams &p, int kb_count, cudaStream_t s);
 // Most pieces a tile can be cut into under the stream-K split over `grid` CTAs.
 int tc_max_slots(int n_tiles, int grid);
 // Merges the per-tile softmax statistics of the LM head (epi_mode 1): for packed

@@ -21,6 +21,12 @@ constexpr int QT = 128;  // queries per CTA
 constexpr int KS = 64;   // keys per sub-chunk
 constexpr int NST = 4;   // K/V sub-chunk buffers: NST - 1 loads in flight ahead of the one in use
 
+// Q tile bytes (padded rows), rounded to 1024 so the K / V ring that follows
+// is aligned for the 128-byte swizzle.
+__host__ __device__ constexpr uint32_t attn_q_bytes(int hd) {
+  return ((uint32_t)QT * (uint32_t)(hd + 8) * 2u + 1023u) & ~1023u;
+}
+
 __device__ __forceinline__ uint32_t smem_u32a(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -59,31 +65,66 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 struct AttnArgs {
+  CUtensorMap kmap, vmap;   // the layer's K / V as [B*Hkv*N rows][hd], box 64 x 64, 128-byte swizzle
   const bf16 *Q;            // [cap][H][hd]
   const bf16 *Kc, *Vc;      // [B][Hkv][N][hd]
   bf16 *out;                // [cap][H][hd]
   const int32_t *seq_off;   // [B + 1] packed-row offsets of the sequences
   float *part_o;            // [splits][cap * H][hd] partial outputs
   float2 *part_ml;          // [splits][cap * H] (max, sum) in log2 units
+  int32_t *status;          // device status word (DCU_ST_TIMEOUT)
   int B, N, H, Hkv, splits, kc, qt_grid;
   float scale_log2;         // log2(e) / sqrt(hd)
 };
 
+// Shared-memory address of the 16-byte chunk holding elements d .. d+7 of key
+// row `key` in a K / V stage written by TMA with the 128-byte swizzle: hd is
+// split in 64-wide boxes of 64 rows x 128 B, chunk c of row r sits at chunk
+// c ^ (r & 7), so the 8 rows an ldmatrix reads hit 8 different bank groups.
+__device__ __forceinline__ uint32_t kv_addr(uint32_t base, int key, int d) {
+  return base + (uint32_t)(d >> 6) * 8192u + (uint32_t)key * 128u + ((uint32_t)(((d & 63) >> 3) ^ (key & 7)) << 4);
+}
+
+__device__ __forceinline__ void tma_load_2d_a(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// Bounded wait on a K / V stage (all threads).  False after ~1 s: the caller
+// abandons the tile (the host sees DCU_ST_TIMEOUT).
+__device__ __forceinline__ bool kv_wait(uint32_t bar, uint32_t parity, int32_t *status) {
+  for (uint32_t it = 0; it < (1u << 24); ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+  }
+  if (status) atomicOr(status, DCU_ST_TIMEOUT);
+  return false;
+}
+
+// Stage layout: K boxes (HD / 64 of 8 KB) then V boxes; NST stages from `ring`.
+// Returns false if a K / V stage never landed (the kernel then stops).
 template <int HD>
-__device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b, int kvh, int ks, int qt, int row0,
-                                          int nq) {
-  constexpr int LD = HD + 8;  // padded row (elements): 16-byte shift per row, conflict-free ldmatrix
+__device__ __forceinline__ bool attn_tile(const AttnArgs &a, uint8_t *sm, uint32_t ring, uint32_t bar0,
+                                          uint32_t &chunk_ctr, int b, int kvh, int ks, int qt, int row0, int nq) {
+  constexpr int LD = HD + 8;  // padded Q row (elements): 16-byte shift per row, conflict-free ldmatrix
   constexpr int CPR = HD / 8;  // 16-byte chunks per row
+  constexpr uint32_t KVB = (uint32_t)HD * 128u;  // bytes of one chunk's K (or V): HD/64 boxes of 8 KB
+  constexpr uint32_t STAGE = 2u * KVB;
   bf16 *Qs = reinterpret_cast<bf16 *>(sm);  // [QT][LD]
-  bf16 *Ks = Qs + QT * LD;                   // [NST][KS][LD]
-  bf16 *Vs = Ks + NST * KS * LD;             // [NST][KS][LD]
   const int G = a.H / a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int k_begin = ks * a.kc;
   const int k_end = min(a.N, k_begin + a.kc);
-  const bf16 *Kb = a.Kc + ((size_t)b * a.Hkv + kvh) * (size_t)a.N * HD;
-  const bf16 *Vb = a.Vc + ((size_t)b * a.Hkv + kvh) * (size_t)a.N * HD;
+  const int rowbase = (b * a.Hkv + kvh) * a.N;  // first K / V row of this (sequence, kv head)
 
   // Q tile -> shared (query q -> packed row row0 + q / G, head kvh * G + q % G)
   for (int c = tid; c < QT * CPR; c += blockDim.x) {
@@ -93,24 +134,26 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
     const int r = row0 + (ok ? q / G : 0), h = kvh * G + (ok ? q % G : 0);
     cp_async16(smem_u32a(Qs + qi * LD + ch * 8), a.Q + ((size_t)r * a.H + h) * HD + ch * 8, ok);
   }
-  auto load_kv = [&](int buf, int key0) {
-    for (int c = tid; c < KS * CPR; c += blockDim.x) {
-      const int ki = c / CPR, ch = c - ki * CPR;
-      const int key = key0 + ki;
-      const bool ok = key < k_end;
-      const size_t off = (size_t)(ok ? key : k_begin) * HD + ch * 8;
-      cp_async16(smem_u32a(Ks + (buf * KS + ki) * LD + ch * 8), Kb + off, ok);
-      cp_async16(smem_u32a(Vs + (buf * KS + ki) * LD + ch * 8), Vb + off, ok);
+  cp_async_commit();
+  // K / V sub-chunk j of this tile -> stage (chunk_ctr + j) % NST: one thread
+  // issues 2 * HD / 64 TMA boxes (keys past this split are masked below; past
+  // the tensor they are zero-filled)
+  const uint32_t c0 = chunk_ctr;
+  auto load_kv = [&](int j) {
+    const uint32_t st = (c0 + (uint32_t)j) % NST;
+    const uint32_t dst = ring + st * STAGE, bar = bar0 + 8u * st;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(STAGE) : "memory");
+    const int y = rowbase + k_begin + j * KS;
+#pragma unroll
+    for (int h = 0; h < HD / 64; ++h) {
+      tma_load_2d_a(dst + (uint32_t)h * 8192u, &a.kmap, h * 64, y, bar);
+      tma_load_2d_a(dst + KVB + (uint32_t)h * 8192u, &a.vmap, h * 64, y, bar);
     }
   };
   const int n_sub = (k_end - k_begin + KS - 1) / KS;
-  // prologue: sub-chunks 0 .. NST-2 (one commit group each, empty past the end,
-  // so group g always holds sub-chunk g; the Q tile rides in group 0)
-#pragma unroll
-  for (int st = 0; st < NST - 1; ++st) {
-    if (st < n_sub) load_kv(st, k_begin + st * KS);
-    cp_async_commit();
-  }
+  chunk_ctr += (uint32_t)n_sub;
+  if (tid == 0)
+    for (int j = 0; j < NST - 1 && j < n_sub; ++j) load_kv(j);
 
   float o[HD / 8][4];
 #pragma unroll
@@ -120,12 +163,25 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
   const bool warp_active = (qt * QT + warp * 16) < nq;
 
   for (int sc = 0; sc < n_sub; ++sc) {
-    const int buf = sc % NST;
-    const int nxt = sc + NST - 1;  // refills the buffer consumed in iteration sc - 1
-    if (nxt < n_sub) load_kv(nxt % NST, k_begin + nxt * KS);
-    cp_async_commit();
-    cp_async_wait<NST - 1>();  // group sc (sub-chunk sc) has landed
-    __syncthreads();
+    const uint32_t st = (c0 + (uint32_t)sc) % NST;
+    const int nxt = sc + NST - 1;  // refills the stage consumed in iteration sc - 1
+    if (tid == 0 && nxt < n_sub) load_kv(nxt);
+    if (sc == 0) cp_async_wait<0>();
+    const bool landed = kv_wait(bar0 + 8u * st, ((c0 + (uint32_t)sc) / NST) & 1u, a.status);
+    if (__syncthreads_or(!landed)) {
+      // timed out (status is set): wait, bounded, for this tile's copies still
+      // in flight so none lands after the CTA has exited, then give up
+      if (tid == 0) {
+        const int issued = min(n_sub, sc + NST);
+        for (int j = sc; j < issued; ++j) {
+          const uint32_t cj = c0 + (uint32_t)j;
+          kv_wait(bar0 + 8u * (cj % NST), (cj / NST) & 1u, nullptr);
+        }
+      }
+      __syncthreads();
+      return false;
+    }
+    const uint32_t Kt = ring + st * STAGE, Vt = Kt + KVB;
     if (sc == 0 && warp_active) {
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
@@ -134,8 +190,6 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
       }
     }
     if (warp_active) {
-      const bf16 *Kt = Ks + buf * KS * LD;
-      const bf16 *Vt = Vs + buf * KS * LD;
       float s[KS / 8][4];
 #pragma unroll
       for (int j = 0; j < KS / 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
@@ -147,7 +201,7 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
           const int key = j * 16 + (lane & 7) + ((lane >> 4) << 3);
           const int d = kk * 16 + ((lane >> 3) & 1) * 8;
           uint32_t b0, b1, b2, b3;
-          ldsm_x4(smem_u32a(Kt + key * LD + d), b0, b1, b2, b3);
+          ldsm_x4(kv_addr(Kt, key, d), b0, b1, b2, b3);
           mma_bf16(s[2 * j], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
           mma_bf16(s[2 * j + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
         }
@@ -214,7 +268,7 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
           const int key = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
           const int d = i * 16 + (lane >> 4) * 8;
           uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(smem_u32a(Vt + key * LD + d), b0, b1, b2, b3);
+          ldsm_x4_t(kv_addr(Vt, key, d), b0, b1, b2, b3);
           mma_bf16(o[2 * i], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b0, b1);
           mma_bf16(o[2 * i + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], b2, b3);
         }
@@ -238,7 +292,7 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
               __floats2bfloat162_rn(o[i][2 * h2] * inv, o[i][2 * h2 + 1] * inv);
       }
     }
-    return;
+    return true;
   }
   // partials of this split: plane = packed (row, head) pairs of all sequences
   const size_t plane = (size_t)a.seq_off[a.B] * a.H;
@@ -256,13 +310,26 @@ __device__ __forceinline__ void attn_tile(const AttnArgs &a, uint8_t *sm, int b,
       if (t == 0) a.part_ml[(size_t)ks * plane + qidx] = make_float2(m_run[h2], l_run[h2]);
     }
   }
+  return true;
 }
 
 // grid = B x Hkv x splits x qt_grid; the CTA walks query tiles qt, qt + qt_grid, ...
 template <int HD>
-__global__ void __launch_bounds__(256, 1) k_attn_mma(const AttnArgs a) {
+__global__ void __launch_bounds__(256, 1) k_attn_mma(const __grid_constant__ AttnArgs a) {
   pdl_enter();
-  extern __shared__ __align__(16) uint8_t sm[];
+  extern __shared__ __align__(16) uint8_t sm_raw[];
+  __shared__ __align__(8) uint64_t kv_full[NST];
+  // Q tile (padded rows) at a 1024-byte aligned base, then the K / V ring
+  uint8_t *sm = sm_raw + ((1024u - (smem_u32a(sm_raw) & 1023u)) & 1023u);
+  const uint32_t ring = smem_u32a(sm) + attn_q_bytes(HD);
+  const uint32_t bar0 = smem_u32a(kv_full);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < NST; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * i) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  uint32_t chunk_ctr = 0;
   int item = blockIdx.x;
   const int per_b = a.Hkv * a.splits * a.qt_grid;
   const int b = item / per_b;
@@ -274,7 +341,7 @@ __global__ void __launch_bounds__(256, 1) k_attn_mma(const AttnArgs a) {
   const int row0 = a.seq_off[b], nq = (a.seq_off[b + 1] - row0) * (a.H / a.Hkv);
   if (ks * a.kc >= a.N) return;
   for (int qt = qt0; qt * QT < nq; qt += a.qt_grid) {
-    attn_tile<HD>(a, sm, b, kvh, ks, qt, row0, nq);
+    if (!attn_tile<HD>(a, sm, ring, bar0, chunk_ctr, b, kvh, ks, qt, row0, nq)) return;
     __syncthreads();
   }
 }
@@ -325,13 +392,18 @@ __global__ void k_attn_merge(const float *__restrict__ part_o, const float2 *__r
 
 }  // namespace
 
-size_t attn_mma_smem(int hd) { return (size_t)(QT + 2 * NST * KS) * (hd + 8) * sizeof(bf16); }
+// Q tile + NST stages of (K, V) x 64 keys + alignment slack.
+size_t attn_mma_smem(int hd) { return (size_t)attn_q_bytes(hd) + (size_t)NST * 2u * (size_t)hd * 128u + 1024u; }
 
 cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
-                                 const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
-                                 int splits, int qt_grid, int cap_rows, cudaStream_t s) {
-  if ((hd != 64 && hd != 128) || splits < 1 || splits > 8) return cudaErrorInvalidValue;
+                                 const void *Kc, const void *Vc, const CUtensorMap *kmap, const CUtensorMap *vmap,
+                                 void *out, float *part_o, float2 *part_ml, int splits, int qt_grid, int cap_rows,
+                                 int32_t *status, cudaStream_t s) {
+  if ((hd != 64 && hd != 128) || splits < 1 || splits > 8 || !kmap || !vmap) return cudaErrorInvalidValue;
   AttnArgs a;
+  a.kmap = *kmap;
+  a.vmap = *vmap;
+  a.status = status;
   a.Q = (const bf16 *)Q;
   a.Kc = (const bf16 *)Kc;
   a.Vc = (const bf16 *)Vc;

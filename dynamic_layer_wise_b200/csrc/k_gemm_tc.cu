@@ -12,7 +12,8 @@
 //               starts before the previous launch has finished (weights are
 //               never written by a kernel)
 //   warp 6      activation producer (one lane): shallow ring of X tiles (from
-//               L2), after the programmatic-dependency wait
+//               L2, one TMA box of the whole token pass per stage), after the
+//               programmatic-dependency wait
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma (K=16)
 //               per 64-wide k block, tcgen05.commit frees both smem stages
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 tile, coalesced
@@ -242,9 +243,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   // boxes of the rows actually loaded, from L2).  The activation ring only has
   // to cover the L2 latency, so most of shared memory holds weight tiles in
   // flight.
-  const int nb_max = (min(BN, M) + 15) / 16;
-  const uint32_t b_stage = (uint32_t)nb_max * kTcBBoxBytes;
-  const int SB = nb_max >= 12 ? 3 : 4;
+  const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per stage
+  const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned stages
+  const int SB = b_stage > 16384u ? 3 : 4;
   int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage) / kTcABytes);
   SA = SA > kTcMaxA ? kTcMaxA : SA;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -340,14 +341,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           ok = false;
           break;
         }
-        mbar_expect_tx(FULL_B(stage), (uint32_t)cb.nb * kTcBBoxBytes);
-        const int n64 = cb.nb / 4, n16 = cb.nb - 4 * n64;
-        for (int j = 0; j < n64; ++j)
-          tma_load_2d(STAGE_B(stage) + (uint32_t)j * 4u * kTcBBoxBytes, &p.b64, cb.kb * 64, cb.m0 + 64 * j,
-                      FULL_B(stage), pol_x);
-        for (int j = 0; j < n16; ++j)
-          tma_load_2d(STAGE_B(stage) + (uint32_t)(4 * n64 + j) * kTcBBoxBytes, &p.b16, cb.kb * 64,
-                      cb.m0 + 64 * n64 + 16 * j, FULL_B(stage), pol_x);
+        // the whole token pass in one box: TMA throughput is bound by the number
+        // of copies, not their bytes (rows past the packed count are never read
+        // by the MMA; rows past the buffer are zero-filled)
+        mbar_expect_tx(FULL_B(stage), b_bytes);
+        tma_load_2d(STAGE_B(stage), &p.b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
         used[stage] = true;
         fill_parity[stage] = phase;
         cb.advance(p, passes, BN, M);
@@ -505,25 +503,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   }
 }
 
-// L2 prefetch of the weight tiles a later launch of k_gemm_tc with the same
-// parameters will read first: CTA c issues, in order, the first `kb_count` k
-// blocks of GEMM CTA c's stream-K range (first token pass) as bulk tensor
-// prefetches.  It only moves weights (never written by a kernel) into L2, so it
-// may run on a side stream concurrently with anything.
-__global__ void __launch_bounds__(32) k_prefetch_w(const __grid_constant__ TcParams p, int kb_count) {
-  if (threadIdx.x != 0) return;
-  const long long b = sk_begin(p.geo, blockIdx.x), e0 = sk_begin(p.geo, blockIdx.x + 1);
-  const long long e = (b + kb_count < e0) ? b + kb_count : e0;
-  FragIter it{b, e, 0};
-  Frag f;
-  while (next_frag(p, 1, it, f))
-    for (int kb = f.kb0; kb < f.kb1; ++kb)
-      asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                       reinterpret_cast<uint64_t>(&p.a[f.seg])),
-                   "r"(kb * 64), "r"(f.arow)
-                   : "memory");
-}
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -583,16 +562,11 @@ static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
   const int grid = p.geo.grid;
   if (grid <= 0) return cudaSuccess;
+  if (p.b_rows <= 0 || p.b_rows > bn || p.b_rows % 16 != 0) return cudaErrorInvalidValue;
   p.smem_bytes = (uint32_t)kTcSmem;
   if (bn == 128) return launch_bn<128>(p, grid, s);
   if (bn == 256) return launch_bn<256>(p, grid, s);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_prefetch_w(const TcParams &p, int kb_count, cudaStream_t s) {
-  if (p.geo.grid <= 0 || kb_count <= 0) return cudaSuccess;
-  k_prefetch_w<<<p.geo.grid, 32, 0, s>>>(p, kb_count);
-  return cudaGetLastError();
 }
 
 int tc_max_slots(int n_tiles, int grid) { return (grid + n_tiles - 1) / n_tiles + 1; }

@@ -70,8 +70,9 @@ cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m
 // the packed rows.
 size_t attn_mma_smem(int hd);
 cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
-                                 const void *Kc, const void *Vc, void *out, float *part_o, float2 *part_ml,
-                                 int splits, int qt_grid, int cap_rows, cudaStream_t s);
+                                 const void *Kc, const void *Vc, const CUtensorMap *kmap, const CUtensorMap *vmap,
+                                 void *out, float *part_o, float2 *part_ml, int splits, int qt_grid, int cap_rows,
+                                 int32_t *status, cudaStream_t s);
 
 // ---- attention (k_attn.cu): out[r][h] = softmax(q K^T / sqrt(hd)) V over all N keys of row r's sequence
 cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,

@@ -214,20 +214,32 @@ def step_algorithmic_bytes(shape, rows_per_layer, N, batch, n_masked):
     return shape.n_layers * (w_layer + kv) + shape.vocab * shape.d_model * es + act + n_masked * shape.d_model * es
 
 
-def traffic_for(kernel_file: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken on
-    the current source of the kernel."""
+GEMM_SOURCES = ("k_gemm_tc.cu", "tc_ptx.cuh", "gemm_tc.h")
+
+
+def kernel_source_sha(files) -> str:
+    """Hash of the sources a kernel is built from (to tell whether a stored
+    ncu figure still describes the current kernel)."""
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "dynamic_layer_wise_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(key: str, files, algorithmic_bytes_per_launch: float):
+    """DRAM bytes per launch from the committed ncu summary (profiles/traffic.json),
+    scaled from the captured launch to the average launch by algorithmic bytes,
+    if the capture was taken on the current source of the kernel; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         t = json.load(fh)
-    src = os.path.join(ROOT, "dynamic_layer_wise_b200", "csrc", kernel_file)
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    e = t.get(kernel_file)
-    if e and e.get("source_sha") == h:
-        return e.get("dram_bytes_per_launch")
-    return None
+    e = t.get(key)
+    if not e or e.get("source_sha") != kernel_source_sha(files):
+        return None
+    return e["dram_bytes"] / e["algorithmic_bytes"] * algorithmic_bytes_per_launch
 
 
 # ---------------------------------------------------------------- profiling cases
@@ -414,7 +426,8 @@ def main():
     step_bytes = step_algorithmic_bytes(shape, rows, N, B, int(masked.sum().item()) + 1)
     roofline = {"bound": "hbm", "kernel": "gemm (recompute projections + FFN)", "achieved": achieved,
                 "peak": hbm, "unit": "GB/s", "frac": (achieved / hbm) if achieved else None,
-                "traffic": traffic_for("k_gemm_tc.cu"), "peak_source": peak_src,
+                "traffic": traffic_for("k_gemm_tc", GEMM_SOURCES, gemm_bytes / gemm_launches),
+                "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": gemm_bytes / gemm_launches,
                 "step_bytes": step_bytes, "step_roofline_ms": step_bytes / (hbm * 1e9) * 1e3,
                 "step_frac_of_measured": (step_bytes / (hbm * 1e9) * 1e3) / ms_step,

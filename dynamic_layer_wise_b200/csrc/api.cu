@@ -364,7 +364,10 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     Prof p(c, DCU_K_ATTN, s);
     if (c->attn_po) {
       const int G = H / Hkv;
-      const int rows_seq = dense ? c->N : (c->gemm_rows_hint + c->B - 1) / c->B;
+      // query tiles per (sequence, kv head) sized for the typical recompute set
+      // (half the GEMM's rows hint: B_layer + B_window + 1 per sequence); a
+      // larger set makes each CTA walk more than one query tile
+      const int rows_seq = dense ? c->N : (c->gemm_rows_hint / 2 + c->B - 1) / c->B;
       int qt_grid = (rows_seq * G + 127) / 128;
       qt_grid = qt_grid < 1 ? 1 : (qt_grid > c->attn_qt_cap ? c->attn_qt_cap : qt_grid);
       // one wave: (sequence, kv head, query tile) items x key splits <= SM count (one CTA per SM)
@@ -706,6 +709,8 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *
                                    g.rms_eps, g.d_model, c->xs, s));
     }
     GemmSeg lm[1] = {{c->lm_head, g.vocab}};
+    const int lm_tiles = (g.vocab + 127) / 128;
+    const int lm_grid = lm_tiles < c->num_sms ? lm_tiles : c->num_sms;  // one statistics row per CTA
     c->gemm_bn = 256;
     c->gemm_rows_hint = 256;
     if (g.dtype == DCU_BF16) {
@@ -740,7 +745,7 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *
     }
     Prof p(c, DCU_K_LMHEAD, s);
     if (g.dtype == DCU_BF16)
-      LAUNCH(c, launch_lm_combine(c->smx, c->smx_arg, (g.vocab + 127) / 128, cap, c->mrow, c->m_masked(), cap,
+      LAUNCH(c, launch_lm_combine(c->smx, c->smx_arg, lm_grid, cap, c->mrow, c->m_masked(), cap,
                                   c->conf, c->amax, s));
     else
       LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));

@@ -60,10 +60,11 @@ struct TcParams {
   float *out;              // [slots][cap][ldc]
   int32_t *status;         // device status word (DCU_ST_TIMEOUT) or null
   uint32_t smem_bytes;
-  // epi_mode 1 (LM head, tile_aligned): instead of storing logits, every tile
-  // writes per token m its softmax statistics over the tile's 128 vocabulary
-  // entries: smx[tile][m] = (max, sum of exp(z - max)), smx_arg[tile][m] =
-  // lowest id reaching the max; row pitch ldm.
+  // epi_mode 1 (LM head, tile_aligned, BN = 256, one segment): the tokens are
+  // the MMA M dimension and the weight tile (128 vocabulary rows) is N; instead
+  // of storing logits, CTA c writes per token m its softmax statistics over the
+  // vocabulary rows of its whole range: smx[c][m] = (max, sum of exp(z - max)),
+  // smx_arg[c][m] = lowest id reaching the max; row pitch ldm.
   int epi_mode;
   float2 *smx;
   int32_t *smx_arg;
@@ -79,9 +80,9 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s);
 // Most pieces a tile can be cut into under the stream-K split over `grid` CTAs.
 int tc_max_slots(int n_tiles, int grid);
-// Merges the per-tile softmax statistics of the LM head (epi_mode 1): for packed
-// row r (position rowmap[r]), conf = 1 / sum_t s_t exp(m_t - M), argmax = the
-// lowest id reaching M = max_t m_t.
+// Merges the per-CTA softmax statistics of the LM head (epi_mode 1, n_parts =
+// the GEMM's grid): for packed row r (position rowmap[r]), conf =
+// 1 / sum_c s_c exp(m_c - M), argmax = the lowest id reaching M = max_c m_c.
 cudaError_t launch_lm_combine(const float2 *smx, const int32_t *smx_arg, int n_tiles, int ldm,
                               const int32_t *rowmap, const int32_t *m_total, int cap, float *conf, int32_t *amax,
                               cudaStream_t s);

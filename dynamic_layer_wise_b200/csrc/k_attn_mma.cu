@@ -93,10 +93,12 @@ __device__ __forceinline__ void tma_load_2d_a(uint32_t dst, const CUtensorMap *m
       : "memory");
 }
 
-// Bounded wait on a K / V stage (all threads).  False after ~1 s: the caller
-// abandons the tile (the host sees DCU_ST_TIMEOUT).
+// Bounded wait on a K / V stage (all threads): false after 1 s of wall-clock
+// time (%globaltimer; try_wait may suspend, so an iteration count is no time
+// bound), the caller abandons the tile and the host sees DCU_ST_TIMEOUT.
 __device__ __forceinline__ bool kv_wait(uint32_t bar, uint32_t parity, int32_t *status) {
-  for (uint32_t it = 0; it < (1u << 24); ++it) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}\n"
@@ -104,6 +106,12 @@ __device__ __forceinline__ bool kv_wait(uint32_t bar, uint32_t parity, int32_t *
         : "r"(bar), "r"(parity)
         : "memory");
     if (ok) return true;
+    if ((it & 63u) == 0u) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+      if (it == 0) t0 = t;
+      else if (t - t0 > 1000000000ull) break;
+    }
   }
   if (status) atomicOr(status, DCU_ST_TIMEOUT);
   return false;

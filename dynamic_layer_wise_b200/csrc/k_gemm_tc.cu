@@ -27,141 +27,10 @@
 #include "common.cuh"
 #include "gemm_tc.h"
 #include "kernels.h"
+#include "tc_ptx.cuh"
 
 namespace dcu {
 namespace {
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar,
-                                            uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
-               : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish() {
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// 32 TMEM lanes x 16 consecutive 32-bit columns: thread i of the warp gets lane
-// (base lane + i), columns col..col+15.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  // the registers are only valid after wait::ld; tie them to it
-  asm volatile("tcgen05.wait::ld.sync.aligned;"
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                 "+r"(r[15])
-               :
-               : "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Shared-memory matrix descriptor of a K-major tile with the 128-byte swizzle:
-// start address >> 4 in bits [0,14), leading byte offset 0 (unused for this
-// layout), stride byte offset 1024 (8 rows x 128 B) >> 4 in bits [32,46), the
-// fixed descriptor version 1 at bit 46, swizzle mode 2 (128 B) in bits [61,64).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) |
-         ((uint64_t)2 << 61);
-}
-
-// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and B
-// bf16 (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 in bits 17-22,
-// M >> 4 in bits 24-28.
-__device__ __forceinline__ uint32_t idesc_bf16(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-
-constexpr uint32_t kSpinLimit = 1u << 25;
-
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                             int32_t *status) {
-  for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 255u && *abort_flag) return false;
-    if (it >= kSpinLimit) {
-      *abort_flag = 1;
-      if (status) atomicOr(status, DCU_ST_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// Drain wait on the abort path: bounded, ignores the abort flag.
-__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
-  for (uint32_t it = 0; it < (1u << 22); ++it)
-    if (mbar_try_wait(bar, parity)) return;
-}
 
 struct Frag {
   int tile, kb0, kb1, seg, arow, slot;
@@ -195,7 +64,6 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
   return true;
 }
 
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 
 // Position in this CTA's (fragment, k block) sequence.
@@ -223,12 +91,10 @@ struct KCursor {
 
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ float2 smx_w[4][16];
-  __shared__ int smx_i[4][16];
 
   // The row count is written by the select / plan kernel two launches before
   // this one, so it is final even while the previous launch still runs.
@@ -362,12 +228,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     if (lane == 0) {
       int sa = 0, sb = 0;
       uint32_t pa = 0, pb = 0, nfrag = 0;
+      const uint32_t idesc_lm = idesc_bf16(128, 128);
       bool ok = true, issued = false;
       FragIter it{my_begin, my_end, 0};
       Frag f;
       while (ok && next_frag(p, passes, it, f)) {
         const int mrows = min(BN, M - it.pass * BN);
         const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
+        const int lm_halves = mrows > 128 ? 2 : 1;
         const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
         const uint32_t dtm = tmem + acc * (uint32_t)BN;
         if (!wait_bounded(TEMPTY(acc), (use & 1u) ^ 1u, abort_v, p.status)) {
@@ -383,9 +251,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           tc_fence_after();
           const uint64_t ad = sw128_desc(STAGE_A(sa));
           const uint64_t bd = sw128_desc(STAGE_B(sb));
+          if (p.epi_mode == 1) {
+            // LM head: tokens are the MMA M dimension (one or two 128-row halves of
+            // the activation box), the tile's 128 vocabulary rows are N
+            for (int mt = 0; mt < lm_halves; ++mt) {
+              const uint64_t xd = sw128_desc(STAGE_B(sb) + (uint32_t)mt * 16384u);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
-            tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
+              for (int k = 0; k < 4; ++k)
+                tc_mma(dtm + (uint32_t)(mt * 128), xd + (uint64_t)(2 * k), ad + (uint64_t)(2 * k), idesc_lm,
+                       (kb > f.kb0 || k > 0) ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
+              tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
+          }
           issued = true;
           tc_commit(EMPTY_A(sa));  // both stages are free once these MMAs have read them
           tc_commit(EMPTY_B(sb));
@@ -412,59 +292,73 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     uint32_t nfrag = 0;
     FragIter it{my_begin, my_end, 0};
     Frag f;
+    float lm_max[2] = {-INFINITY, -INFINITY};
+    double lm_sum[2] = {0.0, 0.0};  // fp64 running sums: ~1000 terms per CTA
+    int lm_arg[2] = {0x7fffffff, 0x7fffffff};
+    int lm_pass = 0;
+    // LM head: this CTA's statistics of the pass's tokens over its vocabulary range
+    auto lm_flush = [&](int pass) {
+      for (int mt = 0; mt < 2; ++mt) {
+        const int m = pass * BN + mt * 128 + q * 32 + lane;
+        if (m < M) {
+          const size_t o = (size_t)blockIdx.x * p.ldm + (size_t)m;
+          p.smx[o] = make_float2(lm_max[mt], (float)lm_sum[mt]);
+          p.smx_arg[o] = lm_arg[mt];
+        }
+        lm_max[mt] = -INFINITY;
+        lm_sum[mt] = 0.0;
+        lm_arg[mt] = 0x7fffffff;
+      }
+    };
     while (next_frag(p, passes, it, f)) {
       const int m0 = it.pass * BN;
       const int mrows = min(BN, M - m0);
       const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
       const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q * 32) << 16);
-      if (!wait_bounded(TFULL(acc), use & 1u, abort_v, p.status)) break;
+      if (!__all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status))) break;
       tc_fence_after();
       const int rin = f.arow + q * 32 + lane;  // row within the weight segment
       const bool col_ok = rin < p.seg_rows[f.seg];
       const size_t col = (size_t)(p.seg_col0[f.seg] + rin);
       if (p.epi_mode == 1) {
-        // softmax statistics of this tile's 128 vocabulary entries per token
-        for (int c = 0; c < mrows; c += 16) {
-          float v[16];
-          tmem_ld16(tacc + (uint32_t)c, v);
+        // LM head: this thread owns token m = mt * 128 + (TMEM lane) and folds the
+        // tile's 128 logits into its running (max, sum of exp, lowest argmax);
+        // tiles arrive in increasing vocabulary order, so on equal maxima the
+        // earlier (lower) id is kept
+        const int vbase = f.tile * 128;
+        if (it.pass != lm_pass) {
+          lm_flush(lm_pass);
+          lm_pass = it.pass;
+        }
+        for (int mt = 0; mt < (mrows > 128 ? 2 : 1); ++mt) {
+          const uint32_t tm = tmem + acc * (uint32_t)BN + (uint32_t)(mt * 128) + ((uint32_t)(q * 32) << 16);
+          float &RM = lm_max[mt];
+          double &RS = lm_sum[mt];
+          int &RI = lm_arg[mt];
+          for (int c = 0; c < 128; c += 16) {
+            float v[16];
+            tmem_ld16(tm + (uint32_t)c, v);
+            float cm = -INFINITY;
+            int cj = 0;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float mx = col_ok ? v[j] : -INFINITY;
-            int ix = col_ok ? (int)col : 0x7fffffff;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              const float om = __shfl_xor_sync(0xffffffffu, mx, o);
-              const int oi = __shfl_xor_sync(0xffffffffu, ix, o);
-              if (om > mx || (om == mx && oi < ix)) { mx = om; ix = oi; }
+            for (int j = 0; j < 16; ++j) {
+              const bool ok = vbase + c + j < p.seg_rows[0];
+              v[j] = ok ? v[j] : -INFINITY;
+              if (v[j] > cm) { cm = v[j]; cj = j; }
             }
-            float e = col_ok ? expf(v[j] - mx) : 0.f;
+            // no divergent exit from this loop: tmem_ld16 is warp-collective
+            if (cm > RM) {
+              RS = (RM == -INFINITY) ? 0.0 : RS * (double)expf(RM - cm);
+              RM = cm;
+              RI = vbase + c + cj;
+            }
+            if (RM != -INFINITY) {
+              float e = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) e += __shfl_xor_sync(0xffffffffu, e, o);
-            if (lane == j) {  // lane j keeps column c + j of this warp
-              smx_w[q][j] = make_float2(mx, e);
-              smx_i[q][j] = ix;
+              for (int j = 0; j < 16; ++j) e += expf(v[j] - RM);
+              RS += (double)e;
             }
           }
-          epi_bar();
-          if (warp == 2 && lane < 16 && c + lane < mrows) {  // merge the 4 lane quarters of column c + lane
-            float M4 = -INFINITY;
-            int I4 = 0x7fffffff;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const float2 t = smx_w[w][lane];
-              if (t.x > M4 || (t.x == M4 && smx_i[w][lane] < I4)) { M4 = t.x; I4 = smx_i[w][lane]; }
-            }
-            float S4 = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const float2 t = smx_w[w][lane];
-              if (t.x != -INFINITY) S4 += t.y * expf(t.x - M4);
-            }
-            const size_t o = (size_t)f.tile * p.ldm + (size_t)(m0 + c + lane);
-            p.smx[o] = make_float2(M4, S4);
-            p.smx_arg[o] = I4;
-          }
-          epi_bar();
         }
         tc_fence_before();
         __syncwarp();
@@ -487,6 +381,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
       ++nfrag;
     }
+    if (p.epi_mode == 1) lm_flush(lm_pass);
   }
 #undef FULL_A
 #undef EMPTY_A

@@ -12,6 +12,7 @@ namespace dcu {
 
 static constexpr int kSelThreads = 1024;
 static constexpr int kMaxSeq = 16384;
+static constexpr int kSelRankMax = 256;  // candidates ranked directly (else radix select)
 
 // ------------------------------------------------------------------ budget split
 // [DLLM] "关键设计 1", the budget equation B^l = (B_layer * L) s^l / sum_k s^k,
@@ -98,12 +99,14 @@ __global__ void __launch_bounds__(kSelThreads)
              float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
              int32_t *__restrict__ done, int32_t *__restrict__ seq_off, int32_t *__restrict__ status) {
   pdl_enter();
-  extern __shared__ uint8_t smem[];
+  extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *sd = reinterpret_cast<uint32_t *>(smem);     // [N] d bits
   uint8_t *flag = smem + (size_t)N * sizeof(uint32_t);   // [N] 0 none, 1 window, 2 top-B
   __shared__ int hist[256];
   __shared__ int red_i[32];
   __shared__ double red_d[32];
+  __shared__ uint32_t cbits[kSelRankMax];
+  __shared__ int cidx[kSelRankMax];
   __shared__ int s_bin, s_rem;
   __shared__ bool s_last;
 
@@ -111,17 +114,13 @@ __global__ void __launch_bounds__(kSelThreads)
   const int tid = threadIdx.x, nthr = blockDim.x;
   const float *db = d + (size_t)b * N;
 
-  double acc = 0.0;
   for (int i = tid; i < N; i += nthr) {
-    float v = db[i];
-    sd[i] = __float_as_uint(v);
+    sd[i] = __float_as_uint(db[i]);
     flag[i] = 0;
-    acc += (double)v;
   }
   if (d_next_zero)
     for (int i = tid; i < N; i += nthr) d_next_zero[(size_t)b * N + i] = 0.f;
-  acc = block_sum(acc, red_d);
-  if (tid == 0) s_out[(size_t)b * s_stride] = (float)(acc / (double)N);
+  __syncthreads();
 
   // forced window
   int nk = nkeys[b];
@@ -145,9 +144,17 @@ __global__ void __launch_bounds__(kSelThreads)
     }
   }
   __syncthreads();
-  int inW = 0;
-  for (int i = tid; i < N; i += nthr) inW += (flag[i] == 1);
-  inW = block_sum(inW, red_i);
+  int inW = 0, nz = 0;
+  {
+    double acc = 0.0;
+    for (int i = tid; i < N; i += nthr) acc += (double)__uint_as_float(sd[i]);
+    acc = block_sum(acc, red_d);
+    if (tid == 0) s_out[(size_t)b * s_stride] = (float)(acc / (double)N);
+    for (int i = tid; i < N; i += nthr) inW += (flag[i] == 1);
+    inW = block_sum(inW, red_i);
+    for (int i = tid; i < N; i += nthr) nz += (flag[i] == 0 && sd[i] != 0u);
+    nz = block_sum(nz, red_i);
+  }
   const int avail = N - inW;
   int k = budgets[(size_t)b * budget_stride];
   k = k < 0 ? 0 : (k > avail ? avail : k);
@@ -155,14 +162,35 @@ __global__ void __launch_bounds__(kSelThreads)
   uint32_t thr = 0xffffffffu;  // select d > thr, plus `need` ties at thr
   int need = 0;
   bool take_all = (k == avail);
-  int nz = 0;  // candidates with d > 0: when they all fit, the threshold is 0
-  if (k > 0 && !take_all) {
-    for (int i = tid; i < N; i += nthr) nz += (flag[i] == 0 && sd[i] != 0u);
-    nz = block_sum(nz, red_i);
-  }
-  if (k > 0 && !take_all && nz <= k) {
+  if (k > 0 && !take_all && nz <= k) {  // every positive d fits: the threshold is 0
     thr = 0u;
     need = k - nz;
+  } else if (k > 0 && !take_all && nz <= kSelRankMax) {
+    // few candidates (typically the rows the previous layer recomputed): exact
+    // ranks by (d desc, index asc) over the compacted candidate list
+    const int chunk = (N + nthr - 1) / nthr;
+    const int i0 = tid * chunk, i1 = min(N, i0 + chunk);
+    int mine = 0;
+    for (int i = i0; i < i1; ++i) mine += (flag[i] == 0 && sd[i] != 0u);
+    int tot;
+    int pos = block_exclusive_scan(mine, red_i, &tot);
+    for (int i = i0; i < i1; ++i)
+      if (flag[i] == 0 && sd[i] != 0u) {
+        cidx[pos] = i;
+        cbits[pos] = sd[i];
+        ++pos;
+      }
+    __syncthreads();
+    for (int c = tid; c < nz; c += nthr) {
+      const uint32_t v = cbits[c];
+      int rank = 0;
+      for (int j = 0; j < nz; ++j) {
+        const uint32_t w = cbits[j];
+        rank += (w > v) || (w == v && j < c);
+      }
+      if (rank < k) flag[cidx[c]] = 2;
+    }
+    __syncthreads();  // thr / need keep their defaults: the marking below adds nothing
   } else if (k > 0 && !take_all) {
     uint32_t prefix = 0, mask = 0;
     int rem = k;

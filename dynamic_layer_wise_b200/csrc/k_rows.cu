@@ -144,7 +144,9 @@ cudaError_t launch_cosine_distance(int dtype, const void *x, const void *y, cons
 }
 
 // ------------------------------------------------------------------ gather + RMSNorm
-// xs[r] = T(H[rowmap[r]] / sqrt(mean(H^2) + eps) * g) for r < *m_total.
+// xs[r] = T(H[rowmap[r]] / sqrt(mean(H^2) + eps) * g) for r < *m_total.  The
+// row stays in registers between the sum of squares and the scaling (rows of
+// up to 256 threads x 4 vectors; longer rows are re-read).
 template <class T>
 __global__ void k_gather_norm(const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
                               const T *__restrict__ H, const float *__restrict__ g, float eps, int D,
@@ -152,11 +154,23 @@ __global__ void k_gather_norm(const int32_t *__restrict__ rowmap, const int32_t 
   pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
+  constexpr int KEEP = 4;
   const int M = *m_total;
+  const int step = blockDim.x * VN;
   for (int r = blockIdx.x; r < M; r += gridDim.x) {
     const T *x = H + (size_t)rowmap[r] * D;
+    float keep[KEEP][VN];
     double ss = 0;
-    for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
+#pragma unroll
+    for (int q = 0; q < KEEP; ++q) {
+      const int j = threadIdx.x * VN + q * step;
+      if (j < D) {
+        load_vec(x + j, keep[q]);
+#pragma unroll
+        for (int i = 0; i < VN; ++i) ss += (double)keep[q][i] * (double)keep[q][i];
+      }
+    }
+    for (int j = threadIdx.x * VN + KEEP * step; j < D; j += step) {
       float v[VN];
       load_vec(x + j, v);
 #pragma unroll
@@ -165,7 +179,16 @@ __global__ void k_gather_norm(const int32_t *__restrict__ rowmap, const int32_t 
     ss = block_sum(ss, red);
     const float inv = (float)(1.0 / sqrt(ss / (double)D + (double)eps));
     T *o = xs + (size_t)r * D;
-    for (int j = threadIdx.x * VN; j < D; j += blockDim.x * VN) {
+#pragma unroll
+    for (int q = 0; q < KEEP; ++q) {
+      const int j = threadIdx.x * VN + q * step;
+      if (j < D) {
+#pragma unroll
+        for (int i = 0; i < VN; ++i) keep[q][i] = keep[q][i] * inv * g[j + i];
+        store_vec(o + j, keep[q]);
+      }
+    }
+    for (int j = threadIdx.x * VN + KEEP * step; j < D; j += step) {
       float v[VN];
       load_vec(x + j, v);
 #pragma unroll

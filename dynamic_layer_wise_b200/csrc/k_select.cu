@@ -113,6 +113,9 @@ __global__ void __launch_bounds__(kSelThreads)
   const int b = blockIdx.x;
   const int tid = threadIdx.x, nthr = blockDim.x;
   const float *db = d + (size_t)b * N;
+  // independent loads first, so their latencies overlap
+  const int nk_in = nkeys[b];
+  const int k_in = budgets[(size_t)b * budget_stride];
 
   for (int i = tid; i < N; i += nthr) {
     sd[i] = __float_as_uint(db[i]);
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(kSelThreads)
   __syncthreads();
 
   // forced window
-  int nk = nkeys[b];
+  int nk = nk_in;
   if (nk < 0 || nk > N) {
     if (tid == 0 && status) atomicOr(status, DCU_ST_BAD_KEY);
     nk = nk < 0 ? 0 : N;
@@ -156,7 +159,7 @@ __global__ void __launch_bounds__(kSelThreads)
     nz = block_sum(nz, red_i);
   }
   const int avail = N - inW;
-  int k = budgets[(size_t)b * budget_stride];
+  int k = k_in;
   k = k < 0 ? 0 : (k > avail ? avail : k);
 
   uint32_t thr = 0xffffffffu;  // select d > thr, plus `need` ties at thr
@@ -274,6 +277,25 @@ __global__ void __launch_bounds__(kSelThreads)
   for (int i = i0; i < i1; ++i) ns += (flag[i] != 0);
   int pos = block_exclusive_scan(ns, red_i, &tot);
   int32_t *ib = idx + (size_t)b * N;
+  if (rowmap != nullptr && B == 1) {
+    // one sequence: its selection is the packed row plan (offset 0), no
+    // cross-CTA step needed
+    for (int i = i0; i < i1; ++i)
+      if (flag[i] != 0) {
+        ib[pos] = i;
+        rowmap[pos] = i;
+        ++pos;
+      }
+    if (tid == 0) {
+      count[0] = tot;
+      if (seq_off) {
+        seq_off[0] = 0;
+        seq_off[1] = tot;
+      }
+      *m_total = tot;
+    }
+    return;
+  }
   for (int i = i0; i < i1; ++i)
     if (flag[i] != 0) ib[pos++] = i;
   if (tid == 0) count[b] = tot;

@@ -694,14 +694,14 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
   return DCU_OK;
 }
 
-int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
-                   int32_t *out_count, cudaStream_t s) {
+int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_len, uint8_t *masked, int32_t *ids,
+                   int32_t *out_pos, int32_t *out_count, cudaStream_t s) {
   const dcu_cfg &g = c->cfg;
   const int cap = (int)c->cap;
   {
     {
       Prof p(c, DCU_K_LMHEAD, s);
-      LAUNCH(c, launch_plan_masked(masked, c->B, c->N, c->mrow, c->m_masked(), s));
+      LAUNCH(c, launch_plan_masked(masked, c->B, c->N, gen_start, block_len, c->mrow, c->m_masked(), s));
     }
     {
       Prof p(c, DCU_K_LMHEAD, s);
@@ -752,7 +752,8 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, uint8_t *masked, int32_t *
   }
   {
     Prof p(c, DCU_K_COMMIT, s);
-    LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, out_pos, out_count, s));
+    LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, gen_start, block_len,
+                                 out_pos, out_count, s));
   }
   return DCU_OK;
 }
@@ -834,13 +835,16 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
   return rc;
 }
 
-int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
-                  int32_t *out_count, dcu_stream_t stream) {
+int commit_select_block(dcu_ctx *c, int32_t rule, float param, int32_t gen_start, int32_t block_len,
+                        uint8_t *masked, int32_t *ids, int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {
   if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
   if (!c->have_cache) return fail(c, DCU_ESTATE, "commit_select before dcu_full_forward");
   if (rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR)
     return fail(c, DCU_EINVAL, "rule must be DCU_FRECHET, DCU_THRESHOLD or DCU_FACTOR");
   if (!masked || !ids || !out_pos || !out_count) return fail(c, DCU_EINVAL, "a buffer is NULL");
+  if (block_len > 0 && (gen_start < 0 || gen_start >= c->N))
+    return fail(c, DCU_EINVAL, "gen_start must lie in [0, N) when block_len > 0");
+  if (block_len < 0) block_len = 0;
   uint32_t pbits;
   memcpy(&pbits, &param, 4);
   const uint64_t key[10] = {2,
@@ -852,10 +856,15 @@ int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_
                             (uint64_t)(uintptr_t)out_count,
                             ((uint64_t)c->B << 32) | (uint64_t)c->N,
                             (uint64_t)(c->prof_max > 0),
-                            0};
+                            ((uint64_t)(uint32_t)gen_start << 32) | (uint64_t)(uint32_t)block_len};
   return run_graphed(c, key, (cudaStream_t)stream, [&](cudaStream_t s) {
-    return enqueue_commit(c, rule, param, masked, ids, out_pos, out_count, s);
+    return enqueue_commit(c, rule, param, gen_start, block_len, masked, ids, out_pos, out_count, s);
   });
+}
+
+int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
+                  int32_t *out_count, dcu_stream_t stream) {
+  return commit_select_block(c, rule, param, 0, 0, masked, ids, out_pos, out_count, stream);
 }
 
 int dcu_set_graphs(dcu_ctx *c, int32_t on) {
@@ -906,14 +915,20 @@ int dcu_cosine_distance(const void *x, const void *y, const float *gain, int64_t
   return DCU_OK;
 }
 
+int dcu_commit_rule_block(int32_t rule, float param, int32_t gen_start, int32_t block_len, const float *conf,
+                          const int32_t *argmax, uint8_t *masked, int32_t *ids, int32_t B, int32_t N,
+                          int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {
+  if ((rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR) || !conf || !argmax || !masked || !ids ||
+      !out_pos || !out_count || B <= 0 || N <= 0 || N > 16384 || (block_len > 0 && (gen_start < 0 || gen_start >= N)))
+    return fail(nullptr, DCU_EINVAL, "dcu_commit_rule: bad argument");
+  CK(nullptr, launch_commit_rule(rule, param, conf, argmax, masked, ids, B, N, gen_start, block_len > 0 ? block_len : 0,
+                                 out_pos, out_count, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
 int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t *argmax, uint8_t *masked,
                     int32_t *ids, int32_t B, int32_t N, int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {
-  if ((rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR) || !conf || !argmax || !masked || !ids ||
-      !out_pos || !out_count || B <= 0 || N <= 0 || N > 16384)
-    return fail(nullptr, DCU_EINVAL, "dcu_commit_rule: bad argument");
-  CK(nullptr, launch_commit_rule(rule, param, conf, argmax, masked, ids, B, N, out_pos, out_count,
-                                 (cudaStream_t)stream));
-  return DCU_OK;
+  return dcu_commit_rule_block(rule, param, 0, 0, conf, argmax, masked, ids, B, N, out_pos, out_count, stream);
 }
 
 int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout, int32_t dtype, float *Y,

@@ -359,25 +359,60 @@ cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int
 }
 
 // Masked positions of all sequences, in (b, i) order, as packed rows.
-__global__ void __launch_bounds__(1024) k_plan_masked(const uint8_t *__restrict__ masked, int B, int N,
-                                                      int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total) {
+// Open block of the block-wise schedule ([README] "Quick Start": generate_mode
+// "default"): generation positions from gen_start are cut into blocks of
+// block_len and only the leftmost block that still holds a masked position is
+// open.  first = that masked position (N when none is left); [b0, b1) out.
+__device__ __forceinline__ void open_block(int first, int N, int gen_start, int block_len, int &b0, int &b1) {
+  if (first >= N) {
+    b0 = b1 = N;
+    return;
+  }
+  b0 = gen_start + (first - gen_start) / block_len * block_len;
+  b1 = min(N, b0 + block_len);
+}
+
+// Packed rows of the commit's candidates: every masked position, or with
+// block_len > 0 the masked positions of each sequence's open block.
+__global__ void __launch_bounds__(1024) k_plan_masked(const uint8_t *__restrict__ masked, int B, int N, int gen_start,
+                                                      int block_len, int32_t *__restrict__ rowmap,
+                                                      int32_t *__restrict__ m_total) {
   pdl_enter();
   __shared__ int red[32];
+  __shared__ int first[256];  // B <= 255
   const int BN = B * N, nthr = blockDim.x, tid = threadIdx.x;
+  if (block_len > 0) {
+    for (int b = tid; b < B; b += nthr) first[b] = N;
+    __syncthreads();
+    for (int i = tid; i < BN; i += nthr) {
+      const int b = i / N, j = i - b * N;
+      if (j >= gen_start && masked[i]) atomicMin(&first[b], j);
+    }
+    __syncthreads();
+  }
+  auto open = [&](int i) -> bool {
+    if (!masked[i]) return false;
+    if (block_len <= 0) return true;
+    const int b = i / N, j = i - b * N;
+    int b0, b1;
+    open_block(first[b], N, gen_start, block_len, b0, b1);
+    return j >= b0 && j < b1;
+  };
   const int chunk = (BN + nthr - 1) / nthr;
   const int i0 = tid * chunk, i1 = min(BN, i0 + chunk);
   int c = 0;
-  for (int i = i0; i < i1; ++i) c += masked[i] != 0;
+  for (int i = i0; i < i1; ++i) c += open(i);
   int tot;
   int pos = block_exclusive_scan(c, red, &tot);
   for (int i = i0; i < i1; ++i)
-    if (masked[i]) rowmap[pos++] = i;
+    if (open(i)) rowmap[pos++] = i;
   if (tid == 0) *m_total = tot;
 }
 
-cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
-                               cudaStream_t s) {
-  launch_pdl(k_plan_masked, 1, 1024, 0, s, masked, B, N, rowmap, m_total);
+cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int gen_start, int block_len, int32_t *rowmap,
+                               int32_t *m_total, cudaStream_t s) {
+  if (B > 255) return cudaErrorInvalidValue;
+  launch_pdl(k_plan_masked, 1, 1024, 0, s, masked, B, N, gen_start, block_len, rowmap, m_total);
   return cudaGetLastError();
 }
 
@@ -391,26 +426,39 @@ cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *row
 // commit the first n*: ids <- argmax, masked <- 0, out_positions, out_count.
 __global__ void __launch_bounds__(1024)
     k_commit_rule(int rule, float param, const float *__restrict__ conf, const int32_t *__restrict__ amax,
-                  uint8_t *__restrict__ masked, int32_t *__restrict__ ids, int N, int32_t *__restrict__ out_pos,
-                  int32_t *__restrict__ out_count) {
+                  uint8_t *__restrict__ masked, int32_t *__restrict__ ids, int N, int gen_start, int block_len,
+                  int32_t *__restrict__ out_pos, int32_t *__restrict__ out_count) {
   pdl_enter();
   extern __shared__ uint64_t keys[];  // [P]
   __shared__ int red[32];
   __shared__ double redd[32];
-  __shared__ int s_best;
+  __shared__ int s_best, s_first;
   const int b = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
   const uint8_t *mb = masked + (size_t)b * N;
   const float *cb = conf + (size_t)b * N;
-
-  // compact the masked positions (index order) into keys
   const int chunk = (N + nthr - 1) / nthr;
   const int i0 = tid * chunk, i1 = min(N, i0 + chunk);
+
+  // candidates: the masked positions, or those of the open block
+  int b0 = 0, b1 = N;
+  if (block_len > 0) {
+    if (tid == 0) s_first = N;
+    __syncthreads();
+    for (int i = max(i0, gen_start); i < i1; ++i)
+      if (mb[i]) {
+        atomicMin(&s_first, i);
+        break;
+      }
+    __syncthreads();
+    open_block(s_first, N, gen_start, block_len, b0, b1);
+  }
+  // compact the candidates (index order) into keys
   int c = 0;
-  for (int i = i0; i < i1; ++i) c += mb[i] != 0;
+  for (int i = i0; i < i1; ++i) c += (mb[i] != 0 && i >= b0 && i < b1);
   int m;
   int pos = block_exclusive_scan(c, red, &m);
   for (int i = i0; i < i1; ++i)
-    if (mb[i]) keys[pos++] = ((uint64_t)__float_as_uint(cb[i]) << 32) | (uint64_t)(~(uint32_t)i);
+    if (mb[i] && i >= b0 && i < b1) keys[pos++] = ((uint64_t)__float_as_uint(cb[i]) << 32) | (uint64_t)(~(uint32_t)i);
   int P = 1;
   while (P < m) P <<= 1;
   for (int t = m + tid; t < P; t += nthr) keys[t] = 0ull;
@@ -504,7 +552,8 @@ __global__ void __launch_bounds__(1024)
 }
 
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
-                               int32_t *ids, int B, int N, int32_t *out_pos, int32_t *out_count, cudaStream_t s) {
+                               int32_t *ids, int B, int N, int gen_start, int block_len, int32_t *out_pos,
+                               int32_t *out_count, cudaStream_t s) {
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   int P = 1;
   while (P < N) P <<= 1;
@@ -515,8 +564,8 @@ cudaError_t launch_commit_rule(int rule, float param, const float *conf, const i
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  launch_pdl(k_commit_rule, B, 1024, (size_t)P * sizeof(uint64_t), s, rule, param, conf, amax, masked, ids, N, out_pos,
-                                                               out_count);
+  launch_pdl(k_commit_rule, B, 1024, (size_t)P * sizeof(uint64_t), s, rule, param, conf, amax, masked, ids, N,
+             gen_start, block_len, out_pos, out_count);
   return cudaGetLastError();
 }
 

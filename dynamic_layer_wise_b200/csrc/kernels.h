@@ -54,10 +54,11 @@ cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nk
                           int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s);
 // rowmap = identity over B * N rows; seq_off[b] = b * N (B <= 255)
 cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off, cudaStream_t s);
-cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int32_t *rowmap, int32_t *m_total,
-                               cudaStream_t s);
+cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int gen_start, int block_len, int32_t *rowmap,
+                               int32_t *m_total, cudaStream_t s);
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
-                               int32_t *ids, int B, int N, int32_t *out_pos, int32_t *out_count, cudaStream_t s);
+                               int32_t *ids, int B, int N, int gen_start, int block_len, int32_t *out_pos,
+                               int32_t *out_count, cudaStream_t s);
 
 // ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total (m < m_cap when m_total is null)
 cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,

@@ -61,11 +61,13 @@ _SIGS = {
     "dcu_full_forward": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "dcu_step": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _vp]),
     "commit_select": (_i32, [_vp, _i32, _f32, _vp, _vp, _vp, _vp, _vp]),
+    "commit_select_block": (_i32, [_vp, _i32, _f32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "dcu_status": (_i32, [_vp, _vp, ctypes.POINTER(_i32)]),
     "dcu_budget_split": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp]),
     "dcu_select_tokens": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "dcu_cosine_distance": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     "dcu_commit_rule": (_i32, [_i32, _f32, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
+    "dcu_commit_rule_block": (_i32, [_i32, _f32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
     "dcu_tensor_bytes": (_i32, [_vp, _i32, ctypes.POINTER(_i64)]),
     "dcu_get_tensor": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
     "dcu_set_tensor": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
@@ -196,6 +198,15 @@ def commit_select(ctx: Context, rule: int, param: float, masked, token_ids, out_
                                _ptr(out_positions), _ptr(out_count), _stream(stream)), ctx.handle)
 
 
+def commit_select_block(ctx: Context, rule: int, param: float, gen_start: int, block_len: int, masked, token_ids,
+                        out_positions, out_count, stream=None):
+    assert masked.dtype == torch.uint8 and token_ids.dtype == torch.int32
+    assert out_positions.dtype == torch.int32 and out_count.dtype == torch.int32
+    _check(lib().commit_select_block(ctx.handle, int(rule), float(param), int(gen_start), int(block_len),
+                                     _ptr(masked), _ptr(token_ids), _ptr(out_positions), _ptr(out_count),
+                                     _stream(stream)), ctx.handle)
+
+
 def dcu_status(ctx: Context, stream=None) -> int:
     bits = _i32(0)
     rc = lib().dcu_status(ctx.handle, _stream(stream), ctypes.byref(bits))
@@ -237,6 +248,14 @@ def dcu_commit_rule(rule: int, param: float, conf, argmax, masked, token_ids, ou
     B, N = conf.shape
     _check(lib().dcu_commit_rule(int(rule), float(param), _ptr(conf), _ptr(argmax), _ptr(masked), _ptr(token_ids),
                                  B, N, _ptr(out_positions), _ptr(out_count), _stream(stream)))
+
+
+def dcu_commit_rule_block(rule: int, param: float, gen_start: int, block_len: int, conf, argmax, masked, token_ids,
+                          out_positions, out_count, stream=None):
+    B, N = conf.shape
+    _check(lib().dcu_commit_rule_block(int(rule), float(param), int(gen_start), int(block_len), _ptr(conf),
+                                       _ptr(argmax), _ptr(masked), _ptr(token_ids), B, N, _ptr(out_positions),
+                                       _ptr(out_count), _stream(stream)))
 
 
 _KIND_DTYPE = {DCU_T_D: torch.float32, DCU_T_S: torch.float32, DCU_T_S_PREV: torch.float32,

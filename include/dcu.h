@@ -139,6 +139,18 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
 int commit_select(dcu_ctx *ctx, int32_t rule, float param, uint8_t *masked, int32_t *token_ids,
                   int32_t *out_positions, int32_t *out_count, dcu_stream_t stream);
 
+/* commit_select under the block-wise schedule ([README] "Quick Start":
+ * generate_mode "default", fixed-schedule block-wise decoding; [FRECHET]
+ * "实验关键数据": block size 32): per sequence, the positions from gen_start on
+ * are cut into consecutive blocks of block_len and only the masked positions
+ * of the leftmost block that still holds one are candidates (LM head and
+ * rule both); a sequence with no masked position at or after gen_start
+ * commits nothing.  block_len <= 0 is commit_select.  gen_start must lie in
+ * [0, N) when block_len > 0 (DCU_EINVAL otherwise). */
+int commit_select_block(dcu_ctx *ctx, int32_t rule, float param, int32_t gen_start, int32_t block_len,
+                        uint8_t *masked, int32_t *token_ids, int32_t *out_positions, int32_t *out_count,
+                        dcu_stream_t stream);
+
 /* dcu_step and commit_select are captured into CUDA graphs (once per distinct
  * set of pointers, budgets and active shape; at most 16 kept, least recently
  * used evicted) and replayed on the caller's stream.  on = 0 launches every
@@ -184,6 +196,12 @@ int dcu_cosine_distance(const void *x, const void *y, const float *gain, int64_t
 int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t *argmax, uint8_t *masked,
                     int32_t *token_ids, int32_t B, int32_t N, int32_t *out_positions, int32_t *out_count,
                     dcu_stream_t stream);
+
+/* dcu_commit_rule restricted to each sequence's open block (as in
+ * commit_select_block; block_len <= 0: no restriction). */
+int dcu_commit_rule_block(int32_t rule, float param, int32_t gen_start, int32_t block_len, const float *conf,
+                          const int32_t *argmax, uint8_t *masked, int32_t *token_ids, int32_t B, int32_t N,
+                          int32_t *out_positions, int32_t *out_count, dcu_stream_t stream);
 
 /* Y[m][n] = sum_k X[m][k] W[n][k] in fp32: the recompute GEMM (tcgen05 with
  * TMA-staged operands for bf16, CUDA cores for float32) as a stateless call.

@@ -482,15 +482,41 @@ def rule_count(rule: int, c_sorted, param: float) -> int:
     raise ValueError(rule)
 
 
-def commit(c: np.ndarray, amax: np.ndarray, masked: np.ndarray, ids: np.ndarray, rule: int, param: float):
+def active_block(masked: np.ndarray, gen_start: int, block_len: int):
+    """Block-wise schedule ([README] "Quick Start": generate_mode "default",
+    fixed-schedule block-wise decoding; [FRECHET] "实验关键数据": block size 32):
+    the generation region from gen_start is cut into consecutive blocks of
+    block_len positions and only the leftmost block that still holds a masked
+    position is open for commits.  Returns its [b0, b1), or None when no masked
+    position is left at or after gen_start.  block_len <= 0: no blocks (the
+    whole sequence is open)."""
+    masked = np.asarray(masked, dtype=bool)
+    N = masked.shape[0]
+    if block_len <= 0:
+        return 0, N
+    left = np.flatnonzero(masked[gen_start:])
+    if len(left) == 0:
+        return None
+    first = gen_start + int(left[0])
+    b0 = gen_start + (first - gen_start) // block_len * block_len
+    return b0, min(N, b0 + block_len)
+
+
+def commit(c: np.ndarray, amax: np.ndarray, masked: np.ndarray, ids: np.ndarray, rule: int, param: float,
+           gen_start: int = 0, block_len: int = 0):
     """Per-sequence commit ([FRECHET] "整体框架"): sort the masked positions by
     confidence (descending; ties -> lower position), take n* by the rule, set
-    their ids to the argmax and unmask them.
+    their ids to the argmax and unmask them.  With block_len > 0 only the
+    masked positions of the active block (see active_block) are candidates.
 
     c, amax: [N] values at every position (only masked ones are read).
     Returns (positions in descending-confidence order, new ids, new masked)."""
     masked = np.asarray(masked, dtype=bool)
-    pos = np.flatnonzero(masked)
+    blk = active_block(masked, gen_start, block_len)
+    open_ = np.zeros_like(masked)
+    if blk is not None:
+        open_[blk[0]:blk[1]] = True
+    pos = np.flatnonzero(masked & open_)
     cm = np.asarray(c, dtype=np.float32)[pos].astype(np.float64)
     order = pos[np.lexsort((pos, -cm))]
     n = rule_count(rule, np.asarray(c, dtype=np.float32)[order], param)

@@ -416,3 +416,57 @@ def test_rope_matches_transformers_rotate_half():
     rq, rk = ml.apply_rotary_pos_emb(x, torch.tensor(k).permute(1, 0, 2)[None], cos.double(), sin.double())
     np.testing.assert_allclose(O.rope(q, np.arange(N), 10000.0), rq[0].permute(1, 0, 2).numpy(), rtol=1e-6, atol=1e-6)
     np.testing.assert_allclose(O.rope(k, np.arange(N), 10000.0), rk[0].permute(1, 0, 2).numpy(), rtol=1e-6, atol=1e-6)
+
+
+# ---- block-wise schedule ([README] "Quick Start", generate_mode "default")
+
+def test_block_commit_worked_example():
+    """N = 10, generation from 4, blocks of 3: [4, 7) [7, 10).  Masked 5, 8, 9:
+    the open block is [4, 7), so only position 5 can be committed; once it is
+    unmasked the open block moves to [7, 10)."""
+    N = 10
+    masked = np.zeros(N, bool)
+    masked[[5, 8, 9]] = True
+    c = np.full(N, 0.5, np.float32)
+    c[[8, 9]] = 0.99                      # higher confidence outside the open block
+    amax = np.arange(N) + 100
+    ids = np.zeros(N, np.int64)
+    assert O.active_block(masked, 4, 3) == (4, 7)
+    pos, new_ids, new_masked = O.commit(c, amax, masked, ids, O.RULE_THRESHOLD, 0.9, gen_start=4, block_len=3)
+    assert list(pos) == [5] and new_ids[5] == 105 and not new_masked[5] and new_masked[8] and new_masked[9]
+    assert O.active_block(new_masked, 4, 3) == (7, 10)
+    pos2, _, m2 = O.commit(c, amax, new_masked, new_ids, O.RULE_THRESHOLD, 0.9, gen_start=4, block_len=3)
+    assert sorted(pos2) == [8, 9] and not m2.any()
+    assert O.active_block(m2, 4, 3) is None
+    assert len(O.commit(c, amax, m2, ids, O.RULE_FRECHET, 0.1, gen_start=4, block_len=3)[0]) == 0
+
+
+def test_block_commit_reduces_to_plain_commit_and_stays_in_block():
+    """A block covering the whole generation region is the plain commit; any
+    block size commits only inside the leftmost block that holds a masked
+    position (brute force over the blocks)."""
+    rng = np.random.default_rng(5)
+    for trial in range(200):
+        N = int(rng.integers(1, 60))
+        g0 = int(rng.integers(0, N))
+        masked = np.zeros(N, bool)
+        masked[g0:] = rng.random(N - g0) < 0.6
+        c = rng.choice([0.2, 0.5, 0.95, 0.99], N).astype(np.float32)
+        amax = rng.integers(0, 50, N)
+        ids = rng.integers(0, 50, N)
+        rule, param = [(O.RULE_FRECHET, 0.1), (O.RULE_THRESHOLD, 0.9), (O.RULE_FACTOR, 0.9)][trial % 3]
+        full = O.commit(c, amax, masked, ids, rule, param)
+        whole = O.commit(c, amax, masked, ids, rule, param, gen_start=g0, block_len=N)
+        np.testing.assert_array_equal(full[0], whole[0])
+        blen = int(rng.integers(1, 9))
+        pos, _, _ = O.commit(c, amax, masked, ids, rule, param, gen_start=g0, block_len=blen)
+        blocks = [(b, min(N, b + blen)) for b in range(g0, N, blen)]
+        open_ = next(((a, b) for a, b in blocks if masked[a:b].any()), None)
+        if open_ is None:
+            assert len(pos) == 0
+        else:
+            assert len(pos) >= 1 and all(open_[0] <= p < open_[1] and masked[p] for p in pos)
+            inside = np.flatnonzero(masked[open_[0]:open_[1]]) + open_[0]
+            ref = O.commit(np.where(np.isin(np.arange(N), inside), c, 0).astype(np.float32), amax,
+                           np.isin(np.arange(N), inside), ids, rule, param)
+            np.testing.assert_array_equal(pos, ref[0])

@@ -919,6 +919,12 @@ int dcu_cosine_distance(const void *x, const void *y, const float *gain, int64_t
   return DCU_OK;
 }
 
+int dcu_selftest_wait_timeout(int32_t *status, dcu_stream_t stream) {
+  if (!status) return fail(nullptr, DCU_EINVAL, "dcu_selftest_wait_timeout: status is NULL");
+  CK(nullptr, launch_wait_timeout_probe(status, (cudaStream_t)stream));
+  return DCU_OK;
+}
+
 int dcu_commit_rule_block(int32_t rule, float param, int32_t gen_start, int32_t block_len, const float *conf,
                           const int32_t *argmax, uint8_t *masked, int32_t *ids, int32_t B, int32_t N,
                           int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {

@@ -80,4 +80,7 @@ cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, co
                              int N, int H, int Hkv, int hd, const void *Kc, const void *Vc, void *out,
                              cudaStream_t s);
 
+// ---- self-test (k_selftest.cu): one bounded mbarrier wait that must expire
+cudaError_t launch_wait_timeout_probe(int32_t *status, cudaStream_t s);
+
 }  // namespace dcu

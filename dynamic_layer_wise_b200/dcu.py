@@ -68,6 +68,7 @@ _SIGS = {
     "dcu_cosine_distance": (_i32, [_vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     "dcu_commit_rule": (_i32, [_i32, _f32, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
     "dcu_commit_rule_block": (_i32, [_i32, _f32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _vp, _vp, _vp]),
+    "dcu_selftest_wait_timeout": (_i32, [_vp, _vp]),
     "dcu_tensor_bytes": (_i32, [_vp, _i32, ctypes.POINTER(_i64)]),
     "dcu_get_tensor": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
     "dcu_set_tensor": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
@@ -256,6 +257,12 @@ def dcu_commit_rule_block(rule: int, param: float, gen_start: int, block_len: in
     _check(lib().dcu_commit_rule_block(int(rule), float(param), int(gen_start), int(block_len), _ptr(conf),
                                        _ptr(argmax), _ptr(masked), _ptr(token_ids), B, N, _ptr(out_positions),
                                        _ptr(out_count), _stream(stream)))
+
+
+def dcu_selftest_wait_timeout(status, stream=None):
+    """One bounded device wait that must expire: sets DCU_ST_TIMEOUT in status."""
+    assert status.dtype == torch.int32
+    _check(lib().dcu_selftest_wait_timeout(_ptr(status), _stream(stream)))
 
 
 _KIND_DTYPE = {DCU_T_D: torch.float32, DCU_T_S: torch.float32, DCU_T_S_PREV: torch.float32,

@@ -197,6 +197,14 @@ int dcu_commit_rule(int32_t rule, float param, const float *conf, const int32_t 
                     int32_t *token_ids, int32_t B, int32_t N, int32_t *out_positions, int32_t *out_count,
                     dcu_stream_t stream);
 
+/* Self-test of the device-side failure detection (the pages have no
+ * counterpart): launches one CTA whose thread waits on an mbarrier that nothing
+ * arrives on.  The bounded wait gives up after its wall-clock limit (about 1 s)
+ * and ORs DCU_ST_TIMEOUT into *status (dev int32, caller-zeroed); bit 30 would
+ * mean the wait wrongly succeeded, bit 29 that the expiry did not raise the
+ * CTA's abort flag.  The kernel always finishes; the context stays usable. */
+int dcu_selftest_wait_timeout(int32_t *status, dcu_stream_t stream);
+
 /* dcu_commit_rule restricted to each sequence's open block (as in
  * commit_select_block; block_len <= 0: no restriction). */
 int dcu_commit_rule_block(int32_t rule, float param, int32_t gen_start, int32_t block_len, const float *conf,

@@ -175,3 +175,20 @@ def test_commit_rule_worked_profile():
         dcu.dcu_commit_rule(rule, param, c, amax, masked, ids, pos, cnt)
         assert cnt.item() == want
         assert list(pos[0, :want].cpu().numpy()) == [4, 3, 2, 1, 0][:want]
+
+
+def test_bounded_wait_expires_and_reports_timeout():
+    """Failure detection without a fault: a wait on a barrier that nothing
+    arrives on gives up after its wall-clock bound (~1 s), reports
+    DCU_ST_TIMEOUT and the kernel finishes; the context keeps working."""
+    import time
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    dcu.dcu_selftest_wait_timeout(status)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert status.item() == dcu.DCU_ST_TIMEOUT
+    assert 0.5 < dt < 10.0
+    x = torch.ones(4, device="cuda")
+    assert float((x * 2).sum().item()) == 8.0                  # the context is usable afterwards

@@ -374,7 +374,15 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
       const long long items = (long long)c->B * Hkv * qt_grid;
       int splits = (int)(c->num_sms / items);
       const int max_sp = (c->N + 63) / 64;
-      splits = splits < 1 ? 1 : (splits > kAttnMaxSplits ? kAttnMaxSplits : splits);
+      splits = splits < 1 ? 1 : splits;
+      // long sequences: the legacy-MMA attention is compute-bound, so when one
+      // wave leaves more than 2048 keys per CTA, cut them to <= 1024 even past
+      // one wave (the heavy query tiles then spread over all SMs instead of the
+      // few that hold them; measured +12 % attention at N = 8192, while at
+      // N = 2048 x 4 sequences the extra wave and merge cost 10 %)
+      if ((c->N + splits - 1) / splits > 2048)
+        while (splits < kAttnMaxSplits && (c->N + splits - 1) / splits > 1024) splits *= 2;
+      splits = splits > kAttnMaxSplits ? kAttnMaxSplits : splits;
       if (splits > max_sp) splits = max_sp;
       const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
       splits = (c->N + kc - 1) / kc;

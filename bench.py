@@ -83,55 +83,99 @@ def measured_peaks():
 # ---------------------------------------------------------------- clocks sampling
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons of the GPU
+    while running: NVML polled every 2 ms (so a timed region of ~0.1 s still
+    gets dozens of samples), else nvidia-smi every 100 ms.  The GPU is found by
+    the UUID of the CUDA device, so CUDA_VISIBLE_DEVICES cannot point it at
+    another GPU.  Read-only: no setting of the GPU is touched."""
 
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
         self.proc = None
-        self.lines = []
+        self.thread = None
+        self.stop_flag = threading.Event()
+        self.samples = []        # (sm_mhz, sm_max_mhz, set of reason names)
+        self.source = None
+
+    def _uuid(self):
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(self.index).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return None
 
     def start(self):
+        uuid = self._uuid()
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+            import pynvml as N
+            N.nvmlInit()
+            h = N.nvmlDeviceGetHandleByUUID(uuid) if uuid else N.nvmlDeviceGetHandleByIndex(self.index)
+            bits = {"hw_slowdown": getattr(N, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+                    "hw_thermal_slowdown": getattr(N, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+                    "sw_thermal_slowdown": getattr(N, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+                    "sw_power_cap": getattr(N, "nvmlClocksThrottleReasonSwPowerCap", 0x4)}
+            smax = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+
+            def poll():
+                while not self.stop_flag.is_set():
+                    try:
+                        sm = float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                        r = int(N.nvmlDeviceGetCurrentClocksThrottleReasons(h))
+                        self.samples.append((sm, smax, {n for n, b in bits.items() if r & b}))
+                    except Exception:
+                        pass
+                    time.sleep(self.period)
+
+            self.source = "nvml"
+            self.thread = threading.Thread(target=poll, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            pass
+        try:
+            ident = uuid or str(self.index)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={ident}", f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
         except Exception:
             self.proc = None
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
+            f = [x.strip() for x in line.strip().split(",")]
             if len(f) < 9:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                self.samples.append((float(f[1]), float(f[2]),
+                                     {n for n, v in zip(self.NAMES, f[5:9]) if v.lower() == "active"}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+
+    def stop(self) -> dict:
+        self.stop_flag.set()
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"], "samples": 0}
+        sm = [x[0] for x in self.samples]
+        reasons = set().union(*[x[2] for x in self.samples])
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "sm_mhz_min": min(sm), "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 # ---------------------------------------------------------------- CPU oracle sample
@@ -265,8 +309,8 @@ def profile_case_gemm(shape, reps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dcu", choices=["dcu", "reference"])
     ap.add_argument("--workload", default="llada8b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -372,19 +416,18 @@ def main():
         raise RuntimeError("device status word set during warm-up")
     masked_before = int(masked.sum().item())
     clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
     launches0 = dcu.dcu_launch_count(ctx)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.start()                                        # samples span the timed region only
     t0.record(stream)
     for _ in range(args.steps):
         step()
     t1.record(stream)
     torch.cuda.synchronize()
-    barrier()
     clk = clocks.stop()
+    barrier()
     ms_total = t0.elapsed_time(t1)
     launches = dcu.dcu_launch_count(ctx) - launches0
     committed = masked_before - int(masked.sum().item())
@@ -396,7 +439,10 @@ def main():
     # (2) per kernel class: a second timed pass of K steps whose graphs carry an
     # event pair around every launch (captured during its own warm-up)
     per_step_launches_guess = 2 + shape.n_layers * 12 + 6
-    dcu.dcu_profile_enable(ctx, (args.steps + args.warmup) * per_step_launches_guess)
+    # event slots for launches outside graphs (with graphs on, the captured
+    # graphs carry their own event nodes)
+    slots = (args.steps + args.warmup) if args.no_graphs else 2
+    dcu.dcu_profile_enable(ctx, slots * per_step_launches_guess)
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()

@@ -1047,6 +1047,10 @@ static int tensor_ptr(dcu_ctx *c, int kind, int layer, char **p, int64_t *bytes)
       *p = (char *)c->amax;
       *bytes = BN * 4;
       return DCU_OK;
+    case DCU_T_ATTN:
+      *p = c->attn;
+      *bytes = BN * g.n_heads * g.head_dim * (int64_t)c->esz;
+      return DCU_OK;
     default:
       return fail(c, DCU_EINVAL, "unknown tensor kind");
   }
@@ -1057,11 +1061,7 @@ int dcu_tensor_bytes(const dcu_ctx *cc, int32_t kind, int64_t *bytes) {
   dcu_ctx *c = const_cast<dcu_ctx *>(cc);
   if (!c || !bytes) return fail(nullptr, DCU_EINVAL, "ctx or bytes is NULL");
   char *p;
-  int layer = (kind == DCU_T_S || kind == DCU_T_S_PREV || kind == DCU_T_BUDGET || kind == DCU_T_CONF ||
-               kind == DCU_T_ARGMAX)
-                  ? 0
-                  : 0;
-  return tensor_ptr(c, kind, layer, &p, bytes);
+  return tensor_ptr(c, kind, 0, &p, bytes);  // every kind's size is the same at every layer
 }
 
 int dcu_get_tensor(dcu_ctx *c, int32_t kind, int32_t layer, void *dst, int64_t bytes, dcu_stream_t stream) {

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/dcu.h"
 
 namespace dcu {
@@ -164,6 +166,23 @@ inline cudaError_t launch_pdl(void (*kern)(Exp...), dim3 grid, dim3 block, size_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Act &&>(args)...);
+}
+
+// Raises the dynamic shared memory limit of kernel `kern` to `bytes` on the
+// current device, once per device: the attribute belongs to the device's copy
+// of the kernel, so a flag per process would leave a second GPU without it.
+// `done` holds one bit per device (devices 64 and up set it on every call);
+// setting the attribute twice is harmless, so concurrent first calls are safe.
+template <class... Exp>
+inline cudaError_t ensure_smem_limit(void (*kern)(Exp...), int bytes, std::atomic<uint64_t> &done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 // Row r of the packed recompute set -> global row b*N + i (written by the

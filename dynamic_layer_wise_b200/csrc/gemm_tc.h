@@ -69,6 +69,19 @@ struct TcParams {
   float2 *smx;
   int32_t *smx_arg;
   int ldm;
+  // L2 prefetch lookahead of the weight producer: with each TMA load of a
+  // weight tile it prefetches the tile pf_ahead tiles past the shared-memory
+  // ring into L2 (0: off), so more HBM requests are in flight than the ring holds.
+  int pf_ahead;
+  // Prefetch of the next GEMM's weights: after its last TMA load, CTA c
+  // prefetches into L2 the first nx_count (tile, k block) units of the ranges
+  // of CTAs c, c + grid, ... of the next GEMM's stream-K geometry nx_geo over
+  // its weight segments nx_a (0: off).  The next GEMM then finds them in L2.
+  CUtensorMap nx_a[3];
+  int nx_seg_tile0[4];
+  int nx_nseg;
+  SlotGeo nx_geo;
+  int nx_count;
 };
 
 // Row-major bf16 matrix [outer][inner] with row pitch row_bytes, box

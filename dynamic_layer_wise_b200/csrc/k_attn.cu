@@ -69,16 +69,9 @@ cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, co
                              cudaStream_t s) {
   if (hd > 256 || N > 16384) return cudaErrorInvalidValue;
   const size_t smem = (size_t)N * sizeof(float);
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e1 = cudaFuncSetAttribute(k_attn_rowhead<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          16384 * sizeof(float));
-    cudaError_t e2 = cudaFuncSetAttribute(k_attn_rowhead<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          16384 * sizeof(float));
-    if (e1 != cudaSuccess) return e1;
-    if (e2 != cudaSuccess) return e2;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr_bf16{0}, attr_f32{0};
+  if (cudaError_t e = ensure_smem_limit(k_attn_rowhead<bf16>, 16384 * (int)sizeof(float), attr_bf16)) return e;
+  if (cudaError_t e = ensure_smem_limit(k_attn_rowhead<float>, 16384 * (int)sizeof(float), attr_f32)) return e;
   long long items = (long long)cap * H;
   int grid = (int)(items < 148 * 16 ? items : 148 * 16);
   if (grid < 1) grid = 1;

@@ -431,20 +431,12 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
   const int grid = B * Hkv * splits * qt_grid;
   if (grid <= 0) return cudaSuccess;
   if (hd == 128) {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_attn_mma<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (cudaError_t e = ensure_smem_limit(k_attn_mma<128>, (int)smem, attr)) return e;
     launch_pdl(k_attn_mma<128>, grid, 256, smem, s, a);
   } else {
-    static bool attr = false;
-    if (!attr) {
-      cudaError_t e = cudaFuncSetAttribute(k_attn_mma<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    static std::atomic<uint64_t> attr{0};
+    if (cudaError_t e = ensure_smem_limit(k_attn_mma<64>, (int)smem, attr)) return e;
     launch_pdl(k_attn_mma<64>, grid, 256, smem, s, a);
   }
   cudaError_t e = cudaGetLastError();

@@ -166,10 +166,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       for (int s = 0; s < kTcMaxA; ++s) used[s] = false;
       KCursor ca;
       ca.start(p, passes, my_begin, my_end, BN, M);
-      int stage = 0;
+      // L2 prefetch cursor, pf_ahead tiles past the ring (the first SA loads
+      // are issued at once, so it starts at tile SA)
+      KCursor cp;
+      cp.start(p, passes, my_begin, my_end, BN, M);
+      const int look = p.pf_ahead > 0 ? SA + p.pf_ahead : 0;
+      int cp_idx = 0;
+      if (look > 0)
+        while (cp.valid && cp_idx < SA) {
+          cp.advance(p, passes, BN, M);
+          ++cp_idx;
+        }
+      int stage = 0, ld_idx = 0;
       uint32_t phase = 0;
       bool ok = true;
       while (ca.valid) {
+        while (look > 0 && cp.valid && cp_idx <= ld_idx + look) {
+          tma_prefetch_2d(&p.a[cp.f.seg], cp.kb * 64, cp.f.arow);
+          cp.advance(p, passes, BN, M);
+          ++cp_idx;
+        }
         if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
           ok = false;
           break;
@@ -179,14 +195,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         used[stage] = true;
         fill_parity[stage] = phase;
         ca.advance(p, passes, BN, M);
+        ++ld_idx;
         if (++stage == SA) {
           stage = 0;
           phase ^= 1u;
         }
       }
-      if (!ok)
+      if (!ok) {
         for (int s = 0; s < SA; ++s)
           if (used[s]) wait_drain(FULL_A(s), fill_parity[s]);
+      } else if (p.nx_count > 0) {
+        // the next GEMM's first weight tiles into L2 (fire and forget)
+        const int nkb = p.nx_geo.kblocks;
+        for (int c = blockIdx.x; c < p.nx_geo.grid; c += gridDim.x) {
+          const long long b = sk_begin(p.nx_geo, c), e0 = sk_begin(p.nx_geo, c + 1);
+          const long long e = e0 < b + p.nx_count ? e0 : b + p.nx_count;
+          for (long long x = b; x < e; ++x) {
+            const int t = (int)(x / nkb), kb = (int)(x - (long long)t * nkb);
+            int seg = 0;
+            while (seg + 1 < p.nx_nseg && t >= p.nx_seg_tile0[seg + 1]) ++seg;
+            tma_prefetch_2d(&p.nx_a[seg], kb * 64, (t - p.nx_seg_tile0[seg]) * 128);
+          }
+        }
+      }
     }
   } else if (warp == 6) {
     // activation producer: the packed rows are written by the previous launch
@@ -403,16 +434,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  // looked up once per process (a thread-safe static): the driver entry point
+  // does not depend on the device
+  static const EncodeTiledFn fn = [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+      return reinterpret_cast<EncodeTiledFn>(p);
+    return (EncodeTiledFn) nullptr;
+  }();
   return fn;
 }
 
@@ -433,12 +464,8 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
 
 template <int BN>
 static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTcSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  if (cudaError_t e = ensure_smem_limit(k_gemm_tc<BN>, (int)kTcSmem, smem_set)) return e;
   // programmatic dependent launch: the CTAs may start while the previous kernel
   // finishes; they wait (griddepcontrol.wait) before reading its outputs
   cudaLaunchConfig_t cfg = {};

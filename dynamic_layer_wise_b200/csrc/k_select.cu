@@ -329,12 +329,8 @@ cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nk
                           int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s) {
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   size_t smem = (size_t)N * 5;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSeq * 5);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (cudaError_t e = ensure_smem_limit(k_select, kMaxSeq * 5, attr)) return e;
   // short sequences: fewer threads make the ~25 block barriers cheaper
   const int threads = N <= 2048 ? 256 : kSelThreads;
   launch_pdl(k_select, B, threads, smem, s, d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
@@ -557,13 +553,8 @@ cudaError_t launch_commit_rule(int rule, float param, const float *conf, const i
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   int P = 1;
   while (P < N) P <<= 1;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_commit_rule, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxSeq * sizeof(uint64_t));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static std::atomic<uint64_t> attr{0};
+  if (cudaError_t e = ensure_smem_limit(k_commit_rule, kMaxSeq * (int)sizeof(uint64_t), attr)) return e;
   launch_pdl(k_commit_rule, B, 1024, (size_t)P * sizeof(uint64_t), s, rule, param, conf, amax, masked, ids, N,
              gen_start, block_len, out_pos, out_count);
   return cudaGetLastError();

@@ -85,8 +85,10 @@ __global__ void k_na_merge(const float *__restrict__ z, int ldz, int ncols, int 
       if (lane == 0) { smax[0] = best; sidx[0] = bi; }
     }
     __syncthreads();
+    // a chunk with no ordered maximum (every logit NaN) keeps its first id as
+    // the argmax; its sum is then NaN, which the confidence reports
     const float cmax = smax[0];
-    const int carg = sidx[0] + base;
+    const int carg = (sidx[0] == 0x7fffffff ? 0 : sidx[0]) + base;
     double s = 0.0;
     for (int v = threadIdx.x; v < ncols; v += blockDim.x) s += (double)expf(zr[v] - cmax);
     s = dcu::block_sum(s, sred);
@@ -127,6 +129,14 @@ extern "C" int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_
   if (!h_rows || !final_norm || !lm_head || !conf || !argmax || (dtype != DCU_F32 && dtype != DCU_BF16) ||
       m < 0 || D <= 0 || V <= 0 || D % 64 || !(rms_eps > 0.0f))
     return na_fail(DCU_EINVAL, "dcu_lm_confidence_noalloc: bad argument");
+  {
+    // the row, gain and weight loads are 16-byte vectors; outputs are 4-byte words
+    auto mis = [](const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) != 0; };
+    if (mis(h_rows, 16) || mis(final_norm, 16) || mis(lm_head, 16) || mis(conf, 4) || mis(argmax, 4))
+      return na_fail(DCU_EINVAL,
+                     "dcu_lm_confidence_noalloc: h_rows, final_norm and lm_head must be 16-byte aligned, "
+                     "conf and argmax 4-byte aligned");
+  }
   if (m > kNaMaxRows || D > kNaMaxD)
     return na_fail(DCU_ECAPACITY, "dcu_lm_confidence_noalloc: at most 256 rows per call and d_model <= 8192");
   if (m == 0) return DCU_OK;

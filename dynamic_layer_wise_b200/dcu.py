@@ -22,7 +22,7 @@ DCU_F32, DCU_BF16 = 0, 1
 DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR = 0, 1, 2
 DCU_WINDOW_INCLUSIVE, DCU_WINDOW_HALFOPEN = 0, 1
 (DCU_T_H, DCU_T_K, DCU_T_V, DCU_T_D, DCU_T_S, DCU_T_S_PREV, DCU_T_BUDGET, DCU_T_SEL, DCU_T_SEL_COUNT,
- DCU_T_CONF, DCU_T_ARGMAX) = range(11)
+ DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN) = range(12)
 (DCU_K_REFRESH, DCU_K_BUDGET, DCU_K_SELECT, DCU_K_GATHER, DCU_K_GEMM, DCU_K_EPILOGUE, DCU_K_ATTN, DCU_K_SCATTER,
  DCU_K_LMHEAD, DCU_K_COMMIT, DCU_K_COUNT) = range(11)
 
@@ -271,7 +271,7 @@ _KIND_DTYPE = {DCU_T_D: torch.float32, DCU_T_S: torch.float32, DCU_T_S_PREV: tor
 
 
 def _kind_dtype(ctx: Context, kind: int):
-    if kind in (DCU_T_H, DCU_T_K, DCU_T_V):
+    if kind in (DCU_T_H, DCU_T_K, DCU_T_V, DCU_T_ATTN):
         return torch.bfloat16 if ctx.cfg["dtype"] == DCU_BF16 else torch.float32
     return _KIND_DTYPE[kind]
 
@@ -316,6 +316,10 @@ def dcu_lm_confidence_noalloc(h_rows, final_norm, lm_head, rms_eps: float = 1e-5
     m, D = h_rows.shape
     V = lm_head.shape[0]
     dt = {torch.bfloat16: DCU_BF16, torch.float32: DCU_F32}[h_rows.dtype]
+    if lm_head.dtype != h_rows.dtype or lm_head.dim() != 2 or lm_head.shape[1] != D:
+        raise ValueError("lm_head must be [V][D] in the dtype of h_rows")
+    if final_norm.dtype != torch.float32 or final_norm.numel() != D:
+        raise ValueError("final_norm must be float32 [D]")
     conf = torch.empty(m, dtype=torch.float32, device=h_rows.device)
     amax = torch.empty(m, dtype=torch.int32, device=h_rows.device)
     _check(lib().dcu_lm_confidence_noalloc(_ptr(h_rows), _ptr(final_norm), _ptr(lm_head), m, D, V, dt,

@@ -251,6 +251,11 @@ int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_norm, const
 #define DCU_T_SEL_COUNT 8  /* layer 0..L-1 : [B] int32                    */
 #define DCU_T_CONF      9  /* [B][N] float, confidence of the last commit (masked positions) */
 #define DCU_T_ARGMAX   10  /* [B][N] int32, argmax of the last commit (masked positions)      */
+#define DCU_T_ATTN     11  /* [B*N][n_heads*head_dim] dtype: attention output of the rows the
+                              most recent layer recomputed (layer L-1 after dcu_step or
+                              dcu_full_forward), packed sequence by sequence in ascending
+                              position; the first sum_b SEL_COUNT[b] rows (B*N after a dense
+                              forward) are defined, the rest are scratch */
 
 /* Size in bytes of a tensor kind for the active (B, N). */
 int dcu_tensor_bytes(const dcu_ctx *ctx, int32_t kind, int64_t *bytes);

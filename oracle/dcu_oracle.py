@@ -320,20 +320,34 @@ def select_rows(d32: np.ndarray, keys, B_window: int, budget: int, mode: int = 0
     return np.flatnonzero(U)
 
 
-def layer_rows(lw: dict, cfg: Config, x: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+def kv_rows(lw: dict, cfg: Config, x: np.ndarray, pos: np.ndarray):
+    """Keys and values of the given layer-input rows, as the cache stores them:
+    k = RoPE(W_k RMSNorm(x)) at the rows' positions, v = W_v RMSNorm(x).
+    Returns (k, v), each [Hkv, M, hd], rounded to the storage dtype."""
+    M = x.shape[0]
+    Hkv, hd = cfg.n_kv_heads, cfg.head_dim
+    n = rmsnorm(x, lw["attn_norm"], cfg.rms_eps)
+    k = rope((n @ lw["wk"].T).reshape(M, Hkv, hd), pos, cfg.rope_theta)
+    v = (n @ lw["wv"].T).reshape(M, Hkv, hd)
+    return store(k.transpose(1, 0, 2), cfg.dtype), store(v.transpose(1, 0, 2), cfg.dtype)
+
+
+def layer_rows(lw: dict, cfg: Config, x: np.ndarray, pos: np.ndarray, K: np.ndarray, V: np.ndarray,
+               trace: dict | None = None) -> np.ndarray:
     """Recompute the selected rows through one layer, reusing every other row's
     cached K/V ([DLLM] "关键设计 1": only the top tokens are recomputed, the rest
     reuse their cache).  K, V ([Hkv, N, hd]) are updated in place with the new
-    rows (written before attention).  Returns the new layer outputs, stored."""
+    rows (written before attention).  Returns the new layer outputs, stored.
+    When ``trace`` is a dict it receives the attention output ('attn',
+    [M, H*hd], fp64) for checks of that stage alone."""
     M = x.shape[0]
-    H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    H, hd = cfg.n_heads, cfg.head_dim
     n = rmsnorm(x, lw["attn_norm"], cfg.rms_eps)
     q = rope((n @ lw["wq"].T).reshape(M, H, hd), pos, cfg.rope_theta)
-    k = rope((n @ lw["wk"].T).reshape(M, Hkv, hd), pos, cfg.rope_theta)
-    v = (n @ lw["wv"].T).reshape(M, Hkv, hd)
-    K[:, pos, :] = store(k.transpose(1, 0, 2), cfg.dtype)
-    V[:, pos, :] = store(v.transpose(1, 0, 2), cfg.dtype)
+    K[:, pos, :], V[:, pos, :] = kv_rows(lw, cfg, x, pos)
     a = attend(q, K, V).reshape(M, H * hd)
+    if trace is not None:
+        trace["attn"] = a
     h = x + a @ lw["wo"].T
     y = h + ffn(rmsnorm(h, lw["ffn_norm"], cfg.rms_eps), lw)
     return store(y, cfg.dtype)

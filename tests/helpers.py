@@ -128,3 +128,88 @@ def check_commit(pos_gpu, pos_ora, c_ora, masked, eps=1e-5):
     bad = [p for p in diff if abs(float(c_ora[p]) - cut) > eps]
     assert not bad, f"commit differs beyond the near-boundary exemption at {bad}"
     return diff
+
+
+# ---------------------------------------------------------------- teacher forcing
+
+class LayerSnap:
+    """Host copy (fp64) of what one layer of a DCU step read and wrote on the
+    GPU: H_l and H_{l+1}, K_l and V_l before and after the step, and the
+    layer's d, selection and counts after it."""
+
+    def __init__(self, before, after, ctx, l, B, N, shape, dcu):
+        D, Hkv, hd = shape.d_model, shape.n_kv_heads, shape.head_dim
+        f64 = lambda t, *dims: np.asarray(to_np(t), dtype=np.float64).reshape(*dims)  # noqa: E731
+        self.l = l
+        self.H_old = f64(before[0][l], B, N, D)
+        self.H_new = f64(after[0][l], B, N, D)
+        self.Hn_old = f64(before[0][l + 1], B, N, D)
+        self.Hn_new = f64(after[0][l + 1], B, N, D)
+        self.K_old = f64(before[1][l], B, Hkv, N, hd)
+        self.V_old = f64(before[2][l], B, Hkv, N, hd)
+        self.K_new = f64(after[1][l], B, Hkv, N, hd)
+        self.V_new = f64(after[2][l], B, Hkv, N, hd)
+        self.d = dcu.dcu_get_tensor(ctx, dcu.DCU_T_D, l).cpu().numpy().reshape(B, N)
+        self.sel = dcu.dcu_get_tensor(ctx, dcu.DCU_T_SEL, l).cpu().numpy().reshape(B, N)
+        self.cnt = dcu.dcu_get_tensor(ctx, dcu.DCU_T_SEL_COUNT, l).cpu().numpy()
+
+
+def teacher_forced_layer(snap, lw, cfg_o, s_gpu, budgets, keys, bw, mode, tol, attn_gpu=None, label=""):
+    """Per-layer parity with the oracle fed the GPU's own layer inputs (the
+    spec parity contract): from the GPU's H_l before and after the step
+    the oracle computes d (to 2e-7), s (to 1e-5 relative) and the selection
+    with the GPU's budget (exact except indices within 1e-5 of the top-B
+    boundary); from the GPU's selection, H_l and pre-step K_l / V_l it
+    recomputes the rows, whose H_{l+1}, K_l and V_l must agree within the
+    relative-L2 tolerance (and the attention output of the packed rows, when
+    given).  Returns the number of exempt near-boundary indices."""
+    B, N = snap.d.shape
+    g = lw["attn_norm"]
+    exempt = 0
+    attn_rows, attn_ref = [], []
+    for b in range(B):
+        d_o = O.to_f32(O.cosine_distance(snap.H_new[b], snap.H_old[b], g))
+        err = float(np.max(np.abs(snap.d[b].astype(np.float64) - d_o.astype(np.float64))))
+        assert err <= 2e-7, f"{label} seq {b}: d differs by {err:.2e}"
+        s_o = O.layer_dynamics(d_o)
+        assert abs(float(s_gpu[b]) - float(s_o)) <= 1e-5 * abs(float(s_o)) + 1e-12, \
+            f"{label} seq {b}: s {float(s_gpu[b])} vs oracle {float(s_o)}"
+        U = snap.sel[b, :snap.cnt[b]].astype(np.int64)
+        ref = O.select_rows(d_o, keys[b], bw, int(budgets[b]), mode)
+        exempt += len(check_selection(U, ref, d_o, keys[b], bw, int(budgets[b]), mode, N, eps=1e-5))
+        if len(U) == 0:
+            continue
+        K, V = snap.K_old[b].copy(), snap.V_old[b].copy()
+        tr = {}
+        y = O.layer_rows(lw, cfg_o, snap.H_new[b][U], U, K, V, trace=tr)
+        e = rel_l2(snap.Hn_new[b][U], y)
+        assert e <= tol, f"{label} seq {b}: H_{snap.l + 1}[U] rel L2 {e:.3e} > {tol}"
+        for name, gpu, o in (("K", snap.K_new[b], K), ("V", snap.V_new[b], V)):
+            e = rel_l2(gpu[:, U, :], o[:, U, :])
+            assert e <= tol, f"{label} seq {b}: {name}_{snap.l}[U] rel L2 {e:.3e} > {tol}"
+        off = np.setdiff1d(np.arange(N), U)
+        assert np.array_equal(snap.Hn_new[b][off], snap.Hn_old[b][off]), f"{label}: H_{snap.l + 1} changed off U"
+        attn_rows.append(len(U))
+        attn_ref.append(tr["attn"])
+    if attn_gpu is not None and attn_ref:
+        ref = np.concatenate(attn_ref)
+        got = np.asarray(attn_gpu, dtype=np.float64)[:len(ref)]
+        e = rel_l2(got, ref)
+        assert e <= tol, f"{label}: attention output rel L2 {e:.3e} > {tol}"
+    return exempt
+
+
+def dense_layer_check(lw, cfg_o, H0, H1_gpu, K_gpu, V_gpu, sample, tol, label=""):
+    """Dense forward, one layer, teacher-forced on the GPU's layer input H0
+    ([B, N, D]): the oracle's K/V of every row and the layer output of the
+    sampled rows (attending over the oracle's K/V of all rows)."""
+    B, N, _ = H0.shape
+    pos = np.arange(N)
+    for b in range(B):
+        K, V = O.kv_rows(lw, cfg_o, H0[b], pos)
+        for name, gpu, o in (("K", K_gpu[b], K), ("V", V_gpu[b], V)):
+            e = rel_l2(gpu, o)
+            assert e <= tol, f"{label} seq {b}: dense {name} rel L2 {e:.3e} > {tol}"
+        y = O.layer_rows(lw, cfg_o, H0[b][sample], sample, K.copy(), V.copy())
+        e = rel_l2(H1_gpu[b][sample], y)
+        assert e <= tol, f"{label} seq {b}: dense H_1 rel L2 {e:.3e} > {tol}"

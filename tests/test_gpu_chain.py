@@ -1,8 +1,14 @@
 """End-to-end parity of the CUDA path with the oracle: dense forward, DCU
 steps and commits on seeded synthetic models, compared layer by layer.
 
-The oracle runs its own fp64 chain from the same seeded inputs (it takes no
-input from the CUDA path).  Cached tensors must agree within relative L2
+Every DCU step is first checked teacher-forced: per layer, the oracle is fed
+the GPU's own layer inputs (H_l before and after the step, K_l / V_l before
+it, the budgets) and must reproduce d, s, the selection (exact except indices
+within 1e-5 of the top-B boundary), H_{l+1}, K_l and V_l of the recomputed
+rows and the last layer's attention output.
+
+Beside that, the oracle runs its own fp64 chain from the same seeded inputs
+(it takes no input from the CUDA path).  Cached tensors must agree within relative L2
 1e-4 (float32 model) or 2e-2 (bf16 model).  Selections and commits must agree
 exactly except at indices whose oracle d or c lies within 1e-5 of the
 decision boundary; for the bf16 model that band is widened to the measured
@@ -19,10 +25,16 @@ import oracle as O
 from dynamic_layer_wise_b200 import dcu
 from dynamic_layer_wise_b200 import inputs as I
 
-from .helpers import (check_commit, check_selection, check_selection_valid, oracle_cfg, oracle_weights, rel_l2,
-                      to_np)
+from .helpers import (LayerSnap, check_commit, check_selection, check_selection_valid, oracle_cfg, oracle_weights,
+                      rel_l2, teacher_forced_layer, to_np)
 
 pytestmark = pytest.mark.gpu
+
+
+def _snapshot(ctx, L):
+    return ([dcu.dcu_get_tensor(ctx, dcu.DCU_T_H, l).clone() for l in range(L + 1)],
+            [dcu.dcu_get_tensor(ctx, dcu.DCU_T_K, l).clone() for l in range(L)],
+            [dcu.dcu_get_tensor(ctx, dcu.DCU_T_V, l).clone() for l in range(L)])
 
 
 def _gpu_caches(ctx, L, B, N, shape):
@@ -146,10 +158,21 @@ def _run_chain(shape, seed, B, n_prompt, n_gen, plan, B_layer, B_window, rule, p
             for b in range(B):
                 kp[b, :len(keys[b])] = keys[b]
                 nk[b] = len(keys[b])
+            before = _snapshot(ctx, L)
             dcu.dcu_step(ctx, torch.tensor(ids, dtype=torch.int32).cuda(), torch.tensor(kp).cuda(),
                          torch.tensor(nk).cuda(), B_layer, B_window)
             st, tr = O.dcu_step(w_o, cfg_o, st, ids, keys, B_layer, B_window)
             assert dcu.dcu_status(ctx) == 0
+            # teacher-forced: every layer against the oracle fed the GPU's own layer inputs (fixed 1e-5 band)
+            after = _snapshot(ctx, L)
+            bud = dcu.dcu_get_tensor(ctx, dcu.DCU_T_BUDGET).cpu().numpy().reshape(B, L)
+            s_g = dcu.dcu_get_tensor(ctx, dcu.DCU_T_S).cpu().numpy().reshape(B, L)
+            attn = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_ATTN)).reshape(B * N, -1)
+            for l in range(L):
+                snap = LayerSnap(before, after, ctx, l, B, N, shape, dcu)
+                teacher_forced_layer(snap, w_o.layers[l], cfg_o, s_g[:, l], bud[:, l], keys, B_window,
+                                     window_mode, tol, attn_gpu=attn if l == L - 1 else None,
+                                     label=f"step {step} teacher-forced layer {l}")
             _compare_step(ctx, st, tr, shape, B, N, keys, B_window, window_mode, tol, s_rtol, d_atol,
                           f"step {step}")
     ctx.close()

@@ -2,14 +2,19 @@
 configuration bench.py times (CUDA graphs on, the same context sizes).
 
 The oracle cannot run a whole 32-layer chain at these sizes, so each test
-checks (1) what the oracle computes one by one from the seeded inputs —
-layer-0 dynamics and selections exactly, layer-0 K/V rows of sampled
-recomputed positions, LM-head confidence and argmax of sampled masked rows on
-seeded synthetic final-layer rows — and (2) invariants that hold at any size
-at every layer: budgets sum to B_layer * L and stay within one of their quota,
-selections are the window plus the top-B of the GPU's own d, d^{l+1} is exactly
-0 and H_{l+1} / K_l / V_l are bitwise unchanged at every row layer l did not
-recompute, and the commit follows its rule on the GPU's own confidences."""
+checks (0) the dense forward's first layer teacher-forced on the GPU's H_0
+(K/V of every row, H_1 of sampled rows), (1) what the oracle computes from
+the seeded inputs alone -- layer-0 dynamics and selections exactly, LM-head
+confidence and argmax of sampled masked rows on seeded synthetic final-layer
+rows, (1b) teacher-forced layers 0, 1 and L-1 of a DCU step: the oracle is fed
+the GPU's layer inputs and must reproduce d, s, the selection (exact up to the
+1e-5 near-boundary band), H_{l+1}, K_l and V_l of the recomputed rows and, at
+layer L-1, the attention output -- and (2) invariants that hold at any size at
+every layer: budgets sum to B_layer * L, stay within one of their quota and
+equal the oracle's split of the GPU's s, selections are the window plus the
+top-B of the GPU's own d, d^{l+1} is exactly 0 and H_{l+1} / K_l / V_l are
+bitwise unchanged at every row layer l did not recompute, and the commit
+follows its rule on the GPU's own confidences."""
 import math
 
 import numpy as np
@@ -20,7 +25,8 @@ import oracle as O
 from dynamic_layer_wise_b200 import dcu
 from dynamic_layer_wise_b200 import inputs as I
 
-from .helpers import LazyMatrix, check_selection_valid, oracle_cfg, rel_l2
+from .helpers import (LayerSnap, LazyMatrix, check_selection_valid, dense_layer_check, oracle_cfg, rel_l2,
+                      teacher_forced_layer, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,8 +43,11 @@ CONFIGS = {
 
 
 def _layer_weights(shape, seed, l, names):
-    return {n: I.as_f64(I.weight_rows(shape, seed, n, 0, shape.weight_shapes()[n][0], layer=l), shape.dtype)
-            for n in names}
+    """fp64 host copies of layer l's matrices, from the host generator (norm gains are ones)."""
+    lw = {n: I.as_f64(I.weight_rows(shape, seed, n, 0, shape.weight_shapes()[n][0], layer=l), shape.dtype)
+          for n in names}
+    lw["attn_norm"] = lw["ffn_norm"] = np.ones(shape.d_model)
+    return lw
 
 
 def _snapshot(ctx, L):
@@ -59,6 +68,18 @@ def test_fullsize_dcu_step(name):
     ids0 = np.stack([I.sequence_ids(1 + b, b, c["n_prompt"], c["n_gen"], shape.vocab) for b in range(B)])
     t_ids = torch.tensor(ids0, dtype=torch.int32, device="cuda")
     dcu.dcu_full_forward(ctx, t_ids)
+    assert dcu.dcu_status(ctx) == 0
+    cfg_o = oracle_cfg(shape)
+
+    # (0) dense forward, layer 0, teacher-forced on the GPU's H_0: K/V of every row and H_1 of sampled rows
+    lw0 = _layer_weights(shape, seed, 0, I.LAYER_TENSORS)
+    H0 = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_H, 0)).reshape(B, N, D)
+    H1 = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_H, 1)).reshape(B, N, D)
+    K0 = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_K, 0)).reshape(B, Hkv, N, hd)
+    V0 = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_V, 0)).reshape(B, Hkv, N, hd)
+    sample = np.unique(np.concatenate([[0, 1, N // 2, N - 2, N - 1], np.linspace(0, N - 1, 7).astype(int)]))
+    dense_layer_check(lw0, cfg_o, H0, H1, K0, V0, sample, 2e-2, label=f"{name} dense layer 0")
+    del H0, H1, K0, V0
 
     # synthetic unmasking of 3 generated positions per sequence (the same inputs for the oracle)
     ids1 = ids0.copy()
@@ -98,22 +119,20 @@ def test_fullsize_dcu_step(name):
         ref = O.select_rows(d_ora, keys[b], c["B_window"], int(budgets[b, 0]), 0)
         np.testing.assert_array_equal(sel0[b, :cnt0[b]], ref)
 
-    # layer-0 K/V of sampled recomputed rows (key rows and a few others), one row at a time
-    cfg_o = oracle_cfg(shape)
-    lw = _layer_weights(shape, seed, 0, ("wk", "wv"))
-    K0 = after[1][0].view(B, Hkv, N, hd).float().cpu().numpy()
-    V0 = after[2][0].view(B, Hkv, N, hd).float().cpu().numpy()
-    for b in range(B):
-        rows = list(keys[b][:2]) + list(sel0[b, :cnt0[b]][[0, cnt0[b] // 2]])
-        for p in rows:
-            x = emb.get(ids1[b, p])
-            if x is None:
-                x = I.as_f64(I.weight_values(shape, seed, "embed", rows=[ids1[b, p]])[0], shape.dtype)
-            n = O.rmsnorm(x[None], np.ones(D), shape.rms_eps)
-            k = O.rope((n @ lw["wk"].T).reshape(1, Hkv, hd), np.array([p]), shape.rope_theta)[0]
-            v = (n @ lw["wv"].T).reshape(Hkv, hd)
-            assert rel_l2(K0[b, :, p, :], k) < 2e-2, f"K_0 row {p}"
-            assert rel_l2(V0[b, :, p, :], v) < 2e-2, f"V_0 row {p}"
+    # (1b) teacher-forced parity at layers 0, 1 and L-1: the oracle is fed the GPU's H_l (before and
+    # after the step), K_l / V_l before it and the GPU's budgets; at layer L-1 the attention output of
+    # the recomputed rows is compared too (the tensor-core attention's split and merge path)
+    s_gpu = dcu.dcu_get_tensor(ctx, dcu.DCU_T_S).cpu().numpy().reshape(B, L)
+    attn = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_ATTN)).reshape(B * N, shape.n_heads * hd)
+    exempt = 0
+    for l in (0, 1, L - 1):
+        lw = lw0 if l == 0 else _layer_weights(shape, seed, l, I.LAYER_TENSORS)
+        snap = LayerSnap(before, after, ctx, l, B, N, shape, dcu)
+        exempt += teacher_forced_layer(snap, lw, cfg_o, s_gpu[:, l], budgets[:, l], keys, c["B_window"], 0, 2e-2,
+                                       attn_gpu=attn if l == L - 1 else None, label=f"{name} layer {l}")
+        del snap, lw
+    print(f"{name}: teacher-forced layers 0, 1, {L - 1}: {exempt} near-boundary selection differences")
+    del lw0
 
     # (2) invariants at every layer
     for l in range(L):
@@ -146,6 +165,8 @@ def test_fullsize_dcu_step(name):
         if tot > 0:
             q = c["B_layer"] * L * s[b].astype(np.float64) / tot
             assert np.all(np.abs(b2[b] - q) < 1.0 + 1e-9)
+        # bit-exact against the oracle fed the GPU's s
+        np.testing.assert_array_equal(b2[b], O.split_budget(s[b], c["B_layer"], False))
 
     # (1') commit on seeded synthetic final-layer rows (set through the ABI), sampled vs the oracle
     HL = I.normal_values(seed, 9100, 0, B * N * D, 1.0, shape.dtype)

@@ -316,6 +316,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graphs", action="store_true", help="launch every kernel directly (no CUDA graphs)")
+    ap.add_argument("--fused", type=int, default=None,
+                    help="DCU_OPT_FUSED_EPILOGUE (1: epilogues inside the layer GEMMs); default: the library's")
+    ap.add_argument("--l2-prefetch", type=int, default=None,
+                    help="DCU_OPT_L2_PREFETCH (next-GEMM weight units per CTA into L2); default: the library's")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: override the number of layers (the JSON line is then not a bench value)")
     ap.add_argument("--case", default="", choices=["", "gemm"],
@@ -385,6 +389,10 @@ def main():
     W = I.device_weights(shape, 0)
     ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
     dcu.dcu_set_graphs(ctx, not args.no_graphs)
+    if args.fused is not None:
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, args.fused)
+    if args.l2_prefetch is not None:
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_L2_PREFETCH, args.l2_prefetch)
     seq_seed = replica_seed(rank)                         # each replica decodes its own sequences
     ids_h = torch.stack([torch.tensor(I.sequence_ids(seq_seed, b, wl["n_prompt"], wl["n_gen"], shape.vocab),
                                       dtype=torch.int32) for b in range(B)])

@@ -62,6 +62,16 @@ struct dcu_ctx {
   std::vector<const float *> g1, g2;
   // active shape
   int B = 0, N = 0;
+  // periodic full refresh: schedule, DCU steps since the dense forward, and the
+  // positions forced into every layer's recompute set by the step being enqueued
+  int refresh_gen_start = 0, refresh_prompt = 0, refresh_gen = 0;
+  int64_t step_count = 0;
+  int force_lo = 0, force_hi = 0;
+  // select_from: DCU_SELECT_INPUT (layer-input distance) or DCU_SELECT_VALUE;
+  // stale[l][r] = H_l row r was rewritten since layer l last recomputed it
+  int select_from = DCU_SELECT_INPUT;
+  uint8_t *stale = nullptr;
+  int32_t *vrowmap = nullptr;
   bool have_cache = false, first_step = true;
   int64_t cap = 0;  // max_batch * max_seq rows
   // caches
@@ -88,6 +98,16 @@ struct dcu_ctx {
   size_t ws_elems = 0;        // capacity of C in floats
   float2 *smx = nullptr;      // LM-head softmax statistics per (vocab tile, row)
   int32_t *smx_arg = nullptr;
+  // fused GEMM epilogues (bf16, head_dim 64 / 128): arrival counters of the
+  // four layer GEMMs, per-tile row sums of squares (O -> gate|up) and per-tile
+  // partial sums of the next-layer distance (down)
+  bool fused = false;        // fused path in use (DCU_OPT_FUSED_EPILOGUE and supported)
+  bool fused_ok = false;     // the model supports it (bf16, head_dim 64 or 128)
+  int nx_count = 16;         // units per CTA of the next GEMM's weights prefetched into L2 (0: off)
+  int32_t *epi_cnt = nullptr;
+  size_t epi_cnt_ints = 0;
+  int32_t *cnt_tile[4] = {}, *cnt_pass[4] = {};
+  double *ssq = nullptr, *dpart = nullptr;
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
   CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of min(128, cap) and min(256, cap) rows
@@ -104,6 +124,7 @@ struct dcu_ctx {
     for (auto &t : slot_tables)
       if (t.n_tiles == g.n_tiles && t.kblocks == g.kblocks && t.grid == g.grid && t.tile_aligned == g.tile_aligned)
         return t.dev;
+    if (capturing) return nullptr;  // no allocation inside a stream capture: geometries are registered at create
     std::vector<int32_t> h(g.n_tiles);
     for (int i = 0; i < g.n_tiles; ++i) h[i] = sk_nslots(g, i);
     int32_t *d = nullptr;
@@ -133,6 +154,8 @@ struct dcu_ctx {
   int32_t *status() { return ints + 2; }
   int32_t *m_masked() { return ints + 3; }
   int32_t *uniform_flag() { return ints + 4; }  // 1: the next step splits its budget uniformly
+  int32_t *vm_total() { return ints + 5; }      // stale rows of the current layer (select_from = "v")
+  uint8_t *stale_l(int l) { return stale + (size_t)l * cap; }
   size_t hslab() const { return (size_t)cap * cfg.d_model * esz; }
   size_t kvslab() const { return (size_t)cap * cfg.n_kv_heads * cfg.head_dim * esz; }
   void *Hl(int l) { return H + (size_t)l * hslab(); }
@@ -299,15 +322,63 @@ int gemm_params(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const G
   if ((size_t)tc_max_slots(tile, g.grid) * cap * ldc > c->ws_elems)
     return fail(c, DCU_ECUDA, "GEMM workspace too small for the stream-K slots");
   g.nslots = c->slot_table(g);
+  if (!g.nslots) return fail(c, DCU_ECUDA, "stream-K piece table unavailable for this GEMM geometry");
   tp->geo = g;
   return DCU_OK;
 }
 
 // C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
 // stream-K slots described by *geo (geo->grid == 0: a single slot).
+// L2 prefetch target of a GEMM launch: the first units of the next weight
+// stream, GEMM `which` (0 QKV, 1 O, 2 gate|up, 3 down) of layer l, or the LM
+// head when l == n_layers (bf16 models; nothing otherwise).
+void set_prefetch(dcu_ctx *c, int l, int which, TcParams *tp) {
+  const dcu_cfg &g = c->cfg;
+  if (c->lmaps.empty() || c->nx_count <= 0 || l > g.n_layers) return;
+  const int D = g.d_model, F = g.d_ffn, Hhd = g.n_heads * g.head_dim, KVd = g.n_kv_heads * g.head_dim;
+  SlotGeo &q = tp->nx_geo;
+  memset(&q, 0, sizeof(q));
+  if (l == g.n_layers) {  // LM head: tile-aligned ranges over the vocabulary
+    tp->nx_a[0] = c->lm_map;
+    q.n_tiles = (g.vocab + 127) / 128;
+    q.kblocks = D / 64;
+    q.tile_aligned = 1;
+    q.grid = q.n_tiles < c->num_sms ? q.n_tiles : c->num_sms;
+    tp->nx_seg_tile0[0] = 0;
+    tp->nx_seg_tile0[1] = q.n_tiles;
+    tp->nx_nseg = 1;
+  } else {
+    const LayerMaps &m = c->lmaps[l];
+    int rows[3] = {0, 0, 0}, n = 0, K = D;
+    if (which == 0) {
+      tp->nx_a[0] = m.wq, tp->nx_a[1] = m.wk, tp->nx_a[2] = m.wv;
+      rows[0] = Hhd, rows[1] = KVd, rows[2] = KVd, n = 3;
+    } else if (which == 1) {
+      tp->nx_a[0] = m.wo, rows[0] = D, n = 1, K = Hhd;
+    } else if (which == 2) {
+      tp->nx_a[0] = m.wg, tp->nx_a[1] = m.wu, rows[0] = rows[1] = F, n = 2;
+    } else {
+      tp->nx_a[0] = m.wd, rows[0] = D, n = 1, K = F;
+    }
+    int tile = 0;
+    for (int i = 0; i < n; ++i) {
+      tp->nx_seg_tile0[i] = tile;
+      tile += (rows[i] + 127) / 128;
+    }
+    tp->nx_seg_tile0[n] = tile;
+    tp->nx_nseg = n;
+    q.n_tiles = tile;
+    q.kblocks = K / 64;
+    const long long T = (long long)tile * q.kblocks;
+    q.grid = (int)(T < c->num_sms ? T : c->num_sms);
+  }
+  tp->nx_count = c->nx_count;
+}
+
 int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
              const CUtensorMap *const *amaps, int nseg, int ldc, cudaStream_t s, SlotGeo *geo,
-             bool tile_aligned = false, int prof_class = DCU_K_GEMM) {
+             bool tile_aligned = false, int prof_class = DCU_K_GEMM, int epi_mode = EPI_SLOTS,
+             const EpiArgs *ea = nullptr, int next_l = -1, int next_which = 0) {
   Prof p(c, prof_class, s);
   const int cap = (int)c->cap;
   memset(geo, 0, sizeof(*geo));
@@ -317,6 +388,9 @@ int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const Gemm
   }
   TcParams tp;
   if (int rc = gemm_params(c, x, m_total, segs, amaps, nseg, ldc, tile_aligned, &tp)) return rc;
+  tp.epi_mode = epi_mode;
+  if (ea) tp.e = *ea;
+  if (next_l >= 0) set_prefetch(c, next_l, next_which, &tp);
   *geo = tp.geo;
   LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
   return DCU_OK;
@@ -333,10 +407,26 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   // grid size of the row kernels: the expected recompute-set size (their loops
   // stride over the device row count, so any count is covered)
   const int gcap = dense ? cap : std::min(cap, std::max(1, c->gemm_rows_hint));
+  if (!dense && c->select_from == DCU_SELECT_VALUE) {
+    // select_from = "v": d of the stale rows from their recomputed Value
+    // against the cached Value (every other row keeps d = 0)
+    Prof p(c, DCU_K_SELECT, s);
+    const int Wv = Hkv * hd;
+    LAUNCH(c, launch_plan_stale(c->stale_l(l), c->B * c->N, c->vrowmap, c->vm_total(), s));
+    LAUNCH(c, launch_gather_norm(dt, c->vrowmap, c->vm_total(), gcap, c->Hl(l), c->g1[l], g.rms_eps, D, c->xs, s));
+    const LayerMaps *lmv = c->lmaps.empty() ? nullptr : &c->lmaps[l];
+    const ActOperand xv{c->xs, D, D, &c->xs_map[0], &c->xs_map[1]};
+    GemmSeg seg[1] = {{c->wv[l], Wv}};
+    const CUtensorMap *am[1] = {lmv ? &lmv->wv : nullptr};
+    SlotGeo vgeo;
+    if (int rc = run_gemm(c, xv, c->vm_total(), seg, am, 1, Wv, s, &vgeo, false, DCU_K_SELECT)) return rc;
+    LAUNCH(c, launch_value_dist(dt, c->C, Wv, vgeo, c->vrowmap, c->vm_total(), gcap, c->N, Hkv, hd, c->Vl(l),
+                                c->dl(l), s));
+  }
   if (!dense) {
     Prof p(c, DCU_K_SELECT, s);
     LAUNCH(c, launch_select(c->dl(l), keys, nkeys, c->budgets + l, L, c->B, c->N, Bw, g.window_mode,
-                            c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
+                            c->force_lo, c->force_hi, c->sel_idx + (size_t)l * cap, c->sel_cnt + (size_t)l * g.max_batch, c->s_cur + l, L,
                             last ? nullptr : c->dl(l + 1), c->rowmap, c->m_total(), c->done(), c->seq_off,
                             c->status(), s));
   }
@@ -350,15 +440,52 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   const ActOperand ac{c->act, F, F, &c->act_map[0], &c->act_map[1]};
   SlotGeo geo;
   const int nqkv = (H + 2 * Hkv) * hd;
+  // fused epilogues: arguments shared by the four GEMMs of the layer
+  EpiArgs ea;
+  memset(&ea, 0, sizeof(ea));
+  if (c->fused) {
+    ea.rowmap = c->rowmap;
+    ea.N = c->N;
+    ea.cap = cap;
+    ea.H = H;
+    ea.Hkv = Hkv;
+    ea.hd = hd;
+    ea.use_rope = g.rope_theta > 0.0f;
+    ea.rope_tab = c->rope_tab;
+    ea.Q = c->Q;
+    ea.Kc = c->Kl(l);
+    ea.Vc = c->Vl(l);
+    ea.D = D;
+    ea.F = F;
+    ea.eps = g.rms_eps;
+    ea.Hl = c->Hl(l);
+    ea.g2 = c->g2[l];
+    ea.hmid = c->hmid;
+    ea.u = c->xs;
+    ea.ssq = c->ssq;
+    ea.ssq_ld = (D / 128 + 1) & ~1;
+    ea.act = c->act;
+    ea.Hn = c->Hl(l + 1);
+    const bool want_d = !dense && !last;
+    ea.g_next = want_d ? c->g1[l + 1] : nullptr;
+    ea.d_next = want_d ? c->dl(l + 1) : nullptr;
+    ea.dpart = c->dpart;
+    ea.stale_l = c->stale_l(l);
+    ea.stale_next = want_d ? c->stale_l(l + 1) : nullptr;
+  }
   {
     GemmSeg seg[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
     const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo)) return rc;
+    ea.tile_cnt = c->cnt_tile[0];
+    ea.pass_cnt = c->cnt_pass[0];
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo, false, DCU_K_GEMM,
+                          c->fused ? EPI_QKV : EPI_SLOTS, c->fused ? &ea : nullptr, l, 1))
+      return rc;
   }
-  {
+  if (!c->fused) {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), gcap, c->N, H, Hkv,
-                             hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), s));
+                             hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), c->stale_l(l), s));
   }
   {
     Prof p(c, DCU_K_ATTN, s);
@@ -398,9 +525,13 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   {
     GemmSeg seg[1] = {{c->wo[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
-    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
+    ea.tile_cnt = c->cnt_tile[1];
+    ea.pass_cnt = c->cnt_pass[1];
+    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo, false, DCU_K_GEMM,
+                          c->fused ? EPI_O : EPI_SLOTS, c->fused ? &ea : nullptr, l, 2))
+      return rc;
   }
-  {
+  if (!c->fused) {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->Hl(l), c->g2[l],
                            g.rms_eps, D, c->hmid, c->xs, s));
@@ -408,23 +539,32 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   {
     GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
     const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo)) return rc;
+    ea.tile_cnt = c->cnt_tile[2];
+    ea.pass_cnt = c->cnt_pass[2];
+    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo, false, DCU_K_GEMM,
+                          c->fused ? EPI_GU : EPI_SLOTS, c->fused ? &ea : nullptr, l, 3))
+      return rc;
   }
-  {
+  if (!c->fused) {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), gcap, F, c->act, s));
   }
   {
     GemmSeg seg[1] = {{c->wd[l], D}};
     const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
-    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo)) return rc;
+    ea.tile_cnt = c->cnt_tile[3];
+    ea.pass_cnt = c->cnt_pass[3];
+    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo, false, DCU_K_GEMM,
+                          c->fused ? EPI_DOWN : EPI_SLOTS, c->fused ? &ea : nullptr, l + 1, 0))
+      return rc;
   }
-  {
+  if (!c->fused) {
     Prof p(c, DCU_K_SCATTER, s);
     const bool want_d = !dense && !last;
     LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->hmid,
                                       c->Hl(l + 1), want_d ? c->g1[l + 1] : nullptr,
-                                      want_d ? c->dl(l + 1) : nullptr, D, s));
+                                      want_d ? c->dl(l + 1) : nullptr, want_d ? c->stale_l(l + 1) : nullptr, D,
+                                      s));
   }
   return DCU_OK;
 }
@@ -495,9 +635,9 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   if (2 * F > cw) cw = 2 * F;
   if (D > cw) cw = D;
   if (cfg->dtype == DCU_BF16) {
-    const size_t widths[4] = {nqkv, D, 2 * F, D};
-    const size_t ks[4] = {D, Hhd, D, F};
-    for (int i = 0; i < 4; ++i) {
+    const size_t widths[5] = {nqkv, D, 2 * F, D, (size_t)cfg->n_kv_heads * cfg->head_dim};
+    const size_t ks[5] = {D, Hhd, D, F, D};
+    for (int i = 0; i < 5; ++i) {
       const size_t tiles = (widths[i] + 127) / 128;
       const long long T = (long long)tiles * (long long)(ks[i] / 64);
       const int grid = (int)(T < c->num_sms ? T : c->num_sms);
@@ -523,6 +663,8 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   AL(c->sel_idx, (size_t)L * cap * 4);
   AL(c->sel_cnt, (size_t)L * cfg->max_batch * 4);
   AL(c->rowmap, cap * 4);
+  AL(c->vrowmap, cap * 4);
+  AL(c->stale, (size_t)L * cap);
   AL(c->mrow, cap * 4);
   AL(c->ints, 64);
   AL(c->rope_tab, (size_t)cfg->max_seq * (cfg->head_dim / 2) * sizeof(float2));
@@ -545,6 +687,26 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     c->attn_qt_cap = (int)(((size_t)cfg->max_seq * G + 127) / 128);
     AL(c->attn_po, (size_t)kAttnMaxSplits * cap * Hhd * 4);
     AL(c->attn_ml, (size_t)kAttnMaxSplits * cap * cfg->n_heads * sizeof(float2));
+    // fused GEMM epilogues: counters for up to cap / 128 token passes
+    c->fused_ok = true;
+    const size_t passes = (cap + 127) / 128;
+    const size_t tiles[4] = {nqkv / 128, D / 128, 2 * F / 128, D / 128};
+    const size_t pcnt[4] = {0, 0, passes * (F / 128), passes};
+    size_t n = 0;
+    for (int i = 0; i < 4; ++i) n += passes * tiles[i] + pcnt[i];
+    c->epi_cnt_ints = n;
+    AL(c->epi_cnt, n * 4);
+    AL(c->ssq, ((D / 128 + 1) & ~(size_t)1) * cap * sizeof(double));
+    AL(c->dpart, (D / 128) * cap * 4 * sizeof(double));
+    if (e == cudaSuccess) {
+      size_t o = 0;
+      for (int i = 0; i < 4; ++i) {
+        c->cnt_tile[i] = c->epi_cnt + o;
+        o += passes * tiles[i];
+        c->cnt_pass[i] = c->epi_cnt + o;
+        o += pcnt[i];
+      }
+    }
   }
 #undef AL
   if (e != cudaSuccess) {
@@ -556,6 +718,8 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   }
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
+  if (e == cudaSuccess && c->epi_cnt) e = cudaMemset(c->epi_cnt, 0, c->epi_cnt_ints * 4);
+  if (e == cudaSuccess) e = cudaMemset(c->stale, 0, (size_t)L * cap);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
   if (e == cudaSuccess && cfg->rope_theta > 0.0f)
@@ -598,9 +762,10 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     }
     // piece-count tables of the four layer GEMMs' stream-K geometries (built
     // here so that no allocation happens while a step is captured)
-    const size_t widths[4] = {nqkv, D, 2 * F, D};
-    const size_t ks[4] = {D, Hhd, D, F};
-    for (int i = 0; i < 4; ++i) {
+    // (the fifth: the W_v GEMM of select_from = "v")
+    const size_t widths[5] = {nqkv, D, 2 * F, D, (size_t)cfg->n_kv_heads * cfg->head_dim};
+    const size_t ks[5] = {D, Hhd, D, F, D};
+    for (int i = 0; i < 5; ++i) {
       SlotGeo g;
       g.n_tiles = (int)((widths[i] + 127) / 128);
       g.kblocks = (int)(ks[i] / 64);
@@ -654,20 +819,23 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
   {
     Prof p(c, DCU_K_REFRESH, s);
     LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
-                               c->cfg.d_model, c->cfg.vocab, 1, c->status(), s));
+                                   c->cfg.d_model, c->cfg.vocab, 1, c->status(), nullptr, s));
   }
   LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), c->seq_off, s));
+  if (c->epi_cnt) CK(c, cudaMemsetAsync(c->epi_cnt, 0, c->epi_cnt_ints * 4, s));
   c->gemm_bn = 256;
   c->gemm_rows_hint = BN;
   for (int l = 0; l < c->cfg.n_layers; ++l)
     if (int rc = run_layer(c, l, true, nullptr, nullptr, 0, s)) return rc;
   CK(c, cudaMemsetAsync(c->s_prev, 0, (size_t)c->cfg.max_batch * c->cfg.n_layers * 4, s));
+  CK(c, cudaMemsetAsync(c->stale, 0, (size_t)c->cfg.n_layers * c->cap, s));  // every row was just recomputed
   {
     static const int32_t one = 1;
     CK(c, cudaMemcpyAsync(c->uniform_flag(), &one, 4, cudaMemcpyHostToDevice, s));
   }
   c->first_step = true;
   c->have_cache = true;
+  c->step_count = 0;
   return DCU_OK;
 }
 
@@ -682,7 +850,9 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
   const int L = c->cfg.n_layers, BN = c->B * c->N;
   {
     // expected rows per layer: twice the mean budget plus a few windows per sequence
-    const long long est = (long long)c->B * (2LL * B_layer + 2LL * (B_window + 1));
+    // (and the refreshed positions on a refresh step)
+    const long long est =
+        (long long)c->B * (2LL * B_layer + 2LL * (B_window + 1) + 2LL * (c->force_hi - c->force_lo));
     c->gemm_rows_hint = (int)(est < BN ? est : BN);
     // token pass of the GEMMs: 128 rows when the typical recompute set (half the
     // hint) leaves headroom, since the smaller activation box leaves more shared
@@ -690,6 +860,9 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
     // a larger set is still correct (a second pass re-streams the weights)
     c->gemm_bn = (c->gemm_rows_hint / 2) <= 96 ? 128 : 256;
   }
+  // arrival counters of the fused epilogues start from zero (each launch leaves
+  // them at zero; this clears what an aborted launch may have left)
+  if (c->epi_cnt) CK(c, cudaMemsetAsync(c->epi_cnt, 0, c->epi_cnt_ints * 4, s));
   {
     Prof p(c, DCU_K_BUDGET, s);
     LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, 0, c->uniform_flag(), c->budgets, s));
@@ -697,7 +870,7 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
   {
     Prof p(c, DCU_K_REFRESH, s);
     LAUNCH(c, launch_embed_refresh(c->cfg.dtype, ids, c->prev_ids, c->embed, c->Hl(0), c->dl(0), c->g1[0], BN,
-                                   c->cfg.d_model, c->cfg.vocab, 0, c->status(), s));
+                                   c->cfg.d_model, c->cfg.vocab, 0, c->status(), c->stale_l(0), s));
   }
   for (int l = 0; l < L; ++l)
     if (int rc = run_layer(c, l, false, keys, nkeys, B_window, s)) return rc;
@@ -831,6 +1004,15 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
   if (!c->have_cache) return fail(c, DCU_ESTATE, "dcu_step before dcu_full_forward");
   if (!ids || !keys || !nkeys) return fail(c, DCU_EINVAL, "token_ids, key_positions or n_keys is NULL");
   if (B_layer < 0 || B_window < 0) return fail(c, DCU_EINVAL, "B_layer and B_window must be >= 0");
+  // periodic full refresh due at this step (1, 2, ... after the dense forward)
+  const int64_t step = c->step_count + 1;
+  {
+    const int g0 = c->refresh_gen_start < c->N ? c->refresh_gen_start : c->N;
+    const bool pr = c->refresh_prompt > 0 && step % c->refresh_prompt == 0;
+    const bool gr = c->refresh_gen > 0 && step % c->refresh_gen == 0;
+    c->force_lo = pr ? 0 : (gr ? g0 : 0);
+    c->force_hi = gr ? c->N : (pr ? g0 : 0);
+  }
   const uint64_t key[10] = {1,
                             (uint64_t)(uintptr_t)ids,
                             (uint64_t)(uintptr_t)keys,
@@ -839,12 +1021,50 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
                             (uint64_t)B_window,
                             ((uint64_t)c->B << 32) | (uint64_t)c->N,
                             (uint64_t)(c->prof_max > 0),
-                            0,
-                            0};
+                            ((uint64_t)(uint32_t)c->force_lo << 32) | (uint64_t)(uint32_t)c->force_hi,
+                            (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16)};
   int rc = run_graphed(c, key, (cudaStream_t)stream,
                        [&](cudaStream_t s) { return enqueue_step(c, ids, keys, nkeys, B_layer, B_window, s); });
-  if (rc == DCU_OK) c->first_step = false;
+  if (rc == DCU_OK) {
+    c->first_step = false;
+    c->step_count = step;
+  }
   return rc;
+}
+
+int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  switch (option) {
+    case DCU_OPT_FUSED_EPILOGUE:
+      if (value && !c->fused_ok)
+        return fail(c, DCU_EINVAL, "fused epilogues need a bf16 model with head_dim 64 or 128");
+      c->fused = value != 0;
+      return DCU_OK;
+    case DCU_OPT_L2_PREFETCH:
+      if (value < 0 || value > 4096) return fail(c, DCU_EINVAL, "L2 prefetch units must lie in [0, 4096]");
+      c->nx_count = value;
+      return DCU_OK;
+    default:
+      return fail(c, DCU_EINVAL, "unknown option");
+  }
+}
+
+int dcu_set_select_from(dcu_ctx *c, int32_t source) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (source != DCU_SELECT_INPUT && source != DCU_SELECT_VALUE)
+    return fail(c, DCU_EINVAL, "source must be DCU_SELECT_INPUT or DCU_SELECT_VALUE");
+  c->select_from = source;
+  return DCU_OK;
+}
+
+int dcu_set_refresh(dcu_ctx *c, int32_t gen_start, int32_t prompt_interval, int32_t gen_interval) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (gen_start < 0 || prompt_interval < 0 || gen_interval < 0)
+    return fail(c, DCU_EINVAL, "gen_start and the intervals must be >= 0");
+  c->refresh_gen_start = gen_start;
+  c->refresh_prompt = prompt_interval;
+  c->refresh_gen = gen_interval;
+  return DCU_OK;
 }
 
 int commit_select_block(dcu_ctx *c, int32_t rule, float param, int32_t gen_start, int32_t block_len,
@@ -914,7 +1134,7 @@ int dcu_select_tokens(const float *d, const int32_t *keys, const int32_t *nkeys,
   if (!d || !keys || !nkeys || !budgets || !idx || !count || !s || B <= 0 || N <= 0 || N > 16384 ||
       B_window < 0 || (window_mode != 0 && window_mode != 1))
     return fail(nullptr, DCU_EINVAL, "dcu_select_tokens: bad argument");
-  CK(nullptr, launch_select(d, keys, nkeys, budgets, 1, B, N, B_window, window_mode, idx, count, s, 1, nullptr,
+  CK(nullptr, launch_select(d, keys, nkeys, budgets, 1, B, N, B_window, window_mode, 0, 0, idx, count, s, 1, nullptr,
                             nullptr, nullptr, nullptr, nullptr, status, (cudaStream_t)stream));
   return DCU_OK;
 }
@@ -1047,6 +1267,11 @@ static int tensor_ptr(dcu_ctx *c, int kind, int layer, char **p, int64_t *bytes)
       *p = (char *)c->amax;
       *bytes = BN * 4;
       return DCU_OK;
+    case DCU_T_STALE:
+      if (!need(0, L - 1)) break;
+      *p = (char *)c->stale_l(layer);
+      *bytes = BN;
+      return DCU_OK;
     case DCU_T_ATTN:
       *p = c->attn;
       *bytes = BN * g.n_heads * g.head_dim * (int64_t)c->esz;
@@ -1076,8 +1301,8 @@ int dcu_get_tensor(dcu_ctx *c, int32_t kind, int32_t layer, void *dst, int64_t b
 
 int dcu_set_tensor(dcu_ctx *c, int32_t kind, int32_t layer, const void *src, int64_t bytes, dcu_stream_t stream) {
   if (!c || !src) return fail(c, DCU_EINVAL, "ctx or src is NULL");
-  if (kind != DCU_T_H && kind != DCU_T_K && kind != DCU_T_V && kind != DCU_T_S_PREV)
-    return fail(c, DCU_EINVAL, "only H, K, V and S_PREV can be set");
+  if (kind != DCU_T_H && kind != DCU_T_K && kind != DCU_T_V && kind != DCU_T_S_PREV && kind != DCU_T_STALE)
+    return fail(c, DCU_EINVAL, "only H, K, V, S_PREV and STALE can be set");
   char *p;
   int64_t n;
   if (int rc = tensor_ptr(c, kind, layer, &p, &n)) return rc;

@@ -5,6 +5,9 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 #include "../../include/dcu.h"
 
@@ -148,6 +151,26 @@ __device__ __forceinline__ void pdl_enter() {
   allow_dependents();
 }
 
+// Asks for the largest shared-memory carveout for `kern` on the current device
+// (once per kernel and device).  Under programmatic dependent launch the next
+// kernel's CTAs are scheduled while this one runs; a GEMM CTA needs 220 KB of
+// shared memory, which an SM configured for a small carveout cannot give until
+// it drains.
+inline void prefer_max_smem(const void *kern) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void *, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto &d : done)
+    if (d.first == kern && d.second == dev) return;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) ==
+      cudaSuccess)
+    done.emplace_back(kern, dev);
+  else
+    cudaGetLastError();
+}
+
 // Launch with programmatic stream serialization: the kernel's CTAs may be
 // scheduled while its predecessor finishes, hiding the launch latency; the
 // kernel must call pdl_enter() (or griddep_wait()) before touching anything
@@ -165,6 +188,7 @@ inline cudaError_t launch_pdl(void (*kern)(Exp...), dim3 grid, dim3 block, size_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  prefer_max_smem(reinterpret_cast<const void *>(kern));
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Act &&>(args)...);
 }
 

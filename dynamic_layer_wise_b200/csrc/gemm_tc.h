@@ -11,6 +11,7 @@ constexpr int kTcMaxB = 4;                  // deepest activation-tile ring
 constexpr int kTcThreads = 224;             // 7 warps: W producer, MMA, 4 epilogue, X producer
 constexpr uint32_t kTcABytes = 128u * 128u;  // weight tile: 128 rows x 64 bf16
 constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (one CTA per SM)
+constexpr uint32_t kFixBuf = 24u * 1024u;    // fused epilogues: bytes per fix-up staging buffer
 
 // Stream-K schedule: the flattened (tile, k block) space of one token pass,
 // T = n_tiles * kblocks, is cut into G contiguous ranges [c*T/G, (c+1)*T/G)
@@ -41,6 +42,53 @@ __host__ __device__ inline int sk_first(const SlotGeo &g, int tile) { return sk_
 __host__ __device__ inline int sk_nslots(const SlotGeo &g, int tile) {
   return sk_owner(g, (long long)(tile + 1) * g.kblocks - 1) - sk_first(g, tile) + 1;
 }
+
+// Epilogues fused into the GEMM (epi_mode >= 2, bf16 layer GEMMs with head_dim
+// 64 or 128).  Every piece of a tile is stored in its slot as in epi_mode 0;
+// the CTA that stores a tile's last piece (an arrival counter per (pass,
+// tile), no CTA ever waits for another) sums the slots in slot order and
+// applies the layer's epilogue to the tile's 128 columns:
+//   EPI_QKV   RoPE (rotate-half) on q and k, q -> Q[r], k / v -> the K/V cache
+//   EPI_O     hmid = H_l[row] + o (float), u = bf16(hmid * g2) (the gate|up
+//             operand), ssq[r][tile] = sum of hmid^2 over the tile's columns
+//   EPI_GU    the RMSNorm scale 1/sqrt(sum_tiles ssq / D + eps) of the row is
+//             applied to the summed gate / up pre-activations (the norm is
+//             linear in its input); the tile's result goes to slot 0; the second
+//             tile of a (gate j, up j) pair to finish writes act = silu(g) * u
+//   EPI_DOWN  new = hmid + down -> H_{l+1}[row] (scatter); when d_next is set,
+//             fp64 partial sums of the next-layer cosine distance against the
+//             cached row per tile; the last tile of the pass finishes d_next
+// The last arriver stages each chunk of its rows (the pieces, plus the row data
+// the epilogue reads) in shared memory with bulk copies, double-buffered, so
+// the fix-up moves its data at L2 bandwidth rather than at load latency.
+// Counters are zero between launches (each is reset by its last user).
+enum { EPI_SLOTS = 0, EPI_LMHEAD = 1, EPI_QKV = 2, EPI_O = 3, EPI_GU = 4, EPI_DOWN = 5 };
+struct EpiArgs {
+  int32_t *tile_cnt;       // [passes][n_tiles] arrivals
+  int32_t *pass_cnt;       // EPI_GU: [passes][F / 128] pair arrivals; EPI_DOWN: [passes] finished tiles
+  const int32_t *rowmap;   // packed row -> b * N + i
+  int N, cap;              // sequence length; rows of the row-indexed buffers
+  // EPI_QKV
+  int H, Hkv, hd, use_rope;
+  const float2 *rope_tab;  // [max_seq][hd / 2] (cos, sin)
+  void *Q, *Kc, *Vc;       // Q [cap][H * hd]; the layer's K / V cache [B][Hkv][N][hd]
+  // EPI_O / EPI_GU / EPI_DOWN
+  int D, F;
+  float eps;
+  const void *Hl;          // layer input rows [B * N][D]
+  const float *g2;         // FFN norm gain [D]
+  float *hmid;             // [cap][D]
+  void *u;                 // [cap][D] bf16, gate|up operand
+  double *ssq;             // [cap][ssq_ld]: per row, one partial sum per tile of D
+  int ssq_ld;              // D / 128 rounded up to even (16-byte rows)
+  void *act;               // [cap][F] bf16, down operand
+  void *Hn;                // H_{l+1} rows [B * N][D]
+  const float *g_next;     // next layer's attention-norm gain (null: no d)
+  float *d_next;           // next layer's d [B * N] (null: no d)
+  double *dpart;           // [cap][D / 128][4]: dot, |x|^2, |y|^2, bitwise-equal flag
+  uint8_t *stale_l;        // EPI_QKV: cleared at the rows the layer recomputes (may be null)
+  uint8_t *stale_next;     // EPI_DOWN with d_next: set at rows whose H_{l+1} content changed (may be null)
+};
 
 // Kernel parameters (passed as a __grid_constant__ so the tensor maps can be
 // addressed by TMA).  Output column of segment s, row r: seg_col0[s] + r;
@@ -82,6 +130,7 @@ struct TcParams {
   int nx_nseg;
   SlotGeo nx_geo;
   int nx_count;
+  EpiArgs e;               // epi_mode >= 2
 };
 
 // Row-major bf16 matrix [outer][inner] with row pitch row_bytes, box

@@ -89,12 +89,343 @@ struct KCursor {
   }
 };
 
+// ------------------------------------------------------------------ fused epilogues
+// Run by the 4 epilogue warps (128 threads, named barrier 1) of the CTA that
+// stored a tile's last piece.  The rows are processed in chunks staged in
+// shared memory (two buffers, one mbarrier each): one thread issues a bulk
+// copy per (row, piece) and per extra row slice, the 4 warps consume the
+// chunk one row per warp at a time, lane l owning the tile's columns
+// 4l .. 4l + 3, while the next chunk is in flight.
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d, uint32_t (&bits)[4]) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t *>(&lo);
+  u.y = *reinterpret_cast<const uint32_t *>(&hi);
+  bits[0] = u.x & 0xffffu;
+  bits[1] = u.x >> 16;
+  bits[2] = u.y & 0xffffu;
+  bits[3] = u.y >> 16;
+  return u;
+}
+
+__device__ __forceinline__ void unpack_bf16x4(uint2 u, float (&v)[4], uint32_t (&bits)[4]) {
+  bits[0] = u.x & 0xffffu;
+  bits[1] = u.x >> 16;
+  bits[2] = u.y & 0xffffu;
+  bits[3] = u.y >> 16;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(bits[i] << 16);
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Shared-memory staging of the fix-ups.
+struct FixStage {
+  uint32_t sbase;   // smem address of buffer 0 (buffer 1 follows)
+  uint8_t *gbase;   // generic address of buffer 0
+  uint32_t bytes;   // per buffer
+  uint32_t bar;     // mbarriers of buffers 0 and 1 (8 bytes apart)
+  uint32_t uses[2]; // completed phases waited per buffer (the same in every thread)
+  int *rows;        // smem [BN]: global row (rowmap) of each packed row of the tile's pass
+  int32_t *status;
+  volatile int *abort;
+};
+
+// Arrival of this CTA at a counter (after its global stores): true for the
+// arrival that makes it reach `total` (that CTA resets it).  All 128 epilogue
+// threads call it; only they use named barrier 1.
+__device__ __forceinline__ bool epi_arrive(int32_t *cnt, int total, int *s_flag, int ew, int lane) {
+  __threadfence();
+  epi_bar();
+  if (ew == 0 && lane == 0) {
+    const int old = atomicAdd(cnt, 1);
+    const int last = (old == total - 1);
+    if (last) *cnt = 0;  // every arrival has happened: reset for the next launch
+    *s_flag = last;
+  }
+  epi_bar();
+  const bool last = *s_flag != 0;
+  if (last) {
+    __threadfence();
+    fence_proxy_async_global();  // the other CTAs' stores, next read by bulk copies
+  }
+  return last;
+}
+
+// Rows [0, mrows) of a pass in chunks of floor(bytes / row_bytes) rows: issue(r,
+// dst, bar) (one thread) copies packed row r's data to smem address dst;
+// compute(r, src) (one warp) consumes it from generic address src.
+template <class Issue, class Compute>
+__device__ __forceinline__ void staged_rows(FixStage &st, int mrows, uint32_t row_bytes, int ew, int lane,
+                                            Issue issue, Compute compute) {
+  const int R = max(1, min(mrows, (int)(st.bytes / row_bytes)));
+  const int nch = (mrows + R - 1) / R;
+  auto post = [&](int c) {
+    const int b = c & 1, r0 = c * R, r1 = min(mrows, r0 + R);
+    const uint32_t bar = st.bar + 8u * (uint32_t)b;
+    mbar_expect_tx(bar, (uint32_t)(r1 - r0) * row_bytes);
+    for (int r = r0; r < r1; ++r) issue(r, st.sbase + (uint32_t)b * st.bytes + (uint32_t)(r - r0) * row_bytes, bar);
+  };
+  if (ew == 0 && lane == 0) post(0);
+  for (int c = 0; c < nch; ++c) {
+    const int b = c & 1;
+    // buffer b ^ 1 was released by the barrier that ended chunk c - 1
+    if (c + 1 < nch && ew == 0 && lane == 0) post(c + 1);
+    const uint32_t bar = st.bar + 8u * (uint32_t)b, par = st.uses[b] & 1u;
+    if (!wait_bounded(bar, par, st.abort, st.status)) wait_drain(bar, par);  // the copies land before reuse
+    ++st.uses[b];
+    const int r0 = c * R, r1 = min(mrows, r0 + R);
+    for (int r = r0 + ew; r < r1; r += 4) compute(r, st.gbase + (size_t)b * st.bytes + (size_t)(r - r0) * row_bytes);
+    epi_bar();
+  }
+}
+
+__device__ __forceinline__ float4 piece_sum(const uint8_t *src, int ns, int lane) {
+  float4 v = reinterpret_cast<const float4 *>(src)[lane];
+  for (int sp = 1; sp < ns; ++sp) {
+    const float4 w = reinterpret_cast<const float4 *>(src + sp * 512)[lane];
+    v.x += w.x;
+    v.y += w.y;
+    v.z += w.z;
+    v.w += w.w;
+  }
+  return v;
+}
+
+// the ns pieces of packed row pr, 128 fp32 columns from output column col0
+__device__ __forceinline__ void issue_pieces(const TcParams &p, int ns, int pr, size_t col0, uint32_t dst, uint32_t bar) {
+  for (int sp = 0; sp < ns; ++sp)
+    bulk_g2s(dst + 512u * (uint32_t)sp, p.out + (size_t)sp * (size_t)p.geo.slot_stride + (size_t)pr * p.ldc + col0, 512,
+             bar);
+}
+
+// EPI_QKV on tile t of segment seg (0 q, 1 k, 2 v).
+__device__ void fix_qkv(const TcParams &p, FixStage &st, int t, int seg, int m0, int mrows, int ns, int ew,
+                        int lane) {
+  const EpiArgs &e = p.e;
+  const int hd = e.hd, half = hd >> 1;
+  const int tcol0 = (t - p.seg_tile0[seg]) * 128;
+  const int tcol = tcol0 + lane * 4;  // column within the segment
+  const int head = tcol / hd, j4 = tcol - head * hd;
+  const bool first = j4 < half;
+  const int jr = first ? j4 : j4 - half;  // rotation index of the 4 pairs
+  const int xl = half >> 2;               // lane distance to the partner half
+  const size_t col0 = (size_t)p.seg_col0[seg] + (size_t)tcol0;
+  const bool rot = seg < 2 && e.use_rope;
+  bf16 *Q = static_cast<bf16 *>(e.Q), *Kc = static_cast<bf16 *>(e.Kc), *Vc = static_cast<bf16 *>(e.Vc);
+  staged_rows(
+      st, mrows, 512u * (uint32_t)ns, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) { issue_pieces(p, ns, m0 + r, col0, dst, bar); },
+      [&](int r, const uint8_t *src) {
+        const int pr = m0 + r;
+        float4 v = piece_sum(src, ns, lane);
+        const int row = st.rows[r];
+        const int b = row / e.N, i = row - b * e.N;
+        if (rot) {
+          const float o[4] = {__shfl_xor_sync(0xffffffffu, v.x, xl), __shfl_xor_sync(0xffffffffu, v.y, xl),
+                              __shfl_xor_sync(0xffffffffu, v.z, xl), __shfl_xor_sync(0xffffffffu, v.w, xl)};
+          float a[4] = {v.x, v.y, v.z, v.w};
+          const float2 *cs = e.rope_tab + (size_t)i * half + jr;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 c = cs[k];
+            a[k] = first ? a[k] * c.x - o[k] * c.y : a[k] * c.x + o[k] * c.y;
+          }
+          v = make_float4(a[0], a[1], a[2], a[3]);
+        }
+        if (seg == 2 && tcol == 0 && e.stale_l) e.stale_l[row] = 0;  // the layer recomputes this row
+        bf16 *dst = seg == 0 ? Q + (size_t)pr * e.H * hd + (size_t)head * hd
+                             : (seg == 1 ? Kc : Vc) + (((size_t)b * e.Hkv + head) * e.N + i) * hd;
+        uint32_t bits[4];
+        *reinterpret_cast<uint2 *>(dst + j4) = pack_bf16x4(v.x, v.y, v.z, v.w, bits);
+      });
+}
+
+// EPI_O on tile t (columns t * 128 .. of D).
+__device__ void fix_o(const TcParams &p, FixStage &st, int t, int m0, int mrows, int ns, int ew, int lane) {
+  const EpiArgs &e = p.e;
+  const int col0 = t * 128, col = col0 + lane * 4;
+  const bf16 *Hl = static_cast<const bf16 *>(e.Hl);
+  bf16 *u = static_cast<bf16 *>(e.u);
+  const float4 g = *reinterpret_cast<const float4 *>(e.g2 + col);
+  const uint32_t pb = 512u * (uint32_t)ns;
+  staged_rows(
+      st, mrows, pb + 256u, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) {
+        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
+        bulk_g2s(dst + pb, Hl + (size_t)st.rows[r] * e.D + col0, 256, bar);
+      },
+      [&](int r, const uint8_t *src) {
+        const int pr = m0 + r;
+        const float4 v = piece_sum(src, ns, lane);
+        float x[4];
+        uint32_t xb[4];
+        unpack_bf16x4(reinterpret_cast<const uint2 *>(src + pb)[lane], x, xb);
+        const float4 hm = make_float4(x[0] + v.x, x[1] + v.y, x[2] + v.z, x[3] + v.w);
+        *reinterpret_cast<float4 *>(e.hmid + (size_t)pr * e.D + col) = hm;
+        uint32_t bits[4];
+        *reinterpret_cast<uint2 *>(u + (size_t)pr * e.D + col) =
+            pack_bf16x4(hm.x * g.x, hm.y * g.y, hm.z * g.z, hm.w * g.w, bits);
+        double ss = (double)hm.x * (double)hm.x + (double)hm.y * (double)hm.y + (double)hm.z * (double)hm.z +
+                    (double)hm.w * (double)hm.w;
+        ss = warp_sum_d(ss);
+        if (lane == 0) e.ssq[(size_t)pr * e.ssq_ld + t] = ss;
+      });
+}
+
+// EPI_GU on tile t: gate tiles are [0, F/128), up tiles [F/128, 2F/128).
+__device__ void fix_gu(const TcParams &p, FixStage &st, int t, int pass, int m0, int mrows, int ns, int ew,
+                       int lane, int *s_flag) {
+  const EpiArgs &e = p.e;
+  const int ft = e.F / 128, ntd = e.D / 128;
+  const int col0 = t * 128, col = col0 + lane * 4;  // column of [gate | up]
+  const uint32_t pb = 512u * (uint32_t)ns, sb = 8u * (uint32_t)e.ssq_ld;
+  staged_rows(
+      st, mrows, pb + sb, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) {
+        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
+        bulk_g2s(dst + pb, e.ssq + (size_t)(m0 + r) * e.ssq_ld, sb, bar);
+      },
+      [&](int r, const uint8_t *src) {
+        const int pr = m0 + r;
+        float4 v = piece_sum(src, ns, lane);
+        const double *sq = reinterpret_cast<const double *>(src + pb);
+        double ss = 0.0;
+        for (int k = lane; k < ntd; k += 32) ss += sq[k];
+        ss = warp_sum_d(ss);
+        const float inv = (float)(1.0 / sqrt(ss / (double)e.D + (double)e.eps));
+        v.x *= inv;
+        v.y *= inv;
+        v.z *= inv;
+        v.w *= inv;
+        *reinterpret_cast<float4 *>(p.out + (size_t)pr * p.ldc + col) = v;  // slot 0 now holds the result
+      });
+  const int pair = t < ft ? t : t - ft;
+  if (!epi_arrive(e.pass_cnt + (size_t)pass * ft + pair, 2, s_flag, ew, lane)) return;
+  // second tile of the pair: act = silu(gate) * up over the pair's 128 columns
+  const int j0 = pair * 128, j = j0 + lane * 4;
+  bf16 *act = static_cast<bf16 *>(e.act);
+  staged_rows(
+      st, mrows, 1024u, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) {
+        const float *row = p.out + (size_t)(m0 + r) * p.ldc;
+        bulk_g2s(dst, row + j0, 512, bar);
+        bulk_g2s(dst + 512u, row + e.F + j0, 512, bar);
+      },
+      [&](int r, const uint8_t *src) {
+        const float4 gt = reinterpret_cast<const float4 *>(src)[lane];
+        const float4 up = reinterpret_cast<const float4 *>(src + 512)[lane];
+        uint32_t bits[4];
+        *reinterpret_cast<uint2 *>(act + (size_t)(m0 + r) * e.F + j) =
+            pack_bf16x4(gt.x / (1.0f + expf(-gt.x)) * up.x, gt.y / (1.0f + expf(-gt.y)) * up.y,
+                        gt.z / (1.0f + expf(-gt.z)) * up.z, gt.w / (1.0f + expf(-gt.w)) * up.w, bits);
+      });
+}
+
+// EPI_DOWN on tile t (columns t * 128 .. of D).
+__device__ void fix_down(const TcParams &p, FixStage &st, int t, int pass, int m0, int mrows, int ns, int ew,
+                         int lane, int *s_flag) {
+  const EpiArgs &e = p.e;
+  const int ntd = e.D / 128;
+  const int col0 = t * 128, col = col0 + lane * 4;
+  const bool want_d = e.d_next != nullptr;
+  bf16 *Hn = static_cast<bf16 *>(e.Hn);
+  float gg[4] = {0.f, 0.f, 0.f, 0.f};
+  if (want_d) {
+    const float4 g = *reinterpret_cast<const float4 *>(e.g_next + col);
+    gg[0] = g.x;
+    gg[1] = g.y;
+    gg[2] = g.z;
+    gg[3] = g.w;
+  }
+  const uint32_t pb = 512u * (uint32_t)ns;
+  staged_rows(
+      st, mrows, pb + 512u + 256u, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) {
+        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
+        bulk_g2s(dst + pb, e.hmid + (size_t)(m0 + r) * e.D + col0, 512, bar);
+        bulk_g2s(dst + pb + 512u, Hn + (size_t)st.rows[r] * e.D + col0, 256, bar);  // the cached row
+      },
+      [&](int r, const uint8_t *src) {
+        const int pr = m0 + r;
+        const float4 v = piece_sum(src, ns, lane);
+        const float4 hm = reinterpret_cast<const float4 *>(src + pb)[lane];
+        float nv[4] = {hm.x + v.x, hm.y + v.y, hm.z + v.z, hm.w + v.w};
+        uint32_t nb[4];
+        const uint2 packed = pack_bf16x4(nv[0], nv[1], nv[2], nv[3], nb);
+        if (want_d) {
+          float ov[4];
+          uint32_t ob[4];
+          unpack_bf16x4(reinterpret_cast<const uint2 *>(src + pb + 512)[lane], ov, ob);
+          double dot = 0.0, nx = 0.0, ny = 0.0;
+          bool same = true;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            same = same && (nb[k] == ob[k]);
+            const double a = (double)gg[k] * (double)__uint_as_float(nb[k] << 16), b = (double)gg[k] * (double)ov[k];
+            dot += a * b;
+            nx += a * a;
+            ny += b * b;
+          }
+          dot = warp_sum_d(dot);
+          nx = warp_sum_d(nx);
+          ny = warp_sum_d(ny);
+          same = __all_sync(0xffffffffu, same);
+          if (lane == 0) {
+            double *o = e.dpart + ((size_t)pr * ntd + t) * 4;
+            o[0] = dot;
+            o[1] = nx;
+            o[2] = ny;
+            o[3] = same ? 1.0 : 0.0;
+          }
+        }
+        *reinterpret_cast<uint2 *>(Hn + (size_t)st.rows[r] * e.D + col) = packed;
+      });
+  if (!want_d) return;
+  if (!epi_arrive(e.pass_cnt + pass, ntd, s_flag, ew, lane)) return;
+  // last tile of the pass: the next-layer d of every row of the pass
+  staged_rows(
+      st, mrows, 32u * (uint32_t)ntd, ew, lane,
+      [&](int r, uint32_t dst, uint32_t bar) {
+        bulk_g2s(dst, e.dpart + (size_t)(m0 + r) * ntd * 4, 32u * (uint32_t)ntd, bar);
+      },
+      [&](int r, const uint8_t *src) {
+        const double *o = reinterpret_cast<const double *>(src);
+        double dot = 0.0, nx = 0.0, ny = 0.0;
+        bool same = true;
+        for (int k = lane; k < ntd; k += 32) {
+          dot += o[4 * k];
+          nx += o[4 * k + 1];
+          ny += o[4 * k + 2];
+          same = same && (o[4 * k + 3] != 0.0);
+        }
+        dot = warp_sum_d(dot);
+        nx = warp_sum_d(nx);
+        ny = warp_sum_d(ny);
+        same = __all_sync(0xffffffffu, same);
+        if (lane == 0) {
+          const int row = st.rows[r];
+          e.d_next[row] = finish_cosine_distance(dot, nx, ny, same);
+          if (e.stale_next && !same) e.stale_next[row] = 1;  // H_{l+1} row changed
+        }
+      });
+}
+
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
+  __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 7];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
+  __shared__ int s_epi_ok[4], s_epi_flag;
+  __shared__ int s_rows[256];  // fused epilogues: global rows of the pass being fixed up
 
   // The row count is written by the select / plan kernel two launches before
   // this one, so it is final even while the previous launch still runs.
@@ -112,10 +443,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per stage
   const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned stages
   const int SB = b_stage > 16384u ? 3 : 4;
-  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage) / kTcABytes);
+  // fused epilogues: two fix-up staging buffers after the rings (the weight
+  // ring keeps >= 6 stages, which the pure weight stream needs)
+  const uint32_t fix_bytes = p.epi_mode >= EPI_QKV ? 2u * kFixBuf : 0u;
+  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage - fix_bytes) / kTcABytes);
   SA = SA > kTcMaxA ? kTcMaxA : SA;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bbase = sbase + (uint32_t)SA * kTcABytes;
+  const uint32_t fbase = bbase + (uint32_t)SB * b_stage;
   const uint32_t bar0 = smem_u32(bars);
   // two TMEM accumulators (columns [0, BN) and [BN, 2 BN)) alternate between fragments
 #define FULL_A(s) (bar0 + 8u * (uint32_t)(s))
@@ -123,7 +458,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
 #define FULL_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + (s)))
 #define EMPTY_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + kTcMaxB + (s)))
   const uint32_t tfull0 = bar0 + 8u * (uint32_t)(2 * kTcMaxA + 2 * kTcMaxB), tempty0 = tfull0 + 16u,
-                 drain = tfull0 + 32u;
+                 drain = tfull0 + 32u, fixbar = tfull0 + 40u;
 #define TFULL(a) (tfull0 + 8u * (uint32_t)(a))
 #define TEMPTY(a) (tempty0 + 8u * (uint32_t)(a))
 #define STAGE_A(s) (sbase + (uint32_t)(s) * kTcABytes)
@@ -143,6 +478,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       mbar_init(TEMPTY(a), 4);
     }
     mbar_init(drain, 1);
+    mbar_init(fixbar, 1);
+    mbar_init(fixbar + 8u, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -341,12 +678,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         lm_arg[mt] = 0x7fffffff;
       }
     };
+    const bool fused = p.epi_mode >= EPI_QKV;
+    const int ew = warp - 2;  // epilogue warp 0..3 (row interleave of the fused epilogues)
+    FixStage st;
+    st.sbase = fbase;
+    st.gbase = smem_raw + (fbase - smem_u32(smem_raw));
+    st.bytes = kFixBuf;
+    st.bar = fixbar;
+    st.uses[0] = st.uses[1] = 0;
+    st.rows = s_rows;
+    st.status = p.status;
+    st.abort = abort_v;
+    // the fused epilogues read what the previous launches wrote (H_l rows, the
+    // row sums of squares, hmid): wait for them like the activation producer
+    if (fused) griddep_wait();
     while (next_frag(p, passes, it, f)) {
       const int m0 = it.pass * BN;
       const int mrows = min(BN, M - m0);
       const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
       const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q * 32) << 16);
-      if (!__all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status))) break;
+      bool okw = __all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status));
+      if (fused) {
+        // the 4 warps meet at named barriers below: they leave together or not at all
+        if (lane == 0) s_epi_ok[ew] = okw ? 1 : 0;
+        epi_bar();
+        okw = (s_epi_ok[0] & s_epi_ok[1] & s_epi_ok[2] & s_epi_ok[3]) != 0;
+      }
+      if (!okw) break;
       tc_fence_after();
       const int rin = f.arow + q * 32 + lane;  // row within the weight segment
       const bool col_ok = rin < p.seg_rows[f.seg];
@@ -411,6 +769,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       __syncwarp();
       if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
       ++nfrag;
+      if (fused) {
+        const int ns = sk_nslots(p.geo, f.tile);
+        if (epi_arrive(p.e.tile_cnt + (size_t)it.pass * p.geo.n_tiles + f.tile, ns, &s_epi_flag, ew, lane)) {
+          for (int r = threadIdx.x - 64; r < mrows; r += 128) s_rows[r] = p.e.rowmap[m0 + r];
+          epi_bar();
+          if (p.epi_mode == EPI_QKV)
+            fix_qkv(p, st, f.tile, f.seg, m0, mrows, ns, ew, lane);
+          else if (p.epi_mode == EPI_O)
+            fix_o(p, st, f.tile, m0, mrows, ns, ew, lane);
+          else if (p.epi_mode == EPI_GU)
+            fix_gu(p, st, f.tile, it.pass, m0, mrows, ns, ew, lane, &s_epi_flag);
+          else
+            fix_down(p, st, f.tile, it.pass, m0, mrows, ns, ew, lane, &s_epi_flag);
+        }
+      }
     }
     if (p.epi_mode == 1) lm_flush(lm_pass);
   }
@@ -466,6 +839,7 @@ template <int BN>
 static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
   static std::atomic<uint64_t> smem_set{0};
   if (cudaError_t e = ensure_smem_limit(k_gemm_tc<BN>, (int)kTcSmem, smem_set)) return e;
+  prefer_max_smem(reinterpret_cast<const void *>(k_gemm_tc<BN>));
   // programmatic dependent launch: the CTAs may start while the previous kernel
   // finishes; they wait (griddepcontrol.wait) before reading its outputs
   cudaLaunchConfig_t cfg = {};

@@ -63,7 +63,8 @@ __device__ __forceinline__ void dyn_accum(const T *x, const T *y, const float *g
 template <class T>
 __global__ void k_embed_refresh(const int32_t *__restrict__ ids, int32_t *__restrict__ prev_ids,
                                 const T *__restrict__ embed, T *__restrict__ H0, float *__restrict__ d0,
-                                const float *__restrict__ g0, int BN, int D, int V, int full, int32_t *status) {
+                                const float *__restrict__ g0, int BN, int D, int V, int full, int32_t *status,
+                                uint8_t *__restrict__ stale0) {
   pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
@@ -98,20 +99,21 @@ __global__ void k_embed_refresh(const int32_t *__restrict__ ids, int32_t *__rest
     if (threadIdx.x == 0) {
       d0[r] = finish_cosine_distance(dot, nx, ny, same);
       prev_ids[r] = id;
+      if (stale0 && !same) stale0[r] = 1;  // H_0 row changed: layer 0 has not recomputed it yet
     }
   }
 }
 
 cudaError_t launch_embed_refresh(int dtype, const int32_t *ids, int32_t *prev_ids, const void *embed, void *H0,
                                  float *d0, const float *g0, int BN, int D, int V, int full, int32_t *status,
-                                 cudaStream_t s) {
+                                 uint8_t *stale0, cudaStream_t s) {
   if (BN <= 0) return cudaSuccess;
   if (dtype == DCU_BF16)
     launch_pdl(k_embed_refresh<bf16>, row_grid(BN), 256, 0, s, ids, prev_ids, (const bf16 *)embed, (bf16 *)H0, d0, g0, BN,
-                                                        D, V, full, status);
+                                                        D, V, full, status, stale0);
   else
     launch_pdl(k_embed_refresh<float>, row_grid(BN), 256, 0, s, ids, prev_ids, (const float *)embed, (float *)H0, d0, g0,
-                                                         BN, D, V, full, status);
+                                                         BN, D, V, full, status, stale0);
   return cudaGetLastError();
 }
 
@@ -237,9 +239,12 @@ __device__ __forceinline__ void store4<bf16>(bf16 *p, float a, float b, float c,
   *reinterpret_cast<uint2 *>(p) = u;
 }
 
+// Grid of the flattened (row, 4-column) epilogues: at most 4 CTAs of 256
+// threads per SM, so half of each SM's thread slots stay free for the next
+// GEMM's CTAs, which programmatic dependent launch schedules while these run.
 static inline int flat_grid(long long items_cap) {
   long long g = (items_cap + 255) / 256;
-  if (g > 148 * 16) g = 148 * 16;
+  if (g > 148 * 4) g = 148 * 4;
   return g > 0 ? (int)g : 1;
 }
 
@@ -252,7 +257,7 @@ template <class T>
 __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo geo,
                           const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total, int N, int H,
                           int Hkv, int hd, const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q,
-                          T *__restrict__ Kc, T *__restrict__ Vc) {
+                          T *__restrict__ Kc, T *__restrict__ Vc, uint8_t *__restrict__ stale) {
   pdl_enter();
   const int M = *m_total;
   const int half = hd / 2;
@@ -287,6 +292,7 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
     } else {
       const int t = (u - n_rope) * 4;
       const int kvh = t / hd, j = t - kvh * hd;
+      if (t == 0 && stale) stale[row] = 0;  // the layer recomputes this row
       const float4 v = csum4(c, geo, (size_t)(H + Hkv) * hd + t);
       store4<T>(Vc + (((size_t)b * Hkv + kvh) * N + i) * hd + j, v.x, v.y, v.z, v.w);
     }
@@ -295,14 +301,14 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
 
 cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                            const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
-                           int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s) {
+                           int use_rope, void *Q, void *Kc, void *Vc, uint8_t *stale, cudaStream_t s) {
   const long long items = (long long)cap * ((H + Hkv) * (hd / 2) / 4 + Hkv * hd / 4);
   if (dtype == DCU_BF16)
     launch_pdl(k_epi_qkv<bf16>, flat_grid(items), 256, 0, s, C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
-                                                      rope_tab, use_rope, (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc);
+                                                      rope_tab, use_rope, (bf16 *)Q, (bf16 *)Kc, (bf16 *)Vc, stale);
   else
     launch_pdl(k_epi_qkv<float>, flat_grid(items), 256, 0, s, C, ldc, geo, rowmap, m_total, N, H, Hkv, hd,
-                                                       rope_tab, use_rope, (float *)Q, (float *)Kc, (float *)Vc);
+                                                       rope_tab, use_rope, (float *)Q, (float *)Kc, (float *)Vc, stale);
   return cudaGetLastError();
 }
 
@@ -399,7 +405,7 @@ __global__ void __launch_bounds__(512)
     k_epi_down_scatter(const float *__restrict__ C, int ldc, const SlotGeo geo,
                        const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
                        const float *__restrict__ hmid, T *__restrict__ Hn, const float *__restrict__ g_next,
-                       float *__restrict__ d_next, int D) {
+                       float *__restrict__ d_next, uint8_t *__restrict__ stale_next, int D) {
   pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
@@ -442,20 +448,81 @@ __global__ void __launch_bounds__(512)
       dot = block_sum(dot, red);
       nx = block_sum(nx, red);
       ny = block_sum(ny, red);
-      if (threadIdx.x == 0) d_next[row] = finish_cosine_distance(dot, nx, ny, same);
+      if (threadIdx.x == 0) {
+        d_next[row] = finish_cosine_distance(dot, nx, ny, same);
+        if (stale_next && !same) stale_next[row] = 1;  // H_{l+1} row changed
+      }
     }
   }
 }
 
 cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const SlotGeo geo,
                                     const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
-                                    void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s) {
+                                    void *Hnext, const float *g_next, float *d_next, uint8_t *stale_next, int D,
+                                    cudaStream_t s) {
   if (dtype == DCU_BF16)
     launch_pdl(k_epi_down_scatter<bf16>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, hmid,
-                                                            (bf16 *)Hnext, g_next, d_next, D);
+                                                            (bf16 *)Hnext, g_next, d_next, stale_next, D);
   else
     launch_pdl(k_epi_down_scatter<float>, row_grid(cap), 512, 0, s, C, ldc, geo, rowmap, m_total, hmid,
-                                                             (float *)Hnext, g_next, d_next, D);
+                                                             (float *)Hnext, g_next, d_next, stale_next, D);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ Value dynamics (select_from = "v")
+// For packed stale row r (position rowmap[r] = b * N + i): the recomputed Value
+// v = sum of the GEMM's slots over the Hkv * hd columns, rounded to the cache
+// dtype, against the cached Value row (all kv heads): d[row] = 1 - cos(v,
+// v_cached) in fp64 with the equal-row / zero rules ([DLLM] "关键设计 1", the
+// Value comparison it contrasts with the input proxy).  One CTA per row.
+template <class T>
+__global__ void __launch_bounds__(256)
+    k_value_dist(const float *__restrict__ C, int ldc, const SlotGeo geo, const int32_t *__restrict__ rowmap,
+                 const int32_t *__restrict__ m_total, int N, int Hkv, int hd, const T *__restrict__ Vc,
+                 float *__restrict__ d) {
+  pdl_enter();
+  __shared__ double red[32];
+  const int M = *m_total;
+  const int W = Hkv * hd;
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    const int row = rowmap[r];
+    const int b = row / N, i = row - b * N;
+    const float *c = C + (size_t)r * ldc;
+    double dot = 0, nx = 0, ny = 0;
+    bool same = true;
+    for (int j = threadIdx.x * 4; j < W; j += blockDim.x * 4) {
+      const float4 v = csum4(c, geo, (size_t)j);
+      const int kvh = j / hd, jj = j - kvh * hd;
+      const T *cv = Vc + (((size_t)b * Hkv + kvh) * N + i) * hd + jj;
+      const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const T nt = from_f<T>(vv[e]);
+        const T ot = cv[e];
+        same = same && (bits_of<T>(nt) == bits_of<T>(ot));
+        const double a = (double)to_f(nt), o = (double)to_f(ot);
+        dot += a * o;
+        nx += a * a;
+        ny += o * o;
+      }
+    }
+    same = __syncthreads_and(same);
+    dot = block_sum(dot, red);
+    nx = block_sum(nx, red);
+    ny = block_sum(ny, red);
+    if (threadIdx.x == 0) d[row] = finish_cosine_distance(dot, nx, ny, same);
+  }
+}
+
+cudaError_t launch_value_dist(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
+                              const int32_t *m_total, int cap, int N, int Hkv, int hd, const void *Vc, float *d,
+                              cudaStream_t s) {
+  if (dtype == DCU_BF16)
+    launch_pdl(k_value_dist<bf16>, row_grid(cap), 256, 0, s, C, ldc, geo, rowmap, m_total, N, Hkv, hd,
+               (const bf16 *)Vc, d);
+  else
+    launch_pdl(k_value_dist<float>, row_grid(cap), 256, 0, s, C, ldc, geo, rowmap, m_total, N, Hkv, hd,
+               (const float *)Vc, d);
   return cudaGetLastError();
 }
 

@@ -94,8 +94,8 @@ cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, 
 // indices; U = W + selected, compacted in index order.
 __global__ void __launch_bounds__(kSelThreads)
     k_select(const float *__restrict__ d, const int32_t *__restrict__ keys, const int32_t *__restrict__ nkeys,
-             const int32_t *__restrict__ budgets, int budget_stride, int B, int N, int Bw, int mode,
-             int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
+             const int32_t *__restrict__ budgets, int budget_stride, int B, int N, int Bw, int mode, int force_lo,
+             int force_hi, int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
              float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
              int32_t *__restrict__ done, int32_t *__restrict__ seq_off, int32_t *__restrict__ status) {
   pdl_enter();
@@ -146,6 +146,8 @@ __global__ void __launch_bounds__(kSelThreads)
       if (i >= 0 && i < N) flag[i] = 1;
     }
   }
+  // periodic refresh: the forced range joins the window (recomputed whatever the budget)
+  for (int i = max(force_lo, 0) + tid; i < min(force_hi, N); i += nthr) flag[i] = 1;
   __syncthreads();
   int inW = 0, nz = 0;
   {
@@ -324,17 +326,18 @@ __global__ void __launch_bounds__(kSelThreads)
 }
 
 cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
-                          int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
-                          float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
-                          int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s) {
+                          int budget_stride, int B, int N, int Bw, int mode, int force_lo, int force_hi,
+                          int32_t *idx, int32_t *count, float *s_out, int s_stride, float *d_next_zero,
+                          int32_t *rowmap, int32_t *m_total, int32_t *done, int32_t *seq_off, int32_t *status,
+                          cudaStream_t s) {
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   size_t smem = (size_t)N * 5;
   static std::atomic<uint64_t> attr{0};
   if (cudaError_t e = ensure_smem_limit(k_select, kMaxSeq * 5, attr)) return e;
   // short sequences: fewer threads make the ~25 block barriers cheaper
   const int threads = N <= 2048 ? 256 : kSelThreads;
-  launch_pdl(k_select, B, threads, smem, s, d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, idx, count, s_out,
-                                        s_stride, d_next_zero, rowmap, m_total, done, seq_off, status);
+  launch_pdl(k_select, B, threads, smem, s, d, keys, nkeys, budgets, budget_stride, B, N, Bw, mode, force_lo, force_hi,
+             idx, count, s_out, s_stride, d_next_zero, rowmap, m_total, done, seq_off, status);
   return cudaGetLastError();
 }
 
@@ -409,6 +412,28 @@ cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int gen_star
                                int32_t *m_total, cudaStream_t s) {
   if (B > 255) return cudaErrorInvalidValue;
   launch_pdl(k_plan_masked, 1, 1024, 0, s, masked, B, N, gen_start, block_len, rowmap, m_total);
+  return cudaGetLastError();
+}
+
+// Stale rows of one layer (stale[r] != 0), in index order, as packed rows.
+__global__ void __launch_bounds__(1024) k_plan_stale(const uint8_t *__restrict__ stale, int BN,
+                                                     int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total) {
+  pdl_enter();
+  __shared__ int red[32];
+  const int nthr = blockDim.x, tid = threadIdx.x;
+  const int chunk = (BN + nthr - 1) / nthr;
+  const int i0 = tid * chunk, i1 = min(BN, i0 + chunk);
+  int c = 0;
+  for (int i = i0; i < i1; ++i) c += stale[i] != 0;
+  int tot;
+  int pos = block_exclusive_scan(c, red, &tot);
+  for (int i = i0; i < i1; ++i)
+    if (stale[i]) rowmap[pos++] = i;
+  if (tid == 0) *m_total = tot;
+}
+
+cudaError_t launch_plan_stale(const uint8_t *stale, int BN, int32_t *rowmap, int32_t *m_total, cudaStream_t s) {
+  launch_pdl(k_plan_stale, 1, 1024, 0, s, stale, BN, rowmap, m_total);
   return cudaGetLastError();
 }
 

@@ -19,9 +19,10 @@ struct GemmSeg {
 
 // ---- row kernels (k_rows.cu)
 cudaError_t launch_rope_table(float2 *tab, int max_seq, int head_dim, float theta, cudaStream_t s);
+// stale0 (may be null): set to 1 at rows whose H_0 content changed
 cudaError_t launch_embed_refresh(int dtype, const int32_t *ids, int32_t *prev_ids, const void *embed, void *H0,
                                  float *d0, const float *g0, int BN, int D, int V, int full, int32_t *status,
-                                 cudaStream_t s);
+                                 uint8_t *stale0, cudaStream_t s);
 cudaError_t launch_cosine_distance(int dtype, const void *x, const void *y, const float *g, int64_t rows, int D,
                                    float *d, cudaStream_t s);
 cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *m_total, int cap, const void *H,
@@ -29,7 +30,7 @@ cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *
 // C: GEMM output as slots [slot][cap][ldc] under the slot geometry `geo` (geo.grid == 0: one slot).
 cudaError_t launch_epi_qkv(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                            const int32_t *m_total, int cap, int N, int H, int Hkv, int hd, const float2 *rope_tab,
-                           int use_rope, void *Q, void *Kc, void *Vc, cudaStream_t s);
+                           int use_rope, void *Q, void *Kc, void *Vc, uint8_t *stale, cudaStream_t s);
 cudaError_t launch_epi_o(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
                          const int32_t *m_total, int cap, const void *Hl, const float *g2, float eps, int D,
                          float *hmid, void *xs, cudaStream_t s);
@@ -37,7 +38,12 @@ cudaError_t launch_epi_swiglu(int dtype, const float *C, int ldc, const SlotGeo 
                               int cap, int F, void *act, cudaStream_t s);
 cudaError_t launch_epi_down_scatter(int dtype, const float *C, int ldc, const SlotGeo geo,
                                     const int32_t *rowmap, const int32_t *m_total, int cap, const float *hmid,
-                                    void *Hnext, const float *g_next, float *d_next, int D, cudaStream_t s);
+                                    void *Hnext, const float *g_next, float *d_next, uint8_t *stale_next, int D,
+                                    cudaStream_t s);
+// select_from = "v": Value distance of the packed stale rows against the layer's V cache
+cudaError_t launch_value_dist(int dtype, const float *C, int ldc, const SlotGeo geo, const int32_t *rowmap,
+                              const int32_t *m_total, int cap, int N, int Hkv, int hd, const void *Vc, float *d,
+                              cudaStream_t s);
 cudaError_t launch_softmax_max(const float *C, int ldc, const int32_t *rowmap, const int32_t *m_total, int cap,
                                int V, float *conf, int32_t *amax, cudaStream_t s);
 
@@ -47,11 +53,15 @@ cudaError_t launch_budget_split(const float *s_prev, int B, int L, int B_layer, 
                                 const int32_t *uniform_flag, int32_t *budgets, cudaStream_t s);
 // budgets: pointer to element [0] of the layer's column; budget_stride = L.
 // s_out: pointer to the layer's column of s [B][L]; s_stride = L.
-// rowmap / m_total / done may be null (stateless use).
+// rowmap / m_total / done may be null (stateless use).  Positions [force_lo,
+// force_hi) join the window (periodic refresh; an empty range forces nothing).
 cudaError_t launch_select(const float *d, const int32_t *keys, const int32_t *nkeys, const int32_t *budgets,
-                          int budget_stride, int B, int N, int Bw, int mode, int32_t *idx, int32_t *count,
-                          float *s_out, int s_stride, float *d_next_zero, int32_t *rowmap, int32_t *m_total,
-                          int32_t *done, int32_t *seq_off, int32_t *status, cudaStream_t s);
+                          int budget_stride, int B, int N, int Bw, int mode, int force_lo, int force_hi,
+                          int32_t *idx, int32_t *count, float *s_out, int s_stride, float *d_next_zero,
+                          int32_t *rowmap, int32_t *m_total, int32_t *done, int32_t *seq_off, int32_t *status,
+                          cudaStream_t s);
+// stale rows (stale[r] != 0 over B * N rows) as packed rows, one CTA
+cudaError_t launch_plan_stale(const uint8_t *stale, int BN, int32_t *rowmap, int32_t *m_total, cudaStream_t s);
 // rowmap = identity over B * N rows; seq_off[b] = b * N (B <= 255)
 cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off, cudaStream_t s);
 cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int gen_start, int block_len, int32_t *rowmap,

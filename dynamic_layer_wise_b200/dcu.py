@@ -22,7 +22,9 @@ DCU_F32, DCU_BF16 = 0, 1
 DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR = 0, 1, 2
 DCU_WINDOW_INCLUSIVE, DCU_WINDOW_HALFOPEN = 0, 1
 (DCU_T_H, DCU_T_K, DCU_T_V, DCU_T_D, DCU_T_S, DCU_T_S_PREV, DCU_T_BUDGET, DCU_T_SEL, DCU_T_SEL_COUNT,
- DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN) = range(12)
+ DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN, DCU_T_STALE) = range(13)
+DCU_SELECT_INPUT, DCU_SELECT_VALUE = 0, 1
+DCU_OPT_FUSED_EPILOGUE, DCU_OPT_L2_PREFETCH = 1, 2
 (DCU_K_REFRESH, DCU_K_BUDGET, DCU_K_SELECT, DCU_K_GATHER, DCU_K_GEMM, DCU_K_EPILOGUE, DCU_K_ATTN, DCU_K_SCATTER,
  DCU_K_LMHEAD, DCU_K_COMMIT, DCU_K_COUNT) = range(11)
 
@@ -77,6 +79,9 @@ _SIGS = {
     "dcu_kernel_class_name": (ctypes.c_char_p, [_i32]),
     "dcu_launch_count": (_i64, [_vp]),
     "dcu_set_graphs": (_i32, [_vp, _i32]),
+    "dcu_set_refresh": (_i32, [_vp, _i32, _i32, _i32]),
+    "dcu_set_select_from": (_i32, [_vp, _i32]),
+    "dcu_set_option": (_i32, [_vp, _i32, _i32]),
     "dcu_linear": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]),
     "dcu_lm_confidence_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
 }
@@ -267,7 +272,7 @@ def dcu_selftest_wait_timeout(status, stream=None):
 
 _KIND_DTYPE = {DCU_T_D: torch.float32, DCU_T_S: torch.float32, DCU_T_S_PREV: torch.float32,
                DCU_T_BUDGET: torch.int32, DCU_T_SEL: torch.int32, DCU_T_SEL_COUNT: torch.int32,
-               DCU_T_CONF: torch.float32, DCU_T_ARGMAX: torch.int32}
+               DCU_T_CONF: torch.float32, DCU_T_ARGMAX: torch.int32, DCU_T_STALE: torch.uint8}
 
 
 def _kind_dtype(ctx: Context, kind: int):
@@ -339,3 +344,18 @@ def dcu_linear(X, W, stream=None):
 
 def dcu_set_graphs(ctx: Context, on: bool):
     _check(lib().dcu_set_graphs(ctx.handle, int(bool(on))), ctx.handle)
+
+
+def dcu_set_refresh(ctx: Context, gen_start: int, prompt_interval: int, gen_interval: int):
+    """Periodic full refresh of the prompt / generated positions (0 disables an interval)."""
+    _check(lib().dcu_set_refresh(ctx.handle, int(gen_start), int(prompt_interval), int(gen_interval)), ctx.handle)
+
+
+def dcu_set_select_from(ctx: Context, source: int):
+    """DCU_SELECT_INPUT (layer-input distance, default) or DCU_SELECT_VALUE (Value distance)."""
+    _check(lib().dcu_set_select_from(ctx.handle, int(source)), ctx.handle)
+
+
+def dcu_set_option(ctx: Context, option: int, value: int):
+    """Performance option of the context (DCU_OPT_FUSED_EPILOGUE)."""
+    _check(lib().dcu_set_option(ctx.handle, int(option), int(value)), ctx.handle)

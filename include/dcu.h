@@ -63,6 +63,9 @@ extern "C" {
 #define DCU_THRESHOLD 1     /* commit every c_i >= tau, else the top one ([FRECHET] "研究背景与动机") */
 #define DCU_FACTOR    2     /* largest n with (n+1)(1 - c_(n)) < f, else 1 (same section)      */
 
+#define DCU_SELECT_INPUT 0   /* d from the normalised layer inputs ([DLLM] "关键设计 1")          */
+#define DCU_SELECT_VALUE 1   /* d from recomputed vs cached Value rows ([README] select_from="v") */
+
 #define DCU_WINDOW_INCLUSIVE 0  /* [p - Bw/2, p + Bw/2], Bw+1 positions ([DLLM] "关键设计 2") */
 #define DCU_WINDOW_HALFOPEN  1  /* [p - Bw/2, p - Bw/2 + Bw), Bw positions                   */
 
@@ -128,6 +131,50 @@ int dcu_full_forward(dcu_ctx *ctx, const int32_t *token_ids, int32_t B, int32_t 
  * Returns DCU_ESTATE before the first dcu_full_forward. */
 int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_positions, const int32_t *n_keys,
              int32_t B_layer, int32_t B_window, dcu_stream_t stream);
+
+/* Performance options of a context (results agree within the parity
+ * tolerances either way; both paths are tested).
+ *   DCU_OPT_FUSED_EPILOGUE (bf16 models with head_dim 64 or 128; default 0):
+ *     1 = the layer GEMMs apply their epilogues themselves (RoPE and the K/V
+ *     write, residual and the RMSNorm statistics, SwiGLU, residual, scatter
+ *     and next-layer d), the last CTA to finish a tile summing its split-K
+ *     pieces; 0 = separate epilogue kernels.
+ * DCU_EINVAL for an unknown option or an unsupported value. */
+#define DCU_OPT_FUSED_EPILOGUE 1
+/*   DCU_OPT_L2_PREFETCH (default 16): when a layer GEMM has issued its own
+ *     weight loads, each CTA prefetches this many (tile, k block) units of the
+ *     next GEMM's weights (the next layer's QKV, or the LM head after the last
+ *     layer) into L2, so HBM keeps streaming through the dependent kernels in
+ *     between; 0 turns it off, at most 4096. */
+#define DCU_OPT_L2_PREFETCH 2
+int dcu_set_option(dcu_ctx *ctx, int32_t option, int32_t value);
+
+/* Feature source of the token dynamics d ([README] "Quick Start":
+ * select_from; [DLLM] "关键设计 1" contrasts the layer-input proxy with
+ * recomputing and comparing the Value vectors).  DCU_SELECT_INPUT (default):
+ * d compares the normalised layer inputs.  DCU_SELECT_VALUE: per layer, for
+ * every row whose layer input was rewritten with a different value since the
+ * layer last recomputed that row ("stale"; DCU_T_STALE), the Value
+ * W_v RMSNorm(x) is recomputed, rounded to the cache dtype and compared with
+ * the cached Value row over all kv heads, d = 1 - cos; every other row has
+ * d = 0 (its input, hence its Value, is unchanged).  This costs a compaction,
+ * a gather + RMSNorm, a W_v GEMM over the stale rows and a distance kernel per
+ * layer.  Stale flags are kept in both modes.  Takes effect from the next
+ * dcu_step; DCU_EINVAL for another value. */
+int dcu_set_select_from(dcu_ctx *ctx, int32_t source);
+
+/* Periodic full refresh ([README] "Quick Start": prompt_interval_steps,
+ * gen_interval_steps; the pages name the parameters, not their semantics, so
+ * this is the reading taken): counting the DCU steps after the last
+ * dcu_full_forward as 1, 2, ..., a step whose number is a multiple of
+ * prompt_interval forces every prompt position [0, gen_start) into the
+ * recompute set U of every layer, and a multiple of gen_interval every
+ * generated position [gen_start, N) (both: a dense recompute).  Forced
+ * positions join the window: the top-B budget is spent outside them, and d, s
+ * and the next step's budgets are computed as on any step.  0 disables an
+ * interval (the default: no refresh).  gen_start is clamped to N.  Takes
+ * effect from the next dcu_step; DCU_EINVAL for negative arguments. */
+int dcu_set_refresh(dcu_ctx *ctx, int32_t gen_start, int32_t prompt_interval, int32_t gen_interval);
 
 /* Per-step commit ([FRECHET] "整体框架"): final RMSNorm + LM head on the
  * masked positions of H_L only, fused softmax giving the max-probability
@@ -251,6 +298,8 @@ int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_norm, const
 #define DCU_T_SEL_COUNT 8  /* layer 0..L-1 : [B] int32                    */
 #define DCU_T_CONF      9  /* [B][N] float, confidence of the last commit (masked positions) */
 #define DCU_T_ARGMAX   10  /* [B][N] int32, argmax of the last commit (masked positions)      */
+#define DCU_T_STALE    12  /* layer 0..L-1 : [B][N] uint8, 1 = the H_l row was rewritten with a new
+                              value since layer l last recomputed it (settable) */
 #define DCU_T_ATTN     11  /* [B*N][n_heads*head_dim] dtype: attention output of the rows the
                               most recent layer recomputed (layer L-1 after dcu_step or
                               dcu_full_forward), packed sequence by sequence in ascending
@@ -261,7 +310,7 @@ int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_norm, const
 int dcu_tensor_bytes(const dcu_ctx *ctx, int32_t kind, int64_t *bytes);
 /* Device-to-device copy of a tensor kind into dst (dev, `bytes` long). */
 int dcu_get_tensor(dcu_ctx *ctx, int32_t kind, int32_t layer, void *dst, int64_t bytes, dcu_stream_t stream);
-/* Device-to-device copy from src into a tensor kind (H, K, V, S_PREV only). */
+/* Device-to-device copy from src into a tensor kind (H, K, V, S_PREV, STALE only). */
 int dcu_set_tensor(dcu_ctx *ctx, int32_t kind, int32_t layer, const void *src, int64_t bytes, dcu_stream_t stream);
 
 /* ---- per-kernel timing (CUDA events on the launch stream) ---- */

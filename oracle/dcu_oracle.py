@@ -177,10 +177,12 @@ class State:
     ids: np.ndarray                # [B, N] ids the caches were built for
     s_prev: np.ndarray             # [B, L] float32 values of the previous step's s
     first: bool = True             # no previous-step s yet -> uniform split
+    stale: list = None             # stale[l]: [B, N] bool, H_l row rewritten since layer l last recomputed it
 
     def copy(self) -> "State":
         return State([h.copy() for h in self.H], [k.copy() for k in self.K], [v.copy() for v in self.V],
-                     self.ids.copy(), self.s_prev.copy(), self.first)
+                     self.ids.copy(), self.s_prev.copy(), self.first,
+                     None if self.stale is None else [x.copy() for x in self.stale])
 
 
 def full_forward(w: Weights, cfg: Config, ids: np.ndarray) -> State:
@@ -210,7 +212,8 @@ def full_forward(w: Weights, cfg: Config, ids: np.ndarray) -> State:
             h = x + a @ lw["wo"].T
             y = h + ffn(rmsnorm(h, lw["ffn_norm"], cfg.rms_eps), lw)
             Hs[l + 1][b] = store(y, cfg.dtype)
-    return State(Hs, Ks, Vs, ids.copy(), np.zeros((B, L), dtype=np.float32), True)
+    return State(Hs, Ks, Vs, ids.copy(), np.zeros((B, L), dtype=np.float32), True,
+                 [np.zeros((B, N), dtype=bool) for _ in range(L)])
 
 
 # ----------------------------------------------------------------- DCU pieces
@@ -236,6 +239,28 @@ def cosine_distance(x: np.ndarray, y: np.ndarray, g: np.ndarray) -> np.ndarray:
         else:
             out[r] = min(2.0, max(0.0, 1.0 - float(a @ b) / (na * nb)))
     return out
+
+
+def value_dynamics(lw: dict, cfg: Config, x: np.ndarray, V: np.ndarray, stale: np.ndarray) -> np.ndarray:
+    """Token dynamics with select_from = "v" ([README] "Quick Start": the
+    feature source of the similarity is the Value; [DLLM] "关键设计 1" contrasts
+    the input proxy with recomputing the Value vectors and comparing their
+    cosine similarity).  Reading: for every row whose layer input changed since
+    this layer last recomputed it (``stale``), the Value is recomputed from the
+    current input x (W_v RMSNorm(x), rounded as the cache stores it) and
+    compared with the cached Value row over all kv heads: d = 1 - cos(v_new,
+    v_cached) with the zero / equal-row rules of cosine_distance.  Every other
+    row has an unchanged input, hence an unchanged Value, and d = 0.
+    x: [N, D] layer inputs; V: [Hkv, N, hd] cached values; -> float32 [N]."""
+    N = x.shape[0]
+    d = np.zeros(N)
+    idx = np.flatnonzero(np.asarray(stale, dtype=bool))
+    if len(idx):
+        _, v = kv_rows(lw, cfg, x[idx], idx)
+        vn = v.transpose(1, 0, 2).reshape(len(idx), -1)
+        vc = V[:, idx, :].transpose(1, 0, 2).reshape(len(idx), -1)
+        d[idx] = cosine_distance(vn, vc, np.ones(vn.shape[1]))
+    return to_f32(d)
 
 
 def layer_dynamics(d32: np.ndarray) -> np.float32:
@@ -310,14 +335,38 @@ def top_outside(d32: np.ndarray, W: np.ndarray, k: int) -> np.ndarray:
     return np.sort(cand[order[:k]])
 
 
-def select_rows(d32: np.ndarray, keys, B_window: int, budget: int, mode: int = 0) -> np.ndarray:
-    """U = W  union  top-B outside W, as sorted row indices."""
+def select_rows(d32: np.ndarray, keys, B_window: int, budget: int, mode: int = 0, force=None) -> np.ndarray:
+    """U = W  union  top-B outside W, as sorted row indices.  ``force`` = (lo, hi)
+    adds the positions [lo, hi) to W (a periodic refresh, see refresh_range):
+    they are recomputed whatever the budget, which is then spent outside them."""
     N = len(d32)
     W = window_mask(keys, B_window, N, mode)
+    if force is not None:
+        W[max(0, int(force[0])):max(0, min(N, int(force[1])))] = True
     k = int(min(max(int(budget), 0), N - int(W.sum())))
     U = W.copy()
     U[top_outside(d32, W, k)] = True
     return np.flatnonzero(U)
+
+
+def refresh_range(step: int, gen_start: int, N: int, prompt_interval: int, gen_interval: int):
+    """Periodic full refresh ([README] "Quick Start": prompt_interval_steps and
+    gen_interval_steps; the function name _compute_sim_for_budget_full_refresh
+    in the code index).  Reading: DCU step ``step`` (1, 2, ... after the dense
+    forward) recomputes every prompt position [0, gen_start) when
+    prompt_interval > 0 divides it, and every generated position
+    [gen_start, N) when gen_interval > 0 divides it; d and s are still computed,
+    so the next step's budgets follow this step.  Returns the forced range
+    (lo, hi), or None when no refresh is due."""
+    p = prompt_interval > 0 and step % prompt_interval == 0
+    g = gen_interval > 0 and step % gen_interval == 0
+    if p and g:
+        return 0, N
+    if p:
+        return 0, gen_start
+    if g:
+        return gen_start, N
+    return None
 
 
 def kv_rows(lw: dict, cfg: Config, x: np.ndarray, pos: np.ndarray):
@@ -362,7 +411,7 @@ class StepTrace:
 
 
 def dcu_step(w: Weights, cfg: Config, state: State, ids: np.ndarray, keys: list, B_layer: int,
-             B_window: int) -> tuple[State, StepTrace]:
+             B_window: int, force=None, select_from: str = "input") -> tuple[State, StepTrace]:
     """One cached denoising step (the DCU procedure of [DLLM] "关键设计 1/2").
 
     1. Layer-0 inputs of positions whose id changed are replaced by their
@@ -373,6 +422,11 @@ def dcu_step(w: Weights, cfg: Config, state: State, ids: np.ndarray, keys: list,
        elsewhere ("关键设计 2": an unselected token feeds the next layer an
        unchanged input, so its next-layer d is 0).
     3. The step's s becomes the previous-step s of the next step.
+    ``force`` = (lo, hi) forces the positions [lo, hi) into every layer's U
+    (periodic refresh, see refresh_range).  ``select_from`` = "v" ranks the
+    rows by value_dynamics instead of the input distance; the stale flags it
+    needs are kept in either mode (set where a write changes an H_l row, cleared
+    where layer l recomputes it).
     """
     st = state.copy()
     ids = np.asarray(ids, dtype=np.int64)
@@ -381,25 +435,35 @@ def dcu_step(w: Weights, cfg: Config, state: State, ids: np.ndarray, keys: list,
     budgets = np.stack([split_budget(st.s_prev[b], B_layer, st.first) for b in range(B)])
     tr = StepTrace(budgets=budgets, s=np.zeros((B, L), dtype=np.float32))
     d_cur = np.zeros((B, N), dtype=np.float32)
+    if select_from not in ("input", "v"):
+        raise ValueError(select_from)
+    if st.stale is None:
+        st.stale = [np.zeros((B, N), dtype=bool) for _ in range(L)]
     for b in range(B):
         ch = np.flatnonzero(ids[b] != st.ids[b])
         if len(ch):
             xn = store(np.asarray(w.embed[ids[b][ch]], dtype=np.float64), cfg.dtype)
             d_cur[b, ch] = to_f32(cosine_distance(xn, st.H[0][b][ch], w.layers[0]["attn_norm"]))
+            st.stale[0][b][ch[np.any(xn != st.H[0][b][ch], axis=1)]] = True
             st.H[0][b][ch] = xn
     for l in range(L):
+        if select_from == "v":
+            d_cur = np.stack([value_dynamics(w.layers[l], cfg, st.H[l][b], st.V[l][b], st.stale[l][b])
+                              for b in range(B)])
         tr.d.append(d_cur.copy())
         d_next = np.zeros((B, N), dtype=np.float32)
         sel_l = []
         for b in range(B):
             tr.s[b, l] = layer_dynamics(d_cur[b])
-            U = select_rows(d_cur[b], keys[b], B_window, int(budgets[b, l]), cfg.window_mode)
+            U = select_rows(d_cur[b], keys[b], B_window, int(budgets[b, l]), cfg.window_mode, force)
             sel_l.append(U)
             if len(U) == 0:
                 continue
             y = layer_rows(w.layers[l], cfg, st.H[l][b][U], U, st.K[l][b], st.V[l][b])
+            st.stale[l][b][U] = False
             if l + 1 < L:
                 d_next[b, U] = to_f32(cosine_distance(y, st.H[l + 1][b][U], w.layers[l + 1]["attn_norm"]))
+                st.stale[l + 1][b][U[np.any(y != st.H[l + 1][b][U], axis=1)]] = True
             st.H[l + 1][b][U] = y
         tr.sel.append(sel_l)
         d_cur = d_next

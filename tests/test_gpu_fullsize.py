@@ -56,8 +56,9 @@ def _snapshot(ctx, L):
             [dcu.dcu_get_tensor(ctx, dcu.DCU_T_V, l).clone() for l in range(L)])
 
 
-@pytest.mark.parametrize("name", list(CONFIGS))
-def test_fullsize_dcu_step(name):
+@pytest.mark.parametrize("name,fused", [(n, False) for n in CONFIGS] +
+                         [("llada8b_n1024", True), ("llada8b_batch4_n2048", True), ("dream7b_n1024", True)])
+def test_fullsize_dcu_step(name, fused):
     c = CONFIGS[name]
     shape, B = c["shape"], c["B"]
     N = c["n_prompt"] + c["n_gen"]
@@ -65,6 +66,7 @@ def test_fullsize_dcu_step(name):
     seed = 0
     W = I.device_weights(shape, seed)
     ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, int(fused))
     ids0 = np.stack([I.sequence_ids(1 + b, b, c["n_prompt"], c["n_gen"], shape.vocab) for b in range(B)])
     t_ids = torch.tensor(ids0, dtype=torch.int32, device="cuda")
     dcu.dcu_full_forward(ctx, t_ids)

@@ -27,8 +27,9 @@ def _snapshot(ctx, L):
             [dcu.dcu_get_tensor(ctx, dcu.DCU_T_V, l).clone() for l in range(L)])
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("B_layer,B_window", [(32, 32), (200, 16)])
-def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window):
+def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window, fused):
     shape, seed, n_prompt, n_gen = LONG_BF16, 7, 3840, 256
     N, B = n_prompt + n_gen, 1
     L, D, Hkv, hd, H = shape.n_layers, shape.d_model, shape.n_kv_heads, shape.head_dim, shape.n_heads
@@ -36,6 +37,7 @@ def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window):
     w_o = oracle_weights(shape, seed)
     W = I.device_weights(shape, seed)
     ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, int(fused))
     ids = np.stack([I.sequence_ids(seed, 0, n_prompt, n_gen, shape.vocab)])
     t_ids = torch.tensor(ids, dtype=torch.int32).cuda()
     dcu.dcu_full_forward(ctx, t_ids)

@@ -3,6 +3,7 @@
 // points, introspection and per-kernel event timing.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -32,7 +33,7 @@ struct ProfClass {
 // A captured dcu_step or commit_select: instantiated graph, the kernels it
 // launches and (when captured with profiling on) its event-record nodes.
 struct GraphEntry {
-  uint64_t key[10] = {};
+  uint64_t key[12] = {};
   cudaGraphExec_t exec = nullptr;
   int64_t kernels = 0;
   std::vector<std::pair<int, EventPair>> ev;
@@ -70,6 +71,14 @@ struct dcu_ctx {
   // select_from: DCU_SELECT_INPUT (layer-input distance) or DCU_SELECT_VALUE;
   // stale[l][r] = H_l row r was rewritten since layer l last recomputed it
   int select_from = DCU_SELECT_INPUT;
+  // adaptive parallel decoding: parameters, per-position thresholds, the
+  // logits of the current and previous commit ([2][cap][vocab] fp32, flipped
+  // every APD commit) and the last signals
+  bool apd = false;
+  float apd_alpha = 0.f, apd_beta = 0.f, apd_tau0 = 0.9f;
+  float *apd_z = nullptr, *apd_tau = nullptr, *apd_c = nullptr, *apd_h = nullptr;
+  uint8_t *apd_prev = nullptr;
+  int apd_flip = 0;
   uint8_t *stale = nullptr;
   int32_t *vrowmap = nullptr;
   bool have_cache = false, first_step = true;
@@ -833,6 +842,7 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
     static const int32_t one = 1;
     CK(c, cudaMemcpyAsync(c->uniform_flag(), &one, 4, cudaMemcpyHostToDevice, s));
   }
+  if (c->apd) LAUNCH(c, launch_apd_reset(c->apd_tau, c->apd_prev, c->cap, c->apd_tau0, s));  // a new generation
   c->first_step = true;
   c->have_cache = true;
   c->step_count = 0;
@@ -922,6 +932,11 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_l
       tp.smx = c->smx;
       tp.smx_arg = c->smx_arg;
       tp.ldm = cap;
+      if (rule == DCU_APD) {  // this commit's logits, by position, for the APD signals
+        tp.zout = c->apd_z + (size_t)c->apd_flip * cap * g.vocab;
+        tp.zrow = c->mrow;
+        tp.ldz = g.vocab;
+      }
       LAUNCH(c, launch_gemm_tc(tp, 256, s));
     } else {
       SlotGeo geo;
@@ -934,11 +949,22 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_l
                                   c->conf, c->amax, s));
     else
       LAUNCH(c, launch_softmax_max(c->C, g.vocab, c->mrow, c->m_masked(), cap, g.vocab, c->conf, c->amax, s));
+    if (rule == DCU_APD) {
+      // [DLLM] "关键设计 3": concentration, instability and the threshold update
+      float *zcur = c->apd_z + (size_t)c->apd_flip * cap * g.vocab;
+      const float *zprev = c->apd_z + (size_t)(1 - c->apd_flip) * cap * g.vocab;
+      if (g.dtype == DCU_BF16)
+        LAUNCH(c, launch_apd_signals(zcur, g.vocab, 1, nullptr, zprev, c->mrow, c->m_masked(), cap, g.vocab,
+                                     c->apd_prev, c->apd_tau, c->apd_alpha, c->apd_beta, c->apd_c, c->apd_h, s));
+      else  // the float32 LM head left the logits of packed row r in C
+        LAUNCH(c, launch_apd_signals(c->C, g.vocab, 0, zcur, zprev, c->mrow, c->m_masked(), cap, g.vocab,
+                                     c->apd_prev, c->apd_tau, c->apd_alpha, c->apd_beta, c->apd_c, c->apd_h, s));
+    }
   }
   {
     Prof p(c, DCU_K_COMMIT, s);
     LAUNCH(c, launch_commit_rule(rule, param, c->conf, c->amax, masked, ids, c->B, c->N, gen_start, block_len,
-                                 out_pos, out_count, s));
+                                 out_pos, out_count, rule == DCU_APD ? c->apd_tau : nullptr, s));
   }
   return DCU_OK;
 }
@@ -946,7 +972,7 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_l
 // Runs `body` directly, or through a cached CUDA graph keyed by `key` (captured
 // on the context's private stream, launched on s).
 template <class F>
-int run_graphed(dcu_ctx *c, const uint64_t (&key)[10], cudaStream_t s, F &&body) {
+int run_graphed(dcu_ctx *c, const uint64_t (&key)[12], cudaStream_t s, F &&body) {
   if (!c->use_graphs) return body(s);
   GraphEntry *g = nullptr;
   for (auto &e : c->graphs)
@@ -1013,7 +1039,7 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
     c->force_lo = pr ? 0 : (gr ? g0 : 0);
     c->force_hi = gr ? c->N : (pr ? g0 : 0);
   }
-  const uint64_t key[10] = {1,
+  const uint64_t key[12] = {1,
                             (uint64_t)(uintptr_t)ids,
                             (uint64_t)(uintptr_t)keys,
                             (uint64_t)(uintptr_t)nkeys,
@@ -1022,7 +1048,9 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
                             ((uint64_t)c->B << 32) | (uint64_t)c->N,
                             (uint64_t)(c->prof_max > 0),
                             ((uint64_t)(uint32_t)c->force_lo << 32) | (uint64_t)(uint32_t)c->force_hi,
-                            (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16)};
+                            (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16),
+                            0,
+                            0};
   int rc = run_graphed(c, key, (cudaStream_t)stream,
                        [&](cudaStream_t s) { return enqueue_step(c, ids, keys, nkeys, B_layer, B_window, s); });
   if (rc == DCU_OK) {
@@ -1049,6 +1077,35 @@ int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
   }
 }
 
+int dcu_set_apd(dcu_ctx *c, float alpha, float beta, float tau0) {
+  if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
+  if (!(alpha >= 0.0f) || !(beta >= 0.0f) || !std::isfinite(alpha) || !std::isfinite(beta) || !std::isfinite(tau0))
+    return fail(c, DCU_EINVAL, "alpha and beta must be finite and >= 0, tau0 finite");
+  if (c->capturing) return fail(c, DCU_ESTATE, "dcu_set_apd inside a stream capture");
+  if (!c->apd_z) {
+    const size_t cap = (size_t)c->cap, V = (size_t)c->cfg.vocab;
+    cudaError_t e = dalloc(c, &c->apd_z, 2 * cap * V * sizeof(float));
+    if (e == cudaSuccess) e = dalloc(c, &c->apd_tau, cap * sizeof(float));
+    if (e == cudaSuccess) e = dalloc(c, &c->apd_c, cap * sizeof(float));
+    if (e == cudaSuccess) e = dalloc(c, &c->apd_h, cap * sizeof(float));
+    if (e == cudaSuccess) e = dalloc(c, &c->apd_prev, cap);
+    if (e == cudaSuccess) e = cudaMemset(c->apd_c, 0, cap * sizeof(float));
+    if (e == cudaSuccess) e = cudaMemset(c->apd_h, 0, cap * sizeof(float));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(c, DCU_ENOMEM, std::string("APD buffers: ") + cudaGetErrorString(e));
+    }
+  }
+  c->apd = true;
+  c->apd_alpha = alpha;
+  c->apd_beta = beta;
+  c->apd_tau0 = tau0;
+  c->apd_flip = 0;
+  CK(c, launch_apd_reset(c->apd_tau, c->apd_prev, c->cap, tau0, nullptr));
+  CK(c, cudaDeviceSynchronize());
+  return DCU_OK;
+}
+
 int dcu_set_select_from(dcu_ctx *c, int32_t source) {
   if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
   if (source != DCU_SELECT_INPUT && source != DCU_SELECT_VALUE)
@@ -1071,15 +1128,20 @@ int commit_select_block(dcu_ctx *c, int32_t rule, float param, int32_t gen_start
                         uint8_t *masked, int32_t *ids, int32_t *out_pos, int32_t *out_count, dcu_stream_t stream) {
   if (!c) return fail(nullptr, DCU_EINVAL, "ctx is NULL");
   if (!c->have_cache) return fail(c, DCU_ESTATE, "commit_select before dcu_full_forward");
-  if (rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR)
-    return fail(c, DCU_EINVAL, "rule must be DCU_FRECHET, DCU_THRESHOLD or DCU_FACTOR");
+  if (rule != DCU_FRECHET && rule != DCU_THRESHOLD && rule != DCU_FACTOR && rule != DCU_APD)
+    return fail(c, DCU_EINVAL, "rule must be DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR or DCU_APD");
+  if (rule == DCU_APD && !c->apd) return fail(c, DCU_ESTATE, "DCU_APD before dcu_set_apd");
   if (!masked || !ids || !out_pos || !out_count) return fail(c, DCU_EINVAL, "a buffer is NULL");
   if (block_len > 0 && (gen_start < 0 || gen_start >= c->N))
     return fail(c, DCU_EINVAL, "gen_start must lie in [0, N) when block_len > 0");
   if (block_len < 0) block_len = 0;
   uint32_t pbits;
   memcpy(&pbits, &param, 4);
-  const uint64_t key[10] = {2,
+  uint32_t abits = 0, bbits = 0;
+  memcpy(&abits, &c->apd_alpha, 4);
+  memcpy(&bbits, &c->apd_beta, 4);
+  const bool apd = rule == DCU_APD;
+  const uint64_t key[12] = {2,
                             (uint64_t)rule,
                             (uint64_t)pbits,
                             (uint64_t)(uintptr_t)masked,
@@ -1088,10 +1150,14 @@ int commit_select_block(dcu_ctx *c, int32_t rule, float param, int32_t gen_start
                             (uint64_t)(uintptr_t)out_count,
                             ((uint64_t)c->B << 32) | (uint64_t)c->N,
                             (uint64_t)(c->prof_max > 0),
-                            ((uint64_t)(uint32_t)gen_start << 32) | (uint64_t)(uint32_t)block_len};
-  return run_graphed(c, key, (cudaStream_t)stream, [&](cudaStream_t s) {
+                            ((uint64_t)(uint32_t)gen_start << 32) | (uint64_t)(uint32_t)block_len,
+                            apd ? (uint64_t)(1 + c->apd_flip) : 0,
+                            apd ? (((uint64_t)abits << 32) | bbits) : 0};
+  const int rc = run_graphed(c, key, (cudaStream_t)stream, [&](cudaStream_t s) {
     return enqueue_commit(c, rule, param, gen_start, block_len, masked, ids, out_pos, out_count, s);
   });
+  if (rc == DCU_OK && apd) c->apd_flip ^= 1;  // this commit's logits are the next one's previous
+  return rc;
 }
 
 int commit_select(dcu_ctx *c, int32_t rule, float param, uint8_t *masked, int32_t *ids, int32_t *out_pos,
@@ -1160,7 +1226,7 @@ int dcu_commit_rule_block(int32_t rule, float param, int32_t gen_start, int32_t 
       !out_pos || !out_count || B <= 0 || N <= 0 || N > 16384 || (block_len > 0 && (gen_start < 0 || gen_start >= N)))
     return fail(nullptr, DCU_EINVAL, "dcu_commit_rule: bad argument");
   CK(nullptr, launch_commit_rule(rule, param, conf, argmax, masked, ids, B, N, gen_start, block_len > 0 ? block_len : 0,
-                                 out_pos, out_count, (cudaStream_t)stream));
+                                 out_pos, out_count, nullptr, (cudaStream_t)stream));
   return DCU_OK;
 }
 
@@ -1265,6 +1331,13 @@ static int tensor_ptr(dcu_ctx *c, int kind, int layer, char **p, int64_t *bytes)
       return DCU_OK;
     case DCU_T_ARGMAX:
       *p = (char *)c->amax;
+      *bytes = BN * 4;
+      return DCU_OK;
+    case DCU_T_APD_TAU:
+    case DCU_T_APD_C:
+    case DCU_T_APD_H:
+      if (!c->apd) return fail(c, DCU_ESTATE, "APD is not enabled (dcu_set_apd)");
+      *p = (char *)(kind == DCU_T_APD_TAU ? c->apd_tau : (kind == DCU_T_APD_C ? c->apd_c : c->apd_h));
       *bytes = BN * 4;
       return DCU_OK;
     case DCU_T_STALE:

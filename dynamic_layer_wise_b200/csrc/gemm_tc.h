@@ -117,6 +117,11 @@ struct TcParams {
   float2 *smx;
   int32_t *smx_arg;
   int ldm;
+  // epi_mode 1 with zout: the logits of token m are also stored at
+  // zout[zrow[m] * ldz + v] (fp32; the next commit's previous logits for APD)
+  float *zout;
+  const int32_t *zrow;
+  int64_t ldz;
   // L2 prefetch lookahead of the weight producer: with each TMA load of a
   // weight tile it prefetches the tile pf_ahead tiles past the shared-memory
   // ring into L2 (0: off), so more HBM requests are in flight than the ring holds.

@@ -724,9 +724,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           float &RM = lm_max[mt];
           double &RS = lm_sum[mt];
           int &RI = lm_arg[mt];
+          const int tok = it.pass * BN + mt * 128 + q * 32 + lane;
+          float *zdst = (p.zout && tok < M) ? p.zout + (int64_t)p.zrow[tok] * p.ldz + vbase : nullptr;
           for (int c = 0; c < 128; c += 16) {
             float v[16];
             tmem_ld16(tm + (uint32_t)c, v);
+            if (zdst) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (vbase + c + j < p.seg_rows[0]) zdst[c + j] = v[j];
+            }
             float cm = -INFINITY;
             int cj = 0;
 #pragma unroll

@@ -448,7 +448,7 @@ cudaError_t launch_plan_stale(const uint8_t *stale, int BN, int32_t *rowmap, int
 __global__ void __launch_bounds__(1024)
     k_commit_rule(int rule, float param, const float *__restrict__ conf, const int32_t *__restrict__ amax,
                   uint8_t *__restrict__ masked, int32_t *__restrict__ ids, int N, int gen_start, int block_len,
-                  int32_t *__restrict__ out_pos, int32_t *__restrict__ out_count) {
+                  int32_t *__restrict__ out_pos, int32_t *__restrict__ out_count, const float *__restrict__ tau) {
   pdl_enter();
   extern __shared__ uint64_t keys[];  // [P]
   __shared__ int red[32];
@@ -501,6 +501,34 @@ __global__ void __launch_bounds__(1024)
   // n*: each thread takes a contiguous run of sorted entries; fp64 prefix sums
   const int run = (m + nthr - 1) / nthr;
   const int j0 = tid * run, j1 = min(m, j0 + run);
+  if (rule == DCU_APD) {
+    // [DLLM] "关键设计 3": every candidate whose confidence reaches its own
+    // threshold, in descending confidence; none -> the most confident one
+    int cnt = 0;
+    for (int j = j0; j < j1; ++j) {
+      const int p = (int)(~(uint32_t)(keys[j] & 0xffffffffull));
+      cnt += __uint_as_float((uint32_t)(keys[j] >> 32)) >= tau[(size_t)b * N + p];
+    }
+    int total;
+    int k = block_exclusive_scan(cnt, red, &total);
+    if (total > 0) {
+      for (int j = j0; j < j1; ++j) {
+        const int p = (int)(~(uint32_t)(keys[j] & 0xffffffffull));
+        if (__uint_as_float((uint32_t)(keys[j] >> 32)) >= tau[(size_t)b * N + p]) {
+          out_pos[(size_t)b * N + k++] = p;
+          ids[(size_t)b * N + p] = amax[(size_t)b * N + p];
+          masked[(size_t)b * N + p] = 0;
+        }
+      }
+    } else if (tid == 0 && m > 0) {
+      const int p = (int)(~(uint32_t)(keys[0] & 0xffffffffull));
+      out_pos[(size_t)b * N] = p;
+      ids[(size_t)b * N + p] = amax[(size_t)b * N + p];
+      masked[(size_t)b * N + p] = 0;
+    }
+    if (tid == 0) out_count[b] = total > 0 ? total : (m > 0 ? 1 : 0);
+    return;
+  }
   double local = 0.0;
   for (int j = j0; j < j1; ++j) local += (double)__uint_as_float((uint32_t)(keys[j] >> 32));
   // exclusive scan of the per-thread fp64 sums (thread order)
@@ -574,14 +602,15 @@ __global__ void __launch_bounds__(1024)
 
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
                                int32_t *ids, int B, int N, int gen_start, int block_len, int32_t *out_pos,
-                               int32_t *out_count, cudaStream_t s) {
+                               int32_t *out_count, const float *tau, cudaStream_t s) {
   if (N > kMaxSeq || B <= 0) return cudaErrorInvalidValue;
   int P = 1;
   while (P < N) P <<= 1;
   static std::atomic<uint64_t> attr{0};
   if (cudaError_t e = ensure_smem_limit(k_commit_rule, kMaxSeq * (int)sizeof(uint64_t), attr)) return e;
+  if (rule == DCU_APD && !tau) return cudaErrorInvalidValue;
   launch_pdl(k_commit_rule, B, 1024, (size_t)P * sizeof(uint64_t), s, rule, param, conf, amax, masked, ids, N,
-             gen_start, block_len, out_pos, out_count);
+             gen_start, block_len, out_pos, out_count, tau);
   return cudaGetLastError();
 }
 

@@ -66,9 +66,10 @@ cudaError_t launch_plan_stale(const uint8_t *stale, int BN, int32_t *rowmap, int
 cudaError_t launch_plan_all(int B, int N, int32_t *rowmap, int32_t *m_total, int32_t *seq_off, cudaStream_t s);
 cudaError_t launch_plan_masked(const uint8_t *masked, int B, int N, int gen_start, int block_len, int32_t *rowmap,
                                int32_t *m_total, cudaStream_t s);
+// rule DCU_APD: commit every candidate with conf >= tau[b * N + i] (tau required), else the top one
 cudaError_t launch_commit_rule(int rule, float param, const float *conf, const int32_t *amax, uint8_t *masked,
                                int32_t *ids, int B, int N, int gen_start, int block_len, int32_t *out_pos,
-                               int32_t *out_count, cudaStream_t s);
+                               int32_t *out_count, const float *tau, cudaStream_t s);
 
 // ---- GEMM (k_gemm_simt.cu): C[m][n] = sum_k X[m][k] * W[n][k], m < *m_total (m < m_cap when m_total is null)
 cudaError_t launch_gemm_simt(int dtype, const void *X, int ldx, const int32_t *m_total, int m_cap,
@@ -89,6 +90,13 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
 cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,
                              int N, int H, int Hkv, int hd, const void *Kc, const void *Vc, void *out,
                              cudaStream_t s);
+
+// ---- adaptive parallel decoding (k_apd.cu)
+cudaError_t launch_apd_reset(float *tau, uint8_t *has_prev, int64_t n, float tau0, cudaStream_t s);
+// signals and threshold update of the packed candidate rows (see k_apd.cu)
+cudaError_t launch_apd_signals(const float *z_cur, int64_t ld_cur, int by_pos, float *z_copy, const float *z_prev,
+                               const int32_t *rowmap, const int32_t *m_total, int cap, int V, uint8_t *has_prev,
+                               float *tau, float alpha, float beta, float *out_c, float *out_h, cudaStream_t s);
 
 // ---- self-test (k_selftest.cu): one bounded mbarrier wait that must expire
 cudaError_t launch_wait_timeout_probe(int32_t *status, cudaStream_t s);

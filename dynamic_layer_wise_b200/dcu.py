@@ -19,10 +19,10 @@ LIB_PATH = os.path.join(_HERE, "libdcu.so")
 DCU_OK, DCU_EINVAL, DCU_ENOMEM, DCU_ECUDA, DCU_ECAPACITY, DCU_ESTATE, DCU_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 DCU_ST_BAD_KEY, DCU_ST_BAD_TOKEN, DCU_ST_TIMEOUT = 1, 2, 4
 DCU_F32, DCU_BF16 = 0, 1
-DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR = 0, 1, 2
+DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR, DCU_APD = 0, 1, 2, 3
 DCU_WINDOW_INCLUSIVE, DCU_WINDOW_HALFOPEN = 0, 1
 (DCU_T_H, DCU_T_K, DCU_T_V, DCU_T_D, DCU_T_S, DCU_T_S_PREV, DCU_T_BUDGET, DCU_T_SEL, DCU_T_SEL_COUNT,
- DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN, DCU_T_STALE) = range(13)
+ DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN, DCU_T_STALE, DCU_T_APD_TAU, DCU_T_APD_C, DCU_T_APD_H) = range(16)
 DCU_SELECT_INPUT, DCU_SELECT_VALUE = 0, 1
 DCU_OPT_FUSED_EPILOGUE, DCU_OPT_L2_PREFETCH = 1, 2
 (DCU_K_REFRESH, DCU_K_BUDGET, DCU_K_SELECT, DCU_K_GATHER, DCU_K_GEMM, DCU_K_EPILOGUE, DCU_K_ATTN, DCU_K_SCATTER,
@@ -82,6 +82,7 @@ _SIGS = {
     "dcu_set_refresh": (_i32, [_vp, _i32, _i32, _i32]),
     "dcu_set_select_from": (_i32, [_vp, _i32]),
     "dcu_set_option": (_i32, [_vp, _i32, _i32]),
+    "dcu_set_apd": (_i32, [_vp, _f32, _f32, _f32]),
     "dcu_linear": (_i32, [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp]),
     "dcu_lm_confidence_noalloc": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp]),
 }
@@ -272,7 +273,8 @@ def dcu_selftest_wait_timeout(status, stream=None):
 
 _KIND_DTYPE = {DCU_T_D: torch.float32, DCU_T_S: torch.float32, DCU_T_S_PREV: torch.float32,
                DCU_T_BUDGET: torch.int32, DCU_T_SEL: torch.int32, DCU_T_SEL_COUNT: torch.int32,
-               DCU_T_CONF: torch.float32, DCU_T_ARGMAX: torch.int32, DCU_T_STALE: torch.uint8}
+               DCU_T_CONF: torch.float32, DCU_T_ARGMAX: torch.int32, DCU_T_STALE: torch.uint8,
+               DCU_T_APD_TAU: torch.float32, DCU_T_APD_C: torch.float32, DCU_T_APD_H: torch.float32}
 
 
 def _kind_dtype(ctx: Context, kind: int):
@@ -359,3 +361,8 @@ def dcu_set_select_from(ctx: Context, source: int):
 def dcu_set_option(ctx: Context, option: int, value: int):
     """Performance option of the context (DCU_OPT_FUSED_EPILOGUE)."""
     _check(lib().dcu_set_option(ctx.handle, int(option), int(value)), ctx.handle)
+
+
+def dcu_set_apd(ctx: Context, alpha: float, beta: float, tau0: float = 0.9):
+    """Adaptive parallel decoding: enables rule DCU_APD with its alpha, beta and initial tau."""
+    _check(lib().dcu_set_apd(ctx.handle, float(alpha), float(beta), float(tau0)), ctx.handle)

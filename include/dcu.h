@@ -62,6 +62,8 @@ extern "C" {
 #define DCU_FRECHET   0     /* n* = max{n : G_n > delta}, else 1  ([FRECHET] "关键设计 2") */
 #define DCU_THRESHOLD 1     /* commit every c_i >= tau, else the top one ([FRECHET] "研究背景与动机") */
 #define DCU_FACTOR    2     /* largest n with (n+1)(1 - c_(n)) < f, else 1 (same section)      */
+#define DCU_APD       3     /* c_i >= tau_i with per-position adaptive tau, else the top one
+                               ([DLLM] "关键设计 3"; commit_select after dcu_set_apd only)      */
 
 #define DCU_SELECT_INPUT 0   /* d from the normalised layer inputs ([DLLM] "关键设计 1")          */
 #define DCU_SELECT_VALUE 1   /* d from recomputed vs cached Value rows ([README] select_from="v") */
@@ -149,6 +151,24 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
 #define DCU_OPT_L2_PREFETCH 2
 int dcu_set_option(dcu_ctx *ctx, int32_t option, int32_t value);
 
+/* Adaptive parallel decoding, APD ([DLLM] "关键设计 3").  Enables rule DCU_APD of
+ * commit_select / commit_select_block: at every such commit, for each
+ * candidate position i (masked, in the open block),
+ *   c_i = 1 - (second-highest probability of its LM-head distribution),
+ *   H_i = 1 - cos(p_i, p_i^prev), p^prev its distribution at the previous APD
+ *         commit (H_i = 0 the first time a position is a candidate),
+ *   tau_i <- tau_i - alpha c_i + beta H_i     (fp64, stored float32),
+ * then every candidate with confidence >= tau_i is committed (descending
+ * confidence), or the most confident one when none is.  The pages leave
+ * alpha, beta >= 0 open and start tau near 0.9, so all three are parameters.
+ * tau resets to tau0 and the history is cleared here and at every
+ * dcu_full_forward.  Allocates the logits of two commits, 2 x max_batch x
+ * max_seq x vocab floats, the first time (DCU_ENOMEM); synchronises the
+ * device; not inside a stream capture (DCU_ESTATE).  DCU_EINVAL for negative
+ * or non-finite alpha / beta or non-finite tau0.  Thresholds and signals:
+ * DCU_T_APD_TAU, DCU_T_APD_C, DCU_T_APD_H. */
+int dcu_set_apd(dcu_ctx *ctx, float alpha, float beta, float tau0);
+
 /* Feature source of the token dynamics d ([README] "Quick Start":
  * select_from; [DLLM] "关键设计 1" contrasts the layer-input proxy with
  * recomputing and comparing the Value vectors).  DCU_SELECT_INPUT (default):
@@ -235,7 +255,8 @@ int dcu_select_tokens(const float *d, const int32_t *key_positions, const int32_
 int dcu_cosine_distance(const void *x, const void *y, const float *gain, int64_t rows, int32_t D, int32_t dtype,
                         float *d, dcu_stream_t stream);
 
-/* Commit rule alone (the drop-in selector of [FRECHET] "整体框架"): per
+/* Commit rule alone (the drop-in selector of [FRECHET] "整体框架"; rules
+ * DCU_FRECHET, DCU_THRESHOLD, DCU_FACTOR -- DCU_APD needs a context): per
  * sequence, sorts the masked positions by conf (descending, ties to the lower
  * position) and commits n* of them by `rule` (param = delta | tau | f; fp64
  * prefix sums).  conf: dev float [B][N]; argmax: dev int32 [B][N];
@@ -300,6 +321,9 @@ int dcu_lm_confidence_noalloc(const void *h_rows, const float *final_norm, const
 #define DCU_T_ARGMAX   10  /* [B][N] int32, argmax of the last commit (masked positions)      */
 #define DCU_T_STALE    12  /* layer 0..L-1 : [B][N] uint8, 1 = the H_l row was rewritten with a new
                               value since layer l last recomputed it (settable) */
+#define DCU_T_APD_TAU  13  /* [B][N] float: APD thresholds tau (after dcu_set_apd)           */
+#define DCU_T_APD_C    14  /* [B][N] float: APD concentration c of the last APD commit      */
+#define DCU_T_APD_H    15  /* [B][N] float: APD instability H of the last APD commit        */
 #define DCU_T_ATTN     11  /* [B*N][n_heads*head_dim] dtype: attention output of the rows the
                               most recent layer recomputed (layer L-1 after dcu_step or
                               dcu_full_forward), packed sequence by sequence in ascending

@@ -475,16 +475,22 @@ def dcu_step(w: Weights, cfg: Config, state: State, ids: np.ndarray, keys: list,
 
 # ----------------------------------------------------------------- commit
 
-def confidence(h_rows: np.ndarray, final_norm: np.ndarray, lm_head, eps: float, chunk: int = 16384):
-    """LM head on the given final-layer rows, softmax, max probability and argmax
-    ([FRECHET] "整体框架": the argmax of every masked position and its
-    confidence c_i).  c = 1 / sum_v exp(z_v - z_max); argmax ties -> lowest id.
-    Returns (c as float32, argmax as int64)."""
+def logits(h_rows: np.ndarray, final_norm: np.ndarray, lm_head, eps: float, chunk: int = 16384) -> np.ndarray:
+    """z = W_lm RMSNorm(h) for the given final-layer rows, fp64 [m, V]."""
     h = rmsnorm(np.atleast_2d(np.asarray(h_rows, dtype=np.float64)), final_norm, eps)
     V = lm_head.shape[0]
     z = np.empty((h.shape[0], V))
     for v0 in range(0, V, chunk):
         z[:, v0:v0 + chunk] = h @ np.asarray(lm_head[v0:v0 + chunk], dtype=np.float64).T
+    return z
+
+
+def confidence(h_rows: np.ndarray, final_norm: np.ndarray, lm_head, eps: float, chunk: int = 16384):
+    """LM head on the given final-layer rows, softmax, max probability and argmax
+    ([FRECHET] "整体框架": the argmax of every masked position and its
+    confidence c_i).  c = 1 / sum_v exp(z_v - z_max); argmax ties -> lowest id.
+    Returns (c as float32, argmax as int64)."""
+    z = logits(h_rows, final_norm, lm_head, eps, chunk)
     zmax = np.max(z, axis=1)
     amax = np.argmax(z, axis=1)              # first maximum -> lowest id
     c = 1.0 / np.sum(np.exp(z - zmax[:, None]), axis=1)
@@ -547,7 +553,68 @@ def factor_count(c_sorted, f: float) -> int:
     return best if best > 0 else 1
 
 
-RULE_FRECHET, RULE_THRESHOLD, RULE_FACTOR = 0, 1, 2
+RULE_FRECHET, RULE_THRESHOLD, RULE_FACTOR, RULE_APD = 0, 1, 2, 3
+
+
+# ----------------------------------------------------------------- APD (adaptive parallel decoding)
+
+def apd_signals(z: np.ndarray, z_prev) -> tuple:
+    """The two per-token signals of [DLLM] "关键设计 3", from the logits z [m, V]
+    of this step and z_prev (the same positions' logits at the previous step,
+    or None where a position has none, given as a list of arrays / None):
+
+    * confidence concentration c = 1 - max_{v != u} p_v, u = argmax (the second
+      highest probability; with a tie at the top it is the top probability);
+    * temporal instability H = 1 - cos(p, p_prev) of the full probability
+      vectors of adjacent steps; 0 for a position seen for the first time
+      (reading: the page defines H from step t+1, which a first visit lacks).
+
+    Returns (c, H) as fp64 arrays [m]."""
+    z = np.atleast_2d(np.asarray(z, dtype=np.float64))
+    m = z.shape[0]
+    c = np.zeros(m)
+    H = np.zeros(m)
+    for i in range(m):
+        p = softmax_rows(z[i][None])[0]
+        top2 = np.sort(p)[-2:] if len(p) > 1 else np.array([0.0, p[0]])
+        c[i] = 1.0 - top2[0]
+        zp = None if z_prev is None else z_prev[i]
+        if zp is not None:
+            q = softmax_rows(np.asarray(zp, dtype=np.float64)[None])[0]
+            H[i] = 1.0 - float(p @ q) / (math.sqrt(float(p @ p)) * math.sqrt(float(q @ q)))
+    return c, H
+
+
+def apd_update(tau, c, H, alpha: float, beta: float) -> np.ndarray:
+    """[DLLM] "关键设计 3": tau_i^t = tau_i^{t+1} - alpha c_i^t + beta H_i^t, in fp64
+    from the stored float32 thresholds, stored again as float32."""
+    tau = np.asarray(tau, dtype=np.float32).astype(np.float64)
+    return to_f32(tau - float(alpha) * np.asarray(c, dtype=np.float64) + float(beta) * np.asarray(H, dtype=np.float64))
+
+
+def apd_commit(c, amax, masked, ids, tau, gen_start: int = 0, block_len: int = 0):
+    """APD commit ("τ 满足则 unmask": a token is unmasked once its confidence
+    reaches its own threshold): every candidate with c_i >= tau_i (float32),
+    in descending confidence (ties -> lower position); none -> the top one (as
+    the threshold rule, so decoding progresses).  Candidates as in commit().
+    Returns (positions, new ids, new masked)."""
+    masked = np.asarray(masked, dtype=bool)
+    blk = active_block(masked, gen_start, block_len)
+    open_ = np.zeros_like(masked)
+    if blk is not None:
+        open_[blk[0]:blk[1]] = True
+    pos = np.flatnonzero(masked & open_)
+    c32 = np.asarray(c, dtype=np.float32)
+    order = pos[np.lexsort((pos, -c32[pos].astype(np.float64)))]
+    t32 = np.asarray(tau, dtype=np.float32)
+    chosen = np.array([i for i in order if c32[i] >= t32[i]], dtype=np.int64)
+    if len(chosen) == 0 and len(order):
+        chosen = order[:1]
+    new_ids = np.array(ids, dtype=np.int64, copy=True)
+    new_masked = masked.copy()
+    new_ids[chosen] = np.asarray(amax)[chosen]
+    new_masked[chosen] = False
+    return chosen, new_ids, new_masked
 
 
 def rule_count(rule: int, c_sorted, param: float) -> int:

@@ -596,3 +596,60 @@ def test_value_mode_full_budget_equals_dense_forward():
     for l in range(cfg.n_layers + 1):
         np.testing.assert_allclose(st1.H[l], dense.H[l], rtol=0, atol=1e-6)
     assert not any(x.any() for x in st1.stale)
+
+
+# ------------------------------------------------------------------ APD (adaptive parallel decoding)
+
+def test_apd_concentration_closed_forms():
+    """c = 1 - (second-highest probability): p = (0.6, 0.3, 0.1) -> 0.7; a tie at
+    the top makes the second-highest the top probability: (0.4, 0.4, 0.2) -> 0.6."""
+    c, H = O.apd_signals(np.log([[0.6, 0.3, 0.1], [0.4, 0.4, 0.2]]), None)
+    np.testing.assert_allclose(c, [0.7, 0.6], rtol=0, atol=1e-12)
+    assert np.all(H == 0.0)                                # first visit: no instability yet
+
+
+def test_apd_instability_closed_forms_and_scipy():
+    """H = 1 - cos(p, p_prev): 0 for identical distributions; p = (1/2, 1/2, 0)
+    against (1/2, 0, 1/2) gives cos = 1/2; random logits agree with
+    scipy.spatial.distance.cosine of the softmax vectors."""
+    z = np.log(np.array([[0.5, 0.5, 1e-300], [0.2, 0.3, 0.5]]))
+    zp = [np.log(np.array([0.5, 1e-300, 0.5])), np.log(np.array([0.2, 0.3, 0.5]))]
+    _, H = O.apd_signals(z, zp)
+    np.testing.assert_allclose(H, [0.5, 0.0], rtol=0, atol=1e-12)
+    rng = np.random.default_rng(3)
+    z = rng.normal(0, 3, (5, 40))
+    zp = [rng.normal(0, 3, 40) for _ in range(5)]
+    _, H = O.apd_signals(z, zp)
+    ref = [scipy.spatial.distance.cosine(scipy.special.softmax(z[i]), scipy.special.softmax(zp[i])) for i in range(5)]
+    np.testing.assert_allclose(H, ref, rtol=1e-9, atol=1e-12)
+    _, H = O.apd_signals(z, [None, zp[1], None, zp[3], None])
+    assert H[0] == 0.0 and H[2] == 0.0 and H[1] > 0
+
+
+def test_apd_update_and_commit_reduce_to_threshold_rule():
+    """alpha = beta = 0 keeps tau; with H = 0 the threshold drops by alpha c; a
+    constant tau makes the APD commit the threshold rule (a different code path:
+    the sorted prefix with c >= tau); random per-position tau commits exactly
+    {i : c_i >= tau_i} (brute force), else the most confident position."""
+    tau = np.full(6, 0.9, dtype=np.float32)
+    c = np.linspace(0.1, 0.6, 6)
+    np.testing.assert_array_equal(O.apd_update(tau, c, np.ones(6), 0.0, 0.0), tau)
+    np.testing.assert_allclose(O.apd_update(tau, c, np.zeros(6), 0.5, 1.0), 0.9 - 0.5 * c, rtol=0, atol=1e-7)
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        N = int(rng.integers(1, 30))
+        conf = (rng.integers(0, 8, N) / 8).astype(np.float32)
+        masked = rng.random(N) < 0.7
+        ids = np.zeros(N, np.int64)
+        amax = rng.integers(0, 50, N)
+        t0 = float(rng.integers(0, 9) / 8)
+        a = O.apd_commit(conf, amax, masked, ids, np.full(N, t0, np.float32))
+        b = O.commit(conf, amax, masked, ids, O.RULE_THRESHOLD, t0)
+        assert list(a[0]) == list(b[0])
+        tau = (rng.integers(0, 9, N) / 8).astype(np.float32)
+        got = set(O.apd_commit(conf, amax, masked, ids, tau)[0].tolist())
+        want = {i for i in range(N) if masked[i] and conf[i] >= tau[i]}
+        if not want and masked.any():
+            mp = np.flatnonzero(masked)
+            want = {int(sorted(mp, key=lambda i: (-float(conf[i]), i))[0])}
+        assert got == want

@@ -45,6 +45,7 @@ constexpr size_t kMaxGraphs = 16;
 size_t esize(int dtype) { return dtype == DCU_BF16 ? 2 : 4; }
 
 constexpr int kAttnMaxSplits = 8;
+constexpr int kChainBars = 8;  // per layer: QKV launch 2, O + gate|up + down launch 6
 
 }  // namespace
 
@@ -110,13 +111,10 @@ struct dcu_ctx {
   // fused GEMM epilogues (bf16, head_dim 64 / 128): arrival counters of the
   // four layer GEMMs, per-tile row sums of squares (O -> gate|up) and per-tile
   // partial sums of the next-layer distance (down)
-  bool fused = false;        // fused path in use (DCU_OPT_FUSED_EPILOGUE and supported)
-  bool fused_ok = false;     // the model supports it (bf16, head_dim 64 or 128)
+  int fused = 0;             // chained launches in use (DCU_OPT_FUSED_EPILOGUE and supported): 1 or 2
+  bool fused_ok = false;     // the model supports them (bf16, head_dim 64 or 128)
   int nx_count = 16;         // units per CTA of the next GEMM's weights prefetched into L2 (0: off)
-  int32_t *epi_cnt = nullptr;
-  size_t epi_cnt_ints = 0;
-  int32_t *cnt_tile[4] = {}, *cnt_pass[4] = {};
-  double *ssq = nullptr, *dpart = nullptr;
+  int32_t *chain_bar = nullptr;  // grid-barrier counters of the chained launches, kChainBars per layer
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
   CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of min(128, cap) and min(256, cap) rows
@@ -298,29 +296,25 @@ struct ActOperand {
   const CUtensorMap *map128, *map256;  // activation boxes for 128- and 256-token passes
 };
 
-// tcgen05 GEMM parameters of C[m][n] = sum_k X[m][k] W[n][k] over the
+// One tcgen05 GEMM phase: C[m][n] = sum_k X[m][k] W[n][k] over the
 // concatenated weight segments (stream-K over all SMs unless tile_aligned).
-int gemm_params(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
-                const CUtensorMap *const *amaps, int nseg, int ldc, bool tile_aligned, TcParams *tp) {
+int gemm_phase(dcu_ctx *c, const ActOperand &x, const GemmSeg *segs, const CUtensorMap *const *amaps, int nseg,
+               int ldc, bool tile_aligned, TcPhase *ph) {
   const int cap = (int)c->cap;
-  memset(tp, 0, sizeof(*tp));
+  memset(ph, 0, sizeof(*ph));
   int tile = 0, col = 0;
   for (int i = 0; i < nseg; ++i) {
-    tp->a[i] = *amaps[i];
-    tp->seg_tile0[i] = tile;
-    tp->seg_col0[i] = col;
-    tp->seg_rows[i] = segs[i].rows;
+    ph->a[i] = *amaps[i];
+    ph->seg_tile0[i] = tile;
+    ph->seg_col0[i] = col;
+    ph->seg_rows[i] = segs[i].rows;
     tile += (segs[i].rows + 127) / 128;
     col += segs[i].rows;
   }
-  tp->seg_tile0[nseg] = tile;
-  tp->nseg = nseg;
-  tp->b = c->gemm_bn == 128 ? *x.map128 : *x.map256;
-  tp->b_rows = (int)c->act_box[c->gemm_bn == 128 ? 0 : 1];
-  tp->ldc = ldc;
-  tp->m_total = m_total;
-  tp->out = c->C;
-  tp->status = c->status();
+  ph->seg_tile0[nseg] = tile;
+  ph->nseg = nseg;
+  ph->b = c->gemm_bn == 128 ? *x.map128 : *x.map256;
+  ph->ldc = ldc;
   SlotGeo g;
   g.n_tiles = tile;
   g.kblocks = x.K / 64;
@@ -332,8 +326,18 @@ int gemm_params(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const G
     return fail(c, DCU_ECUDA, "GEMM workspace too small for the stream-K slots");
   g.nslots = c->slot_table(g);
   if (!g.nslots) return fail(c, DCU_ECUDA, "stream-K piece table unavailable for this GEMM geometry");
-  tp->geo = g;
+  ph->geo = g;
   return DCU_OK;
+}
+
+// Launch-wide fields of the tcgen05 GEMM (one phase until more are added).
+void gemm_common(dcu_ctx *c, const int32_t *m_total, TcParams *tp) {
+  memset(tp, 0, sizeof(*tp));
+  tp->nphase = 1;
+  tp->b_rows = (int)c->act_box[c->gemm_bn == 128 ? 0 : 1];
+  tp->m_total = m_total;
+  tp->out = c->C;
+  tp->status = c->status();
 }
 
 // C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
@@ -386,8 +390,7 @@ void set_prefetch(dcu_ctx *c, int l, int which, TcParams *tp) {
 
 int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const GemmSeg *segs,
              const CUtensorMap *const *amaps, int nseg, int ldc, cudaStream_t s, SlotGeo *geo,
-             bool tile_aligned = false, int prof_class = DCU_K_GEMM, int epi_mode = EPI_SLOTS,
-             const EpiArgs *ea = nullptr, int next_l = -1, int next_which = 0) {
+             bool tile_aligned = false, int prof_class = DCU_K_GEMM, int next_l = -1, int next_which = 0) {
   Prof p(c, prof_class, s);
   const int cap = (int)c->cap;
   memset(geo, 0, sizeof(*geo));
@@ -396,11 +399,10 @@ int run_gemm(dcu_ctx *c, const ActOperand &x, const int32_t *m_total, const Gemm
     return DCU_OK;
   }
   TcParams tp;
-  if (int rc = gemm_params(c, x, m_total, segs, amaps, nseg, ldc, tile_aligned, &tp)) return rc;
-  tp.epi_mode = epi_mode;
-  if (ea) tp.e = *ea;
+  gemm_common(c, m_total, &tp);
+  if (int rc = gemm_phase(c, x, segs, amaps, nseg, ldc, tile_aligned, &tp.ph[0])) return rc;
   if (next_l >= 0) set_prefetch(c, next_l, next_which, &tp);
-  *geo = tp.geo;
+  *geo = tp.ph[0].geo;
   LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
   return DCU_OK;
 }
@@ -449,13 +451,14 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
   const ActOperand ac{c->act, F, F, &c->act_map[0], &c->act_map[1]};
   SlotGeo geo;
   const int nqkv = (H + 2 * Hkv) * hd;
-  // fused epilogues: arguments shared by the four GEMMs of the layer
+  // chained launches (DCU_OPT_FUSED_EPILOGUE): QKV with its epilogue, then O,
+  // gate|up and down with theirs, each a persistent cooperative launch
+  const bool chained = c->fused;
   EpiArgs ea;
   memset(&ea, 0, sizeof(ea));
-  if (c->fused) {
+  if (chained) {
     ea.rowmap = c->rowmap;
     ea.N = c->N;
-    ea.cap = cap;
     ea.H = H;
     ea.Hkv = Hkv;
     ea.hd = hd;
@@ -464,37 +467,41 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
     ea.Q = c->Q;
     ea.Kc = c->Kl(l);
     ea.Vc = c->Vl(l);
+    ea.stale_l = c->stale_l(l);
     ea.D = D;
     ea.F = F;
     ea.eps = g.rms_eps;
     ea.Hl = c->Hl(l);
     ea.g2 = c->g2[l];
     ea.hmid = c->hmid;
-    ea.u = c->xs;
-    ea.ssq = c->ssq;
-    ea.ssq_ld = (D / 128 + 1) & ~1;
+    ea.xs = c->xs;
     ea.act = c->act;
     ea.Hn = c->Hl(l + 1);
     const bool want_d = !dense && !last;
     ea.g_next = want_d ? c->g1[l + 1] : nullptr;
     ea.d_next = want_d ? c->dl(l + 1) : nullptr;
-    ea.dpart = c->dpart;
-    ea.stale_l = c->stale_l(l);
     ea.stale_next = want_d ? c->stale_l(l + 1) : nullptr;
   }
   {
     GemmSeg seg[3] = {{c->wq[l], H * hd}, {c->wk[l], Hkv * hd}, {c->wv[l], Hkv * hd}};
     const CUtensorMap *am[3] = {lm ? &lm->wq : nullptr, lm ? &lm->wk : nullptr, lm ? &lm->wv : nullptr};
-    ea.tile_cnt = c->cnt_tile[0];
-    ea.pass_cnt = c->cnt_pass[0];
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo, false, DCU_K_GEMM,
-                          c->fused ? EPI_QKV : EPI_SLOTS, c->fused ? &ea : nullptr, l, 1))
-      return rc;
-  }
-  if (!c->fused) {
-    Prof p(c, DCU_K_EPILOGUE, s);
-    LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), gcap, c->N, H, Hkv,
-                             hd, c->rope_tab, g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), c->stale_l(l), s));
+    if (chained) {
+      Prof p(c, DCU_K_GEMM, s);
+      TcParams tp;
+      gemm_common(c, c->m_total(), &tp);
+      if (int rc = gemm_phase(c, xs, seg, am, 3, nqkv, false, &tp.ph[0])) return rc;
+      tp.ph[0].epi = EPI_QKV;
+      tp.chain = c->fused;
+      tp.bar = c->chain_bar + (size_t)l * kChainBars;
+      tp.e = ea;
+      set_prefetch(c, l, 1, &tp);
+      LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
+    } else {
+      if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 3, nqkv, s, &geo, false, DCU_K_GEMM, l, 1)) return rc;
+      Prof p(c, DCU_K_EPILOGUE, s);
+      LAUNCH(c, launch_epi_qkv(dt, c->C, nqkv, geo, c->rowmap, c->m_total(), gcap, c->N, H, Hkv, hd, c->rope_tab,
+                               g.rope_theta > 0.0f, c->Q, c->Kl(l), c->Vl(l), c->stale_l(l), s));
+    }
   }
   {
     Prof p(c, DCU_K_ATTN, s);
@@ -531,43 +538,40 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
                                  c->attn, s));
     }
   }
-  {
-    GemmSeg seg[1] = {{c->wo[l], D}};
-    const CUtensorMap *am[1] = {lm ? &lm->wo : nullptr};
-    ea.tile_cnt = c->cnt_tile[1];
-    ea.pass_cnt = c->cnt_pass[1];
-    if (int rc = run_gemm(c, at, c->m_total(), seg, am, 1, D, s, &geo, false, DCU_K_GEMM,
-                          c->fused ? EPI_O : EPI_SLOTS, c->fused ? &ea : nullptr, l, 2))
-      return rc;
+  GemmSeg seg_o[1] = {{c->wo[l], D}}, seg_gu[2] = {{c->wg[l], F}, {c->wu[l], F}}, seg_d[1] = {{c->wd[l], D}};
+  const CUtensorMap *am_o[1] = {lm ? &lm->wo : nullptr}, *am_gu[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr},
+                    *am_d[1] = {lm ? &lm->wd : nullptr};
+  if (chained) {
+    Prof p(c, DCU_K_GEMM, s);
+    TcParams tp;
+    gemm_common(c, c->m_total(), &tp);
+    if (int rc = gemm_phase(c, at, seg_o, am_o, 1, D, false, &tp.ph[0])) return rc;
+    if (int rc = gemm_phase(c, xs, seg_gu, am_gu, 2, 2 * F, false, &tp.ph[1])) return rc;
+    if (int rc = gemm_phase(c, ac, seg_d, am_d, 1, D, false, &tp.ph[2])) return rc;
+    tp.ph[0].epi = EPI_O;
+    tp.ph[1].epi = EPI_GU;
+    tp.ph[2].epi = EPI_DOWN;
+    tp.nphase = 3;
+    tp.chain = c->fused;
+    tp.bar = c->chain_bar + (size_t)l * kChainBars + 2;
+    tp.e = ea;
+    set_prefetch(c, l + 1, 0, &tp);
+    LAUNCH(c, launch_gemm_tc(tp, c->gemm_bn, s));
+    return DCU_OK;
   }
-  if (!c->fused) {
+  if (int rc = run_gemm(c, at, c->m_total(), seg_o, am_o, 1, D, s, &geo, false, DCU_K_GEMM, l, 2)) return rc;
+  {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_o(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->Hl(l), c->g2[l],
                            g.rms_eps, D, c->hmid, c->xs, s));
   }
+  if (int rc = run_gemm(c, xs, c->m_total(), seg_gu, am_gu, 2, 2 * F, s, &geo, false, DCU_K_GEMM, l, 3)) return rc;
   {
-    GemmSeg seg[2] = {{c->wg[l], F}, {c->wu[l], F}};
-    const CUtensorMap *am[2] = {lm ? &lm->wg : nullptr, lm ? &lm->wu : nullptr};
-    ea.tile_cnt = c->cnt_tile[2];
-    ea.pass_cnt = c->cnt_pass[2];
-    if (int rc = run_gemm(c, xs, c->m_total(), seg, am, 2, 2 * F, s, &geo, false, DCU_K_GEMM,
-                          c->fused ? EPI_GU : EPI_SLOTS, c->fused ? &ea : nullptr, l, 3))
-      return rc;
-  }
-  if (!c->fused) {
     Prof p(c, DCU_K_EPILOGUE, s);
     LAUNCH(c, launch_epi_swiglu(dt, c->C, 2 * F, geo, c->m_total(), gcap, F, c->act, s));
   }
+  if (int rc = run_gemm(c, ac, c->m_total(), seg_d, am_d, 1, D, s, &geo, false, DCU_K_GEMM, l + 1, 0)) return rc;
   {
-    GemmSeg seg[1] = {{c->wd[l], D}};
-    const CUtensorMap *am[1] = {lm ? &lm->wd : nullptr};
-    ea.tile_cnt = c->cnt_tile[3];
-    ea.pass_cnt = c->cnt_pass[3];
-    if (int rc = run_gemm(c, ac, c->m_total(), seg, am, 1, D, s, &geo, false, DCU_K_GEMM,
-                          c->fused ? EPI_DOWN : EPI_SLOTS, c->fused ? &ea : nullptr, l + 1, 0))
-      return rc;
-  }
-  if (!c->fused) {
     Prof p(c, DCU_K_SCATTER, s);
     const bool want_d = !dense && !last;
     LAUNCH(c, launch_epi_down_scatter(dt, c->C, D, geo, c->rowmap, c->m_total(), gcap, c->hmid,
@@ -696,26 +700,9 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
     c->attn_qt_cap = (int)(((size_t)cfg->max_seq * G + 127) / 128);
     AL(c->attn_po, (size_t)kAttnMaxSplits * cap * Hhd * 4);
     AL(c->attn_ml, (size_t)kAttnMaxSplits * cap * cfg->n_heads * sizeof(float2));
-    // fused GEMM epilogues: counters for up to cap / 128 token passes
+    // chained launches: grid-barrier counters
     c->fused_ok = true;
-    const size_t passes = (cap + 127) / 128;
-    const size_t tiles[4] = {nqkv / 128, D / 128, 2 * F / 128, D / 128};
-    const size_t pcnt[4] = {0, 0, passes * (F / 128), passes};
-    size_t n = 0;
-    for (int i = 0; i < 4; ++i) n += passes * tiles[i] + pcnt[i];
-    c->epi_cnt_ints = n;
-    AL(c->epi_cnt, n * 4);
-    AL(c->ssq, ((D / 128 + 1) & ~(size_t)1) * cap * sizeof(double));
-    AL(c->dpart, (D / 128) * cap * 4 * sizeof(double));
-    if (e == cudaSuccess) {
-      size_t o = 0;
-      for (int i = 0; i < 4; ++i) {
-        c->cnt_tile[i] = c->epi_cnt + o;
-        o += passes * tiles[i];
-        c->cnt_pass[i] = c->epi_cnt + o;
-        o += pcnt[i];
-      }
-    }
+    AL(c->chain_bar, (size_t)L * kChainBars * 4);
   }
 #undef AL
   if (e != cudaSuccess) {
@@ -727,7 +714,7 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   }
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
-  if (e == cudaSuccess && c->epi_cnt) e = cudaMemset(c->epi_cnt, 0, c->epi_cnt_ints * 4);
+  if (e == cudaSuccess && c->chain_bar) e = cudaMemset(c->chain_bar, 0, (size_t)L * kChainBars * 4);
   if (e == cudaSuccess) e = cudaMemset(c->stale, 0, (size_t)L * cap);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
@@ -831,7 +818,7 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
                                    c->cfg.d_model, c->cfg.vocab, 1, c->status(), nullptr, s));
   }
   LAUNCH(c, launch_plan_all(B, N, c->rowmap, c->m_total(), c->seq_off, s));
-  if (c->epi_cnt) CK(c, cudaMemsetAsync(c->epi_cnt, 0, c->epi_cnt_ints * 4, s));
+  if (c->chain_bar) CK(c, cudaMemsetAsync(c->chain_bar, 0, (size_t)c->cfg.n_layers * kChainBars * 4, s));
   c->gemm_bn = 256;
   c->gemm_rows_hint = BN;
   for (int l = 0; l < c->cfg.n_layers; ++l)
@@ -870,9 +857,8 @@ int enqueue_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int3
     // a larger set is still correct (a second pass re-streams the weights)
     c->gemm_bn = (c->gemm_rows_hint / 2) <= 96 ? 128 : 256;
   }
-  // arrival counters of the fused epilogues start from zero (each launch leaves
-  // them at zero; this clears what an aborted launch may have left)
-  if (c->epi_cnt) CK(c, cudaMemsetAsync(c->epi_cnt, 0, c->epi_cnt_ints * 4, s));
+  // grid-barrier counters of the chained launches count up from zero once per step
+  if (c->chain_bar) CK(c, cudaMemsetAsync(c->chain_bar, 0, (size_t)L * kChainBars * 4, s));
   {
     Prof p(c, DCU_K_BUDGET, s);
     LAUNCH(c, launch_budget_split(c->s_prev, c->B, L, B_layer, 0, c->uniform_flag(), c->budgets, s));
@@ -913,22 +899,24 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_l
       Prof p(c, DCU_K_LMHEAD, s);
       TcParams tp;
       memset(&tp, 0, sizeof(tp));
-      tp.a[0] = c->lm_map;
-      tp.b = c->xs_map[1];
+      tp.nphase = 1;
+      TcPhase &q = tp.ph[0];
+      q.a[0] = c->lm_map;
+      q.b = c->xs_map[1];
       tp.b_rows = (int)c->act_box[1];
       const int tiles = (g.vocab + 127) / 128;
-      tp.seg_tile0[0] = 0;
-      tp.seg_tile0[1] = tiles;
-      tp.seg_rows[0] = g.vocab;
-      tp.nseg = 1;
-      tp.geo.n_tiles = tiles;
-      tp.geo.kblocks = g.d_model / 64;
-      tp.geo.grid = tiles < c->num_sms ? tiles : c->num_sms;
-      tp.geo.tile_aligned = 1;
-      tp.ldc = g.vocab;
+      q.seg_tile0[0] = 0;
+      q.seg_tile0[1] = tiles;
+      q.seg_rows[0] = g.vocab;
+      q.nseg = 1;
+      q.geo.n_tiles = tiles;
+      q.geo.kblocks = g.d_model / 64;
+      q.geo.grid = tiles < c->num_sms ? tiles : c->num_sms;
+      q.geo.tile_aligned = 1;
+      q.ldc = g.vocab;
       tp.m_total = c->m_masked();
       tp.status = c->status();
-      tp.epi_mode = 1;
+      tp.epi_mode = EPI_LMHEAD;
       tp.smx = c->smx;
       tp.smx_arg = c->smx_arg;
       tp.ldm = cap;
@@ -1066,7 +1054,8 @@ int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
     case DCU_OPT_FUSED_EPILOGUE:
       if (value && !c->fused_ok)
         return fail(c, DCU_EINVAL, "fused epilogues need a bf16 model with head_dim 64 or 128");
-      c->fused = value != 0;
+      if (value < 0 || value > 2) return fail(c, DCU_EINVAL, "DCU_OPT_FUSED_EPILOGUE takes 0, 1 or 2");
+      c->fused = value;
       return DCU_OK;
     case DCU_OPT_L2_PREFETCH:
       if (value < 0 || value > 4096) return fail(c, DCU_EINVAL, "L2 prefetch units must lie in [0, 4096]");
@@ -1250,19 +1239,21 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
   }
   TcParams tp;
   memset(&tp, 0, sizeof(tp));
+  tp.nphase = 1;
+  TcPhase &q = tp.ph[0];
   const int bn = M <= 128 ? 128 : 256;
   const int m16 = (M + 15) / 16 * 16, b_rows = m16 < bn ? m16 : bn;  // activation box rows (multiple of 16)
-  if (!encode_tmap_bf16(&tp.a[0], W, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, 64, 128) ||
-      !encode_tmap_bf16(&tp.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)b_rows))
+  if (!encode_tmap_bf16(&q.a[0], W, (uint64_t)K, (uint64_t)Nout, (uint64_t)K * 2, 64, 128) ||
+      !encode_tmap_bf16(&q.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)b_rows))
     return fail(nullptr, DCU_ECUDA, "dcu_linear: cuTensorMapEncodeTiled failed");
   tp.b_rows = b_rows;
   const int tiles = (Nout + 127) / 128;
-  tp.seg_tile0[0] = 0;
-  tp.seg_tile0[1] = tiles;
-  tp.seg_col0[0] = 0;
-  tp.seg_rows[0] = Nout;
-  tp.nseg = 1;
-  tp.ldc = Nout;
+  q.seg_tile0[0] = 0;
+  q.seg_tile0[1] = tiles;
+  q.seg_col0[0] = 0;
+  q.seg_rows[0] = Nout;
+  q.nseg = 1;
+  q.ldc = Nout;
   tp.m_total = nullptr;
   tp.m_host = M;
   tp.out = Y;
@@ -1270,10 +1261,10 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  tp.geo.n_tiles = tiles;
-  tp.geo.kblocks = K / 64;
-  tp.geo.tile_aligned = 1;
-  tp.geo.grid = tiles < sms ? tiles : sms;
+  q.geo.n_tiles = tiles;
+  q.geo.kblocks = K / 64;
+  q.geo.tile_aligned = 1;
+  q.geo.grid = tiles < sms ? tiles : sms;
   CK(nullptr, launch_gemm_tc(tp, bn, s));
   return DCU_OK;
 }

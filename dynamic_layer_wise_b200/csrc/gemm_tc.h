@@ -11,7 +11,6 @@ constexpr int kTcMaxB = 4;                  // deepest activation-tile ring
 constexpr int kTcThreads = 224;             // 7 warps: W producer, MMA, 4 epilogue, X producer
 constexpr uint32_t kTcABytes = 128u * 128u;  // weight tile: 128 rows x 64 bf16
 constexpr size_t kTcSmem = 220u * 1024u;     // dynamic shared memory per CTA (one CTA per SM)
-constexpr uint32_t kFixBuf = 24u * 1024u;    // fused epilogues: bytes per fix-up staging buffer
 
 // Stream-K schedule: the flattened (tile, k block) space of one token pass,
 // T = n_tiles * kblocks, is cut into G contiguous ranges [c*T/G, (c+1)*T/G)
@@ -43,69 +42,72 @@ __host__ __device__ inline int sk_nslots(const SlotGeo &g, int tile) {
   return sk_owner(g, (long long)(tile + 1) * g.kblocks - 1) - sk_first(g, tile) + 1;
 }
 
-// Epilogues fused into the GEMM (epi_mode >= 2, bf16 layer GEMMs with head_dim
-// 64 or 128).  Every piece of a tile is stored in its slot as in epi_mode 0;
-// the CTA that stores a tile's last piece (an arrival counter per (pass,
-// tile), no CTA ever waits for another) sums the slots in slot order and
-// applies the layer's epilogue to the tile's 128 columns:
+// Epilogue kinds.  EPI_NONE: the pieces stay in their slots (separate
+// epilogue kernels sum them).  EPI_LMHEAD: softmax statistics of the LM head.
+// The other four are the layer epilogues of a chained launch (see TcParams):
 //   EPI_QKV   RoPE (rotate-half) on q and k, q -> Q[r], k / v -> the K/V cache
-//   EPI_O     hmid = H_l[row] + o (float), u = bf16(hmid * g2) (the gate|up
-//             operand), ssq[r][tile] = sum of hmid^2 over the tile's columns
-//   EPI_GU    the RMSNorm scale 1/sqrt(sum_tiles ssq / D + eps) of the row is
-//             applied to the summed gate / up pre-activations (the norm is
-//             linear in its input); the tile's result goes to slot 0; the second
-//             tile of a (gate j, up j) pair to finish writes act = silu(g) * u
-//   EPI_DOWN  new = hmid + down -> H_{l+1}[row] (scatter); when d_next is set,
-//             fp64 partial sums of the next-layer cosine distance against the
-//             cached row per tile; the last tile of the pass finishes d_next
-// The last arriver stages each chunk of its rows (the pieces, plus the row data
-// the epilogue reads) in shared memory with bulk copies, double-buffered, so
-// the fix-up moves its data at L2 bandwidth rather than at load latency.
-// Counters are zero between launches (each is reset by its last user).
-enum { EPI_SLOTS = 0, EPI_LMHEAD = 1, EPI_QKV = 2, EPI_O = 3, EPI_GU = 4, EPI_DOWN = 5 };
+//   EPI_O     hmid = H_l[row] + o (float); xs = bf16(RMSNorm(hmid) * g2)
+//   EPI_GU    act = bf16(silu(gate) * up)
+//   EPI_DOWN  new = hmid + down -> H_{l+1}[row] (scatter), next-layer d and
+//             stale flag against the cached row before it is overwritten
+enum { EPI_NONE = 0, EPI_LMHEAD = 1, EPI_QKV = 2, EPI_O = 3, EPI_GU = 4, EPI_DOWN = 5 };
+constexpr int kTcMaxPhases = 3;
+
+// Arguments of the chained epilogues.
 struct EpiArgs {
-  int32_t *tile_cnt;       // [passes][n_tiles] arrivals
-  int32_t *pass_cnt;       // EPI_GU: [passes][F / 128] pair arrivals; EPI_DOWN: [passes] finished tiles
   const int32_t *rowmap;   // packed row -> b * N + i
-  int N, cap;              // sequence length; rows of the row-indexed buffers
+  int N;                   // sequence length
   // EPI_QKV
   int H, Hkv, hd, use_rope;
   const float2 *rope_tab;  // [max_seq][hd / 2] (cos, sin)
   void *Q, *Kc, *Vc;       // Q [cap][H * hd]; the layer's K / V cache [B][Hkv][N][hd]
+  uint8_t *stale_l;        // cleared at the recomputed rows (may be null)
   // EPI_O / EPI_GU / EPI_DOWN
   int D, F;
   float eps;
   const void *Hl;          // layer input rows [B * N][D]
   const float *g2;         // FFN norm gain [D]
   float *hmid;             // [cap][D]
-  void *u;                 // [cap][D] bf16, gate|up operand
-  double *ssq;             // [cap][ssq_ld]: per row, one partial sum per tile of D
-  int ssq_ld;              // D / 128 rounded up to even (16-byte rows)
+  void *xs;                // [cap][D] bf16, gate|up operand
   void *act;               // [cap][F] bf16, down operand
   void *Hn;                // H_{l+1} rows [B * N][D]
   const float *g_next;     // next layer's attention-norm gain (null: no d)
   float *d_next;           // next layer's d [B * N] (null: no d)
-  double *dpart;           // [cap][D / 128][4]: dot, |x|^2, |y|^2, bitwise-equal flag
-  uint8_t *stale_l;        // EPI_QKV: cleared at the rows the layer recomputes (may be null)
-  uint8_t *stale_next;     // EPI_DOWN with d_next: set at rows whose H_{l+1} content changed (may be null)
+  uint8_t *stale_next;     // set at rows whose H_{l+1} content changed (may be null)
 };
 
-// Kernel parameters (passed as a __grid_constant__ so the tensor maps can be
-// addressed by TMA).  Output column of segment s, row r: seg_col0[s] + r;
-// every segment but the last has rows % 128 == 0, so column n lies in tile n / 128.
-// out[slot][m][n] = the piece `slot` of sum_k X[m][k] * W[n][k] for m < M.
-struct TcParams {
+// One GEMM of a launch: out[slot][m][n] = the piece `slot` of
+// sum_k X[m][k] * W[n][k] over the concatenated weight segments (output
+// column of segment s, row r: seg_col0[s] + r; every segment but the last has
+// rows % 128 == 0, so column n lies in tile n / 128).
+struct TcPhase {
   CUtensorMap a[3];        // weight segments, bf16 [rows][K], box 64 x 128, 128-byte swizzle
   CUtensorMap b;           // packed activations, bf16 [cap][K], box 64 x b_rows, 128-byte swizzle
-  int b_rows;              // rows of the activation box: the token pass (BN) or fewer when cap < BN
   int seg_tile0[4];        // first 128-row tile of segment s; seg_tile0[nseg] = n_tiles
   int seg_col0[3];         // first output column of segment s
   int seg_rows[3];         // rows of segment s
   int nseg, ldc;
-  SlotGeo geo;             // n_tiles, kblocks, grid (= gridDim.x), tile_aligned, slot stride
+  SlotGeo geo;             // n_tiles, kblocks, grid, tile_aligned, slot stride, piece table
+  int epi;                 // chained launches: the epilogue run after this phase
+};
+
+// Kernel parameters (passed as a __grid_constant__ so the tensor maps can be
+// addressed by TMA).  A launch runs nphase GEMMs over the same packed rows.
+// chain = 0: one GEMM (nphase = 1), its pieces in slots, or the LM head
+// (epi_mode 1).  chain = 1 (a cooperative launch, one CTA per SM): after each
+// phase every CTA meets a grid barrier, the phase's epilogue runs spread over
+// all CTAs, a second barrier publishes its outputs, and the next phase's
+// activation loads wait for that barrier while its weight loads have been
+// streaming all along.  bar: 2 * nphase counters, zero before the launch.
+struct TcParams {
+  TcPhase ph[kTcMaxPhases];
+  int nphase;
+  int chain;
+  int32_t *bar;
+  int b_rows;              // rows of the activation box: the token pass (BN) or fewer when cap < BN
   const int32_t *m_total;  // device row count M (or null: m_host)
   int m_host;
-  float *out;              // [slots][cap][ldc]
+  float *out;              // slots [slot][cap][ldc] (every phase uses the same buffer in turn)
   int32_t *status;         // device status word (DCU_ST_TIMEOUT) or null
   uint32_t smem_bytes;
   // epi_mode 1 (LM head, tile_aligned, BN = 256, one segment): the tokens are
@@ -122,10 +124,6 @@ struct TcParams {
   float *zout;
   const int32_t *zrow;
   int64_t ldz;
-  // L2 prefetch lookahead of the weight producer: with each TMA load of a
-  // weight tile it prefetches the tile pf_ahead tiles past the shared-memory
-  // ring into L2 (0: off), so more HBM requests are in flight than the ring holds.
-  int pf_ahead;
   // Prefetch of the next GEMM's weights: after its last TMA load, CTA c
   // prefetches into L2 the first nx_count (tile, k block) units of the ranges
   // of CTAs c, c + grid, ... of the next GEMM's stream-K geometry nx_geo over
@@ -135,7 +133,7 @@ struct TcParams {
   int nx_nseg;
   SlotGeo nx_geo;
   int nx_count;
-  EpiArgs e;               // epi_mode >= 2
+  EpiArgs e;               // chained epilogues
 };
 
 // Row-major bf16 matrix [outer][inner] with row pitch row_bytes, box
@@ -143,7 +141,8 @@ struct TcParams {
 // missing or the encoding is rejected.
 bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                       uint32_t box_inner, uint32_t box_outer);
-// bn: token rows per pass (128 or 256); the grid is p.geo.grid CTAs.
+// bn: token rows per pass (128 or 256); the grid is p.ph[0].geo.grid CTAs (a
+// cooperative launch when p.chain).
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s);
 // Most pieces a tile can be cut into under the stream-K split over `grid` CTAs.
 int tc_max_slots(int n_tiles, int grid);

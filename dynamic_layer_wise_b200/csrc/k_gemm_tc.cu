@@ -10,18 +10,21 @@
 // Warp roles (224 threads, one CTA per SM, persistent over work units):
 //   warp 0      weight producer (one lane): deep ring of 16 KB W tiles; it
 //               starts before the previous launch has finished (weights are
-//               never written by a kernel)
+//               never written by a kernel) and runs through every phase
 //   warp 6      activation producer (one lane): shallow ring of X tiles (from
 //               L2, one TMA box of the whole token pass per stage), after the
-//               programmatic-dependency wait
+//               programmatic-dependency wait (phase 0) or the grid barrier that
+//               publishes the previous phase's epilogue (chained phases)
 //   warp 1      TMEM allocator + MMA issuer (one lane): 4 x tcgen05.mma (K=16)
 //               per 64-wide k block, tcgen05.commit frees both smem stages
 //   warps 2..5  epilogue: tcgen05.ld of the 128 x BN fp32 tile, coalesced
-//               stores of the split-K partial (32 lanes = 32 consecutive n)
+//               stores of the split-K partial (32 lanes = 32 consecutive n);
+//               in a chained launch also the grid barriers and their share of
+//               each phase's epilogue (128 threads, named barrier 1)
 // A work unit is (weight tile, k split, token pass); the row count M is read
 // from the device, so one launch serves any recompute-set size inside a graph.
-// Every mbarrier wait is bounded: on expiry the CTA sets DCU_ST_TIMEOUT,
-// drains its own copies / MMAs in flight, frees TMEM and exits.
+// Every mbarrier wait and grid barrier is bounded: on expiry the CTA sets
+// DCU_ST_TIMEOUT, drains its own copies / MMAs in flight, frees TMEM and exits.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -36,18 +39,34 @@ struct Frag {
   int tile, kb0, kb1, seg, arow, slot;
 };
 
-// Fragment iterator over this CTA's stream-K range, pass by pass.
+// Fragment iterator over this CTA's stream-K range of one phase, pass by pass.
 struct FragIter {
   long long pos, end;
-  int pass;
+  int pass, ph;
 };
 
+__device__ __forceinline__ FragIter frag_begin(const TcParams &p, int ph) {
+  const SlotGeo &g = p.ph[ph].geo;
+  FragIter it;
+  it.ph = ph;
+  it.pass = 0;
+  if ((int)blockIdx.x < g.grid) {
+    it.pos = sk_begin(g, blockIdx.x);
+    it.end = sk_begin(g, blockIdx.x + 1);
+  } else {  // more CTAs than this phase has ranges
+    it.pos = it.end = 0;
+  }
+  return it;
+}
+
 __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIter &it, Frag &f) {
+  const TcPhase &q = p.ph[it.ph];
+  if ((int)blockIdx.x >= q.geo.grid) return false;  // no range in this phase
   while (it.pos >= it.end) {
     if (++it.pass >= passes) return false;
-    it.pos = sk_begin(p.geo, blockIdx.x);
+    it.pos = sk_begin(q.geo, blockIdx.x);
   }
-  const int KB = p.geo.kblocks;
+  const int KB = q.geo.kblocks;
   const int t = (int)(it.pos / KB);
   const int kb0 = (int)(it.pos - (long long)t * KB);
   const long long left = it.end - it.pos;
@@ -57,140 +76,100 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
   f.kb0 = kb0;
   f.kb1 = kb1;
   int seg = 0;
-  while (seg + 1 < p.nseg && t >= p.seg_tile0[seg + 1]) ++seg;
+  while (seg + 1 < q.nseg && t >= q.seg_tile0[seg + 1]) ++seg;
   f.seg = seg;
-  f.arow = (t - p.seg_tile0[seg]) * 128;
-  f.slot = (int)blockIdx.x - sk_first(p.geo, t);
+  f.arow = (t - q.seg_tile0[seg]) * 128;
+  f.slot = (int)blockIdx.x - sk_first(q.geo, t);
   return true;
 }
 
-
-
-// Position in this CTA's (fragment, k block) sequence.
+// Position in this CTA's (phase, fragment, k block) sequence.
 struct KCursor {
   FragIter it;
   Frag f;
-  int kb, m0, nb;
+  int kb, m0;
   bool valid;
-  __device__ __forceinline__ void load_frag(int BN, int M) {
-    kb = f.kb0;
-    m0 = it.pass * BN;
-    nb = (min(BN, M - m0) + 15) / 16;
-  }
-  __device__ __forceinline__ void start(const TcParams &p, int passes, long long b, long long e, int BN, int M) {
-    it = FragIter{b, e, 0};
+  __device__ __forceinline__ void start(const TcParams &p, int ph, int passes, int BN) {
+    it = frag_begin(p, ph);
     valid = next_frag(p, passes, it, f);
-    if (valid) load_frag(BN, M);
+    if (valid) {
+      kb = f.kb0;
+      m0 = it.pass * BN;
+    }
   }
-  __device__ __forceinline__ void advance(const TcParams &p, int passes, int BN, int M) {
+  __device__ __forceinline__ void advance(const TcParams &p, int passes, int BN) {
     if (++kb < f.kb1) return;
     valid = next_frag(p, passes, it, f);
-    if (valid) load_frag(BN, M);
+    if (valid) {
+      kb = f.kb0;
+      m0 = it.pass * BN;
+    }
   }
 };
 
-// ------------------------------------------------------------------ fused epilogues
-// Run by the 4 epilogue warps (128 threads, named barrier 1) of the CTA that
-// stored a tile's last piece.  The rows are processed in chunks staged in
-// shared memory (two buffers, one mbarrier each): one thread issues a bulk
-// copy per (row, piece) and per extra row slice, the 4 warps consume the
-// chunk one row per warp at a time, lane l owning the tile's columns
-// 4l .. 4l + 3, while the next chunk is in flight.
+// ------------------------------------------------------------------ chained launches
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d, uint32_t (&bits)[4]) {
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
-  uint2 u;
-  u.x = *reinterpret_cast<const uint32_t *>(&lo);
-  u.y = *reinterpret_cast<const uint32_t *>(&hi);
-  bits[0] = u.x & 0xffffu;
-  bits[1] = u.x >> 16;
-  bits[2] = u.y & 0xffffu;
-  bits[3] = u.y >> 16;
-  return u;
-}
-
-__device__ __forceinline__ void unpack_bf16x4(uint2 u, float (&v)[4], uint32_t (&bits)[4]) {
-  bits[0] = u.x & 0xffffu;
-  bits[1] = u.x >> 16;
-  bits[2] = u.y & 0xffffu;
-  bits[3] = u.y >> 16;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(bits[i] << 16);
-}
-
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
-// Shared-memory staging of the fix-ups.
-struct FixStage {
-  uint32_t sbase;   // smem address of buffer 0 (buffer 1 follows)
-  uint8_t *gbase;   // generic address of buffer 0
-  uint32_t bytes;   // per buffer
-  uint32_t bar;     // mbarriers of buffers 0 and 1 (8 bytes apart)
-  uint32_t uses[2]; // completed phases waited per buffer (the same in every thread)
-  int *rows;        // smem [BN]: global row (rowmap) of each packed row of the tile's pass
-  int32_t *status;
-  volatile int *abort;
-};
+// Spins (bounded by wall-clock time) until *ctr reaches target.
+__device__ __forceinline__ bool spin_count(const int32_t *ctr, int target, volatile int *abort_flag,
+                                           int32_t *status) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire(ctr) >= target) return true;
+    if ((it & 15u) == 15u) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        if (status) atomicOr(status, DCU_ST_TIMEOUT);
+        return false;
+      }
+    }
+    __nanosleep(128);
+  }
+}
 
-// Arrival of this CTA at a counter (after its global stores): true for the
-// arrival that makes it reach `total` (that CTA resets it).  All 128 epilogue
-// threads call it; only they use named barrier 1.
-__device__ __forceinline__ bool epi_arrive(int32_t *cnt, int total, int *s_flag, int ew, int lane) {
+// Grid barrier of the epilogue warps (all 128 threads of every CTA call it):
+// the CTA's earlier global stores are published, one arrival per CTA, then
+// every CTA waits for all gridDim.x arrivals.  False if the wait gave up.
+__device__ __forceinline__ bool grid_sync(int32_t *ctr, int ew, int lane, volatile int *abort_flag,
+                                          int32_t *status, int *s_flag) {
   __threadfence();
   epi_bar();
   if (ew == 0 && lane == 0) {
-    const int old = atomicAdd(cnt, 1);
-    const int last = (old == total - 1);
-    if (last) *cnt = 0;  // every arrival has happened: reset for the next launch
-    *s_flag = last;
+    atomicAdd(ctr, 1);
+    *s_flag = spin_count(ctr, (int)gridDim.x, abort_flag, status) ? 1 : 0;
   }
   epi_bar();
-  const bool last = *s_flag != 0;
-  if (last) {
-    __threadfence();
-    fence_proxy_async_global();  // the other CTAs' stores, next read by bulk copies
-  }
-  return last;
+  const bool ok = *s_flag != 0;
+  __threadfence();
+  return ok;
 }
 
-// Rows [0, mrows) of a pass in chunks of floor(bytes / row_bytes) rows: issue(r,
-// dst, bar) (one thread) copies packed row r's data to smem address dst;
-// compute(r, src) (one warp) consumes it from generic address src.
-template <class Issue, class Compute>
-__device__ __forceinline__ void staged_rows(FixStage &st, int mrows, uint32_t row_bytes, int ew, int lane,
-                                            Issue issue, Compute compute) {
-  const int R = max(1, min(mrows, (int)(st.bytes / row_bytes)));
-  const int nch = (mrows + R - 1) / R;
-  auto post = [&](int c) {
-    const int b = c & 1, r0 = c * R, r1 = min(mrows, r0 + R);
-    const uint32_t bar = st.bar + 8u * (uint32_t)b;
-    mbar_expect_tx(bar, (uint32_t)(r1 - r0) * row_bytes);
-    for (int r = r0; r < r1; ++r) issue(r, st.sbase + (uint32_t)b * st.bytes + (uint32_t)(r - r0) * row_bytes, bar);
-  };
-  if (ew == 0 && lane == 0) post(0);
-  for (int c = 0; c < nch; ++c) {
-    const int b = c & 1;
-    // buffer b ^ 1 was released by the barrier that ended chunk c - 1
-    if (c + 1 < nch && ew == 0 && lane == 0) post(c + 1);
-    const uint32_t bar = st.bar + 8u * (uint32_t)b, par = st.uses[b] & 1u;
-    if (!wait_bounded(bar, par, st.abort, st.status)) wait_drain(bar, par);  // the copies land before reuse
-    ++st.uses[b];
-    const int r0 = c * R, r1 = min(mrows, r0 + R);
-    for (int r = r0 + ew; r < r1; r += 4) compute(r, st.gbase + (size_t)b * st.bytes + (size_t)(r - r0) * row_bytes);
-    epi_bar();
-  }
+// Sum of the 128 epilogue threads' values (fixed tree; every thread gets it).
+__device__ __forceinline__ double sum128(double v, double *red, int ew, int lane) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  epi_bar();
+  if (lane == 0) red[ew] = v;
+  epi_bar();
+  return (red[0] + red[1]) + (red[2] + red[3]);
 }
 
-__device__ __forceinline__ float4 piece_sum(const uint8_t *src, int ns, int lane) {
-  float4 v = reinterpret_cast<const float4 *>(src)[lane];
+// 4 consecutive outputs of packed row r: the pieces of their tile summed in
+// slot order (read through L2: other CTAs of this launch wrote them).
+__device__ __forceinline__ float4 slot_sum4(const TcParams &p, const TcPhase &q, int r, int col) {
+  const float *c = p.out + (size_t)r * q.ldc + col;
+  float4 v = __ldcg(reinterpret_cast<const float4 *>(c));
+  const int ns = __ldg(q.geo.nslots + (col >> 7));
   for (int sp = 1; sp < ns; ++sp) {
-    const float4 w = reinterpret_cast<const float4 *>(src + sp * 512)[lane];
+    const float4 w = __ldcg(reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)q.geo.slot_stride));
     v.x += w.x;
     v.y += w.y;
     v.z += w.z;
@@ -199,258 +178,192 @@ __device__ __forceinline__ float4 piece_sum(const uint8_t *src, int ns, int lane
   return v;
 }
 
-// the ns pieces of packed row pr, 128 fp32 columns from output column col0
-__device__ __forceinline__ void issue_pieces(const TcParams &p, int ns, int pr, size_t col0, uint32_t dst, uint32_t bar) {
-  for (int sp = 0; sp < ns; ++sp)
-    bulk_g2s(dst + 512u * (uint32_t)sp, p.out + (size_t)sp * (size_t)p.geo.slot_stride + (size_t)pr * p.ldc + col0, 512,
-             bar);
+__device__ __forceinline__ uint2 pack_bf16x4(float a, float b, float c, float d) {
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+  uint2 u;
+  u.x = *reinterpret_cast<const uint32_t *>(&lo);
+  u.y = *reinterpret_cast<const uint32_t *>(&hi);
+  return u;
 }
 
-// EPI_QKV on tile t of segment seg (0 q, 1 k, 2 v).
-__device__ void fix_qkv(const TcParams &p, FixStage &st, int t, int seg, int m0, int mrows, int ns, int ew,
-                        int lane) {
+// EPI_QKV, items of 4 consecutive RoPE pairs or 4 v values over all rows.
+__device__ void epi_qkv(const TcParams &p, const TcPhase &q, int M, int t128) {
   const EpiArgs &e = p.e;
-  const int hd = e.hd, half = hd >> 1;
-  const int tcol0 = (t - p.seg_tile0[seg]) * 128;
-  const int tcol = tcol0 + lane * 4;  // column within the segment
-  const int head = tcol / hd, j4 = tcol - head * hd;
-  const bool first = j4 < half;
-  const int jr = first ? j4 : j4 - half;  // rotation index of the 4 pairs
-  const int xl = half >> 2;               // lane distance to the partner half
-  const size_t col0 = (size_t)p.seg_col0[seg] + (size_t)tcol0;
-  const bool rot = seg < 2 && e.use_rope;
+  const int H = e.H, Hkv = e.Hkv, hd = e.hd, half = hd / 2, N = e.N;
+  const int n_rope = (H + Hkv) * half / 4, n_v = Hkv * hd / 4;
+  const int per_row = n_rope + n_v;
   bf16 *Q = static_cast<bf16 *>(e.Q), *Kc = static_cast<bf16 *>(e.Kc), *Vc = static_cast<bf16 *>(e.Vc);
-  staged_rows(
-      st, mrows, 512u * (uint32_t)ns, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) { issue_pieces(p, ns, m0 + r, col0, dst, bar); },
-      [&](int r, const uint8_t *src) {
-        const int pr = m0 + r;
-        float4 v = piece_sum(src, ns, lane);
-        const int row = st.rows[r];
-        const int b = row / e.N, i = row - b * e.N;
-        if (rot) {
-          const float o[4] = {__shfl_xor_sync(0xffffffffu, v.x, xl), __shfl_xor_sync(0xffffffffu, v.y, xl),
-                              __shfl_xor_sync(0xffffffffu, v.z, xl), __shfl_xor_sync(0xffffffffu, v.w, xl)};
-          float a[4] = {v.x, v.y, v.z, v.w};
-          const float2 *cs = e.rope_tab + (size_t)i * half + jr;
+  for (long long it = (long long)blockIdx.x * 128 + t128; it < (long long)M * per_row; it += (long long)gridDim.x * 128) {
+    const int r = (int)(it / per_row), u = (int)(it - (long long)r * per_row);
+    const int row = e.rowmap[r];
+    const int b = row / N, i = row - b * N;
+    if (u < n_rope) {
+      const int t = u * 4;
+      const int head = t / half, j = t - head * half;
+      const int base = head * hd;  // q heads first, then k heads (contiguous in the output)
+      const float4 a = slot_sum4(p, q, r, base + j), bb = slot_sum4(p, q, r, base + j + half);
+      float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+      if (e.use_rope) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const float2 c = cs[k];
-            a[k] = first ? a[k] * c.x - o[k] * c.y : a[k] * c.x + o[k] * c.y;
-          }
-          v = make_float4(a[0], a[1], a[2], a[3]);
+        for (int k = 0; k < 4; ++k) {
+          const float2 cs = e.rope_tab[(size_t)i * half + j + k];
+          const float a2 = av[k] * cs.x - bv[k] * cs.y;
+          const float b2 = bv[k] * cs.x + av[k] * cs.y;
+          av[k] = a2;
+          bv[k] = b2;
         }
-        if (seg == 2 && tcol == 0 && e.stale_l) e.stale_l[row] = 0;  // the layer recomputes this row
-        bf16 *dst = seg == 0 ? Q + (size_t)pr * e.H * hd + (size_t)head * hd
-                             : (seg == 1 ? Kc : Vc) + (((size_t)b * e.Hkv + head) * e.N + i) * hd;
-        uint32_t bits[4];
-        *reinterpret_cast<uint2 *>(dst + j4) = pack_bf16x4(v.x, v.y, v.z, v.w, bits);
-      });
-}
-
-// EPI_O on tile t (columns t * 128 .. of D).
-__device__ void fix_o(const TcParams &p, FixStage &st, int t, int m0, int mrows, int ns, int ew, int lane) {
-  const EpiArgs &e = p.e;
-  const int col0 = t * 128, col = col0 + lane * 4;
-  const bf16 *Hl = static_cast<const bf16 *>(e.Hl);
-  bf16 *u = static_cast<bf16 *>(e.u);
-  const float4 g = *reinterpret_cast<const float4 *>(e.g2 + col);
-  const uint32_t pb = 512u * (uint32_t)ns;
-  staged_rows(
-      st, mrows, pb + 256u, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) {
-        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
-        bulk_g2s(dst + pb, Hl + (size_t)st.rows[r] * e.D + col0, 256, bar);
-      },
-      [&](int r, const uint8_t *src) {
-        const int pr = m0 + r;
-        const float4 v = piece_sum(src, ns, lane);
-        float x[4];
-        uint32_t xb[4];
-        unpack_bf16x4(reinterpret_cast<const uint2 *>(src + pb)[lane], x, xb);
-        const float4 hm = make_float4(x[0] + v.x, x[1] + v.y, x[2] + v.z, x[3] + v.w);
-        *reinterpret_cast<float4 *>(e.hmid + (size_t)pr * e.D + col) = hm;
-        uint32_t bits[4];
-        *reinterpret_cast<uint2 *>(u + (size_t)pr * e.D + col) =
-            pack_bf16x4(hm.x * g.x, hm.y * g.y, hm.z * g.z, hm.w * g.w, bits);
-        double ss = (double)hm.x * (double)hm.x + (double)hm.y * (double)hm.y + (double)hm.z * (double)hm.z +
-                    (double)hm.w * (double)hm.w;
-        ss = warp_sum_d(ss);
-        if (lane == 0) e.ssq[(size_t)pr * e.ssq_ld + t] = ss;
-      });
-}
-
-// EPI_GU on tile t: gate tiles are [0, F/128), up tiles [F/128, 2F/128).
-__device__ void fix_gu(const TcParams &p, FixStage &st, int t, int pass, int m0, int mrows, int ns, int ew,
-                       int lane, int *s_flag) {
-  const EpiArgs &e = p.e;
-  const int ft = e.F / 128, ntd = e.D / 128;
-  const int col0 = t * 128, col = col0 + lane * 4;  // column of [gate | up]
-  const uint32_t pb = 512u * (uint32_t)ns, sb = 8u * (uint32_t)e.ssq_ld;
-  staged_rows(
-      st, mrows, pb + sb, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) {
-        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
-        bulk_g2s(dst + pb, e.ssq + (size_t)(m0 + r) * e.ssq_ld, sb, bar);
-      },
-      [&](int r, const uint8_t *src) {
-        const int pr = m0 + r;
-        float4 v = piece_sum(src, ns, lane);
-        const double *sq = reinterpret_cast<const double *>(src + pb);
-        double ss = 0.0;
-        for (int k = lane; k < ntd; k += 32) ss += sq[k];
-        ss = warp_sum_d(ss);
-        const float inv = (float)(1.0 / sqrt(ss / (double)e.D + (double)e.eps));
-        v.x *= inv;
-        v.y *= inv;
-        v.z *= inv;
-        v.w *= inv;
-        *reinterpret_cast<float4 *>(p.out + (size_t)pr * p.ldc + col) = v;  // slot 0 now holds the result
-      });
-  const int pair = t < ft ? t : t - ft;
-  if (!epi_arrive(e.pass_cnt + (size_t)pass * ft + pair, 2, s_flag, ew, lane)) return;
-  // second tile of the pair: act = silu(gate) * up over the pair's 128 columns
-  const int j0 = pair * 128, j = j0 + lane * 4;
-  bf16 *act = static_cast<bf16 *>(e.act);
-  staged_rows(
-      st, mrows, 1024u, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) {
-        const float *row = p.out + (size_t)(m0 + r) * p.ldc;
-        bulk_g2s(dst, row + j0, 512, bar);
-        bulk_g2s(dst + 512u, row + e.F + j0, 512, bar);
-      },
-      [&](int r, const uint8_t *src) {
-        const float4 gt = reinterpret_cast<const float4 *>(src)[lane];
-        const float4 up = reinterpret_cast<const float4 *>(src + 512)[lane];
-        uint32_t bits[4];
-        *reinterpret_cast<uint2 *>(act + (size_t)(m0 + r) * e.F + j) =
-            pack_bf16x4(gt.x / (1.0f + expf(-gt.x)) * up.x, gt.y / (1.0f + expf(-gt.y)) * up.y,
-                        gt.z / (1.0f + expf(-gt.z)) * up.z, gt.w / (1.0f + expf(-gt.w)) * up.w, bits);
-      });
-}
-
-// EPI_DOWN on tile t (columns t * 128 .. of D).
-__device__ void fix_down(const TcParams &p, FixStage &st, int t, int pass, int m0, int mrows, int ns, int ew,
-                         int lane, int *s_flag) {
-  const EpiArgs &e = p.e;
-  const int ntd = e.D / 128;
-  const int col0 = t * 128, col = col0 + lane * 4;
-  const bool want_d = e.d_next != nullptr;
-  bf16 *Hn = static_cast<bf16 *>(e.Hn);
-  float gg[4] = {0.f, 0.f, 0.f, 0.f};
-  if (want_d) {
-    const float4 g = *reinterpret_cast<const float4 *>(e.g_next + col);
-    gg[0] = g.x;
-    gg[1] = g.y;
-    gg[2] = g.z;
-    gg[3] = g.w;
+      }
+      bf16 *dst = head < H ? Q + (size_t)r * H * hd + (size_t)head * hd
+                           : Kc + (((size_t)b * Hkv + (head - H)) * N + i) * hd;
+      *reinterpret_cast<uint2 *>(dst + j) = pack_bf16x4(av[0], av[1], av[2], av[3]);
+      *reinterpret_cast<uint2 *>(dst + j + half) = pack_bf16x4(bv[0], bv[1], bv[2], bv[3]);
+    } else {
+      const int t = (u - n_rope) * 4;
+      const int kvh = t / hd, j = t - kvh * hd;
+      if (t == 0 && e.stale_l) e.stale_l[row] = 0;  // the layer recomputes this row
+      const float4 v = slot_sum4(p, q, r, (H + Hkv) * hd + t);
+      *reinterpret_cast<uint2 *>(Vc + (((size_t)b * Hkv + kvh) * N + i) * hd + j) = pack_bf16x4(v.x, v.y, v.z, v.w);
+    }
   }
-  const uint32_t pb = 512u * (uint32_t)ns;
-  staged_rows(
-      st, mrows, pb + 512u + 256u, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) {
-        issue_pieces(p, ns, m0 + r, (size_t)col0, dst, bar);
-        bulk_g2s(dst + pb, e.hmid + (size_t)(m0 + r) * e.D + col0, 512, bar);
-        bulk_g2s(dst + pb + 512u, Hn + (size_t)st.rows[r] * e.D + col0, 256, bar);  // the cached row
-      },
-      [&](int r, const uint8_t *src) {
-        const int pr = m0 + r;
-        const float4 v = piece_sum(src, ns, lane);
-        const float4 hm = reinterpret_cast<const float4 *>(src + pb)[lane];
-        float nv[4] = {hm.x + v.x, hm.y + v.y, hm.z + v.z, hm.w + v.w};
-        uint32_t nb[4];
-        const uint2 packed = pack_bf16x4(nv[0], nv[1], nv[2], nv[3], nb);
-        if (want_d) {
-          float ov[4];
-          uint32_t ob[4];
-          unpack_bf16x4(reinterpret_cast<const uint2 *>(src + pb + 512)[lane], ov, ob);
-          double dot = 0.0, nx = 0.0, ny = 0.0;
-          bool same = true;
+}
+
+// EPI_O, one row per CTA: hmid = H_l[row] + o; xs = bf16(hmid / rms(hmid) * g2).
+__device__ void epi_o(const TcParams &p, const TcPhase &q, int M, int t128, int ew, int lane, double *red) {
+  const EpiArgs &e = p.e;
+  const int D = e.D;
+  const bf16 *Hl = static_cast<const bf16 *>(e.Hl);
+  bf16 *xs = static_cast<bf16 *>(e.xs);
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    const bf16 *x = Hl + (size_t)e.rowmap[r] * D;
+    float *hm = e.hmid + (size_t)r * D;
+    double ss = 0;
+    for (int j = t128 * 8; j < D; j += 128 * 8) {
+      float v[8];
+      load_vec(x + j, v);
+      const float4 c0 = slot_sum4(p, q, r, j), c1 = slot_sum4(p, q, r, j + 4);
+      v[0] += c0.x; v[1] += c0.y; v[2] += c0.z; v[3] += c0.w;
+      v[4] += c1.x; v[5] += c1.y; v[6] += c1.z; v[7] += c1.w;
+      *reinterpret_cast<float4 *>(hm + j) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4 *>(hm + j + 4) = make_float4(v[4], v[5], v[6], v[7]);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            same = same && (nb[k] == ob[k]);
-            const double a = (double)gg[k] * (double)__uint_as_float(nb[k] << 16), b = (double)gg[k] * (double)ov[k];
-            dot += a * b;
-            nx += a * a;
-            ny += b * b;
-          }
-          dot = warp_sum_d(dot);
-          nx = warp_sum_d(nx);
-          ny = warp_sum_d(ny);
-          same = __all_sync(0xffffffffu, same);
-          if (lane == 0) {
-            double *o = e.dpart + ((size_t)pr * ntd + t) * 4;
-            o[0] = dot;
-            o[1] = nx;
-            o[2] = ny;
-            o[3] = same ? 1.0 : 0.0;
-          }
+      for (int k = 0; k < 8; ++k) ss += (double)v[k] * (double)v[k];
+    }
+    ss = sum128(ss, red, ew, lane);
+    const float inv = (float)(1.0 / sqrt(ss / (double)D + (double)e.eps));
+    bf16 *o = xs + (size_t)r * D;
+    for (int j = t128 * 8; j < D; j += 128 * 8) {
+      const float4 h0 = *reinterpret_cast<const float4 *>(hm + j), h1 = *reinterpret_cast<const float4 *>(hm + j + 4);
+      const float *g = e.g2 + j;
+      *reinterpret_cast<uint2 *>(o + j) =
+          pack_bf16x4(h0.x * inv * g[0], h0.y * inv * g[1], h0.z * inv * g[2], h0.w * inv * g[3]);
+      *reinterpret_cast<uint2 *>(o + j + 4) =
+          pack_bf16x4(h1.x * inv * g[4], h1.y * inv * g[5], h1.z * inv * g[6], h1.w * inv * g[7]);
+    }
+  }
+}
+
+// EPI_GU, items of 4 consecutive columns over all rows: act = silu(gate) * up.
+__device__ void epi_gu(const TcParams &p, const TcPhase &q, int M, int t128) {
+  const EpiArgs &e = p.e;
+  const int F = e.F, per_row = F / 4;
+  bf16 *act = static_cast<bf16 *>(e.act);
+  for (long long it = (long long)blockIdx.x * 128 + t128; it < (long long)M * per_row; it += (long long)gridDim.x * 128) {
+    const int r = (int)(it / per_row), j = (int)(it - (long long)r * per_row) * 4;
+    const float4 gt = slot_sum4(p, q, r, j), up = slot_sum4(p, q, r, F + j);
+    *reinterpret_cast<uint2 *>(act + (size_t)r * F + j) =
+        pack_bf16x4(gt.x / (1.0f + expf(-gt.x)) * up.x, gt.y / (1.0f + expf(-gt.y)) * up.y,
+                    gt.z / (1.0f + expf(-gt.z)) * up.z, gt.w / (1.0f + expf(-gt.w)) * up.w);
+  }
+}
+
+// EPI_DOWN, one row per CTA: new = bf16(hmid + down); with d_next, the next
+// layer's distance against the cached row (before it is overwritten) and the
+// stale flag; H_{l+1}[row] = new.
+__device__ void epi_down(const TcParams &p, const TcPhase &q, int M, int t128, int ew, int lane, double *red,
+                         int *s_flag) {
+  const EpiArgs &e = p.e;
+  const int D = e.D;
+  bf16 *Hn = static_cast<bf16 *>(e.Hn);
+  const bool want_d = e.d_next != nullptr;
+  for (int r = blockIdx.x; r < M; r += gridDim.x) {
+    const int row = e.rowmap[r];
+    const float *hm = e.hmid + (size_t)r * D;
+    bf16 *dst = Hn + (size_t)row * D;
+    double dot = 0, nx = 0, ny = 0;
+    bool same = true;
+    for (int j = t128 * 8; j < D; j += 128 * 8) {
+      const float4 c0 = slot_sum4(p, q, r, j), c1 = slot_sum4(p, q, r, j + 4);
+      const float4 h0 = __ldcg(reinterpret_cast<const float4 *>(hm + j)),
+                   h1 = __ldcg(reinterpret_cast<const float4 *>(hm + j + 4));
+      float v[8] = {h0.x + c0.x, h0.y + c0.y, h0.z + c0.z, h0.w + c0.w,
+                    h1.x + c1.x, h1.y + c1.y, h1.z + c1.z, h1.w + c1.w};
+      if (want_d) {
+        float ov[8];
+        uint32_t ob[8];
+        load_vec(dst + j, ov, ob);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const bf16 nt = __float2bfloat16_rn(v[k]);
+          const float nv = __bfloat162float(nt);
+          same = same && ((uint32_t)__bfloat16_as_ushort(nt) == ob[k]);
+          const double gg = (double)e.g_next[j + k];
+          const double a = gg * (double)nv, b = gg * (double)ov[k];
+          dot += a * b;
+          nx += a * a;
+          ny += b * b;
         }
-        *reinterpret_cast<uint2 *>(Hn + (size_t)st.rows[r] * e.D + col) = packed;
-      });
-  if (!want_d) return;
-  if (!epi_arrive(e.pass_cnt + pass, ntd, s_flag, ew, lane)) return;
-  // last tile of the pass: the next-layer d of every row of the pass
-  staged_rows(
-      st, mrows, 32u * (uint32_t)ntd, ew, lane,
-      [&](int r, uint32_t dst, uint32_t bar) {
-        bulk_g2s(dst, e.dpart + (size_t)(m0 + r) * ntd * 4, 32u * (uint32_t)ntd, bar);
-      },
-      [&](int r, const uint8_t *src) {
-        const double *o = reinterpret_cast<const double *>(src);
-        double dot = 0.0, nx = 0.0, ny = 0.0;
-        bool same = true;
-        for (int k = lane; k < ntd; k += 32) {
-          dot += o[4 * k];
-          nx += o[4 * k + 1];
-          ny += o[4 * k + 2];
-          same = same && (o[4 * k + 3] != 0.0);
-        }
-        dot = warp_sum_d(dot);
-        nx = warp_sum_d(nx);
-        ny = warp_sum_d(ny);
-        same = __all_sync(0xffffffffu, same);
-        if (lane == 0) {
-          const int row = st.rows[r];
-          e.d_next[row] = finish_cosine_distance(dot, nx, ny, same);
-          if (e.stale_next && !same) e.stale_next[row] = 1;  // H_{l+1} row changed
-        }
-      });
+      }
+      store_vec(dst + j, v);
+    }
+    if (want_d) {
+      epi_bar();
+      if (ew == 0 && lane == 0) *s_flag = 1;
+      epi_bar();
+      if (!same) *s_flag = 0;
+      dot = sum128(dot, red, ew, lane);
+      nx = sum128(nx, red, ew, lane);
+      ny = sum128(ny, red, ew, lane);
+      const bool all_same = *s_flag != 0;
+      if (ew == 0 && lane == 0) {
+        e.d_next[row] = finish_cosine_distance(dot, nx, ny, all_same);
+        if (e.stale_next && !all_same) e.stale_next[row] = 1;  // H_{l+1} row changed
+      }
+      epi_bar();
+    }
+  }
 }
 
 template <int BN>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 7];
+  __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
-  __shared__ int s_epi_ok[4], s_epi_flag;
-  __shared__ int s_rows[256];  // fused epilogues: global rows of the pass being fixed up
+  __shared__ int s_epi_ok[4], s_flag, s_same;
+  __shared__ double s_red[4];
 
   // The row count is written by the select / plan kernel two launches before
   // this one, so it is final even while the previous launch still runs.
   const int M = p.m_total ? *p.m_total : p.m_host;
-  if (M <= 0) return;
+  if (M <= 0) return;  // every CTA of a chained launch leaves here, or none
   const int passes = (M + BN - 1) / BN;
-  const long long my_begin = sk_begin(p.geo, blockIdx.x), my_end = sk_begin(p.geo, blockIdx.x + 1);
-  if (my_begin >= my_end) return;
+  if (!p.chain) {  // a CTA without work may leave (no barrier waits for it)
+    const FragIter it0 = frag_begin(p, 0);
+    if (it0.pos >= it0.end) return;
+  }
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Two rings: weight tiles (16 KB, from HBM) and activation tiles (16-row
-  // boxes of the rows actually loaded, from L2).  The activation ring only has
+  // Two rings: weight tiles (16 KB, from HBM) and activation tiles (one TMA
+  // box of the token pass per stage, from L2).  The activation ring only has
   // to cover the L2 latency, so most of shared memory holds weight tiles in
   // flight.
   const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per stage
   const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned stages
   const int SB = b_stage > 16384u ? 3 : 4;
-  // fused epilogues: two fix-up staging buffers after the rings (the weight
-  // ring keeps >= 6 stages, which the pure weight stream needs)
-  const uint32_t fix_bytes = p.epi_mode >= EPI_QKV ? 2u * kFixBuf : 0u;
-  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage - fix_bytes) / kTcABytes);
+  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage) / kTcABytes);
   SA = SA > kTcMaxA ? kTcMaxA : SA;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bbase = sbase + (uint32_t)SA * kTcABytes;
-  const uint32_t fbase = bbase + (uint32_t)SB * b_stage;
   const uint32_t bar0 = smem_u32(bars);
   // two TMEM accumulators (columns [0, BN) and [BN, 2 BN)) alternate between fragments
 #define FULL_A(s) (bar0 + 8u * (uint32_t)(s))
@@ -458,7 +371,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
 #define FULL_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + (s)))
 #define EMPTY_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + kTcMaxB + (s)))
   const uint32_t tfull0 = bar0 + 8u * (uint32_t)(2 * kTcMaxA + 2 * kTcMaxB), tempty0 = tfull0 + 16u,
-                 drain = tfull0 + 32u, fixbar = tfull0 + 40u;
+                 drain = tfull0 + 32u;
 #define TFULL(a) (tfull0 + 8u * (uint32_t)(a))
 #define TEMPTY(a) (tempty0 + 8u * (uint32_t)(a))
 #define STAGE_A(s) (sbase + (uint32_t)(s) * kTcABytes)
@@ -478,8 +391,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       mbar_init(TEMPTY(a), 4);
     }
     mbar_init(drain, 1);
-    mbar_init(fixbar, 1);
-    mbar_init(fixbar + 8u, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -495,47 +406,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
 
   if (warp == 0) {
     // weight producer: the weights are never written by a kernel, so the ring
-    // fills before (and while) the previous launch finishes
+    // fills before (and while) the previous launch or phase finishes
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();  // weights stream through once
       uint32_t fill_parity[kTcMaxA];
       bool used[kTcMaxA];
       for (int s = 0; s < kTcMaxA; ++s) used[s] = false;
-      KCursor ca;
-      ca.start(p, passes, my_begin, my_end, BN, M);
-      // L2 prefetch cursor, pf_ahead tiles past the ring (the first SA loads
-      // are issued at once, so it starts at tile SA)
-      KCursor cp;
-      cp.start(p, passes, my_begin, my_end, BN, M);
-      const int look = p.pf_ahead > 0 ? SA + p.pf_ahead : 0;
-      int cp_idx = 0;
-      if (look > 0)
-        while (cp.valid && cp_idx < SA) {
-          cp.advance(p, passes, BN, M);
-          ++cp_idx;
-        }
-      int stage = 0, ld_idx = 0;
+      int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      while (ca.valid) {
-        while (look > 0 && cp.valid && cp_idx <= ld_idx + look) {
-          tma_prefetch_2d(&p.a[cp.f.seg], cp.kb * 64, cp.f.arow);
-          cp.advance(p, passes, BN, M);
-          ++cp_idx;
-        }
-        if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        mbar_expect_tx(FULL_A(stage), kTcABytes);
-        tma_load_2d(STAGE_A(stage), &p.a[ca.f.seg], ca.kb * 64, ca.f.arow, FULL_A(stage), pol_w);
-        used[stage] = true;
-        fill_parity[stage] = phase;
-        ca.advance(p, passes, BN, M);
-        ++ld_idx;
-        if (++stage == SA) {
-          stage = 0;
-          phase ^= 1u;
+      for (int ph = 0; ph < p.nphase && ok; ++ph) {
+        KCursor ca;
+        ca.start(p, ph, passes, BN);
+        while (ca.valid) {
+          if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(FULL_A(stage), kTcABytes);
+          tma_load_2d(STAGE_A(stage), &p.ph[ph].a[ca.f.seg], ca.kb * 64, ca.f.arow, FULL_A(stage), pol_w);
+          used[stage] = true;
+          fill_parity[stage] = phase;
+          ca.advance(p, passes, BN);
+          if (++stage == SA) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok) {
@@ -558,6 +454,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     }
   } else if (warp == 6) {
     // activation producer: the packed rows are written by the previous launch
+    // (phase 0) or by the previous phase's epilogue (chained phases)
     if (lane == 0) {
       griddep_wait();
       allow_dependents();  // the next kernel may be scheduled (it waits for this grid)
@@ -565,27 +462,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       uint32_t fill_parity[kTcMaxB];
       bool used[kTcMaxB];
       for (int s = 0; s < kTcMaxB; ++s) used[s] = false;
-      KCursor cb;
-      cb.start(p, passes, my_begin, my_end, BN, M);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      while (cb.valid) {
-        if (!wait_bounded(EMPTY_B(stage), phase ^ 1u, abort_v, p.status)) {
-          ok = false;
-          break;
+      for (int ph = 0; ph < p.nphase && ok; ++ph) {
+        if (ph > 0 && p.chain) {
+          // the barrier after phase ph - 1's epilogue: its outputs are this phase's operand
+          if (!spin_count(p.bar + 2 * (ph - 1) + 1, (int)gridDim.x, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          fence_proxy_async_global();  // generic-proxy stores of other CTAs, read next by TMA
         }
-        // the whole token pass in one box: TMA throughput is bound by the number
-        // of copies, not their bytes (rows past the packed count are never read
-        // by the MMA; rows past the buffer are zero-filled)
-        mbar_expect_tx(FULL_B(stage), b_bytes);
-        tma_load_2d(STAGE_B(stage), &p.b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
-        used[stage] = true;
-        fill_parity[stage] = phase;
-        cb.advance(p, passes, BN, M);
-        if (++stage == SB) {
-          stage = 0;
-          phase ^= 1u;
+        KCursor cb;
+        cb.start(p, ph, passes, BN);
+        while (cb.valid) {
+          if (!wait_bounded(EMPTY_B(stage), phase ^ 1u, abort_v, p.status)) {
+            ok = false;
+            break;
+          }
+          // the whole token pass in one box: TMA throughput is bound by the number
+          // of copies, not their bytes (rows past the packed count are never read
+          // by the MMA; rows past the buffer are zero-filled)
+          mbar_expect_tx(FULL_B(stage), b_bytes);
+          tma_load_2d(STAGE_B(stage), &p.ph[ph].b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
+          used[stage] = true;
+          fill_parity[stage] = phase;
+          cb.advance(p, passes, BN);
+          if (++stage == SB) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok)
@@ -598,57 +505,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       uint32_t pa = 0, pb = 0, nfrag = 0;
       const uint32_t idesc_lm = idesc_bf16(128, 128);
       bool ok = true, issued = false;
-      FragIter it{my_begin, my_end, 0};
-      Frag f;
-      while (ok && next_frag(p, passes, it, f)) {
-        const int mrows = min(BN, M - it.pass * BN);
-        const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
-        const int lm_halves = mrows > 128 ? 2 : 1;
-        const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
-        const uint32_t dtm = tmem + acc * (uint32_t)BN;
-        if (!wait_bounded(TEMPTY(acc), (use & 1u) ^ 1u, abort_v, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int kb = f.kb0; kb < f.kb1; ++kb) {
-          if (!wait_bounded(FULL_A(sa), pa, abort_v, p.status) || !wait_bounded(FULL_B(sb), pb, abort_v, p.status)) {
+      for (int ph = 0; ph < p.nphase && ok; ++ph) {
+        FragIter it = frag_begin(p, ph);
+        Frag f;
+        while (ok && next_frag(p, passes, it, f)) {
+          const int mrows = min(BN, M - it.pass * BN);
+          const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
+          const int lm_halves = mrows > 128 ? 2 : 1;
+          const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
+          const uint32_t dtm = tmem + acc * (uint32_t)BN;
+          if (!wait_bounded(TEMPTY(acc), (use & 1u) ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sw128_desc(STAGE_A(sa));
-          const uint64_t bd = sw128_desc(STAGE_B(sb));
-          if (p.epi_mode == 1) {
-            // LM head: tokens are the MMA M dimension (one or two 128-row halves of
-            // the activation box), the tile's 128 vocabulary rows are N
-            for (int mt = 0; mt < lm_halves; ++mt) {
-              const uint64_t xd = sw128_desc(STAGE_B(sb) + (uint32_t)mt * 16384u);
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                tc_mma(dtm + (uint32_t)(mt * 128), xd + (uint64_t)(2 * k), ad + (uint64_t)(2 * k), idesc_lm,
-                       (kb > f.kb0 || k > 0) ? 1u : 0u);
+          for (int kb = f.kb0; kb < f.kb1; ++kb) {
+            if (!wait_bounded(FULL_A(sa), pa, abort_v, p.status) ||
+                !wait_bounded(FULL_B(sb), pb, abort_v, p.status)) {
+              ok = false;
+              break;
             }
-          } else {
+            tc_fence_after();
+            const uint64_t ad = sw128_desc(STAGE_A(sa));
+            const uint64_t bd = sw128_desc(STAGE_B(sb));
+            if (p.epi_mode == EPI_LMHEAD) {
+              // LM head: tokens are the MMA M dimension (one or two 128-row halves of
+              // the activation box), the tile's 128 vocabulary rows are N
+              for (int mt = 0; mt < lm_halves; ++mt) {
+                const uint64_t xd = sw128_desc(STAGE_B(sb) + (uint32_t)mt * 16384u);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
-              tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
+                for (int k = 0; k < 4; ++k)
+                  tc_mma(dtm + (uint32_t)(mt * 128), xd + (uint64_t)(2 * k), ad + (uint64_t)(2 * k), idesc_lm,
+                         (kb > f.kb0 || k > 0) ? 1u : 0u);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
+                tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
+            }
+            issued = true;
+            tc_commit(EMPTY_A(sa));  // both stages are free once these MMAs have read them
+            tc_commit(EMPTY_B(sb));
+            if (++sa == SA) {
+              sa = 0;
+              pa ^= 1u;
+            }
+            if (++sb == SB) {
+              sb = 0;
+              pb ^= 1u;
+            }
           }
-          issued = true;
-          tc_commit(EMPTY_A(sa));  // both stages are free once these MMAs have read them
-          tc_commit(EMPTY_B(sb));
-          if (++sa == SA) {
-            sa = 0;
-            pa ^= 1u;
-          }
-          if (++sb == SB) {
-            sb = 0;
-            pb ^= 1u;
-          }
+          if (!ok) break;
+          tc_commit(TFULL(acc));
+          ++nfrag;
         }
-        if (!ok) break;
-        tc_commit(TFULL(acc));
-        ++nfrag;
       }
       if (!ok && issued) {
         tc_commit(drain);
@@ -656,10 +566,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       }
     }
   } else if (warp >= 2 && warp <= 5) {
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q4 = warp & 3;  // TMEM lane quarter this warp may access
+    const int ew = warp - 2, t128 = threadIdx.x - 64;
     uint32_t nfrag = 0;
-    FragIter it{my_begin, my_end, 0};
-    Frag f;
     float lm_max[2] = {-INFINITY, -INFINITY};
     double lm_sum[2] = {0.0, 0.0};  // fp64 running sums: ~1000 terms per CTA
     int lm_arg[2] = {0x7fffffff, 0x7fffffff};
@@ -667,7 +576,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     // LM head: this CTA's statistics of the pass's tokens over its vocabulary range
     auto lm_flush = [&](int pass) {
       for (int mt = 0; mt < 2; ++mt) {
-        const int m = pass * BN + mt * 128 + q * 32 + lane;
+        const int m = pass * BN + mt * 128 + q4 * 32 + lane;
         if (m < M) {
           const size_t o = (size_t)blockIdx.x * p.ldm + (size_t)m;
           p.smx[o] = make_float2(lm_max[mt], (float)lm_sum[mt]);
@@ -678,121 +587,121 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         lm_arg[mt] = 0x7fffffff;
       }
     };
-    const bool fused = p.epi_mode >= EPI_QKV;
-    const int ew = warp - 2;  // epilogue warp 0..3 (row interleave of the fused epilogues)
-    FixStage st;
-    st.sbase = fbase;
-    st.gbase = smem_raw + (fbase - smem_u32(smem_raw));
-    st.bytes = kFixBuf;
-    st.bar = fixbar;
-    st.uses[0] = st.uses[1] = 0;
-    st.rows = s_rows;
-    st.status = p.status;
-    st.abort = abort_v;
-    // the fused epilogues read what the previous launches wrote (H_l rows, the
-    // row sums of squares, hmid): wait for them like the activation producer
-    if (fused) griddep_wait();
-    while (next_frag(p, passes, it, f)) {
-      const int m0 = it.pass * BN;
-      const int mrows = min(BN, M - m0);
-      const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
-      const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q * 32) << 16);
-      bool okw = __all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status));
-      if (fused) {
-        // the 4 warps meet at named barriers below: they leave together or not at all
-        if (lane == 0) s_epi_ok[ew] = okw ? 1 : 0;
-        epi_bar();
-        okw = (s_epi_ok[0] & s_epi_ok[1] & s_epi_ok[2] & s_epi_ok[3]) != 0;
-      }
-      if (!okw) break;
-      tc_fence_after();
-      const int rin = f.arow + q * 32 + lane;  // row within the weight segment
-      const bool col_ok = rin < p.seg_rows[f.seg];
-      const size_t col = (size_t)(p.seg_col0[f.seg] + rin);
-      if (p.epi_mode == 1) {
-        // LM head: this thread owns token m = mt * 128 + (TMEM lane) and folds the
-        // tile's 128 logits into its running (max, sum of exp, lowest argmax);
-        // tiles arrive in increasing vocabulary order, so on equal maxima the
-        // earlier (lower) id is kept
-        const int vbase = f.tile * 128;
-        if (it.pass != lm_pass) {
-          lm_flush(lm_pass);
-          lm_pass = it.pass;
+    bool alive = true;
+    for (int ph = 0; ph < p.nphase && alive; ++ph) {
+      const TcPhase &q = p.ph[ph];
+      FragIter it = frag_begin(p, ph);
+      Frag f;
+      while (next_frag(p, passes, it, f)) {
+        const int m0 = it.pass * BN;
+        const int mrows = min(BN, M - m0);
+        const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
+        const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q4 * 32) << 16);
+        bool okw = __all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status));
+        if (p.chain) {
+          // the 4 warps meet at named barriers below: they leave together or not at all
+          if (lane == 0) s_epi_ok[ew] = okw ? 1 : 0;
+          epi_bar();
+          okw = (s_epi_ok[0] & s_epi_ok[1] & s_epi_ok[2] & s_epi_ok[3]) != 0;
+          epi_bar();
         }
-        for (int mt = 0; mt < (mrows > 128 ? 2 : 1); ++mt) {
-          const uint32_t tm = tmem + acc * (uint32_t)BN + (uint32_t)(mt * 128) + ((uint32_t)(q * 32) << 16);
-          float &RM = lm_max[mt];
-          double &RS = lm_sum[mt];
-          int &RI = lm_arg[mt];
-          const int tok = it.pass * BN + mt * 128 + q * 32 + lane;
-          float *zdst = (p.zout && tok < M) ? p.zout + (int64_t)p.zrow[tok] * p.ldz + vbase : nullptr;
-          for (int c = 0; c < 128; c += 16) {
-            float v[16];
-            tmem_ld16(tm + (uint32_t)c, v);
-            if (zdst) {
+        if (!okw) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        const int rin = f.arow + q4 * 32 + lane;  // row within the weight segment
+        const bool col_ok = rin < q.seg_rows[f.seg];
+        const size_t col = (size_t)(q.seg_col0[f.seg] + rin);
+        if (p.epi_mode == EPI_LMHEAD) {
+          // LM head: this thread owns token m = mt * 128 + (TMEM lane) and folds the
+          // tile's 128 logits into its running (max, sum of exp, lowest argmax);
+          // tiles arrive in increasing vocabulary order, so on equal maxima the
+          // earlier (lower) id is kept
+          const int vbase = f.tile * 128;
+          if (it.pass != lm_pass) {
+            lm_flush(lm_pass);
+            lm_pass = it.pass;
+          }
+          for (int mt = 0; mt < (mrows > 128 ? 2 : 1); ++mt) {
+            const uint32_t tm = tmem + acc * (uint32_t)BN + (uint32_t)(mt * 128) + ((uint32_t)(q4 * 32) << 16);
+            float &RM = lm_max[mt];
+            double &RS = lm_sum[mt];
+            int &RI = lm_arg[mt];
+            const int tok = it.pass * BN + mt * 128 + q4 * 32 + lane;
+            float *zdst = (p.zout && tok < M) ? p.zout + (int64_t)p.zrow[tok] * p.ldz + vbase : nullptr;
+            for (int c = 0; c < 128; c += 16) {
+              float v[16];
+              tmem_ld16(tm + (uint32_t)c, v);
+              if (zdst) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (vbase + c + j < p.seg_rows[0]) zdst[c + j] = v[j];
-            }
-            float cm = -INFINITY;
-            int cj = 0;
+                for (int j = 0; j < 16; ++j)
+                  if (vbase + c + j < q.seg_rows[0]) zdst[c + j] = v[j];
+              }
+              float cm = -INFINITY;
+              int cj = 0;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const bool ok = vbase + c + j < p.seg_rows[0];
-              v[j] = ok ? v[j] : -INFINITY;
-              if (v[j] > cm) { cm = v[j]; cj = j; }
-            }
-            // no divergent exit from this loop: tmem_ld16 is warp-collective
-            if (cm > RM) {
-              RS = (RM == -INFINITY) ? 0.0 : RS * (double)expf(RM - cm);
-              RM = cm;
-              RI = vbase + c + cj;
-            }
-            if (RM != -INFINITY) {
-              float e = 0.f;
+              for (int j = 0; j < 16; ++j) {
+                const bool ok = vbase + c + j < q.seg_rows[0];
+                v[j] = ok ? v[j] : -INFINITY;
+                if (v[j] > cm) { cm = v[j]; cj = j; }
+              }
+              // no divergent exit from this loop: tmem_ld16 is warp-collective
+              if (cm > RM) {
+                RS = (RM == -INFINITY) ? 0.0 : RS * (double)expf(RM - cm);
+                RM = cm;
+                RI = vbase + c + cj;
+              }
+              if (RM != -INFINITY) {
+                float e = 0.f;
 #pragma unroll
-              for (int j = 0; j < 16; ++j) e += expf(v[j] - RM);
-              RS += (double)e;
+                for (int j = 0; j < 16; ++j) e += expf(v[j] - RM);
+                RS += (double)e;
+              }
             }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(TEMPTY(acc));
+          ++nfrag;
+          continue;
+        }
+        float *dst = p.out + (size_t)f.slot * (size_t)q.geo.slot_stride + col;
+        for (int c = 0; c < mrows; c += 16) {
+          float v[16];
+          tmem_ld16(tacc + (uint32_t)c, v);
+          if (col_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (c + j < mrows) dst[(size_t)(m0 + c + j) * q.ldc] = v[j];
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(TEMPTY(acc));
+        if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
         ++nfrag;
-        continue;
       }
-      float *dst = p.out + (size_t)f.slot * (size_t)p.geo.slot_stride + col;
-      for (int c = 0; c < mrows; c += 16) {
-        float v[16];
-        tmem_ld16(tacc + (uint32_t)c, v);
-        if (col_ok) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c + j < mrows) dst[(size_t)(m0 + c + j) * p.ldc] = v[j];
-        }
+      if (!alive || !p.chain) continue;
+      // chained launch: every piece of this phase is stored once all CTAs are here
+      if (!grid_sync(p.bar + 2 * ph, ew, lane, abort_v, p.status, &s_flag)) {
+        alive = false;
+        break;
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
-      ++nfrag;
-      if (fused) {
-        const int ns = sk_nslots(p.geo, f.tile);
-        if (epi_arrive(p.e.tile_cnt + (size_t)it.pass * p.geo.n_tiles + f.tile, ns, &s_epi_flag, ew, lane)) {
-          for (int r = threadIdx.x - 64; r < mrows; r += 128) s_rows[r] = p.e.rowmap[m0 + r];
-          epi_bar();
-          if (p.epi_mode == EPI_QKV)
-            fix_qkv(p, st, f.tile, f.seg, m0, mrows, ns, ew, lane);
-          else if (p.epi_mode == EPI_O)
-            fix_o(p, st, f.tile, m0, mrows, ns, ew, lane);
-          else if (p.epi_mode == EPI_GU)
-            fix_gu(p, st, f.tile, it.pass, m0, mrows, ns, ew, lane, &s_epi_flag);
-          else
-            fix_down(p, st, f.tile, it.pass, m0, mrows, ns, ew, lane, &s_epi_flag);
-        }
+      if (q.epi == EPI_QKV)
+        epi_qkv(p, q, M, t128);
+      else if (q.epi == EPI_O)
+        epi_o(p, q, M, t128, ew, lane, s_red);
+      else if (q.epi == EPI_GU)
+        epi_gu(p, q, M, t128);
+      else if (q.epi == EPI_DOWN)
+        epi_down(p, q, M, t128, ew, lane, s_red, &s_same);
+      // the epilogue's outputs are the next phase's operand
+      if (ph + 1 < p.nphase && !grid_sync(p.bar + 2 * ph + 1, ew, lane, abort_v, p.status, &s_flag)) {
+        alive = false;
+        break;
       }
     }
-    if (p.epi_mode == 1) lm_flush(lm_pass);
+    if (p.epi_mode == EPI_LMHEAD) lm_flush(lm_pass);
   }
 #undef FULL_A
 #undef EMPTY_A
@@ -854,17 +763,23 @@ static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = kTcSmem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // chained phases meet at grid barriers: every CTA must be resident at once
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.chain == 1 ? 2 : 1;  // chain 2: programmatic launch only (all CTAs fit one per SM)
   return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN>, p);
 }
 
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
-  const int grid = p.geo.grid;
+  int grid = p.ph[0].geo.grid;
+  if (p.nphase < 1 || p.nphase > kTcMaxPhases) return cudaErrorInvalidValue;
+  for (int i = 1; i < p.nphase; ++i) grid = p.ph[i].geo.grid > grid ? p.ph[i].geo.grid : grid;
   if (grid <= 0) return cudaSuccess;
+  if (p.chain && !p.bar) return cudaErrorInvalidValue;
   if (p.b_rows <= 0 || p.b_rows > bn || p.b_rows % 16 != 0) return cudaErrorInvalidValue;
   p.smem_bytes = (uint32_t)kTcSmem;
   if (bn == 128) return launch_bn<128>(p, grid, s);

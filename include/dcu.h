@@ -135,12 +135,18 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
              int32_t B_layer, int32_t B_window, dcu_stream_t stream);
 
 /* Performance options of a context (results agree within the parity
- * tolerances either way; both paths are tested).
+ * tolerances either way; every path is tested).
  *   DCU_OPT_FUSED_EPILOGUE (bf16 models with head_dim 64 or 128; default 0):
- *     1 = the layer GEMMs apply their epilogues themselves (RoPE and the K/V
- *     write, residual and the RMSNorm statistics, SwiGLU, residual, scatter
- *     and next-layer d), the last CTA to finish a tile summing its split-K
- *     pieces; 0 = separate epilogue kernels.
+ *     0 = each layer GEMM stores its split-K pieces and separate kernels apply
+ *     the epilogues (RoPE and the K/V write, residual + RMSNorm, SwiGLU,
+ *     residual + scatter + next-layer d);
+ *     1 = chained launches: the QKV GEMM with its epilogue, and the O, gate|up
+ *     and down GEMMs with theirs, each run as one persistent cooperative
+ *     launch (one CTA per SM) whose phases are separated by grid barriers and
+ *     whose epilogues are spread over all CTAs;
+ *     2 = as 1 without the cooperative launch attribute (every CTA still fits
+ *     one per SM; every barrier wait is time-bounded and reports
+ *     DCU_ST_TIMEOUT if a CTA never arrives).
  * DCU_EINVAL for an unknown option or an unsupported value. */
 #define DCU_OPT_FUSED_EPILOGUE 1
 /*   DCU_OPT_L2_PREFETCH (default 16): when a layer GEMM has issued its own

@@ -401,18 +401,29 @@ def main():
     pos = torch.zeros((B, N), dtype=torch.int32, device="cuda")
     cnt = torch.zeros(B, dtype=torch.int32, device="cuda")
 
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    dcu.dcu_full_forward(ctx, ids)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    full_ms = e0.elapsed_time(e1)
-    dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
+    def new_generation():
+        """Every timed pass starts from the same state: the prompt and an all-masked
+        generated tail, the dense forward, the first commit (none of it timed), so
+        the passes decode the same steps of a generation (the LM head of the commit
+        covers the still-masked rows, which shrink as the generation proceeds)."""
+        ids.copy_(ids_h)
+        masked.copy_((ids == shape.mask_id).to(torch.uint8))
+        pos.zero_()
+        cnt.zero_()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        dcu.dcu_full_forward(ctx, ids)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
+        return g0.elapsed_time(g1)
 
     def step():
         dcu.dcu_step(ctx, ids, pos, cnt, wl["B_layer"], wl["B_window"])
         dcu.commit_select(ctx, wl["rule"], wl["param"], masked, ids, pos, cnt)
+
+    full_ms = new_generation()
 
     # (1) the headline: K steps with nothing but the step's own kernels in the
     # graph (event-record nodes would split it and cut the programmatic edges
@@ -438,7 +449,9 @@ def main():
     barrier()
     ms_total = t0.elapsed_time(t1)
     launches = dcu.dcu_launch_count(ctx) - launches0
-    committed = masked_before - int(masked.sum().item())
+    masked_after = int(masked.sum().item())
+    committed = masked_before - masked_after
+    config["masked_rows_first_last_step"] = [masked_before, masked_after]
     ms_step = max_over_ranks(ms_total / args.steps)
     steps_all = args.steps * world
     value = aggregate_rate(args.steps, world, ms_step, args.steps)
@@ -451,6 +464,7 @@ def main():
     # graphs carry their own event nodes)
     slots = (args.steps + args.warmup) if args.no_graphs else 2
     dcu.dcu_profile_enable(ctx, slots * per_step_launches_guess)
+    new_generation()
     for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -490,6 +504,10 @@ def main():
     e2e = None
     if not args.no_e2e:
         # through the C ABI with host buffers: ids/keys in from pinned memory, result out, every step
+        new_generation()
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
         h_ids = ids.cpu().pin_memory()
         h_pos = pos.cpu().pin_memory()
         h_cnt = cnt.cpu().pin_memory()

@@ -320,6 +320,8 @@ def main():
                     help="DCU_OPT_FUSED_EPILOGUE (1: epilogues inside the layer GEMMs); default: the library's")
     ap.add_argument("--l2-prefetch", type=int, default=None,
                     help="DCU_OPT_L2_PREFETCH (next-GEMM weight units per CTA into L2); default: the library's")
+    ap.add_argument("--attention", choices=["tcgen05", "mma_sync"], default=None,
+                    help="attention implementation (DCU_OPT_ATTENTION; default: the library's)")
     ap.add_argument("--layers", type=int, default=0,
                     help="profiling only: override the number of layers (the JSON line is then not a bench value)")
     ap.add_argument("--case", default="", choices=["", "gemm"],
@@ -393,6 +395,10 @@ def main():
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, args.fused)
     if args.l2_prefetch is not None:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_L2_PREFETCH, args.l2_prefetch)
+    if args.attention is not None:
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION,
+                           dcu.DCU_ATTN_TCGEN05 if args.attention == "tcgen05" else dcu.DCU_ATTN_MMA_SYNC)
+        config["attention"] = args.attention
     seq_seed = replica_seed(rank)                         # each replica decodes its own sequences
     ids_h = torch.stack([torch.tensor(I.sequence_ids(seq_seed, b, wl["n_prompt"], wl["n_gen"], shape.vocab),
                                       dtype=torch.int32) for b in range(B)])

@@ -108,9 +108,7 @@ struct dcu_ctx {
   size_t ws_elems = 0;        // capacity of C in floats
   float2 *smx = nullptr;      // LM-head softmax statistics per (vocab tile, row)
   int32_t *smx_arg = nullptr;
-  // fused GEMM epilogues (bf16, head_dim 64 / 128): arrival counters of the
-  // four layer GEMMs, per-tile row sums of squares (O -> gate|up) and per-tile
-  // partial sums of the next-layer distance (down)
+  // chained GEMM launches with their epilogues (bf16, head_dim 64 / 128)
   int fused = 0;             // chained launches in use (DCU_OPT_FUSED_EPILOGUE and supported): 1 or 2
   bool fused_ok = false;     // the model supports them (bf16, head_dim 64 or 128)
   int nx_count = 16;         // units per CTA of the next GEMM's weights prefetched into L2 (0: off)
@@ -119,8 +117,10 @@ struct dcu_ctx {
   CUtensorMap lm_map;
   CUtensorMap xs_map[2], attn_map[2], act_map[2];  // boxes of min(128, cap) and min(256, cap) rows
   uint32_t act_box[2] = {128, 256};
-  // per layer: K and V of the active shape as [B*Hkv*N rows][hd], box 64 x 64 (attention)
-  std::vector<CUtensorMap> kv_maps;
+  // per layer: K and V of the active shape as [B*Hkv*N rows][hd], box 64 x 64
+  // (mma.sync attention) and box 64 x 128 (tcgen05 attention)
+  std::vector<CUtensorMap> kv_maps, kv_maps_tc;
+  int attn_impl = DCU_ATTN_TCGEN05;  // DCU_OPT_ATTENTION
   // per-tile piece counts of each stream-K geometry used so far (device tables)
   struct SlotTable {
     int n_tiles, kblocks, grid, tile_aligned;
@@ -516,23 +516,37 @@ int run_layer(dcu_ctx *c, int l, bool dense, const int32_t *keys, const int32_t 
       // one wave: (sequence, kv head, query tile) items x key splits <= SM count (one CTA per SM)
       const long long items = (long long)c->B * Hkv * qt_grid;
       int splits = (int)(c->num_sms / items);
-      const int max_sp = (c->N + 63) / 64;
-      splits = splits < 1 ? 1 : splits;
-      // long sequences: the legacy-MMA attention is compute-bound, so when one
-      // wave leaves more than 2048 keys per CTA, cut them to <= 1024 even past
-      // one wave (the heavy query tiles then spread over all SMs instead of the
-      // few that hold them; measured +12 % attention at N = 8192, while at
-      // N = 2048 x 4 sequences the extra wave and merge cost 10 %)
-      if ((c->N + splits - 1) / splits > 2048)
-        while (splits < kAttnMaxSplits && (c->N + splits - 1) / splits > 1024) splits *= 2;
-      splits = splits > kAttnMaxSplits ? kAttnMaxSplits : splits;
-      if (splits > max_sp) splits = max_sp;
-      const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
-      splits = (c->N + kc - 1) / kc;
-      LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
-                                     &c->kv_maps[2 * l], &c->kv_maps[2 * l + 1], c->attn, c->attn_po, c->attn_ml,
-                                     splits, qt_grid, gcap, c->status(), s));
-      if (splits > 1) ++c->launches;  // the merge kernel
+      if (c->attn_impl == DCU_ATTN_TCGEN05) {
+        // tensor cores to spare: one wave of CTAs, each streaming whole 128-key
+        // chunks; the splits of a query tile form a cluster, so the split count
+        // is also capped by how many such clusters can be resident at once
+        const int max_tc = (c->N + 127) / 128;
+        splits = splits < 1 ? 1 : (splits > kAttnMaxSplits ? kAttnMaxSplits : splits);
+        if (splits > max_tc) splits = max_tc;
+        while (splits > 1 && (long long)attn_tc_max_clusters(hd, splits) < items) --splits;
+        const int kc = ((c->N + splits - 1) / splits + 127) / 128 * 128;
+        splits = (c->N + kc - 1) / kc;
+        LAUNCH(c, launch_attention_tc(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, &c->kv_maps_tc[2 * l],
+                                      &c->kv_maps_tc[2 * l + 1], c->attn, splits, qt_grid, c->status(), s));
+      } else {
+        const int max_sp = (c->N + 63) / 64;
+        splits = splits < 1 ? 1 : splits;
+        // long sequences: the legacy-MMA attention is compute-bound, so when one
+        // wave leaves more than 2048 keys per CTA, cut them to <= 1024 even past
+        // one wave (the heavy query tiles then spread over all SMs instead of the
+        // few that hold them; measured +12 % attention at N = 8192, while at
+        // N = 2048 x 4 sequences the extra wave and merge cost 10 %)
+        if ((c->N + splits - 1) / splits > 2048)
+          while (splits < kAttnMaxSplits && (c->N + splits - 1) / splits > 1024) splits *= 2;
+        splits = splits > kAttnMaxSplits ? kAttnMaxSplits : splits;
+        if (splits > max_sp) splits = max_sp;
+        const int kc = ((c->N + splits - 1) / splits + 63) / 64 * 64;
+        splits = (c->N + kc - 1) / kc;
+        LAUNCH(c, launch_attention_mma(c->Q, c->seq_off, c->B, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
+                                       &c->kv_maps[2 * l], &c->kv_maps[2 * l + 1], c->attn, c->attn_po, c->attn_ml,
+                                       splits, qt_grid, gcap, c->status(), s));
+        if (splits > 1) ++c->launches;  // the merge kernel
+      }
     } else {
       LAUNCH(c, launch_attention(dt, c->Q, c->rowmap, c->m_total(), gcap, c->N, H, Hkv, hd, c->Kl(l), c->Vl(l),
                                  c->attn, s));
@@ -715,6 +729,8 @@ int dcu_create(const dcu_weights *w, const dcu_cfg *cfg, dcu_ctx **out) {
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaMemset(c->ints, 0, 64);
   if (e == cudaSuccess && c->chain_bar) e = cudaMemset(c->chain_bar, 0, (size_t)L * kChainBars * 4);
+  if (e == cudaSuccess && c->attn_po)  // cluster residency of the tcgen05 attention, queried outside any capture
+    for (int sp = 1; sp <= kAttnMaxSplits; ++sp) attn_tc_max_clusters(cfg->head_dim, sp);
   if (e == cudaSuccess) e = cudaMemset(c->stale, 0, (size_t)L * cap);
   if (e == cudaSuccess) e = cudaMemset(c->d, 0, (size_t)L * cap * 4);
   if (e == cudaSuccess) e = cudaMemset(c->s_prev, 0, (size_t)cfg->max_batch * L * 4);
@@ -806,10 +822,13 @@ int dcu_full_forward(dcu_ctx *c, const int32_t *ids, int32_t B, int32_t N, dcu_s
   if (c->attn_po) {  // K / V tensor maps of the tensor-core attention for this shape
     const dcu_cfg &g = c->cfg;
     c->kv_maps.resize(2 * (size_t)g.n_layers);
+    c->kv_maps_tc.resize(2 * (size_t)g.n_layers);
     const uint64_t rows = (uint64_t)B * g.n_kv_heads * N, hd = (uint64_t)g.head_dim;
     for (int l = 0; l < g.n_layers; ++l)
       if (!encode_tmap_bf16(&c->kv_maps[2 * l], c->Kl(l), hd, rows, hd * 2, 64, 64) ||
-          !encode_tmap_bf16(&c->kv_maps[2 * l + 1], c->Vl(l), hd, rows, hd * 2, 64, 64))
+          !encode_tmap_bf16(&c->kv_maps[2 * l + 1], c->Vl(l), hd, rows, hd * 2, 64, 64) ||
+          !encode_tmap_bf16(&c->kv_maps_tc[2 * l], c->Kl(l), hd, rows, hd * 2, 64, 128) ||
+          !encode_tmap_bf16(&c->kv_maps_tc[2 * l + 1], c->Vl(l), hd, rows, hd * 2, 64, 128))
         return fail(c, DCU_ECUDA, "cuTensorMapEncodeTiled failed for the K / V cache");
   }
   {
@@ -1036,7 +1055,8 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
                             ((uint64_t)c->B << 32) | (uint64_t)c->N,
                             (uint64_t)(c->prof_max > 0),
                             ((uint64_t)(uint32_t)c->force_lo << 32) | (uint64_t)(uint32_t)c->force_hi,
-                            (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16),
+                            (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16) |
+                                ((uint64_t)c->attn_impl << 32),
                             0,
                             0};
   int rc = run_graphed(c, key, (cudaStream_t)stream,
@@ -1060,6 +1080,11 @@ int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
     case DCU_OPT_L2_PREFETCH:
       if (value < 0 || value > 4096) return fail(c, DCU_EINVAL, "L2 prefetch units must lie in [0, 4096]");
       c->nx_count = value;
+      return DCU_OK;
+    case DCU_OPT_ATTENTION:
+      if (value != DCU_ATTN_TCGEN05 && value != DCU_ATTN_MMA_SYNC)
+        return fail(c, DCU_EINVAL, "DCU_OPT_ATTENTION takes DCU_ATTN_TCGEN05 or DCU_ATTN_MMA_SYNC");
+      c->attn_impl = value;
       return DCU_OK;
     default:
       return fail(c, DCU_EINVAL, "unknown option");

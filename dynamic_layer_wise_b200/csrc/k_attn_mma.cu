@@ -441,6 +441,12 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
+  return launch_attn_merge(part_o, part_ml, seq_off, B, H, hd, splits, cap_rows, out, s);
+}
+
+cudaError_t launch_attn_merge(const float *part_o, const float2 *part_ml, const int32_t *seq_off, int B, int H,
+                              int hd, int splits, int cap_rows, void *out, cudaStream_t s) {
+  if ((hd != 64 && hd != 128) || splits < 2 || splits > 8) return cudaErrorInvalidValue;
   const long long items = (long long)cap_rows * H * (hd / 4);
   long long mg = (items + 255) / 256;
   const int mgrid = (int)(mg < 148 * 8 ? mg : 148 * 8);

@@ -86,6 +86,21 @@ cudaError_t launch_attention_mma(const void *Q, const int32_t *seq_off, int B, i
                                  void *out, float *part_o, float2 *part_ml, int splits, int qt_grid, int cap_rows,
                                  int32_t *status, cudaStream_t s);
 
+// the split merge of both tensor-core attentions: out = sum_s w_s O_s / sum_s w_s l_s (2 <= splits <= 8)
+cudaError_t launch_attn_merge(const float *part_o, const float2 *part_ml, const int32_t *seq_off, int B, int H,
+                              int hd, int splits, int cap_rows, void *out, cudaStream_t s);
+
+// ---- tcgen05 attention (k_attn_tc.cu), bf16, head_dim 64 or 128: same packing
+// as above; K / V maps with a box of 64 x 128 keys; key splits (<= 8) of whole
+// 128-key chunks, each split holding keys, merged inside the launch (the
+// splits of a query tile form one cluster) -- one launch
+size_t attn_tc_smem(int hd);
+// clusters of `splits` CTAs of the kernel that can be resident at once (0: unknown)
+int attn_tc_max_clusters(int hd, int splits);
+cudaError_t launch_attention_tc(const void *Q, const int32_t *seq_off, int B, int N, int H, int Hkv, int hd,
+                                const CUtensorMap *kmap, const CUtensorMap *vmap, void *out, int splits, int qt_grid,
+                                int32_t *status, cudaStream_t s);
+
 // ---- attention (k_attn.cu): out[r][h] = softmax(q K^T / sqrt(hd)) V over all N keys of row r's sequence
 cudaError_t launch_attention(int dtype, const void *Q, const int32_t *rowmap, const int32_t *m_total, int cap,
                              int N, int H, int Hkv, int hd, const void *Kc, const void *Vc, void *out,

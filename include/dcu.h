@@ -155,6 +155,15 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
  *     layer) into L2, so HBM keeps streaming through the dependent kernels in
  *     between; 0 turns it off, at most 4096. */
 #define DCU_OPT_L2_PREFETCH 2
+/*   DCU_OPT_ATTENTION (bf16 models with head_dim 64 or 128): the attention of
+ *     the recomputed rows over all N keys.  DCU_ATTN_TCGEN05 (default): 5th-gen
+ *     tensor cores, S and O accumulated in tensor memory, 128-key chunks;
+ *     DCU_ATTN_MMA_SYNC: warp-level mma.sync with the online softmax in
+ *     registers, 64-key chunks.  Both split the keys over at most 8 CTAs per
+ *     (sequence, kv head, query tile) and merge the splits in split order. */
+#define DCU_OPT_ATTENTION 3
+#define DCU_ATTN_TCGEN05 0
+#define DCU_ATTN_MMA_SYNC 1
 int dcu_set_option(dcu_ctx *ctx, int32_t option, int32_t value);
 
 /* Adaptive parallel decoding, APD ([DLLM] "关键设计 3").  Enables rule DCU_APD of

@@ -78,4 +78,5 @@ def test_stateless_entry_points_reject_bad_args_on_host(libs):
     assert L.dcu_full_forward(None, None, 1, 8, None) == dcu.DCU_EINVAL
     assert L.dcu_step(None, None, None, None, 1, 1, None) == dcu.DCU_EINVAL
     assert L.commit_select(None, 0, 0.1, None, None, None, None, None) == dcu.DCU_EINVAL
+    assert L.dcu_set_option(None, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_TCGEN05) == dcu.DCU_EINVAL
     assert dcu.dcu_kernel_class_name(dcu.DCU_K_GEMM) == "gemm"

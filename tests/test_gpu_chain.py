@@ -105,7 +105,7 @@ def _oracle_commit(w, cfg, st, masked, ids, rule, param):
 
 
 def _run_chain(shape, seed, B, n_prompt, n_gen, plan, B_layer, B_window, rule, param, window_mode, tol, s_rtol,
-               d_atol, c_rtol, graphs=True, fused=False):
+               d_atol, c_rtol, graphs=True, fused=False, attn="tcgen05"):
     N = n_prompt + n_gen
     L, V = shape.n_layers, shape.vocab
     cfg_o = oracle_cfg(shape, window_mode)
@@ -115,6 +115,8 @@ def _run_chain(shape, seed, B, n_prompt, n_gen, plan, B_layer, B_window, rule, p
     dcu.dcu_set_graphs(ctx, graphs)
     if fused:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, 1)
+    if attn != "tcgen05":
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_MMA_SYNC)
     ids = np.stack([I.sequence_ids(seed, b, n_prompt, n_gen, V) for b in range(B)])
     masked = (ids == shape.mask_id).astype(np.uint8)
 
@@ -200,23 +202,24 @@ SMALL_BF16 = I.ModelShape(n_layers=3, d_model=256, n_heads=4, n_kv_heads=2, head
                           dtype="bf16")
 
 
-@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("fused,attn", [(False, "tcgen05"), (True, "tcgen05"), (False, "mma_sync")])
 @pytest.mark.parametrize("rule,param,mode", [(O.RULE_FRECHET, 0.1, 0), (O.RULE_THRESHOLD, 0.9, 1),
                                              (O.RULE_FACTOR, 0.9, 0)])
-def test_small_bf16_batched_chain(rule, param, mode, fused):
+def test_small_bf16_batched_chain(rule, param, mode, fused, attn):
     """bf16, GQA (4 query / 2 kv heads), ragged vocab (1000) and sequence
     (N = 300), batch of 2 sequences, three commit + DCU rounds."""
     _run_chain(SMALL_BF16, 3, 2, 236, 64, ["commit", "dcu", "commit", "dcu", "commit", "dcu", "commit"],
-               8, 8, rule, param, mode, tol=2e-2, s_rtol=2e-2, d_atol=2e-3, c_rtol=2e-2, fused=fused)
+               8, 8, rule, param, mode, tol=2e-2, s_rtol=2e-2, d_atol=2e-3, c_rtol=2e-2, fused=fused, attn=attn)
 
 
 HD128_BF16 = I.ModelShape(n_layers=2, d_model=256, n_heads=4, n_kv_heads=2, head_dim=128, d_ffn=512, vocab=640,
                           dtype="bf16")
 
 
-@pytest.mark.parametrize("fused", [False, True])
-def test_bf16_head_dim_128_gqa_chain(fused):
+@pytest.mark.parametrize("fused,attn", [(False, "tcgen05"), (True, "tcgen05"), (False, "mma_sync")])
+def test_bf16_head_dim_128_gqa_chain(fused, attn):
     """head_dim 128 (the tensor-core attention's LLaDA / Dream tile), GQA 4/2,
-    N = 200 (ragged against the 64-key sub-chunks), two commit + DCU rounds."""
+    N = 200 (ragged against the 64- and 128-key chunks), two commit + DCU
+    rounds, with either attention."""
     _run_chain(HD128_BF16, 5, 1, 160, 40, ["commit", "dcu", "commit", "dcu", "commit"], 12, 6, O.RULE_FRECHET, 0.1, 0,
-               tol=2e-2, s_rtol=2e-2, d_atol=2e-3, c_rtol=2e-2, fused=fused)
+               tol=2e-2, s_rtol=2e-2, d_atol=2e-3, c_rtol=2e-2, fused=fused, attn=attn)

@@ -192,3 +192,18 @@ def test_bounded_wait_expires_and_reports_timeout():
     assert 0.5 < dt < 10.0
     x = torch.ones(4, device="cuda")
     assert float((x * 2).sum().item()) == 8.0                  # the context is usable afterwards
+
+
+def test_options_refuse_bad_values():
+    """dcu_set_option: unknown options and values out of range are refused
+    (DCU_EINVAL); the context stays usable and a valid setting is accepted."""
+    shape = I.ModelShape(n_layers=1, d_model=256, n_heads=4, n_kv_heads=2, head_dim=64, d_ffn=512, vocab=500,
+                         dtype="bf16")
+    ctx = dcu.dcu_create(I.device_weights(shape, 2), I.cfg_dict(shape, 1, 64))
+    for opt, val in [(dcu.DCU_OPT_ATTENTION, 2), (dcu.DCU_OPT_ATTENTION, -1), (dcu.DCU_OPT_FUSED_EPILOGUE, 3),
+                     (dcu.DCU_OPT_L2_PREFETCH, -1), (dcu.DCU_OPT_L2_PREFETCH, 4097), (99, 0)]:
+        with pytest.raises(dcu.DcuError):
+            dcu.dcu_set_option(ctx, opt, val)
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_MMA_SYNC)
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_TCGEN05)
+    ctx.close()

@@ -1,9 +1,9 @@
 """Teacher-forced parity on a small bf16 model with a long sequence (N = 4096),
-so that every CTA of the tensor-core attention walks many 64-key chunks: the
-dense forward gives each (kv head, 128-query tile) CTA all 4096 keys (64
-chunks), a DCU step splits the keys 8 ways (8 chunks per CTA), so the 4-stage
-TMA ring wraps its mbarrier phase and the online-softmax rescale runs across
-chunks.  Every layer is compared with the oracle fed the GPU's own layer
+so that every CTA of both tensor-core attentions walks many key chunks: the
+dense forward gives each (kv head, 128-query tile) CTA all 4096 keys (32
+chunks of 128 keys on tcgen05, 64 of 64 keys on mma.sync), a DCU step splits
+the keys 8 ways (4 or 8 chunks per CTA), so the TMA rings wrap their mbarrier
+phases and the online-softmax rescale runs across chunks.  Every layer is compared with the oracle fed the GPU's own layer
 inputs; the attention output of the last layer is compared directly."""
 import numpy as np
 import pytest
@@ -27,9 +27,9 @@ def _snapshot(ctx, L):
             [dcu.dcu_get_tensor(ctx, dcu.DCU_T_V, l).clone() for l in range(L)])
 
 
-@pytest.mark.parametrize("fused", [False, True])
+@pytest.mark.parametrize("fused,attn", [(False, "tcgen05"), (True, "tcgen05"), (False, "mma_sync")])
 @pytest.mark.parametrize("B_layer,B_window", [(32, 32), (200, 16)])
-def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window, fused):
+def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window, fused, attn):
     shape, seed, n_prompt, n_gen = LONG_BF16, 7, 3840, 256
     N, B = n_prompt + n_gen, 1
     L, D, Hkv, hd, H = shape.n_layers, shape.d_model, shape.n_kv_heads, shape.head_dim, shape.n_heads
@@ -38,6 +38,8 @@ def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window, fu
     W = I.device_weights(shape, seed)
     ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
     dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, int(fused))
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION,
+                       dcu.DCU_ATTN_TCGEN05 if attn == "tcgen05" else dcu.DCU_ATTN_MMA_SYNC)
     ids = np.stack([I.sequence_ids(seed, 0, n_prompt, n_gen, shape.vocab)])
     t_ids = torch.tensor(ids, dtype=torch.int32).cuda()
     dcu.dcu_full_forward(ctx, t_ids)

@@ -320,6 +320,8 @@ def main():
                     help="DCU_OPT_FUSED_EPILOGUE (1: epilogues inside the layer GEMMs); default: the library's")
     ap.add_argument("--l2-prefetch", type=int, default=None,
                     help="DCU_OPT_L2_PREFETCH (next-GEMM weight units per CTA into L2); default: the library's")
+    ap.add_argument("--gemm-smem-kb", type=int, default=None,
+                    help="DCU_OPT_GEMM_SMEM_KB (layer GEMM shared memory per CTA); default: the library's")
     ap.add_argument("--attention", choices=["tcgen05", "mma_sync"], default=None,
                     help="attention implementation (DCU_OPT_ATTENTION; default: the library's)")
     ap.add_argument("--layers", type=int, default=0,
@@ -395,6 +397,9 @@ def main():
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_FUSED_EPILOGUE, args.fused)
     if args.l2_prefetch is not None:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_L2_PREFETCH, args.l2_prefetch)
+    if args.gemm_smem_kb is not None:
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_GEMM_SMEM_KB, args.gemm_smem_kb)
+        config["gemm_smem_kb"] = args.gemm_smem_kb
     if args.attention is not None:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION,
                            dcu.DCU_ATTN_TCGEN05 if args.attention == "tcgen05" else dcu.DCU_ATTN_MMA_SYNC)

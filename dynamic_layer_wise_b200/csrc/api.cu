@@ -112,6 +112,7 @@ struct dcu_ctx {
   int fused = 0;             // chained launches in use (DCU_OPT_FUSED_EPILOGUE and supported): 1 or 2
   bool fused_ok = false;     // the model supports them (bf16, head_dim 64 or 128)
   int nx_count = 16;         // units per CTA of the next GEMM's weights prefetched into L2 (0: off)
+  size_t gemm_smem = kTcSmem;  // dynamic shared memory of a layer GEMM CTA (DCU_OPT_GEMM_SMEM_KB)
   int32_t *chain_bar = nullptr;  // grid-barrier counters of the chained launches, kChainBars per layer
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
@@ -338,6 +339,7 @@ void gemm_common(dcu_ctx *c, const int32_t *m_total, TcParams *tp) {
   tp->m_total = m_total;
   tp->out = c->C;
   tp->status = c->status();
+  tp->smem_bytes = (uint32_t)c->gemm_smem;  // layer GEMMs (the LM head keeps the default)
 }
 
 // C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
@@ -1056,7 +1058,7 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
                             (uint64_t)(c->prof_max > 0),
                             ((uint64_t)(uint32_t)c->force_lo << 32) | (uint64_t)(uint32_t)c->force_hi,
                             (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16) |
-                                ((uint64_t)c->attn_impl << 32),
+                                ((uint64_t)c->attn_impl << 32) | ((uint64_t)(c->gemm_smem >> 10) << 36),
                             0,
                             0};
   int rc = run_graphed(c, key, (cudaStream_t)stream,
@@ -1080,6 +1082,11 @@ int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
     case DCU_OPT_L2_PREFETCH:
       if (value < 0 || value > 4096) return fail(c, DCU_EINVAL, "L2 prefetch units must lie in [0, 4096]");
       c->nx_count = value;
+      return DCU_OK;
+    case DCU_OPT_GEMM_SMEM_KB:
+      if (value < 136 || (size_t)value * 1024u > kTcSmem)
+        return fail(c, DCU_EINVAL, "DCU_OPT_GEMM_SMEM_KB must lie in [136, 220]");
+      c->gemm_smem = (size_t)value * 1024u;
       return DCU_OK;
     case DCU_OPT_ATTENTION:
       if (value != DCU_ATTN_TCGEN05 && value != DCU_ATTN_MMA_SYNC)

@@ -24,14 +24,24 @@ struct SlotGeo {
   const int32_t *nslots = nullptr;  // device table [n_tiles] of sk_nslots (consumers), or null
 };
 
+// (Every product below is at most n_tiles * kblocks * grid; when that fits in
+// 32 bits -- every shape of these models -- the divisions run in 32-bit
+// arithmetic, which the GPU does natively, with the same results.)
+__host__ __device__ inline bool sk_small(const SlotGeo &g) {
+  return (unsigned long long)g.n_tiles * (unsigned)g.kblocks * (unsigned)g.grid < (1ull << 32);
+}
 __host__ __device__ inline long long sk_begin(const SlotGeo &g, int c) {
+  if (sk_small(g)) {
+    if (g.tile_aligned) return (long long)((unsigned)g.n_tiles * (unsigned)c / (unsigned)g.grid * (unsigned)g.kblocks);
+    return (long long)((unsigned)g.n_tiles * (unsigned)g.kblocks * (unsigned)c / (unsigned)g.grid);
+  }
   if (g.tile_aligned) return (long long)g.n_tiles * c / g.grid * g.kblocks;
   return (long long)g.n_tiles * g.kblocks * c / g.grid;
 }
 // CTA whose range holds flattened index x
 __host__ __device__ inline int sk_owner(const SlotGeo &g, long long x) {
   const long long T = (long long)g.n_tiles * g.kblocks;
-  int c = (int)((x * (long long)g.grid) / T);
+  int c = sk_small(g) ? (int)((unsigned)x * (unsigned)g.grid / (unsigned)T) : (int)((x * (long long)g.grid) / T);
   if (c >= g.grid) c = g.grid - 1;
   while (c + 1 < g.grid && sk_begin(g, c + 1) <= x) ++c;
   while (c > 0 && sk_begin(g, c) > x) --c;

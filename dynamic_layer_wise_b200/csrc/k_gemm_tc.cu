@@ -37,17 +37,59 @@ namespace {
 
 struct Frag {
   int tile, kb0, kb1, seg, arow, slot;
+  int col0, rows;  // first output column and row count of the fragment's weight segment
 };
+
+// The fields of a phase that the per-fragment bookkeeping reads, copied out of
+// the kernel parameters with constant indices.  (Indexing the parameter
+// struct with a run-time phase number, or its small arrays with a run-time
+// segment number, turns every access into a generic load from parameter
+// memory; at the start of a CTA those dependent loads cost microseconds.)
+struct PhaseLite {
+  SlotGeo geo;
+  int nseg, ldc;
+  int t1, t2, t3;   // seg_tile0[1..3]
+  int c0, c1, c2;   // seg_col0[0..2]
+  int r0, r1, r2;   // seg_rows[0..2]
+};
+
+__device__ __forceinline__ void copy_phase(const TcPhase &q, PhaseLite &l) {
+  l.geo = q.geo;
+  l.nseg = q.nseg;
+  l.ldc = q.ldc;
+  l.t1 = q.seg_tile0[1];
+  l.t2 = q.seg_tile0[2];
+  l.t3 = q.seg_tile0[3];
+  l.c0 = q.seg_col0[0];
+  l.c1 = q.seg_col0[1];
+  l.c2 = q.seg_col0[2];
+  l.r0 = q.seg_rows[0];
+  l.r1 = q.seg_rows[1];
+  l.r2 = q.seg_rows[2];
+}
+
+__device__ __forceinline__ PhaseLite phase_lite(const TcParams &p, int ph) {
+  PhaseLite l;
+  if (ph == 0)
+    copy_phase(p.ph[0], l);
+  else if (ph == 1)
+    copy_phase(p.ph[1], l);
+  else
+    copy_phase(p.ph[2], l);
+  return l;
+}
 
 // Fragment iterator over this CTA's stream-K range of one phase, pass by pass.
 struct FragIter {
   long long pos, end;
   int pass, ph;
+  PhaseLite l;
 };
 
 __device__ __forceinline__ FragIter frag_begin(const TcParams &p, int ph) {
-  const SlotGeo &g = p.ph[ph].geo;
   FragIter it;
+  it.l = phase_lite(p, ph);
+  const SlotGeo &g = it.l.geo;
   it.ph = ph;
   it.pass = 0;
   if ((int)blockIdx.x < g.grid) {
@@ -60,14 +102,14 @@ __device__ __forceinline__ FragIter frag_begin(const TcParams &p, int ph) {
 }
 
 __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIter &it, Frag &f) {
-  const TcPhase &q = p.ph[it.ph];
+  const PhaseLite &q = it.l;
   if ((int)blockIdx.x >= q.geo.grid) return false;  // no range in this phase
   while (it.pos >= it.end) {
     if (++it.pass >= passes) return false;
     it.pos = sk_begin(q.geo, blockIdx.x);
   }
   const int KB = q.geo.kblocks;
-  const int t = (int)(it.pos / KB);
+  const int t = sk_small(q.geo) ? (int)((unsigned)it.pos / (unsigned)KB) : (int)(it.pos / KB);
   const int kb0 = (int)(it.pos - (long long)t * KB);
   const long long left = it.end - it.pos;
   const int kb1 = (int)((long long)kb0 + left < KB ? kb0 + left : KB);
@@ -75,10 +117,14 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
   f.tile = t;
   f.kb0 = kb0;
   f.kb1 = kb1;
-  int seg = 0;
-  while (seg + 1 < q.nseg && t >= q.seg_tile0[seg + 1]) ++seg;
+  // segment of tile t (segment starts ascend): selects with constant indices
+  int seg = 0, tile0 = 0, col0 = q.c0, rows = q.r0;
+  if (q.nseg > 1 && t >= q.t1) { seg = 1; tile0 = q.t1; col0 = q.c1; rows = q.r1; }
+  if (q.nseg > 2 && t >= q.t2) { seg = 2; tile0 = q.t2; col0 = q.c2; rows = q.r2; }
   f.seg = seg;
-  f.arow = (t - q.seg_tile0[seg]) * 128;
+  f.arow = (t - tile0) * 128;
+  f.col0 = col0;
+  f.rows = rows;
   f.slot = (int)blockIdx.x - sk_first(q.geo, t);
   return true;
 }
@@ -333,8 +379,14 @@ __device__ void epi_down(const TcParams &p, const TcPhase &q, int M, int t128, i
   }
 }
 
-template <int BN>
+// MODE (compile time, so each instantiation carries only its own code paths
+// and stays small in the instruction cache): kPlain -- stream-K pieces into
+// slots; kLmHead -- epi_mode EPI_LMHEAD; kChained -- chained phases (chain != 0).
+enum { kPlain = 0, kLmHead = 1, kChained = 2 };
+
+template <int BN, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
+  constexpr bool kChain = MODE == kChained, kLm = MODE == kLmHead;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
   __shared__ uint32_t tmem_slot;
@@ -342,17 +394,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   __shared__ int s_epi_ok[4], s_flag, s_same;
   __shared__ double s_red[4];
 
-  // The row count is written by the select / plan kernel two launches before
-  // this one, so it is final even while the previous launch still runs.
-  const int M = p.m_total ? *p.m_total : p.m_host;
-  if (M <= 0) return;  // every CTA of a chained launch leaves here, or none
-  const int passes = (M + BN - 1) / BN;
-  if (!p.chain) {  // a CTA without work may leave (no barrier waits for it)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!kChain) {  // a CTA without work may leave (no barrier waits for it)
     const FragIter it0 = frag_begin(p, 0);
     if (it0.pos >= it0.end) return;
   }
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the first loads' tensor maps into the descriptor cache while the CTA sets up
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.ph[0].nseg; ++s) prefetch_tmap(&p.ph[0].a[s]);
+    prefetch_tmap(&p.ph[0].b);
+  }
+  // The row count is written by the select / plan kernel two launches before
+  // this one, so it is final even while the previous launch still runs; its
+  // load overlaps the set-up below and is checked after it.
+  const int M = p.m_total ? *p.m_total : p.m_host;
   // Two rings: weight tiles (16 KB, from HBM) and activation tiles (one TMA
   // box of the token pass per stage, from L2).  The activation ring only has
   // to cover the L2 latency, so most of shared memory holds weight tiles in
@@ -403,15 +458,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
   volatile int *abort_v = &abort_flag;
+  if (M <= 0) {  // nothing to multiply (uniform: every CTA of the launch leaves here, or none)
+    if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+    return;
+  }
+  const int passes = (M + BN - 1) / BN;
 
   if (warp == 0) {
     // weight producer: the weights are never written by a kernel, so the ring
     // fills before (and while) the previous launch or phase finishes
     if (lane == 0) {
       const uint64_t pol_w = policy_evict_first();  // weights stream through once
-      uint32_t fill_parity[kTcMaxA];
-      bool used[kTcMaxA];
-      for (int s = 0; s < kTcMaxA; ++s) used[s] = false;
+      uint32_t used = 0, fill_parity = 0;  // per stage bit: loaded at least once / parity of its last fill
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -425,8 +483,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           }
           mbar_expect_tx(FULL_A(stage), kTcABytes);
           tma_load_2d(STAGE_A(stage), &p.ph[ph].a[ca.f.seg], ca.kb * 64, ca.f.arow, FULL_A(stage), pol_w);
-          used[stage] = true;
-          fill_parity[stage] = phase;
+          used |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           ca.advance(p, passes, BN);
           if (++stage == SA) {
             stage = 0;
@@ -436,7 +494,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       }
       if (!ok) {
         for (int s = 0; s < SA; ++s)
-          if (used[s]) wait_drain(FULL_A(s), fill_parity[s]);
+          if ((used >> s) & 1u) wait_drain(FULL_A(s), (fill_parity >> s) & 1u);
       } else if (p.nx_count > 0) {
         // the next GEMM's first weight tiles into L2 (fire and forget)
         const int nkb = p.nx_geo.kblocks;
@@ -459,14 +517,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       griddep_wait();
       allow_dependents();  // the next kernel may be scheduled (it waits for this grid)
       const uint64_t pol_x = policy_evict_last();  // activations are re-read by every tile
-      uint32_t fill_parity[kTcMaxB];
-      bool used[kTcMaxB];
-      for (int s = 0; s < kTcMaxB; ++s) used[s] = false;
+      uint32_t used = 0, fill_parity = 0;  // per stage bit: loaded at least once / parity of its last fill
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int ph = 0; ph < p.nphase && ok; ++ph) {
-        if (ph > 0 && p.chain) {
+        if (kChain && ph > 0) {
           // the barrier after phase ph - 1's epilogue: its outputs are this phase's operand
           if (!spin_count(p.bar + 2 * (ph - 1) + 1, (int)gridDim.x, abort_v, p.status)) {
             ok = false;
@@ -486,8 +542,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           // by the MMA; rows past the buffer are zero-filled)
           mbar_expect_tx(FULL_B(stage), b_bytes);
           tma_load_2d(STAGE_B(stage), &p.ph[ph].b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
-          used[stage] = true;
-          fill_parity[stage] = phase;
+          used |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           cb.advance(p, passes, BN);
           if (++stage == SB) {
             stage = 0;
@@ -497,7 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       }
       if (!ok)
         for (int s = 0; s < SB; ++s)
-          if (used[s]) wait_drain(FULL_B(s), fill_parity[s]);
+          if ((used >> s) & 1u) wait_drain(FULL_B(s), (fill_parity >> s) & 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -528,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
             tc_fence_after();
             const uint64_t ad = sw128_desc(STAGE_A(sa));
             const uint64_t bd = sw128_desc(STAGE_B(sb));
-            if (p.epi_mode == EPI_LMHEAD) {
+            if (kLm) {
               // LM head: tokens are the MMA M dimension (one or two 128-row halves of
               // the activation box), the tile's 128 vocabulary rows are N
               for (int mt = 0; mt < lm_halves; ++mt) {
@@ -598,7 +654,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
         const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q4 * 32) << 16);
         bool okw = __all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status));
-        if (p.chain) {
+        if (kChain) {
           // the 4 warps meet at named barriers below: they leave together or not at all
           if (lane == 0) s_epi_ok[ew] = okw ? 1 : 0;
           epi_bar();
@@ -611,9 +667,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         }
         tc_fence_after();
         const int rin = f.arow + q4 * 32 + lane;  // row within the weight segment
-        const bool col_ok = rin < q.seg_rows[f.seg];
-        const size_t col = (size_t)(q.seg_col0[f.seg] + rin);
-        if (p.epi_mode == EPI_LMHEAD) {
+        const bool col_ok = rin < f.rows;
+        const size_t col = (size_t)(f.col0 + rin);
+        if (kLm) {
           // LM head: this thread owns token m = mt * 128 + (TMEM lane) and folds the
           // tile's 128 logits into its running (max, sum of exp, lowest argmax);
           // tiles arrive in increasing vocabulary order, so on equal maxima the
@@ -636,13 +692,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
               if (zdst) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                  if (vbase + c + j < q.seg_rows[0]) zdst[c + j] = v[j];
+                  if (vbase + c + j < f.rows) zdst[c + j] = v[j];
               }
               float cm = -INFINITY;
               int cj = 0;
 #pragma unroll
               for (int j = 0; j < 16; ++j) {
-                const bool ok = vbase + c + j < q.seg_rows[0];
+                const bool ok = vbase + c + j < f.rows;
                 v[j] = ok ? v[j] : -INFINITY;
                 if (v[j] > cm) { cm = v[j]; cj = j; }
               }
@@ -666,14 +722,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           ++nfrag;
           continue;
         }
-        float *dst = p.out + (size_t)f.slot * (size_t)q.geo.slot_stride + col;
+        float *dst = p.out + (size_t)f.slot * (size_t)it.l.geo.slot_stride + col;
+        const size_t ldc = (size_t)it.l.ldc;
         for (int c = 0; c < mrows; c += 16) {
           float v[16];
           tmem_ld16(tacc + (uint32_t)c, v);
           if (col_ok) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (c + j < mrows) dst[(size_t)(m0 + c + j) * q.ldc] = v[j];
+              if (c + j < mrows) dst[(size_t)(m0 + c + j) * ldc] = v[j];
           }
         }
         tc_fence_before();
@@ -681,7 +738,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         if (lane == 0) mbar_arrive(TEMPTY(acc));  // the accumulator may be reused from here on
         ++nfrag;
       }
-      if (!alive || !p.chain) continue;
+      if (!alive || !kChain) continue;
       // chained launch: every piece of this phase is stored once all CTAs are here
       if (!grid_sync(p.bar + 2 * ph, ew, lane, abort_v, p.status, &s_flag)) {
         alive = false;
@@ -701,7 +758,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         break;
       }
     }
-    if (p.epi_mode == EPI_LMHEAD) lm_flush(lm_pass);
+    if (kLm) lm_flush(lm_pass);
   }
 #undef FULL_A
 #undef EMPTY_A
@@ -751,17 +808,17 @@ bool encode_tmap_bf16(CUtensorMap *map, const void *ptr, uint64_t inner, uint64_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, int MODE>
 static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
   static std::atomic<uint64_t> smem_set{0};
-  if (cudaError_t e = ensure_smem_limit(k_gemm_tc<BN>, (int)kTcSmem, smem_set)) return e;
-  prefer_max_smem(reinterpret_cast<const void *>(k_gemm_tc<BN>));
+  if (cudaError_t e = ensure_smem_limit(k_gemm_tc<BN, MODE>, (int)kTcSmem, smem_set)) return e;
+  prefer_max_smem(reinterpret_cast<const void *>(k_gemm_tc<BN, MODE>));
   // programmatic dependent launch: the CTAs may start while the previous kernel
   // finishes; they wait (griddepcontrol.wait) before reading its outputs
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = kTcSmem;
+  cfg.dynamicSmemBytes = p.smem_bytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -771,7 +828,14 @@ static cudaError_t launch_bn(const TcParams &p, int grid, cudaStream_t s) {
   attr[1].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = p.chain == 1 ? 2 : 1;  // chain 2: programmatic launch only (all CTAs fit one per SM)
-  return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN>, p);
+  return cudaLaunchKernelEx(&cfg, k_gemm_tc<BN, MODE>, p);
+}
+
+template <int BN>
+static cudaError_t launch_mode(const TcParams &p, int grid, cudaStream_t s) {
+  if (p.chain) return launch_bn<BN, kChained>(p, grid, s);
+  if (p.epi_mode == EPI_LMHEAD) return launch_bn<BN, kLmHead>(p, grid, s);
+  return launch_bn<BN, kPlain>(p, grid, s);
 }
 
 cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
@@ -780,10 +844,20 @@ cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
   for (int i = 1; i < p.nphase; ++i) grid = p.ph[i].geo.grid > grid ? p.ph[i].geo.grid : grid;
   if (grid <= 0) return cudaSuccess;
   if (p.chain && !p.bar) return cudaErrorInvalidValue;
+  if (p.chain && p.epi_mode == EPI_LMHEAD) return cudaErrorInvalidValue;
   if (p.b_rows <= 0 || p.b_rows > bn || p.b_rows % 16 != 0) return cudaErrorInvalidValue;
-  p.smem_bytes = (uint32_t)kTcSmem;
-  if (bn == 128) return launch_bn<128>(p, grid, s);
-  if (bn == 256) return launch_bn<256>(p, grid, s);
+  // dynamic shared memory: the default fills the SM; a smaller ring (at least
+  // the activation stages and 4 weight tiles) leaves room for the CTAs of the
+  // neighbouring small kernels, so this launch's CTAs become resident (and
+  // start their weight stream) while those still run
+  {
+    const uint32_t b_stage = ((uint32_t)p.b_rows * 128u + 1023u) & ~1023u;
+    const uint32_t need = 1024u + (b_stage > 16384u ? 3u : 4u) * b_stage + 4u * kTcABytes;
+    if (p.smem_bytes == 0 || p.smem_bytes > (uint32_t)kTcSmem) p.smem_bytes = (uint32_t)kTcSmem;
+    if (p.smem_bytes < need) p.smem_bytes = need;
+  }
+  if (bn == 128) return launch_mode<128>(p, grid, s);
+  if (bn == 256) return launch_mode<256>(p, grid, s);
   return cudaErrorInvalidValue;
 }
 

@@ -70,6 +70,12 @@ __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *map, int x, i
                : "memory");
 }
 
+// Brings a tensor map (a kernel parameter) into the descriptor cache ahead of
+// its first TMA use.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

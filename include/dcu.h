@@ -162,6 +162,11 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
  *     registers, 64-key chunks.  Both split the keys over at most 8 CTAs per
  *     (sequence, kv head, query tile) and merge the splits in split order. */
 #define DCU_OPT_ATTENTION 3
+/*   DCU_OPT_GEMM_SMEM_KB (136 .. 220, default 220): dynamic shared memory of a
+ *     layer GEMM CTA (its weight ring).  A smaller ring leaves room on each SM
+ *     for the CTAs of the small kernels before it, so the GEMM's CTAs become
+ *     resident, and start streaming weights, while those still run. */
+#define DCU_OPT_GEMM_SMEM_KB 4
 #define DCU_ATTN_TCGEN05 0
 #define DCU_ATTN_MMA_SYNC 1
 int dcu_set_option(dcu_ctx *ctx, int32_t option, int32_t value);

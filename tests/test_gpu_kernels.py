@@ -201,9 +201,11 @@ def test_options_refuse_bad_values():
                          dtype="bf16")
     ctx = dcu.dcu_create(I.device_weights(shape, 2), I.cfg_dict(shape, 1, 64))
     for opt, val in [(dcu.DCU_OPT_ATTENTION, 2), (dcu.DCU_OPT_ATTENTION, -1), (dcu.DCU_OPT_FUSED_EPILOGUE, 3),
-                     (dcu.DCU_OPT_L2_PREFETCH, -1), (dcu.DCU_OPT_L2_PREFETCH, 4097), (99, 0)]:
+                     (dcu.DCU_OPT_L2_PREFETCH, -1), (dcu.DCU_OPT_L2_PREFETCH, 4097), (dcu.DCU_OPT_GEMM_SMEM_KB, 135),
+                     (dcu.DCU_OPT_GEMM_SMEM_KB, 221), (99, 0)]:
         with pytest.raises(dcu.DcuError):
             dcu.dcu_set_option(ctx, opt, val)
     dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_MMA_SYNC)
     dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION, dcu.DCU_ATTN_TCGEN05)
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_GEMM_SMEM_KB, 160)
     ctx.close()

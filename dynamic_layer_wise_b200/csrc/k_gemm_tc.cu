@@ -101,6 +101,9 @@ __device__ __forceinline__ FragIter frag_begin(const TcParams &p, int ph) {
   return it;
 }
 
+// kSlot: also find the fragment's output slot (a search over the stream-K
+// ranges that only the epilogue needs; the loaders and the MMA skip it).
+template <bool kSlot>
 __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIter &it, Frag &f) {
   const PhaseLite &q = it.l;
   if ((int)blockIdx.x >= q.geo.grid) return false;  // no range in this phase
@@ -125,7 +128,7 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
   f.arow = (t - tile0) * 128;
   f.col0 = col0;
   f.rows = rows;
-  f.slot = (int)blockIdx.x - sk_first(q.geo, t);
+  if (kSlot) f.slot = (int)blockIdx.x - sk_first(q.geo, t);
   return true;
 }
 
@@ -135,9 +138,10 @@ struct KCursor {
   Frag f;
   int kb, m0;
   bool valid;
-  __device__ __forceinline__ void start(const TcParams &p, int ph, int passes, int BN) {
-    it = frag_begin(p, ph);
-    valid = next_frag(p, passes, it, f);
+  // it0: this CTA's iterator of phase ph, fresh from frag_begin
+  __device__ __forceinline__ void start(const TcParams &p, const FragIter &it0, int passes, int BN) {
+    it = it0;
+    valid = next_frag<false>(p, passes, it, f);
     if (valid) {
       kb = f.kb0;
       m0 = it.pass * BN;
@@ -145,7 +149,7 @@ struct KCursor {
   }
   __device__ __forceinline__ void advance(const TcParams &p, int passes, int BN) {
     if (++kb < f.kb1) return;
-    valid = next_frag(p, passes, it, f);
+    valid = next_frag<false>(p, passes, it, f);
     if (valid) {
       kb = f.kb0;
       m0 = it.pass * BN;
@@ -395,10 +399,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   __shared__ double s_red[4];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (!kChain) {  // a CTA without work may leave (no barrier waits for it)
-    const FragIter it0 = frag_begin(p, 0);
-    if (it0.pos >= it0.end) return;
-  }
+  // this CTA's stream-K range of the first phase (every role starts from it)
+  const FragIter it_first = frag_begin(p, 0);
+  if (!kChain && it_first.pos >= it_first.end) return;  // a CTA without work may leave (no barrier waits for it)
   // the first loads' tensor maps into the descriptor cache while the CTA sets up
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.ph[0].nseg; ++s) prefetch_tmap(&p.ph[0].a[s]);
@@ -437,13 +440,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       mbar_init(FULL_A(s), 1);
       mbar_init(EMPTY_A(s), 1);
     }
-    for (int s = 0; s < SB; ++s) {
-      mbar_init(FULL_B(s), 1);
-      mbar_init(EMPTY_B(s), 1);
-    }
     for (int a = 0; a < 2; ++a) {
       mbar_init(TFULL(a), 1);
       mbar_init(TEMPTY(a), 4);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(FULL_B(s), 1);
+      mbar_init(EMPTY_B(s), 1);
     }
     mbar_init(drain, 1);
     abort_flag = 0;
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       bool ok = true;
       for (int ph = 0; ph < p.nphase && ok; ++ph) {
         KCursor ca;
-        ca.start(p, ph, passes, BN);
+        ca.start(p, ph == 0 ? it_first : frag_begin(p, ph), passes, BN);
         while (ca.valid) {
           if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
             ok = false;
@@ -514,9 +517,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     // activation producer: the packed rows are written by the previous launch
     // (phase 0) or by the previous phase's epilogue (chained phases)
     if (lane == 0) {
+      const uint64_t pol_x = policy_evict_last();  // activations are re-read by every tile
+      KCursor cb0;  // the first phase's cursor, ready before the wait
+      cb0.start(p, it_first, passes, BN);
       griddep_wait();
       allow_dependents();  // the next kernel may be scheduled (it waits for this grid)
-      const uint64_t pol_x = policy_evict_last();  // activations are re-read by every tile
       uint32_t used = 0, fill_parity = 0;  // per stage bit: loaded at least once / parity of its last fill
       int stage = 0;
       uint32_t phase = 0;
@@ -530,8 +535,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           }
           fence_proxy_async_global();  // generic-proxy stores of other CTAs, read next by TMA
         }
-        KCursor cb;
-        cb.start(p, ph, passes, BN);
+        KCursor cb = cb0;
+        if (ph > 0) cb.start(p, frag_begin(p, ph), passes, BN);
         while (cb.valid) {
           if (!wait_bounded(EMPTY_B(stage), phase ^ 1u, abort_v, p.status)) {
             ok = false;
@@ -562,9 +567,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       const uint32_t idesc_lm = idesc_bf16(128, 128);
       bool ok = true, issued = false;
       for (int ph = 0; ph < p.nphase && ok; ++ph) {
-        FragIter it = frag_begin(p, ph);
+        FragIter it = ph == 0 ? it_first : frag_begin(p, ph);
         Frag f;
-        while (ok && next_frag(p, passes, it, f)) {
+        while (ok && next_frag<false>(p, passes, it, f)) {
           const int mrows = min(BN, M - it.pass * BN);
           const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
           const int lm_halves = mrows > 128 ? 2 : 1;
@@ -646,9 +651,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     bool alive = true;
     for (int ph = 0; ph < p.nphase && alive; ++ph) {
       const TcPhase &q = p.ph[ph];
-      FragIter it = frag_begin(p, ph);
+      FragIter it = ph == 0 ? it_first : frag_begin(p, ph);
       Frag f;
-      while (next_frag(p, passes, it, f)) {
+      while (next_frag<true>(p, passes, it, f)) {
         const int m0 = it.pass * BN;
         const int mrows = min(BN, M - m0);
         const uint32_t acc = nfrag & 1u, use = nfrag >> 1;

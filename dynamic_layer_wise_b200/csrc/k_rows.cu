@@ -209,11 +209,45 @@ cudaError_t launch_gather_norm(int dtype, const int32_t *rowmap, const int32_t *
   return cudaGetLastError();
 }
 
-// 4 consecutive GEMM outputs (j % 4 == 0): the pieces of column j's 128-wide
-// tile summed in slot order (one piece when geo.grid == 0).
+// Pieces of column j's 128-wide tile (1 when geo.grid == 0).  The piece tables
+// are written when a geometry is first used, long before an epilogue reads them.
+__device__ __forceinline__ int slot_count(const SlotGeo &geo, size_t j) {
+  return geo.grid <= 0 ? 1 : (geo.nslots ? __ldg(geo.nslots + (j >> 7)) : sk_nslots(geo, (int)(j >> 7)));
+}
+
+// 4 consecutive GEMM outputs (j % 4 == 0) summed over their ns pieces in slot
+// order; the loads of up to K pieces are all issued before the first add (a
+// tile of the 32-tile GEMMs over 148 CTAs has up to 6 pieces).
+template <int K = 8>
+__device__ __forceinline__ float4 csum4n(const float *c, long long stride, size_t j, int ns) {
+  float4 w[K];
+#pragma unroll
+  for (int sp = 0; sp < K; ++sp)
+    if (sp < ns) w[sp] = *reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)stride + j);
+  float4 v = w[0];
+#pragma unroll
+  for (int sp = 1; sp < K; ++sp)
+    if (sp < ns) {
+      v.x += w[sp].x;
+      v.y += w[sp].y;
+      v.z += w[sp].z;
+      v.w += w[sp].w;
+    }
+  for (int sp = K; sp < ns; ++sp) {
+    const float4 u = *reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)stride + j);
+    v.x += u.x;
+    v.y += u.y;
+    v.z += u.z;
+    v.w += u.w;
+  }
+  return v;
+}
+
+// The same sum with one load in flight at a time: few registers, for the
+// flattened epilogues whose occupancy matters more than one row's latency.
 __device__ __forceinline__ float4 csum4(const float *c, const SlotGeo &geo, size_t j) {
   float4 v = *reinterpret_cast<const float4 *>(c + j);
-  const int ns = geo.grid <= 0 ? 1 : (geo.nslots ? __ldg(geo.nslots + (j >> 7)) : sk_nslots(geo, (int)(j >> 7)));
+  const int ns = slot_count(geo, j);
   for (int sp = 1; sp < ns; ++sp) {
     const float4 w = *reinterpret_cast<const float4 *>(c + (size_t)sp * (size_t)geo.slot_stride + j);
     v.x += w.x;
@@ -223,6 +257,12 @@ __device__ __forceinline__ float4 csum4(const float *c, const SlotGeo &geo, size
   }
   return v;
 }
+
+// The row epilogues (O, down) run right after a GEMM under programmatic
+// dependent launch.  Only the GEMM's slots come from the launch they wait for;
+// the row count, the row plan, the piece tables and the other operands were
+// written two or more launches earlier (final once this launch has started),
+// so they are loaded before the wait and only the slot loads follow it.
 
 template <class T>
 __device__ __forceinline__ void store4(T *p, float a, float b, float c, float d);
@@ -320,23 +360,49 @@ __global__ void __launch_bounds__(512)
     k_epi_o(const float *__restrict__ C, int ldc, const SlotGeo geo, const int32_t *__restrict__ rowmap,
             const int32_t *__restrict__ m_total, const T *__restrict__ Hl, const float *__restrict__ g2, float eps,
             int D, float *__restrict__ hmid, T *__restrict__ xs) {
-  pdl_enter();
   __shared__ double red[32];
   const int M = *m_total;
-  for (int r = blockIdx.x; r < M; r += gridDim.x) {
-    const T *x = Hl + (size_t)rowmap[r] * D;
+  const int r0 = blockIdx.x, j0 = threadIdx.x * 8;
+  // the first row's operands other than the slots, before the wait
+  const bool pre = r0 < M && j0 < D;
+  int row0 = 0, ns0 = 1;
+  float xv[8], gv[8];
+  if (pre) {
+    row0 = rowmap[r0];
+    const T *x = Hl + (size_t)row0 * D + j0;
+    if (Vec<T>::n == 8) {
+      load_vec(x, *reinterpret_cast<float(*)[Vec<T>::n]>(xv));
+    } else {
+      load_vec(x, *reinterpret_cast<float(*)[Vec<T>::n]>(xv));
+      load_vec(x + 4, *reinterpret_cast<float(*)[Vec<T>::n]>(xv + 4));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) gv[e] = g2[j0 + e];
+    ns0 = slot_count(geo, j0);
+  }
+  griddep_wait();
+  allow_dependents();
+  for (int r = r0; r < M; r += gridDim.x) {
+    const bool first = r == r0;
+    const int row = first ? row0 : rowmap[r];
+    const T *x = Hl + (size_t)row * D;
     const float *c = C + (size_t)r * ldc;
     float *hm = hmid + (size_t)r * D;
     double ss = 0;
-    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
+    for (int j = j0; j < D; j += blockDim.x * 8) {
+      const bool p0 = first && j == j0;
       float v[8];
-      if (Vec<T>::n == 8) {
+      if (p0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = xv[e];
+      } else if (Vec<T>::n == 8) {
         load_vec(x + j, *reinterpret_cast<float(*)[Vec<T>::n]>(v));
       } else {
         load_vec(x + j, *reinterpret_cast<float(*)[Vec<T>::n]>(v));
         load_vec(x + j + 4, *reinterpret_cast<float(*)[Vec<T>::n]>(v + 4));
       }
-      const float4 c0 = csum4(c, geo, j), c1 = csum4(c, geo, j + 4);
+      const int ns = p0 ? ns0 : slot_count(geo, j);  // j and j + 4 share their tile
+      const float4 c0 = csum4n<6>(c, geo.slot_stride, j, ns), c1 = csum4n<6>(c, geo.slot_stride, j + 4, ns);
       v[0] += c0.x; v[1] += c0.y; v[2] += c0.z; v[3] += c0.w;
       v[4] += c1.x; v[5] += c1.y; v[6] += c1.z; v[7] += c1.w;
       *reinterpret_cast<float4 *>(hm + j) = make_float4(v[0], v[1], v[2], v[3]);
@@ -347,11 +413,13 @@ __global__ void __launch_bounds__(512)
     ss = block_sum(ss, red);
     const float inv = (float)(1.0 / sqrt(ss / (double)D + (double)eps));
     T *o = xs + (size_t)r * D;
-    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
+    for (int j = j0; j < D; j += blockDim.x * 8) {
       const float4 h0 = *reinterpret_cast<const float4 *>(hm + j), h1 = *reinterpret_cast<const float4 *>(hm + j + 4);
-      store4<T>(o + j, h0.x * inv * g2[j], h0.y * inv * g2[j + 1], h0.z * inv * g2[j + 2], h0.w * inv * g2[j + 3]);
-      store4<T>(o + j + 4, h1.x * inv * g2[j + 4], h1.y * inv * g2[j + 5], h1.z * inv * g2[j + 6],
-                h1.w * inv * g2[j + 7]);
+      float g[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = (first && j == j0) ? gv[e] : g2[j + e];
+      store4<T>(o + j, h0.x * inv * g[0], h0.y * inv * g[1], h0.z * inv * g[2], h0.w * inv * g[3]);
+      store4<T>(o + j + 4, h1.x * inv * g[4], h1.y * inv * g[5], h1.z * inv * g[6], h1.w * inv * g[7]);
     }
   }
 }
@@ -406,28 +474,63 @@ __global__ void __launch_bounds__(512)
                        const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total,
                        const float *__restrict__ hmid, T *__restrict__ Hn, const float *__restrict__ g_next,
                        float *__restrict__ d_next, uint8_t *__restrict__ stale_next, int D) {
-  pdl_enter();
   __shared__ double red[32];
   constexpr int VN = Vec<T>::n;
   const int M = *m_total;
-  for (int r = blockIdx.x; r < M; r += gridDim.x) {
-    const int row = rowmap[r];
+  const int r0 = blockIdx.x, j0 = threadIdx.x * 8;
+  // the first row's operands other than the slots, before the wait: hmid (the
+  // O epilogue's, three launches back) and the cached H_{l+1} row that the
+  // distance compares against (only this launch rewrites it)
+  const bool pre = r0 < M && j0 < D;
+  int row0 = 0, ns0 = 1;
+  float4 h0p = make_float4(0.f, 0.f, 0.f, 0.f), h1p = h0p;
+  float ovp[8];
+  uint32_t obp[8];
+  if (pre) {
+    row0 = rowmap[r0];
+    ns0 = slot_count(geo, j0);
+    const float *hm = hmid + (size_t)r0 * D;
+    h0p = *reinterpret_cast<const float4 *>(hm + j0);
+    h1p = *reinterpret_cast<const float4 *>(hm + j0 + 4);
+    if (d_next) {
+      const T *dst = Hn + (size_t)row0 * D;
+#pragma unroll
+      for (int q = 0; q < 8; q += VN)
+        load_vec(dst + j0 + q, *reinterpret_cast<float(*)[VN]>(ovp + q), *reinterpret_cast<uint32_t(*)[VN]>(obp + q));
+    }
+  }
+  griddep_wait();
+  allow_dependents();
+  for (int r = r0; r < M; r += gridDim.x) {
+    const bool first = r == r0;
+    const int row = first ? row0 : rowmap[r];
     const float *c = C + (size_t)r * ldc;
     const float *hm = hmid + (size_t)r * D;
     T *dst = Hn + (size_t)row * D;
     double dot = 0, nx = 0, ny = 0;
     bool same = true;
-    for (int j = threadIdx.x * 8; j < D; j += blockDim.x * 8) {
-      const float4 c0 = csum4(c, geo, j), c1 = csum4(c, geo, j + 4);
-      const float4 h0 = *reinterpret_cast<const float4 *>(hm + j), h1 = *reinterpret_cast<const float4 *>(hm + j + 4);
+    for (int j = j0; j < D; j += blockDim.x * 8) {
+      const bool p0 = first && j == j0;
+      const int ns = p0 ? ns0 : slot_count(geo, j);  // j and j + 4 share their tile
+      const float4 c0 = csum4n<6>(c, geo.slot_stride, j, ns), c1 = csum4n<6>(c, geo.slot_stride, j + 4, ns);
+      const float4 h0 = p0 ? h0p : *reinterpret_cast<const float4 *>(hm + j);
+      const float4 h1 = p0 ? h1p : *reinterpret_cast<const float4 *>(hm + j + 4);
       float v[8] = {h0.x + c0.x, h0.y + c0.y, h0.z + c0.z, h0.w + c0.w,
                     h1.x + c1.x, h1.y + c1.y, h1.z + c1.z, h1.w + c1.w};
       if (d_next) {
         float ov[8];
         uint32_t ob[8];
+        if (p0) {
 #pragma unroll
-        for (int q = 0; q < 8; q += VN)
-          load_vec(dst + j + q, *reinterpret_cast<float(*)[VN]>(ov + q), *reinterpret_cast<uint32_t(*)[VN]>(ob + q));
+          for (int e = 0; e < 8; ++e) {
+            ov[e] = ovp[e];
+            ob[e] = obp[e];
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; q += VN)
+            load_vec(dst + j + q, *reinterpret_cast<float(*)[VN]>(ov + q), *reinterpret_cast<uint32_t(*)[VN]>(ob + q));
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const T nt = from_f<T>(v[e]);

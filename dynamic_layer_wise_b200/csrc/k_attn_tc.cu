@@ -175,6 +175,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     abort_flag = 0;
     fence_barrier_init();
   }
+  // This split's first K / V chunks into L2 while the previous launch (the QKV
+  // epilogue, which rewrites only the recomputed rows) still runs; L2 stays
+  // coherent with those writes, so the loads after the wait see them.
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&a.kmap);
+    prefetch_tmap(&a.vmap);
+    const int y0 = (b * a.Hkv + kvh) * a.N + k_begin;
+    const int npf = nch < 4 ? nch : 4;
+    for (int j = 0; j < npf; ++j)
+#pragma unroll
+      for (int h = 0; h < HD / 64; ++h) {
+        tma_prefetch_2d(&a.kmap, h * 64, y0 + j * kKC);
+        tma_prefetch_2d(&a.vmap, h * 64, y0 + j * kKC);
+      }
+  }
   if (warp == 0) {
     tmem_alloc(smem_u32(&tmem_slot), C::kTmemCols);
     tmem_relinquish();

@@ -98,7 +98,6 @@ __global__ void __launch_bounds__(kSelThreads)
              int force_hi, int32_t *__restrict__ idx, int32_t *__restrict__ count, float *__restrict__ s_out, int s_stride,
              float *__restrict__ d_next_zero, int32_t *__restrict__ rowmap, int32_t *__restrict__ m_total,
              int32_t *__restrict__ done, int32_t *__restrict__ seq_off, int32_t *__restrict__ status) {
-  pdl_enter();
   extern __shared__ __align__(16) uint8_t smem[];
   uint32_t *sd = reinterpret_cast<uint32_t *>(smem);     // [N] d bits
   uint8_t *flag = smem + (size_t)N * sizeof(uint32_t);   // [N] 0 none, 1 window, 2 top-B
@@ -113,18 +112,17 @@ __global__ void __launch_bounds__(kSelThreads)
   const int b = blockIdx.x;
   const int tid = threadIdx.x, nthr = blockDim.x;
   const float *db = d + (size_t)b * N;
-  // independent loads first, so their latencies overlap
+
+  // Everything but d is written two or more launches earlier (key positions and
+  // budgets before the step; the next layer's d is read only by later
+  // launches), so the window is marked and d_next cleared before the wait for
+  // the previous launch (the scatter that wrote this layer's d).
   const int nk_in = nkeys[b];
   const int k_in = budgets[(size_t)b * budget_stride];
-
-  for (int i = tid; i < N; i += nthr) {
-    sd[i] = __float_as_uint(db[i]);
-    flag[i] = 0;
-  }
+  for (int i = tid; i < N; i += nthr) flag[i] = 0;
   if (d_next_zero)
     for (int i = tid; i < N; i += nthr) d_next_zero[(size_t)b * N + i] = 0.f;
   __syncthreads();
-
   // forced window
   int nk = nk_in;
   if (nk < 0 || nk > N) {
@@ -149,14 +147,19 @@ __global__ void __launch_bounds__(kSelThreads)
   // periodic refresh: the forced range joins the window (recomputed whatever the budget)
   for (int i = max(force_lo, 0) + tid; i < min(force_hi, N); i += nthr) flag[i] = 1;
   __syncthreads();
-  int inW = 0, nz = 0;
+  int inW = 0;
+  for (int i = tid; i < N; i += nthr) inW += (flag[i] == 1);
+  inW = block_sum(inW, red_i);
+
+  pdl_enter();  // this layer's d is final from here on
+  for (int i = tid; i < N; i += nthr) sd[i] = __float_as_uint(db[i]);
+  __syncthreads();
+  int nz = 0;
   {
     double acc = 0.0;
     for (int i = tid; i < N; i += nthr) acc += (double)__uint_as_float(sd[i]);
     acc = block_sum(acc, red_d);
     if (tid == 0) s_out[(size_t)b * s_stride] = (float)(acc / (double)N);
-    for (int i = tid; i < N; i += nthr) inW += (flag[i] == 1);
-    inW = block_sum(inW, red_i);
     for (int i = tid; i < N; i += nthr) nz += (flag[i] == 0 && sd[i] != 0u);
     nz = block_sum(nz, red_i);
   }

@@ -298,15 +298,30 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
                           const int32_t *__restrict__ rowmap, const int32_t *__restrict__ m_total, int N, int H,
                           int Hkv, int hd, const float2 *__restrict__ rope_tab, int use_rope, T *__restrict__ Q,
                           T *__restrict__ Kc, T *__restrict__ Vc, uint8_t *__restrict__ stale) {
-  pdl_enter();
   const int M = *m_total;
   const int half = hd / 2;
   const int n_rope = (H + Hkv) * half / 4, n_v = Hkv * hd / 4;
   const int per_row = n_rope + n_v;
-  for (long long it = blockIdx.x * (long long)blockDim.x + threadIdx.x; it < (long long)M * per_row;
-       it += (long long)gridDim.x * blockDim.x) {
+  // the first item's row and RoPE factors (written long before this launch),
+  // loaded before the wait for the QKV GEMM
+  const long long it0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  int row0 = 0;
+  float2 cs0[4];
+  if (it0 < (long long)M * per_row) {
+    const int r = (int)(it0 / per_row), u = (int)(it0 - (long long)r * per_row);
+    row0 = rowmap[r];
+    if (u < n_rope && use_rope) {
+      const int t = u * 4, head = t / half, j = t - head * half;
+      const int i = row0 - (row0 / N) * N;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) cs0[e] = rope_tab[(size_t)i * half + j + e];
+    }
+  }
+  pdl_enter();
+  for (long long it = it0; it < (long long)M * per_row; it += (long long)gridDim.x * blockDim.x) {
+    const bool first = it == it0;
     const int r = (int)(it / per_row), u = (int)(it - (long long)r * per_row);
-    const int row = rowmap[r];
+    const int row = first ? row0 : rowmap[r];
     const int b = row / N, i = row - b * N;
     const float *c = C + (size_t)r * ldc;
     if (u < n_rope) {
@@ -318,7 +333,7 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
       if (use_rope) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 cs = rope_tab[(size_t)i * half + j + e];
+          const float2 cs = first ? cs0[e] : rope_tab[(size_t)i * half + j + e];
           const float a2 = av[e] * cs.x - bv[e] * cs.y;
           const float b2 = bv[e] * cs.x + av[e] * cs.y;
           av[e] = a2;

@@ -322,6 +322,8 @@ def main():
                     help="DCU_OPT_L2_PREFETCH (next-GEMM weight units per CTA into L2); default: the library's")
     ap.add_argument("--gemm-smem-kb", type=int, default=None,
                     help="DCU_OPT_GEMM_SMEM_KB (layer GEMM shared memory per CTA); default: the library's")
+    ap.add_argument("--gemm-pass-sweep", type=int, choices=[0, 1], default=None,
+                    help="DCU_OPT_GEMM_PASS_SWEEP (token passes sharing each weight tile); default: the library's")
     ap.add_argument("--attention", choices=["tcgen05", "mma_sync"], default=None,
                     help="attention implementation (DCU_OPT_ATTENTION; default: the library's)")
     ap.add_argument("--layers", type=int, default=0,
@@ -400,6 +402,9 @@ def main():
     if args.gemm_smem_kb is not None:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_GEMM_SMEM_KB, args.gemm_smem_kb)
         config["gemm_smem_kb"] = args.gemm_smem_kb
+    if args.gemm_pass_sweep is not None:
+        dcu.dcu_set_option(ctx, dcu.DCU_OPT_GEMM_PASS_SWEEP, args.gemm_pass_sweep)
+        config["gemm_pass_sweep"] = args.gemm_pass_sweep
     if args.attention is not None:
         dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION,
                            dcu.DCU_ATTN_TCGEN05 if args.attention == "tcgen05" else dcu.DCU_ATTN_MMA_SYNC)

@@ -113,6 +113,7 @@ struct dcu_ctx {
   bool fused_ok = false;     // the model supports them (bf16, head_dim 64 or 128)
   int nx_count = 16;         // units per CTA of the next GEMM's weights prefetched into L2 (0: off)
   size_t gemm_smem = kTcSmem;  // dynamic shared memory of a layer GEMM CTA (DCU_OPT_GEMM_SMEM_KB)
+  int pass_sweep = 1;          // DCU_OPT_GEMM_PASS_SWEEP
   int32_t *chain_bar = nullptr;  // grid-barrier counters of the chained launches, kChainBars per layer
   std::vector<LayerMaps> lmaps;
   CUtensorMap lm_map;
@@ -340,6 +341,10 @@ void gemm_common(dcu_ctx *c, const int32_t *m_total, TcParams *tp) {
   tp->out = c->C;
   tp->status = c->status();
   tp->smem_bytes = (uint32_t)c->gemm_smem;  // layer GEMMs (the LM head keeps the default)
+  // pass sweep with the 256-row pass (recompute sets expected past 192 rows):
+  // its activation stages take shared memory from the weight ring, which the
+  // 128-row pass of the small sets keeps whole
+  tp->sweep = (c->pass_sweep && c->gemm_bn == 256) ? 2 : 0;
 }
 
 // C[m][n] = sum_k X[m][k] W[n][k] over the concatenated segments: ctx->C as
@@ -1058,7 +1063,8 @@ int dcu_step(dcu_ctx *c, const int32_t *ids, const int32_t *keys, const int32_t 
                             (uint64_t)(c->prof_max > 0),
                             ((uint64_t)(uint32_t)c->force_lo << 32) | (uint64_t)(uint32_t)c->force_hi,
                             (uint64_t)c->select_from | ((uint64_t)c->fused << 8) | ((uint64_t)c->nx_count << 16) |
-                                ((uint64_t)c->attn_impl << 32) | ((uint64_t)(c->gemm_smem >> 10) << 36),
+                                ((uint64_t)c->attn_impl << 32) | ((uint64_t)(c->gemm_smem >> 10) << 36) |
+                                ((uint64_t)c->pass_sweep << 48),
                             0,
                             0};
   int rc = run_graphed(c, key, (cudaStream_t)stream,
@@ -1092,6 +1098,10 @@ int dcu_set_option(dcu_ctx *c, int32_t option, int32_t value) {
       if (value != DCU_ATTN_TCGEN05 && value != DCU_ATTN_MMA_SYNC)
         return fail(c, DCU_EINVAL, "DCU_OPT_ATTENTION takes DCU_ATTN_TCGEN05 or DCU_ATTN_MMA_SYNC");
       c->attn_impl = value;
+      return DCU_OK;
+    case DCU_OPT_GEMM_PASS_SWEEP:
+      if (value != 0 && value != 1) return fail(c, DCU_EINVAL, "DCU_OPT_GEMM_PASS_SWEEP takes 0 or 1");
+      c->pass_sweep = value;
       return DCU_OK;
     default:
       return fail(c, DCU_EINVAL, "unknown option");
@@ -1279,6 +1289,7 @@ int dcu_linear(const void *X, const void *W, int32_t M, int32_t K, int32_t Nout,
       !encode_tmap_bf16(&q.b, X, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, (uint32_t)b_rows))
     return fail(nullptr, DCU_ECUDA, "dcu_linear: cuTensorMapEncodeTiled failed");
   tp.b_rows = b_rows;
+  tp.sweep = 512 / bn;  // several token passes share each weight tile
   const int tiles = (Nout + 127) / 128;
   q.seg_tile0[0] = 0;
   q.seg_tile0[1] = tiles;

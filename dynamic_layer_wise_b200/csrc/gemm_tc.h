@@ -115,6 +115,13 @@ struct TcParams {
   int chain;
   int32_t *bar;
   int b_rows;              // rows of the activation box: the token pass (BN) or fewer when cap < BN
+  // Pass sweep (chain = 0, epi_mode 0): when M spans more than one token pass,
+  // up to `sweep` passes share each weight tile while it is in shared memory
+  // (one activation box per pass in a stage, one TMEM accumulator per pass),
+  // so the weights stream from HBM once per group of passes instead of once
+  // per pass.  0 or 1: every pass re-streams the weights.  launch_gemm_tc
+  // lowers it to what TMEM (512 columns) and the shared memory hold.
+  int sweep;
   const int32_t *m_total;  // device row count M (or null: m_host)
   int m_host;
   float *out;              // slots [slot][cap][ldc] (every phase uses the same buffer in turn)

@@ -79,7 +79,8 @@ __device__ __forceinline__ PhaseLite phase_lite(const TcParams &p, int ph) {
   return l;
 }
 
-// Fragment iterator over this CTA's stream-K range of one phase, pass by pass.
+// Fragment iterator over this CTA's stream-K range of one phase, group by
+// group of token passes (a group is one pass unless the launch sweeps).
 struct FragIter {
   long long pos, end;
   int pass, ph;
@@ -104,11 +105,11 @@ __device__ __forceinline__ FragIter frag_begin(const TcParams &p, int ph) {
 // kSlot: also find the fragment's output slot (a search over the stream-K
 // ranges that only the epilogue needs; the loaders and the MMA skip it).
 template <bool kSlot>
-__device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIter &it, Frag &f) {
+__device__ __forceinline__ bool next_frag(const TcParams &p, int ngroups, FragIter &it, Frag &f) {
   const PhaseLite &q = it.l;
   if ((int)blockIdx.x >= q.geo.grid) return false;  // no range in this phase
   while (it.pos >= it.end) {
-    if (++it.pass >= passes) return false;
+    if (++it.pass >= ngroups) return false;
     it.pos = sk_begin(q.geo, blockIdx.x);
   }
   const int KB = q.geo.kblocks;
@@ -132,27 +133,28 @@ __device__ __forceinline__ bool next_frag(const TcParams &p, int passes, FragIte
   return true;
 }
 
-// Position in this CTA's (phase, fragment, k block) sequence.
+// Position in this CTA's (phase, fragment, k block) sequence; m0 is the first
+// row of the fragment's group of token passes (grows rows per group).
 struct KCursor {
   FragIter it;
   Frag f;
   int kb, m0;
   bool valid;
   // it0: this CTA's iterator of phase ph, fresh from frag_begin
-  __device__ __forceinline__ void start(const TcParams &p, const FragIter &it0, int passes, int BN) {
+  __device__ __forceinline__ void start(const TcParams &p, const FragIter &it0, int ngroups, int grows) {
     it = it0;
-    valid = next_frag<false>(p, passes, it, f);
+    valid = next_frag<false>(p, ngroups, it, f);
     if (valid) {
       kb = f.kb0;
-      m0 = it.pass * BN;
+      m0 = it.pass * grows;
     }
   }
-  __device__ __forceinline__ void advance(const TcParams &p, int passes, int BN) {
+  __device__ __forceinline__ void advance(const TcParams &p, int ngroups, int grows) {
     if (++kb < f.kb1) return;
-    valid = next_frag<false>(p, passes, it, f);
+    valid = next_frag<false>(p, ngroups, it, f);
     if (valid) {
       kb = f.kb0;
-      m0 = it.pass * BN;
+      m0 = it.pass * grows;
     }
   }
 };
@@ -385,12 +387,13 @@ __device__ void epi_down(const TcParams &p, const TcPhase &q, int M, int t128, i
 
 // MODE (compile time, so each instantiation carries only its own code paths
 // and stays small in the instruction cache): kPlain -- stream-K pieces into
-// slots; kLmHead -- epi_mode EPI_LMHEAD; kChained -- chained phases (chain != 0).
-enum { kPlain = 0, kLmHead = 1, kChained = 2 };
+// slots; kSweep -- the same with the pass sweep (sweep > 1); kLmHead --
+// epi_mode EPI_LMHEAD; kChained -- chained phases (chain != 0).
+enum { kPlain = 0, kLmHead = 1, kChained = 2, kSweep = 3 };
 
 template <int BN, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant__ TcParams p) {
-  constexpr bool kChain = MODE == kChained, kLm = MODE == kLmHead;
+  constexpr bool kChain = MODE == kChained, kLm = MODE == kLmHead, kSw = MODE == kSweep;
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t bars[2 * kTcMaxA + 2 * kTcMaxB + 5];
   __shared__ uint32_t tmem_slot;
@@ -415,15 +418,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   // box of the token pass per stage, from L2).  The activation ring only has
   // to cover the L2 latency, so most of shared memory holds weight tiles in
   // flight.
-  const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per stage
-  const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned stages
-  const int SB = b_stage > 16384u ? 3 : 4;
-  int SA = (int)((p.smem_bytes - 1024u - (uint32_t)SB * b_stage) / kTcABytes);
+  // Shared memory: the weight ring, then the activation region.  With a pass
+  // sweep an activation stage holds G boxes, one per token pass of the group;
+  // the region is sized for the launch's largest G, so the weight ring's depth
+  // does not depend on M (the weight producer starts before M is loaded) and
+  // only the activation ring's depth follows G.
+  const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per token pass
+  const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned boxes
+  const int gmax = kSw ? p.sweep : 1;
+  const uint32_t x_region = gmax > 1 ? 2u * (uint32_t)gmax * b_stage : (b_stage > 16384u ? 3u : 4u) * b_stage;
+  int SA = (int)((p.smem_bytes - 1024u - x_region) / kTcABytes);
   SA = SA > kTcMaxA ? kTcMaxA : SA;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t bbase = sbase + (uint32_t)SA * kTcABytes;
   const uint32_t bar0 = smem_u32(bars);
-  // two TMEM accumulators (columns [0, BN) and [BN, 2 BN)) alternate between fragments
+  // TMEM: one accumulator of G x BN columns per fragment, two alternating
+  // between fragments while they fit (always for G = 1)
+  const uint32_t tcols = kSw ? 512u : 2u * (uint32_t)BN;
 #define FULL_A(s) (bar0 + 8u * (uint32_t)(s))
 #define EMPTY_A(s) (bar0 + 8u * (uint32_t)(kTcMaxA + (s)))
 #define FULL_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + (s)))
@@ -433,7 +444,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
 #define TFULL(a) (tfull0 + 8u * (uint32_t)(a))
 #define TEMPTY(a) (tempty0 + 8u * (uint32_t)(a))
 #define STAGE_A(s) (sbase + (uint32_t)(s) * kTcABytes)
-#define STAGE_B(s) (bbase + (uint32_t)(s) * b_stage)
+#define STAGE_B(s) (bbase + (uint32_t)(s) * x_stage)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
@@ -444,7 +455,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       mbar_init(TFULL(a), 1);
       mbar_init(TEMPTY(a), 4);
     }
-    for (int s = 0; s < SB; ++s) {
+    for (int s = 0; s < kTcMaxB; ++s) {  // every stage: the depth follows G, known once M is
       mbar_init(FULL_B(s), 1);
       mbar_init(EMPTY_B(s), 1);
     }
@@ -453,7 +464,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&tmem_slot), 2 * BN);
+    tmem_alloc(smem_u32(&tmem_slot), tcols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -462,10 +473,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   const uint32_t tmem = tmem_slot;
   volatile int *abort_v = &abort_flag;
   if (M <= 0) {  // nothing to multiply (uniform: every CTA of the launch leaves here, or none)
-    if (warp == 1) tmem_dealloc(tmem, 2 * BN);
+    if (warp == 1) tmem_dealloc(tmem, tcols);
     return;
   }
   const int passes = (M + BN - 1) / BN;
+  // G token passes per weight tile (a group); the fragment iterators walk groups
+  const int G = kSw ? min(passes, gmax) : 1;
+  const int ngroups = (passes + G - 1) / G, grows = G * BN;
+  const bool dbuf = 2u * (uint32_t)grows <= tcols;  // two accumulators alternate
+  const uint32_t x_stage = (uint32_t)G * b_stage;
+  const int SB = min(kTcMaxB, (int)(x_region / x_stage));
 
   if (warp == 0) {
     // weight producer: the weights are never written by a kernel, so the ring
@@ -478,7 +495,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       bool ok = true;
       for (int ph = 0; ph < p.nphase && ok; ++ph) {
         KCursor ca;
-        ca.start(p, ph == 0 ? it_first : frag_begin(p, ph), passes, BN);
+        ca.start(p, ph == 0 ? it_first : frag_begin(p, ph), ngroups, grows);
         while (ca.valid) {
           if (!wait_bounded(EMPTY_A(stage), phase ^ 1u, abort_v, p.status)) {
             ok = false;
@@ -488,7 +505,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           tma_load_2d(STAGE_A(stage), &p.ph[ph].a[ca.f.seg], ca.kb * 64, ca.f.arow, FULL_A(stage), pol_w);
           used |= 1u << stage;
           fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-          ca.advance(p, passes, BN);
+          ca.advance(p, ngroups, grows);
           if (++stage == SA) {
             stage = 0;
             phase ^= 1u;
@@ -519,7 +536,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     if (lane == 0) {
       const uint64_t pol_x = policy_evict_last();  // activations are re-read by every tile
       KCursor cb0;  // the first phase's cursor, ready before the wait
-      cb0.start(p, it_first, passes, BN);
+      cb0.start(p, it_first, ngroups, grows);
       griddep_wait();
       allow_dependents();  // the next kernel may be scheduled (it waits for this grid)
       uint32_t used = 0, fill_parity = 0;  // per stage bit: loaded at least once / parity of its last fill
@@ -536,7 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           fence_proxy_async_global();  // generic-proxy stores of other CTAs, read next by TMA
         }
         KCursor cb = cb0;
-        if (ph > 0) cb.start(p, frag_begin(p, ph), passes, BN);
+        if (ph > 0) cb.start(p, frag_begin(p, ph), ngroups, grows);
         while (cb.valid) {
           if (!wait_bounded(EMPTY_B(stage), phase ^ 1u, abort_v, p.status)) {
             ok = false;
@@ -545,11 +562,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           // the whole token pass in one box: TMA throughput is bound by the number
           // of copies, not their bytes (rows past the packed count are never read
           // by the MMA; rows past the buffer are zero-filled)
-          mbar_expect_tx(FULL_B(stage), b_bytes);
-          tma_load_2d(STAGE_B(stage), &p.ph[ph].b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
+          if (!kSw || G == 1) {
+            mbar_expect_tx(FULL_B(stage), b_bytes);
+            tma_load_2d(STAGE_B(stage), &p.ph[ph].b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
+          } else {  // one box per token pass of the group
+            const int npg = min(G, passes - cb.it.pass * G);
+            mbar_expect_tx(FULL_B(stage), (uint32_t)npg * b_bytes);
+            for (int q = 0; q < npg; ++q)
+              tma_load_2d(STAGE_B(stage) + (uint32_t)q * b_stage, &p.ph[ph].b, cb.kb * 64, cb.m0 + q * BN,
+                          FULL_B(stage), pol_x);
+          }
           used |= 1u << stage;
           fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-          cb.advance(p, passes, BN);
+          cb.advance(p, ngroups, grows);
           if (++stage == SB) {
             stage = 0;
             phase ^= 1u;
@@ -569,12 +594,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       for (int ph = 0; ph < p.nphase && ok; ++ph) {
         FragIter it = ph == 0 ? it_first : frag_begin(p, ph);
         Frag f;
-        while (ok && next_frag<false>(p, passes, it, f)) {
-          const int mrows = min(BN, M - it.pass * BN);
+        while (ok && next_frag<false>(p, ngroups, it, f)) {
+          const int mrows = min(BN, M - it.pass * grows);  // rows of the group's first pass
           const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
           const int lm_halves = mrows > 128 ? 2 : 1;
-          const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
-          const uint32_t dtm = tmem + acc * (uint32_t)BN;
+          const int npg = min(G, passes - it.pass * G);
+          const uint32_t acc = dbuf ? (nfrag & 1u) : 0u, use = dbuf ? nfrag >> 1 : nfrag;
+          const uint32_t dtm = tmem + acc * (uint32_t)grows;
           if (!wait_bounded(TEMPTY(acc), (use & 1u) ^ 1u, abort_v, p.status)) {
             ok = false;
             break;
@@ -603,6 +629,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
 #pragma unroll
               for (int k = 0; k < 4; ++k)  // 4 x K=16 (32 bytes) inside the 128-byte swizzle atom
                 tc_mma(dtm, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, (kb > f.kb0 || k > 0) ? 1u : 0u);
+              // the group's further passes: their boxes follow in the stage, their
+              // accumulators in TMEM
+              for (int q = 1; kSw && q < npg; ++q) {
+                const int mq = min(BN, M - it.pass * grows - q * BN);
+                const uint32_t idq = idesc_bf16(128, (mq + 15) & ~15);
+                const uint64_t bq = sw128_desc(STAGE_B(sb) + (uint32_t)q * b_stage);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                  tc_mma(dtm + (uint32_t)(q * BN), ad + (uint64_t)(2 * k), bq + (uint64_t)(2 * k), idq,
+                         (kb > f.kb0 || k > 0) ? 1u : 0u);
+              }
             }
             issued = true;
             tc_commit(EMPTY_A(sa));  // both stages are free once these MMAs have read them
@@ -653,11 +690,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
       const TcPhase &q = p.ph[ph];
       FragIter it = ph == 0 ? it_first : frag_begin(p, ph);
       Frag f;
-      while (next_frag<true>(p, passes, it, f)) {
-        const int m0 = it.pass * BN;
-        const int mrows = min(BN, M - m0);
-        const uint32_t acc = nfrag & 1u, use = nfrag >> 1;
-        const uint32_t tacc = tmem + acc * (uint32_t)BN + ((uint32_t)(q4 * 32) << 16);
+      while (next_frag<true>(p, ngroups, it, f)) {
+        const int mg = it.pass * grows;  // first row of the group
+        const uint32_t acc = dbuf ? (nfrag & 1u) : 0u, use = dbuf ? nfrag >> 1 : nfrag;
+        const uint32_t tacc = tmem + acc * (uint32_t)grows + ((uint32_t)(q4 * 32) << 16);
         bool okw = __all_sync(0xffffffffu, wait_bounded(TFULL(acc), use & 1u, abort_v, p.status));
         if (kChain) {
           // the 4 warps meet at named barriers below: they leave together or not at all
@@ -684,8 +720,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
             lm_flush(lm_pass);
             lm_pass = it.pass;
           }
+          const int mrows = min(BN, M - mg);
           for (int mt = 0; mt < (mrows > 128 ? 2 : 1); ++mt) {
-            const uint32_t tm = tmem + acc * (uint32_t)BN + (uint32_t)(mt * 128) + ((uint32_t)(q4 * 32) << 16);
+            const uint32_t tm = tmem + acc * (uint32_t)grows + (uint32_t)(mt * 128) + ((uint32_t)(q4 * 32) << 16);
             float &RM = lm_max[mt];
             double &RS = lm_sum[mt];
             int &RI = lm_arg[mt];
@@ -729,13 +766,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         }
         float *dst = p.out + (size_t)f.slot * (size_t)it.l.geo.slot_stride + col;
         const size_t ldc = (size_t)it.l.ldc;
-        for (int c = 0; c < mrows; c += 16) {
+        const int mend = min(M, mg + grows);  // the group's rows: [mg, mend), pass q at columns q * BN
+        for (int c = 0; c < mend - mg; c += 16) {
           float v[16];
           tmem_ld16(tacc + (uint32_t)c, v);
           if (col_ok) {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (c + j < mrows) dst[(size_t)(m0 + c + j) * ldc] = v[j];
+              if (mg + c + j < mend) dst[(size_t)(mg + c + j) * ldc] = v[j];
           }
         }
         tc_fence_before();
@@ -776,7 +814,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, tcols);
   }
 }
 
@@ -840,6 +878,7 @@ template <int BN>
 static cudaError_t launch_mode(const TcParams &p, int grid, cudaStream_t s) {
   if (p.chain) return launch_bn<BN, kChained>(p, grid, s);
   if (p.epi_mode == EPI_LMHEAD) return launch_bn<BN, kLmHead>(p, grid, s);
+  if (p.sweep > 1) return launch_bn<BN, kSweep>(p, grid, s);
   return launch_bn<BN, kPlain>(p, grid, s);
 }
 
@@ -860,6 +899,12 @@ cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
     const uint32_t need = 1024u + (b_stage > 16384u ? 3u : 4u) * b_stage + 4u * kTcABytes;
     if (p.smem_bytes == 0 || p.smem_bytes > (uint32_t)kTcSmem) p.smem_bytes = (uint32_t)kTcSmem;
     if (p.smem_bytes < need) p.smem_bytes = need;
+    // pass sweep: G passes' accumulators in 512 TMEM columns, and two stages of
+    // G activation boxes beside at least 4 weight tiles in shared memory
+    int g = (p.chain || p.epi_mode == EPI_LMHEAD) ? 0 : p.sweep;
+    if (g > 512 / bn) g = 512 / bn;
+    while (g > 1 && 1024u + 2u * (uint32_t)g * b_stage + 4u * kTcABytes > p.smem_bytes) --g;
+    p.sweep = g > 1 ? g : 0;
   }
   if (bn == 128) return launch_mode<128>(p, grid, s);
   if (bn == 256) return launch_mode<256>(p, grid, s);

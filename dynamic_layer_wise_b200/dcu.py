@@ -25,6 +25,7 @@ DCU_WINDOW_INCLUSIVE, DCU_WINDOW_HALFOPEN = 0, 1
  DCU_T_CONF, DCU_T_ARGMAX, DCU_T_ATTN, DCU_T_STALE, DCU_T_APD_TAU, DCU_T_APD_C, DCU_T_APD_H) = range(16)
 DCU_SELECT_INPUT, DCU_SELECT_VALUE = 0, 1
 DCU_OPT_FUSED_EPILOGUE, DCU_OPT_L2_PREFETCH, DCU_OPT_ATTENTION, DCU_OPT_GEMM_SMEM_KB = 1, 2, 3, 4
+DCU_OPT_GEMM_PASS_SWEEP = 5
 DCU_ATTN_TCGEN05, DCU_ATTN_MMA_SYNC = 0, 1
 (DCU_K_REFRESH, DCU_K_BUDGET, DCU_K_SELECT, DCU_K_GATHER, DCU_K_GEMM, DCU_K_EPILOGUE, DCU_K_ATTN, DCU_K_SCATTER,
  DCU_K_LMHEAD, DCU_K_COMMIT, DCU_K_COUNT) = range(11)

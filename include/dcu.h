@@ -167,6 +167,14 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
  *     for the CTAs of the small kernels before it, so the GEMM's CTAs become
  *     resident, and start streaming weights, while those still run. */
 #define DCU_OPT_GEMM_SMEM_KB 4
+/*   DCU_OPT_GEMM_PASS_SWEEP (0 or 1, default 1): a layer GEMM multiplies its
+ *     rows in token passes of 128 rows (small expected recompute sets) or 256
+ *     (larger ones, and the dense forward).  With 256-row passes and more than
+ *     one pass, 1 multiplies each weight tile held in shared memory by two
+ *     passes of activations, each into its own tensor-memory accumulator, so
+ *     the weights stream from HBM once per two passes; 0 streams them once per
+ *     pass.  Results are bit-identical either way. */
+#define DCU_OPT_GEMM_PASS_SWEEP 5
 #define DCU_ATTN_TCGEN05 0
 #define DCU_ATTN_MMA_SYNC 1
 int dcu_set_option(dcu_ctx *ctx, int32_t option, int32_t value);

@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("M,K,Nout", [(1, 64, 128), (17, 256, 1000), (65, 4096, 384), (128, 512, 256),
-                                      (130, 1024, 640), (300, 128, 200), (1024, 256, 128)])
+                                      (130, 1024, 640), (300, 128, 200), (1024, 256, 128),
+                                      (520, 192, 130), (777, 128, 384)])
 def test_linear_parity(dtype, M, K, Nout):
     """The recompute GEMM (tcgen05 for bf16) against an fp64 product of the same
     stored values; fp32 accumulation bounds the error by ~K * 2^-24 * sum|x||w|."""

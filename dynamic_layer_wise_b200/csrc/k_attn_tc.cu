@@ -7,20 +7,23 @@
 // TMEM lane.  The split's keys are walked in chunks of 128:
 //
 //   warp 0   TMA producer: K and V chunks (128 keys x hd, 128-byte swizzle)
-//            into a ring of stages
+//            into two rings (a K stage is free once S_j is computed, a V
+//            stage once P_j V_j is accumulated)
 //   warp 1   MMA issuer (one thread): S_j = Q K_j^T into one of two TMEM S
 //            buffers (M = 128 queries, N = 128 keys, K = hd), and
-//            O += P_j V_j (M = 128, N = hd, K = 128 keys; V is the B operand
-//            in MN-major form, straight from its TMA layout)
+//            O += P_j V_j (M = 128, N = hd, K = 128 keys) with P_j read from
+//            tensor memory and V the B operand in MN-major form, straight
+//            from its TMA layout
 //   warps 2-9  softmax, two warpgroups: thread = (query row, half of the
 //            chunk's keys); reads its half S row from TMEM, combines the row
 //            max with its partner thread, keeps the running max and its share
 //            of the sum (log2 domain), rescales its half of the O row in TMEM
-//            when the max grows, writes its half of P (bf16) into shared
-//            memory in the K-major 128-byte-swizzled operand layout, and
-//            finally stores its half of O
+//            when the max grows, writes its half of P (bf16 pairs) over the
+//            chunk's own S columns, and finally stores its half of O
 //
-// S_{j+1} is computed while the softmax of chunk j runs.  With one key split
+// S_{j+1} is computed while the softmax of chunk j runs, and P_j lives in
+// S_j's buffer, so the softmax of chunk j + 1 does not wait for P_j V_j
+// unless the running max moved and O must be rescaled.  With one key split
 // the CTA normalises and stores bf16 rows.  With several, the splits of one
 // (sequence, kv head, query tile) run as one thread-block cluster: each CTA
 // stages its (O, max, sum) rows in its own shared memory and, after a cluster
@@ -43,11 +46,12 @@ template <int HD>
 struct TcAttnCfg {
   static constexpr uint32_t kQBytes = (uint32_t)kQT * HD * 2;      // Q tile, HD / 64 swizzle blocks of 16 KB
   static constexpr uint32_t kKVBytes = (uint32_t)kKC * HD * 2;     // K (or V) of one chunk
-  static constexpr uint32_t kStage = 2 * kKVBytes;                 // K then V
-  static constexpr int kStages = HD == 128 ? 2 : 4;                // K / V ring depth
-  static constexpr uint32_t kPBytes = (uint32_t)kQT * kKC * 2;     // P tile, 2 swizzle blocks of 16 KB
-  static constexpr uint32_t kSmem = kQBytes + kStages * kStage + kPBytes + 1024;  // + alignment slack
-  static constexpr uint32_t kTmemCols = 512;  // S buffers [0, 128), [128, 256); O [256, 256 + HD)
+  static constexpr int kKStages = HD == 128 ? 3 : 4;               // K ring depth
+  static constexpr int kVStages = HD == 128 ? 2 : 4;               // V ring depth
+  static constexpr uint32_t kSmem = kQBytes + (kKStages + kVStages) * kKVBytes + 1024;  // + alignment slack
+  // S / P buffers [0, 128), [128, 256) (P_j as bf16 pairs in the first 64
+  // columns of S_j's buffer); O [256, 256 + HD)
+  static constexpr uint32_t kTmemCols = 512;
 };
 
 struct TcAttnArgs {
@@ -124,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
   using C = TcAttnCfg<HD>;
   constexpr uint32_t kStagePitch = (uint32_t)HD * 4u + 16u;  // staged O row (fp32), padded against bank conflicts
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[2 * 4 + 2 + 2 + 1 + 1 + 1 + 1];
+  __shared__ __align__(8) uint64_t bars[4 * 4 + 2 + 1 + 1 + 1 + 1];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ float s_w[kQT][8];     // split weights of the merge
@@ -150,25 +154,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
   const int nch = (k_end - k_begin + kKC - 1) / kKC;
 
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t q_s = sbase, kv_s = sbase + C::kQBytes, p_s = kv_s + (uint32_t)C::kStages * C::kStage;
+  // kv_s: the K ring, then the V ring (after the last chunk of a tile, the
+  // staging area of the cluster merge)
+  const uint32_t q_s = sbase, kv_s = sbase + C::kQBytes, v_s = kv_s + (uint32_t)C::kKStages * C::kKVBytes;
   const uint32_t bar0 = smem_u32(bars);
-#define KV_FULL(s) (bar0 + 8u * (uint32_t)(s))
-#define KV_EMPTY(s) (bar0 + 8u * (uint32_t)(4 + (s)))
-#define S_FULL(i) (bar0 + 8u * (uint32_t)(8 + (i)))
-#define S_FREE(i) (bar0 + 8u * (uint32_t)(10 + (i)))
-  const uint32_t P_FULL = bar0 + 8u * 12u, O_DONE = bar0 + 8u * 13u, DRAIN = bar0 + 8u * 14u,
-                 Q_FULL = bar0 + 8u * 15u;
+#define K_FULL(s) (bar0 + 8u * (uint32_t)(s))
+#define K_EMPTY(s) (bar0 + 8u * (uint32_t)(4 + (s)))
+#define V_FULL(s) (bar0 + 8u * (uint32_t)(8 + (s)))
+#define V_EMPTY(s) (bar0 + 8u * (uint32_t)(12 + (s)))
+#define S_FULL(i) (bar0 + 8u * (uint32_t)(16 + (i)))
+  const uint32_t P_FULL = bar0 + 8u * 18u, O_DONE = bar0 + 8u * 19u, DRAIN = bar0 + 8u * 20u,
+                 Q_FULL = bar0 + 8u * 21u;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(KV_FULL(s), 1);
-      mbar_init(KV_EMPTY(s), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(K_FULL(s), 1);
+      mbar_init(K_EMPTY(s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(S_FULL(i), 1);
-      mbar_init(S_FREE(i), 8);  // one arrive per softmax warp
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(V_FULL(s), 1);
+      mbar_init(V_EMPTY(s), 1);
     }
-    mbar_init(P_FULL, 8);
+    for (int i = 0; i < 2; ++i) mbar_init(S_FULL(i), 1);
+    mbar_init(P_FULL, 8);  // one arrive per softmax warp
     mbar_init(O_DONE, 1);
     mbar_init(DRAIN, 1);
     mbar_init(Q_FULL, 8);  // one arrive per softmax warp
@@ -219,28 +227,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
       // ---- TMA producer
       if (lane == 0) {
         bool ok = true;
-        uint32_t issued = 0;
+        uint32_t issued_k = 0, issued_v = 0;
         const uint64_t pol = policy_evict_normal();
         for (int j = 0; j < nch; ++j) {
-          const uint32_t g = cbase + (uint32_t)j, st = g % C::kStages, use = g / C::kStages;
-          if (!wait_bounded(KV_EMPTY(st), (use & 1u) ^ 1u, abort_v, a.status)) {
+          const uint32_t g = cbase + (uint32_t)j;
+          const uint32_t ks = g % C::kKStages, vs = g % C::kVStages;
+          const int y = rowbase + k_begin + j * kKC;  // rows past the split are masked, past the tensor zero
+          if (!wait_bounded(K_EMPTY(ks), ((g / C::kKStages) & 1u) ^ 1u, abort_v, a.status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(KV_FULL(st), C::kStage);
-          const uint32_t dst = kv_s + st * C::kStage;
-          const int y = rowbase + k_begin + j * kKC;  // rows past the split are masked, past the tensor zero
+          mbar_expect_tx(K_FULL(ks), C::kKVBytes);
 #pragma unroll
-          for (int h = 0; h < HD / 64; ++h) {
-            tma_load_2d(dst + (uint32_t)h * 16384u, &a.kmap, h * 64, y, KV_FULL(st), pol);
-            tma_load_2d(dst + C::kKVBytes + (uint32_t)h * 16384u, &a.vmap, h * 64, y, KV_FULL(st), pol);
+          for (int h = 0; h < HD / 64; ++h)
+            tma_load_2d(kv_s + ks * C::kKVBytes + (uint32_t)h * 16384u, &a.kmap, h * 64, y, K_FULL(ks), pol);
+          ++issued_k;
+          if (!wait_bounded(V_EMPTY(vs), ((g / C::kVStages) & 1u) ^ 1u, abort_v, a.status)) {
+            ok = false;
+            break;
           }
-          ++issued;
+          mbar_expect_tx(V_FULL(vs), C::kKVBytes);
+#pragma unroll
+          for (int h = 0; h < HD / 64; ++h)
+            tma_load_2d(v_s + vs * C::kKVBytes + (uint32_t)h * 16384u, &a.vmap, h * 64, y, V_FULL(vs), pol);
+          ++issued_v;
         }
         if (!ok) {  // wait, bounded, for the copies this tile still has in flight
-          for (uint32_t j = 0; j < issued; ++j) {
+          for (uint32_t j = 0; j < issued_k; ++j) {
             const uint32_t g = cbase + j;
-            wait_drain(KV_FULL(g % C::kStages), (g / C::kStages) & 1u);
+            wait_drain(K_FULL(g % C::kKStages), (g / C::kKStages) & 1u);
+          }
+          for (uint32_t j = 0; j < issued_v; ++j) {
+            const uint32_t g = cbase + j;
+            wait_drain(V_FULL(g % C::kVStages), (g / C::kVStages) & 1u);
           }
         }
       }
@@ -251,32 +270,37 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const uint32_t idesc_o = idesc_bf16_bmn(kQT, HD);
         const uint32_t o_tm = tmem + 256u;
         bool ok = true, any = false;
+        // P_i from TMEM (S_i's buffer, 16 keys = 8 columns per K step), V_i from
+        // its stage.  The tensor core runs one thread's MMAs in issue order, so
+        // S_{i+2}, issued after this, overwrites P_i only once it has been read.
         auto issue_pv = [&](int i) -> bool {
-          const uint32_t g = cbase + (uint32_t)i, st = g % C::kStages;
-          if (!wait_bounded(P_FULL, g & 1u, abort_v, a.status)) return false;
+          const uint32_t g = cbase + (uint32_t)i, vs = g % C::kVStages;
+          if (!wait_bounded(P_FULL, g & 1u, abort_v, a.status) ||
+              !wait_bounded(V_FULL(vs), (g / C::kVStages) & 1u, abort_v, a.status))
+            return false;
           tc_fence_after();
-          const uint32_t vb = kv_s + st * C::kStage + C::kKVBytes;
+          const uint32_t vb = v_s + vs * C::kKVBytes, p_tm = tmem + (g & 1u) * (uint32_t)kKC;
 #pragma unroll
           for (int kk = 0; kk < kKC / 16; ++kk) {
-            const uint64_t pd = sw128_desc(p_s + (uint32_t)(kk >> 2) * 16384u) + (uint64_t)(2 * (kk & 3));
             const uint64_t vd = sw128_mn_desc(vb + (uint32_t)kk * 2048u, 16384u);
-            tc_mma(o_tm, pd, vd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(o_tm, p_tm + (uint32_t)(kk * 8), vd, idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
           }
-          tc_commit(KV_EMPTY(st));  // the stage may be refilled once these MMAs have read it
+          tc_commit(V_EMPTY(vs));  // the stage may be refilled once these MMAs have read it
           tc_commit(O_DONE);
           return true;
         };
         if (!wait_bounded(Q_FULL, ntile & 1u, abort_v, a.status)) ok = false;
         tc_fence_after();
+        // S_j's buffer was last read as P_{j-2}, whose MMAs were issued before
+        // these (after the softmax had finished with S_{j-2}: P_FULL)
         for (int j = 0; j < nch && ok; ++j) {
-          const uint32_t g = cbase + (uint32_t)j, st = g % C::kStages, sb = g & 1u;
-          if (!wait_bounded(KV_FULL(st), (g / C::kStages) & 1u, abort_v, a.status) ||
-              !wait_bounded(S_FREE(sb), ((g >> 1) & 1u) ^ 1u, abort_v, a.status)) {
+          const uint32_t g = cbase + (uint32_t)j, ks = g % C::kKStages, sb = g & 1u;
+          if (!wait_bounded(K_FULL(ks), (g / C::kKStages) & 1u, abort_v, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t kb = kv_s + st * C::kStage;
+          const uint32_t kb = kv_s + ks * C::kKVBytes;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             const uint64_t qd = sw128_desc(q_s + (uint32_t)(kk >> 2) * 16384u) + (uint64_t)(2 * (kk & 3));
@@ -284,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             tc_mma(tmem + sb * (uint32_t)kKC, qd, kd, idesc_s, kk > 0 ? 1u : 0u);
           }
           any = true;
+          tc_commit(K_EMPTY(ks));
           tc_commit(S_FULL(sb));
           if (j >= 1 && !issue_pv(j - 1)) ok = false;
         }
@@ -358,7 +383,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         // raw S here; the scale (> 0) commutes with the max and enters the exponent below
         float mc = sc * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         s_mx[j & 1][hf][qi] = mc;
+        // (the barrier also orders both halves' S loads before the P stores
+        // below, which overwrite the first 64 columns of S_j)
+        tc_fence_before();
         pair_sync();
+        tc_fence_after();
         mc = fmaxf(mc, s_mx[j & 1][hf ^ 1][qi]);  // the row's chunk max (identical in both halves)
         if (!alive) continue;
         // The running max only moves when the chunk's max exceeds it by more than
@@ -367,12 +396,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const bool grow = mc > m_run + 8.f;  // always on the first chunk (m_run = -inf)
         const float m_new = grow ? mc : m_run;
         const float alpha = grow ? (m_run == -INFINITY ? 0.f : ex2_approx(m_run - m_new)) : 1.f;
-        // P_{j-1} V_{j-1} must be complete before P is overwritten and O rescaled
-        if (j >= 1) {
+        // a rescale of O needs P_{j-1} V_{j-1} accumulated first (P_j has a
+        // buffer of its own, so otherwise nothing waits for it).  P_j V_j cannot
+        // complete before this warp's P_FULL arrival below, so the barrier is at
+        // most one phase ahead and the parity wait is exact.
+        if (j >= 1 && __any_sync(0xffffffffu, grow)) {  // warp-uniform: tcgen05.ld / st are collective
           alive = __all_sync(0xffffffffu, wait_bounded(O_DONE, (g - 1u) & 1u, abort_v, a.status));
           if (!alive) continue;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, grow)) {  // warp-uniform: tcgen05.ld / st are collective
+          {
 #pragma unroll
             for (int c = 0; c < HD / 64; ++c) {  // this half's HD / 2 columns, 32 at a time
               uint32_t orr[32];
@@ -386,29 +418,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
           }
         }
         m_run = m_new;
-        // P = 2^(s - m) of this half's valid keys (0 past them); the half's 64
-        // keys are exactly one 128-byte swizzle block of the P tile
+        // P = 2^(s - m) of this half's valid keys (0 past them), as bf16 pairs:
+        // keys 64 hf + 2c, 64 hf + 2c + 1 in column 32 hf + c of S_j's buffer
+        // (the K-major A operand of P_j V_j in tensor memory)
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t pk[4];
+        for (int h = 0; h < 2; ++h) {  // 16 columns at a time
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float p0 = ex2_approx(fmaf(sv[8 * c + 2 * e], sc, -m_new));
-            const float p1 = ex2_approx(fmaf(sv[8 * c + 2 * e + 1], sc, -m_new));
-            ps[e] += p0 + p1;
-            pk[e] = pack2_bf16(p0, p1);
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ex2_approx(fmaf(sv[32 * h + 2 * c], sc, -m_new));
+            const float p1 = ex2_approx(fmaf(sv[32 * h + 2 * c + 1], sc, -m_new));
+            ps[c & 3] += p0 + p1;
+            pk[c] = pack2_bf16(p0, p1);
           }
-          st_shared_v4(p_s + sw128_off(qi, hf * 8 + c), pk[0], pk[1], pk[2], pk[3]);
+          tmem_st16u(tmem + sb * (uint32_t)kKC + lane_off + (uint32_t)(hf * 32 + h * 16), pk);
         }
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-        fence_proxy_async_smem();  // P is read by the MMA through the async proxy
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(S_FREE(sb));  // the S buffer may take S_{j+2}
-          mbar_arrive(P_FULL);
-        }
+        if (lane == 0) mbar_arrive(P_FULL);
       }
       if (alive) {
         const uint32_t g = cbase + (uint32_t)(nch - 1);
@@ -514,10 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     cbase += (uint32_t)nch;
     __syncthreads();  // the next tile reuses Q, P, the TMEM buffers and the merge weights
   }
-#undef KV_FULL
-#undef KV_EMPTY
+#undef K_FULL
+#undef K_EMPTY
+#undef V_FULL
+#undef V_EMPTY
 #undef S_FULL
-#undef S_FREE
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();

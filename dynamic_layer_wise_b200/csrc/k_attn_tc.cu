@@ -18,11 +18,11 @@
 //            chunk's keys); reads its half S row from TMEM, combines the row
 //            max with its partner thread, keeps the running max and its share
 //            of the sum (log2 domain), rescales its half of the O row in TMEM
-//            when the max grows, writes its half of P (bf16 pairs) over the
-//            chunk's own S columns, and finally stores its half of O
+//            when the max grows, writes its half of P (bf16 pairs) into one
+//            of two TMEM P buffers, and finally stores its half of O
 //
-// S_{j+1} is computed while the softmax of chunk j runs, and P_j lives in
-// S_j's buffer, so the softmax of chunk j + 1 does not wait for P_j V_j
+// S_{j+1} is computed while the softmax of chunk j runs, and P_j has a TMEM
+// buffer of its own, so the softmax of chunk j + 1 does not wait for P_j V_j
 // unless the running max moved and O must be rescaled.  With one key split
 // the CTA normalises and stores bf16 rows.  With several, the splits of one
 // (sequence, kv head, query tile) run as one thread-block cluster: each CTA
@@ -49,9 +49,11 @@ struct TcAttnCfg {
   static constexpr int kKStages = HD == 128 ? 3 : 4;               // K ring depth
   static constexpr int kVStages = HD == 128 ? 2 : 4;               // V ring depth
   static constexpr uint32_t kSmem = kQBytes + (kKStages + kVStages) * kKVBytes + 1024;  // + alignment slack
-  // S / P buffers [0, 128), [128, 256) (P_j as bf16 pairs in the first 64
-  // columns of S_j's buffer); O [256, 256 + HD)
+  // S buffers [0, 128), [128, 256); O [256, 256 + HD); P buffers (128 keys
+  // as bf16 pairs) [384, 448), [448, 512)
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kPCol = 384;
+  static_assert(256 + HD <= kPCol, "O and the P buffers overlap");
 };
 
 struct TcAttnArgs {
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
   using C = TcAttnCfg<HD>;
   constexpr uint32_t kStagePitch = (uint32_t)HD * 4u + 16u;  // staged O row (fp32), padded against bank conflicts
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bars[4 * 4 + 2 + 1 + 1 + 1 + 1];
+  __shared__ __align__(8) uint64_t bars[4 * 4 + 2 + 2 + 1 + 1 + 1 + 1];
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   __shared__ float s_w[kQT][8];     // split weights of the merge
@@ -163,8 +165,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
 #define V_FULL(s) (bar0 + 8u * (uint32_t)(8 + (s)))
 #define V_EMPTY(s) (bar0 + 8u * (uint32_t)(12 + (s)))
 #define S_FULL(i) (bar0 + 8u * (uint32_t)(16 + (i)))
-  const uint32_t P_FULL = bar0 + 8u * 18u, O_DONE = bar0 + 8u * 19u, DRAIN = bar0 + 8u * 20u,
-                 Q_FULL = bar0 + 8u * 21u;
+  // P_FULL per S / P buffer: the softmax warps are not in step with one
+  // another (only the two of a row pair are), and a warp may finish P_{j+1}
+  // before a slower one finishes P_j; with one barrier for both, such early
+  // arrivals would count towards chunk j's phase.  A warp reaches P_{j+2}
+  // only after every warp's P_j (S_{j+2} follows P_j V_j), so per buffer the
+  // phases stay in order.
+#define P_FULL(i) (bar0 + 8u * (uint32_t)(18 + (i)))
+  // O_DONE: once per chunk, after P_j V_j (the rescale waits); O_FINAL: once
+  // per query tile, after its last P V.  The softmax skips O_DONE phases, so
+  // its wait for the tile's last chunk could alias an older phase; O_FINAL
+  // cannot.
+  const uint32_t O_DONE = bar0 + 8u * 20u, DRAIN = bar0 + 8u * 21u, Q_FULL = bar0 + 8u * 22u,
+                 O_FINAL = bar0 + 8u * 23u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kKStages; ++s) {
@@ -175,9 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
       mbar_init(V_FULL(s), 1);
       mbar_init(V_EMPTY(s), 1);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(S_FULL(i), 1);
-    mbar_init(P_FULL, 8);  // one arrive per softmax warp
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(S_FULL(i), 1);
+      mbar_init(P_FULL(i), 8);  // one arrive per softmax warp
+    }
     mbar_init(O_DONE, 1);
+    mbar_init(O_FINAL, 1);
     mbar_init(DRAIN, 1);
     mbar_init(Q_FULL, 8);  // one arrive per softmax warp
     abort_flag = 0;
@@ -224,42 +240,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     // the tiles, every wait now failing at once, so their cluster barriers match
     if (a.splits == 1 && *abort_v) break;
     if (warp == 0) {
-      // ---- TMA producer
-      if (lane == 0) {
+      // ---- TMA producers: lane 0 fills the K ring, lane 1 the V ring, so a K
+      // load never queues behind a V stage still held by P V
+      if (lane < 2) {
+        const bool is_v = lane == 1;
+        const uint32_t stages = is_v ? (uint32_t)C::kVStages : (uint32_t)C::kKStages;
+        const uint32_t ring = is_v ? v_s : kv_s;
+        const uint32_t full0 = is_v ? V_FULL(0) : K_FULL(0), empty0 = is_v ? V_EMPTY(0) : K_EMPTY(0);
+        const CUtensorMap *map = is_v ? &a.vmap : &a.kmap;
         bool ok = true;
-        uint32_t issued_k = 0, issued_v = 0;
+        uint32_t issued = 0;
         const uint64_t pol = policy_evict_normal();
         for (int j = 0; j < nch; ++j) {
-          const uint32_t g = cbase + (uint32_t)j;
-          const uint32_t ks = g % C::kKStages, vs = g % C::kVStages;
+          const uint32_t g = cbase + (uint32_t)j, st = g % stages;
           const int y = rowbase + k_begin + j * kKC;  // rows past the split are masked, past the tensor zero
-          if (!wait_bounded(K_EMPTY(ks), ((g / C::kKStages) & 1u) ^ 1u, abort_v, a.status)) {
+          if (!wait_bounded(empty0 + 8u * st, ((g / stages) & 1u) ^ 1u, abort_v, a.status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(K_FULL(ks), C::kKVBytes);
+          mbar_expect_tx(full0 + 8u * st, C::kKVBytes);
 #pragma unroll
           for (int h = 0; h < HD / 64; ++h)
-            tma_load_2d(kv_s + ks * C::kKVBytes + (uint32_t)h * 16384u, &a.kmap, h * 64, y, K_FULL(ks), pol);
-          ++issued_k;
-          if (!wait_bounded(V_EMPTY(vs), ((g / C::kVStages) & 1u) ^ 1u, abort_v, a.status)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(V_FULL(vs), C::kKVBytes);
-#pragma unroll
-          for (int h = 0; h < HD / 64; ++h)
-            tma_load_2d(v_s + vs * C::kKVBytes + (uint32_t)h * 16384u, &a.vmap, h * 64, y, V_FULL(vs), pol);
-          ++issued_v;
+            tma_load_2d(ring + st * C::kKVBytes + (uint32_t)h * 16384u, map, h * 64, y, full0 + 8u * st, pol);
+          ++issued;
         }
         if (!ok) {  // wait, bounded, for the copies this tile still has in flight
-          for (uint32_t j = 0; j < issued_k; ++j) {
+          for (uint32_t j = 0; j < issued; ++j) {
             const uint32_t g = cbase + j;
-            wait_drain(K_FULL(g % C::kKStages), (g / C::kKStages) & 1u);
-          }
-          for (uint32_t j = 0; j < issued_v; ++j) {
-            const uint32_t g = cbase + j;
-            wait_drain(V_FULL(g % C::kVStages), (g / C::kVStages) & 1u);
+            wait_drain(full0 + 8u * (g % stages), (g / stages) & 1u);
           }
         }
       }
@@ -270,16 +278,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const uint32_t idesc_o = idesc_bf16_bmn(kQT, HD);
         const uint32_t o_tm = tmem + 256u;
         bool ok = true, any = false;
-        // P_i from TMEM (S_i's buffer, 16 keys = 8 columns per K step), V_i from
-        // its stage.  The tensor core runs one thread's MMAs in issue order, so
-        // S_{i+2}, issued after this, overwrites P_i only once it has been read.
+        // P_i from its TMEM buffer (16 keys = 8 columns per K step), V_i from its
+        // stage.  The softmax writes P_{i+2} into the same buffer only after
+        // S_{i+2}, whose commit follows the completion of these MMAs.
         auto issue_pv = [&](int i) -> bool {
           const uint32_t g = cbase + (uint32_t)i, vs = g % C::kVStages;
-          if (!wait_bounded(P_FULL, g & 1u, abort_v, a.status) ||
+          if (!wait_bounded(P_FULL(g & 1u), (g >> 1) & 1u, abort_v, a.status) ||
               !wait_bounded(V_FULL(vs), (g / C::kVStages) & 1u, abort_v, a.status))
             return false;
           tc_fence_after();
-          const uint32_t vb = v_s + vs * C::kKVBytes, p_tm = tmem + (g & 1u) * (uint32_t)kKC;
+          const uint32_t vb = v_s + vs * C::kKVBytes, p_tm = tmem + C::kPCol + (g & 1u) * 64u;
 #pragma unroll
           for (int kk = 0; kk < kKC / 16; ++kk) {
             const uint64_t vd = sw128_mn_desc(vb + (uint32_t)kk * 2048u, 16384u);
@@ -291,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         };
         if (!wait_bounded(Q_FULL, ntile & 1u, abort_v, a.status)) ok = false;
         tc_fence_after();
-        // S_j's buffer was last read as P_{j-2}, whose MMAs were issued before
-        // these (after the softmax had finished with S_{j-2}: P_FULL)
+        // S_j's buffer was last read by the softmax of chunk j - 2, which had
+        // finished (P_FULL) before P_{j-2} V_{j-2}, issued before these
         for (int j = 0; j < nch && ok; ++j) {
           const uint32_t g = cbase + (uint32_t)j, ks = g % C::kKStages, sb = g & 1u;
           if (!wait_bounded(K_FULL(ks), (g / C::kKStages) & 1u, abort_v, a.status)) {
@@ -313,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
           if (j >= 1 && !issue_pv(j - 1)) ok = false;
         }
         if (ok && !issue_pv(nch - 1)) ok = false;
+        if (ok) tc_commit(O_FINAL);  // every P V of the tile is accumulated
         if (!ok && any) {
           tc_commit(DRAIN);
           wait_drain(DRAIN, 0);
@@ -383,11 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         // raw S here; the scale (> 0) commutes with the max and enters the exponent below
         float mc = sc * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         s_mx[j & 1][hf][qi] = mc;
-        // (the barrier also orders both halves' S loads before the P stores
-        // below, which overwrite the first 64 columns of S_j)
-        tc_fence_before();
         pair_sync();
-        tc_fence_after();
         mc = fmaxf(mc, s_mx[j & 1][hf ^ 1][qi]);  // the row's chunk max (identical in both halves)
         if (!alive) continue;
         // The running max only moves when the chunk's max exceeds it by more than
@@ -397,9 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const float m_new = grow ? mc : m_run;
         const float alpha = grow ? (m_run == -INFINITY ? 0.f : ex2_approx(m_run - m_new)) : 1.f;
         // a rescale of O needs P_{j-1} V_{j-1} accumulated first (P_j has a
-        // buffer of its own, so otherwise nothing waits for it).  P_j V_j cannot
-        // complete before this warp's P_FULL arrival below, so the barrier is at
-        // most one phase ahead and the parity wait is exact.
+        // buffer of its own, so otherwise nothing waits for it).  The parity
+        // wait is exact: P_j V_j cannot complete before this warp's P_FULL
+        // arrival below, and S_j (seen above) completed after P_{j-2} V_{j-2},
+        // issued before it, so O_DONE has completed chunk j - 2 or j - 1.
         if (j >= 1 && __any_sync(0xffffffffu, grow)) {  // warp-uniform: tcgen05.ld / st are collective
           alive = __all_sync(0xffffffffu, wait_bounded(O_DONE, (g - 1u) & 1u, abort_v, a.status));
           if (!alive) continue;
@@ -419,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         }
         m_run = m_new;
         // P = 2^(s - m) of this half's valid keys (0 past them), as bf16 pairs:
-        // keys 64 hf + 2c, 64 hf + 2c + 1 in column 32 hf + c of S_j's buffer
+        // keys 64 hf + 2c, 64 hf + 2c + 1 in column 32 hf + c of P buffer j % 2
         // (the K-major A operand of P_j V_j in tensor memory)
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -432,18 +438,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             ps[c & 3] += p0 + p1;
             pk[c] = pack2_bf16(p0, p1);
           }
-          tmem_st16u(tmem + sb * (uint32_t)kKC + lane_off + (uint32_t)(hf * 32 + h * 16), pk);
+          tmem_st16u(tmem + C::kPCol + sb * 64u + lane_off + (uint32_t)(hf * 32 + h * 16), pk);
         }
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(P_FULL);
+        if (lane == 0) mbar_arrive(P_FULL(sb));
       }
-      if (alive) {
-        const uint32_t g = cbase + (uint32_t)(nch - 1);
-        alive = __all_sync(0xffffffffu, wait_bounded(O_DONE, g & 1u, abort_v, a.status));
-      }
+      if (alive) alive = __all_sync(0xffffffffu, wait_bounded(O_FINAL, ntile & 1u, abort_v, a.status));
       // the row sum: this half's share plus the partner's, in half order
       s_l[hf][qi] = l_run;
       pair_sync();
@@ -549,6 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
 #undef V_FULL
 #undef V_EMPTY
 #undef S_FULL
+#undef P_FULL
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();

@@ -88,3 +88,48 @@ def test_long_sequence_multichunk_attention_teacher_forced(B_layer, B_window, fu
                                  attn_gpu=attn if l == L - 1 else None, label=f"step {step} layer {l}")
         s_prev = s_g[0].copy()
     ctx.close()
+
+
+@pytest.mark.parametrize("attn", ["tcgen05", "mma_sync"])
+def test_query_tiles_beyond_the_expected_set_teacher_forced(attn):
+    """Many unmasked keys with wide windows and a small budget: each sequence
+    recomputes ~250 rows (~500 queries per kv head) while the launch geometry
+    is sized for the expected ~25 rows, so every attention CTA walks several
+    128-query tiles in turn (and, with 8 key splits, merges each tile in its
+    cluster).  Teacher-forced against the oracle, attention output included."""
+    shape, seed, n_prompt, n_gen, B = LONG_BF16, 11, 1536, 512, 2
+    N, L, H, hd = n_prompt + n_gen, shape.n_layers, shape.n_heads, shape.head_dim
+    B_layer, B_window, n_keys = 8, 16, 24
+    cfg_o = oracle_cfg(shape)
+    w_o = oracle_weights(shape, seed)
+    W = I.device_weights(shape, seed)
+    ctx = dcu.dcu_create(W, I.cfg_dict(shape, B, N))
+    dcu.dcu_set_option(ctx, dcu.DCU_OPT_ATTENTION,
+                       dcu.DCU_ATTN_TCGEN05 if attn == "tcgen05" else dcu.DCU_ATTN_MMA_SYNC)
+    ids = np.stack([I.sequence_ids(seed, b, n_prompt, n_gen, shape.vocab) for b in range(B)])
+    t_ids = torch.tensor(ids, dtype=torch.int32).cuda()
+    dcu.dcu_full_forward(ctx, t_ids)
+    assert dcu.dcu_status(ctx) == 0
+    keys = []
+    kp = np.zeros((B, N), np.int32)
+    for b in range(B):
+        pos, new = I.unmask_draw(seed + 1, b, np.arange(n_prompt, N), n_keys, shape.vocab)
+        ids[b, pos] = new
+        keys.append(list(pos))
+        kp[b, :n_keys] = pos
+    before = _snapshot(ctx, L)
+    t_ids.copy_(torch.tensor(ids, dtype=torch.int32))
+    dcu.dcu_step(ctx, t_ids, torch.tensor(kp).cuda(), torch.full((B,), n_keys, dtype=torch.int32).cuda(), B_layer,
+                 B_window)
+    assert dcu.dcu_status(ctx) == 0
+    after = _snapshot(ctx, L)
+    cnt = dcu.dcu_get_tensor(ctx, dcu.DCU_T_SEL_COUNT, 0).cpu().numpy()
+    assert int(cnt.min()) > 150, cnt  # >= 3 query tiles per (sequence, kv head)
+    bud = dcu.dcu_get_tensor(ctx, dcu.DCU_T_BUDGET).cpu().numpy().reshape(B, L)
+    s_g = dcu.dcu_get_tensor(ctx, dcu.DCU_T_S).cpu().numpy().reshape(B, L)
+    attn_out = to_np(dcu.dcu_get_tensor(ctx, dcu.DCU_T_ATTN)).reshape(B * N, H * hd)
+    for l in range(L):
+        snap = LayerSnap(before, after, ctx, l, B, N, shape, dcu)
+        teacher_forced_layer(snap, w_o.layers[l], cfg_o, s_g[:, l], bud[:, l], keys, B_window, 0, 2e-2,
+                             attn_gpu=attn_out if l == L - 1 else None, label=f"layer {l}")
+    ctx.close()

@@ -14,12 +14,13 @@
 //            O += P_j V_j (M = 128, N = hd, K = 128 keys) with P_j read from
 //            tensor memory and V the B operand in MN-major form, straight
 //            from its TMA layout
-//   warps 2-9  softmax, two warpgroups: thread = (query row, half of the
-//            chunk's keys); reads its half S row from TMEM, combines the row
-//            max with its partner thread, keeps the running max and its share
-//            of the sum (log2 domain), rescales its half of the O row in TMEM
-//            when the max grows, writes its half of P (bf16 pairs) into one
-//            of two TMEM P buffers, and finally stores its half of O
+//   warps 2-17 softmax, four warpgroups: thread = (query row, one of four
+//            32-key parts of the chunk); reads its part of the S row from
+//            TMEM, combines the row max with the other parts' threads, keeps
+//            the running max and its share of the sum (log2 domain), rescales
+//            its quarter of the O row in TMEM when the max grows, writes its
+//            part of P (bf16 pairs) into one of two TMEM P buffers, and
+//            finally stores its quarter of O
 //
 // S_{j+1} is computed while the softmax of chunk j runs, and P_j has a TMEM
 // buffer of its own, so the softmax of chunk j + 1 does not wait for P_j V_j
@@ -40,7 +41,10 @@ namespace {
 
 constexpr int kQT = 128;      // queries per tile (TMEM lanes)
 constexpr int kKC = 128;      // keys per chunk (S columns)
-constexpr int kThreads = 320;  // 10 warps: TMA, MMA, 8 softmax (two warpgroups)
+constexpr int kParts = 4;                     // softmax warpgroups: key parts of a chunk
+constexpr int kPartKeys = kKC / kParts;        // keys of a part (32)
+constexpr int kSoftThreads = 128 * kParts;     // softmax threads
+constexpr int kThreads = 64 + kSoftThreads;   // warps: TMA, MMA, 4 x kParts softmax
 
 template <int HD>
 struct TcAttnCfg {
@@ -135,8 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
   __shared__ int abort_flag;
   __shared__ float s_w[kQT][8];     // split weights of the merge
   __shared__ float2 s_ml[kQT];      // this split's (max, sum) per query row
-  __shared__ float s_mx[2][2][kQT];  // [chunk parity][half] chunk max per row (softmax pair exchange)
-  __shared__ float s_l[2][kQT];      // [half] share of the row sum
+  __shared__ float s_mx[2][kParts][kQT];  // [chunk parity][part] chunk max per row (row-group exchange)
+  __shared__ float s_l[kParts][kQT];      // [part] share of the row sum
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int item = blockIdx.x;
@@ -190,12 +194,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(S_FULL(i), 1);
-      mbar_init(P_FULL(i), 8);  // one arrive per softmax warp
+      mbar_init(P_FULL(i), kSoftThreads / 32);  // one arrive per softmax warp
     }
     mbar_init(O_DONE, 1);
     mbar_init(O_FINAL, 1);
     mbar_init(DRAIN, 1);
-    mbar_init(Q_FULL, 8);  // one arrive per softmax warp
+    mbar_init(Q_FULL, kSoftThreads / 32);  // one arrive per softmax warp
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -328,22 +332,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         }
       }
     } else {
-      // ---- softmax: two warpgroups; thread = (query row = TMEM lane, half of
-      // the key columns).  Warps 2-5 take keys [0, 64) of every chunk, warps
-      // 6-9 keys [64, 128); warps w and w + 4 share the rows 32 (w % 4) ..
-      // and combine their row max (and at the end their sums) through shared
-      // memory at a named barrier of the pair.
+      // ---- softmax: kParts warpgroups; thread = (query row = TMEM lane, part
+      // of the key columns).  Warp w takes keys [32 p, 32 p + 32) of every
+      // chunk, p = (w - 2) / 4; the kParts warps w = 2 + 4 p + (w % 4) share
+      // the rows 32 (w % 4) .. and combine their row max (and at the end their
+      // sums) through shared memory at a named barrier of the row group.
+      constexpr int OC = HD / kParts;          // O columns of a part
       const int q4 = warp & 3;
       const int qi = q4 * 32 + lane;
-      const int hf = (warp - 2) >> 2;          // 0: keys [0, 64), 1: keys [64, 128)
-      const int st_id = threadIdx.x - 64;      // 0 .. 255 among the softmax threads
+      const int pt = (warp - 2) >> 2;          // key part
+      const int st_id = threadIdx.x - 64;      // 0 .. kSoftThreads - 1
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-      const uint32_t o_tm = tmem + 256u + lane_off + (uint32_t)(hf * (HD / 2));  // this half's O columns
+      const uint32_t o_tm = tmem + 256u + lane_off + (uint32_t)(pt * OC);  // this part's O columns
       const float sc = a.scale_log2;
-      auto pair_sync = [&]() { asm volatile("bar.sync %0, 64;" ::"r"(1 + q4) : "memory"); };
-      // Q tile -> shared memory (the 256 softmax threads; zero rows past nq),
-      // while the producer already streams K / V
-      for (int c = st_id; c < kQT * (HD / 8); c += 256) {
+      auto group_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + q4), "r"(32 * kParts) : "memory"); };
+      // Q tile -> shared memory (the softmax threads; zero rows past nq),
+      // while the producers already stream K / V
+      for (int c = st_id; c < kQT * (HD / 8); c += kSoftThreads) {
         const int qr = c / (HD / 8), ch = c - qr * (HD / 8);
         const int q = qt * kQT + qr;
         const bool ok = q < nq;
@@ -355,45 +360,42 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
       fence_proxy_async_smem();  // the MMA reads Q through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(Q_FULL);
-      float m_run = -INFINITY, l_run = 0.f;  // l_run: this half's share of the row sum
+      float m_run = -INFINITY, l_run = 0.f;  // l_run: this part's share of the row sum
       bool alive = true;
-      // Every softmax warp walks all nch chunks and meets its partner at each
-      // pair barrier, also after a timed-out wait (it then skips the work), so
+      // Every softmax warp walks all nch chunks and meets its row group at each
+      // named barrier, also after a timed-out wait (it then skips the work), so
       // the named barriers always match.
       for (int j = 0; j < nch; ++j) {
         const uint32_t g = cbase + (uint32_t)j, sb = g & 1u;
         if (alive) alive = __all_sync(0xffffffffu, wait_bounded(S_FULL(sb), (g >> 1) & 1u, abort_v, a.status));
-        const int nvalid = min(kKC, k_end - (k_begin + j * kKC)) - hf * 64;  // valid keys of this half (may be <= 0)
-        float sv[64];
-        float mx[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = -INFINITY;
+        const int nvalid = min(kKC, k_end - (k_begin + j * kKC)) - pt * kPartKeys;  // valid keys of this part
+        float sv[kPartKeys];
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         if (alive) {
           tc_fence_after();
-          uint32_t sr[64];
-          const uint32_t s_tm = tmem + sb * (uint32_t)kKC + lane_off + (uint32_t)(hf * 64);
-          tmem_ld32_issue(s_tm, sr);
-          tmem_ld32_issue(s_tm + 32u, sr + 32);
-          tmem_wait_ld_tie64(sr);
-          if (nvalid >= 64) {  // a full half (every chunk but a ragged last one)
+          uint32_t sr[kPartKeys];
+          tmem_ld32_issue(tmem + sb * (uint32_t)kKC + lane_off + (uint32_t)(pt * kPartKeys), sr);
+          tmem_wait_ld_tie32(sr);
+          if (nvalid >= kPartKeys) {  // a full part (every chunk but a ragged last one)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
+            for (int c = 0; c < kPartKeys; ++c) {
               sv[c] = __uint_as_float(sr[c]);
-              mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+              mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
+            for (int c = 0; c < kPartKeys; ++c) {
               sv[c] = c < nvalid ? __uint_as_float(sr[c]) : -INFINITY;
-              mx[c & 7] = fmaxf(mx[c & 7], sv[c]);
+              mx[c & 3] = fmaxf(mx[c & 3], sv[c]);
             }
           }
         }
         // raw S here; the scale (> 0) commutes with the max and enters the exponent below
-        float mc = sc * fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        s_mx[j & 1][hf][qi] = mc;
-        pair_sync();
-        mc = fmaxf(mc, s_mx[j & 1][hf ^ 1][qi]);  // the row's chunk max (identical in both halves)
+        float mc = sc * fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        s_mx[j & 1][pt][qi] = mc;
+        group_sync();
+#pragma unroll
+        for (int o = 0; o < kParts; ++o) mc = fmaxf(mc, s_mx[j & 1][o][qi]);  // the row's chunk max
         if (!alive) continue;
         // The running max only moves when the chunk's max exceeds it by more than
         // 8 (log2 units): P then stays below 2^8 and most chunks need no O
@@ -410,36 +412,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
           alive = __all_sync(0xffffffffu, wait_bounded(O_DONE, (g - 1u) & 1u, abort_v, a.status));
           if (!alive) continue;
           tc_fence_after();
-          {
 #pragma unroll
-            for (int c = 0; c < HD / 64; ++c) {  // this half's HD / 2 columns, 32 at a time
-              uint32_t orr[32];
-              tmem_ld32_issue(o_tm + (uint32_t)(c * 32), orr);
-              tmem_wait_ld_tie32(orr);
+          for (int c = 0; c < OC / 16; ++c) {  // this part's OC columns, 16 at a time
+            float ov[16];
+            tmem_ld16(o_tm + (uint32_t)(c * 16), ov);
 #pragma unroll
-              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-              tmem_st32(o_tm + (uint32_t)(c * 32), orr);
-            }
-            tmem_wait_st();
+            for (int e = 0; e < 16; ++e) ov[e] *= alpha;
+            tmem_st16(o_tm + (uint32_t)(c * 16), ov);
           }
+          tmem_wait_st();
         }
         m_run = m_new;
-        // P = 2^(s - m) of this half's valid keys (0 past them), as bf16 pairs:
-        // keys 64 hf + 2c, 64 hf + 2c + 1 in column 32 hf + c of P buffer j % 2
+        // P = 2^(s - m) of this part's valid keys (0 past them), as bf16 pairs:
+        // keys 32 pt + 2c, 32 pt + 2c + 1 in column 16 pt + c of P buffer j % 2
         // (the K-major A operand of P_j V_j in tensor memory)
         float ps[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[kPartKeys / 2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 16 columns at a time
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float p0 = ex2_approx(fmaf(sv[32 * h + 2 * c], sc, -m_new));
-            const float p1 = ex2_approx(fmaf(sv[32 * h + 2 * c + 1], sc, -m_new));
-            ps[c & 3] += p0 + p1;
-            pk[c] = pack2_bf16(p0, p1);
-          }
-          tmem_st16u(tmem + C::kPCol + sb * 64u + lane_off + (uint32_t)(hf * 32 + h * 16), pk);
+        for (int c = 0; c < kPartKeys / 2; ++c) {
+          const float p0 = ex2_approx(fmaf(sv[2 * c], sc, -m_new));
+          const float p1 = ex2_approx(fmaf(sv[2 * c + 1], sc, -m_new));
+          ps[c & 3] += p0 + p1;
+          pk[c] = pack2_bf16(p0, p1);
         }
+        tmem_st16u(tmem + C::kPCol + sb * 64u + lane_off + (uint32_t)(pt * (kPartKeys / 2)), pk);
         l_run = l_run * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
         tmem_wait_st();
         tc_fence_before();
@@ -447,37 +443,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         if (lane == 0) mbar_arrive(P_FULL(sb));
       }
       if (alive) alive = __all_sync(0xffffffffu, wait_bounded(O_FINAL, ntile & 1u, abort_v, a.status));
-      // the row sum: this half's share plus the partner's, in half order
-      s_l[hf][qi] = l_run;
-      pair_sync();
-      const float l_row = s_l[0][qi] + s_l[1][qi];
+      // the row sum: the parts' shares in part order
+      s_l[pt][qi] = l_run;
+      group_sync();
+      float l_row = 0.f;
+#pragma unroll
+      for (int o = 0; o < kParts; ++o) l_row += s_l[o][qi];
       if (alive) {
         tc_fence_after();
-        uint32_t orr[HD / 2];
+        float orr[OC];
 #pragma unroll
-        for (int c = 0; c < HD / 64; ++c) tmem_ld32_issue(o_tm + (uint32_t)(c * 32), orr + c * 32);
-        tmem_wait_tie(orr);
+        for (int c = 0; c < OC / 16; ++c) tmem_ld16(o_tm + (uint32_t)(c * 16), *reinterpret_cast<float(*)[16]>(orr + 16 * c));
         const int q = qt * kQT + qi;
         if (q < nq) {
           const int r = row0 + q / G, h = kvh * G + q % G;
           const size_t qidx = (size_t)r * a.H + h;
           if (a.splits == 1) {
             const float inv = 1.f / l_row;
-            uint4 *dst = reinterpret_cast<uint4 *>(a.out + qidx * HD + hf * (HD / 2));
+            uint4 *dst = reinterpret_cast<uint4 *>(a.out + qidx * HD + pt * OC);
 #pragma unroll
-            for (int c = 0; c < HD / 16; ++c)
-              dst[c] = make_uint4(pack2_bf16(__uint_as_float(orr[8 * c]) * inv, __uint_as_float(orr[8 * c + 1]) * inv),
-                                  pack2_bf16(__uint_as_float(orr[8 * c + 2]) * inv, __uint_as_float(orr[8 * c + 3]) * inv),
-                                  pack2_bf16(__uint_as_float(orr[8 * c + 4]) * inv, __uint_as_float(orr[8 * c + 5]) * inv),
-                                  pack2_bf16(__uint_as_float(orr[8 * c + 6]) * inv, __uint_as_float(orr[8 * c + 7]) * inv));
+            for (int c = 0; c < OC / 8; ++c)
+              dst[c] = make_uint4(pack2_bf16(orr[8 * c] * inv, orr[8 * c + 1] * inv),
+                                  pack2_bf16(orr[8 * c + 2] * inv, orr[8 * c + 3] * inv),
+                                  pack2_bf16(orr[8 * c + 4] * inv, orr[8 * c + 5] * inv),
+                                  pack2_bf16(orr[8 * c + 6] * inv, orr[8 * c + 7] * inv));
           } else {
             // this split's (O, max, sum) of the row, staged in this CTA's shared
-            // memory for the cluster merge (the K / V ring is idle by now)
-            const uint32_t dst = kv_s + (uint32_t)qi * kStagePitch + (uint32_t)(hf * (HD / 2)) * 4u;
+            // memory for the cluster merge (the K / V rings are idle by now)
+            const uint32_t dst = kv_s + (uint32_t)qi * kStagePitch + (uint32_t)(pt * OC) * 4u;
 #pragma unroll
-            for (int c = 0; c < HD / 8; ++c)
-              st_shared_v4(dst + (uint32_t)c * 16u, orr[4 * c], orr[4 * c + 1], orr[4 * c + 2], orr[4 * c + 3]);
-            if (hf == 0) s_ml[qi] = make_float2(m_run, l_row);
+            for (int c = 0; c < OC / 4; ++c)
+              st_shared_v4(dst + (uint32_t)c * 16u, __float_as_uint(orr[4 * c]), __float_as_uint(orr[4 * c + 1]),
+                           __float_as_uint(orr[4 * c + 2]), __float_as_uint(orr[4 * c + 3]));
+            if (pt == 0) s_ml[qi] = make_float2(m_run, l_row);
           }
         }
       }

@@ -946,6 +946,7 @@ int enqueue_commit(dcu_ctx *c, int rule, float param, int gen_start, int block_l
       tp.smx = c->smx;
       tp.smx_arg = c->smx_arg;
       tp.ldm = cap;
+      tp.sweep = c->pass_sweep ? 2 : 0;  // more than 256 masked rows: two passes per weight tile
       if (rule == DCU_APD) {  // this commit's logits, by position, for the APD signals
         tp.zout = c->apd_z + (size_t)c->apd_flip * cap * g.vocab;
         tp.zrow = c->mrow;

@@ -115,7 +115,7 @@ struct TcParams {
   int chain;
   int32_t *bar;
   int b_rows;              // rows of the activation box: the token pass (BN) or fewer when cap < BN
-  // Pass sweep (chain = 0, epi_mode 0): when M spans more than one token pass,
+  // Pass sweep (chain = 0; layer GEMMs and the LM head): when M spans more than one token pass,
   // up to `sweep` passes share each weight tile while it is in shared memory
   // (one activation box per pass in a stage, one TMEM accumulator per pass),
   // so the weights stream from HBM once per group of passes instead of once

@@ -422,10 +422,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   // sweep an activation stage holds G boxes, one per token pass of the group;
   // the region is sized for the launch's largest G, so the weight ring's depth
   // does not depend on M (the weight producer starts before M is loaded) and
-  // only the activation ring's depth follows G.
+  // only the activation ring's depth follows G.  (The LM head, which runs
+  // once per step, sizes it from M itself: a set within one pass keeps the
+  // deeper weight ring.)
   const uint32_t b_bytes = (uint32_t)p.b_rows * 128u;            // one TMA box per token pass
   const uint32_t b_stage = (b_bytes + 1023u) & ~1023u;             // 1024-byte aligned boxes
-  const int gmax = kSw ? p.sweep : 1;
+  const int gmax = kSw ? p.sweep : (kLm && p.sweep > 1 && M > BN ? p.sweep : 1);
   const uint32_t x_region = gmax > 1 ? 2u * (uint32_t)gmax * b_stage : (b_stage > 16384u ? 3u : 4u) * b_stage;
   int SA = (int)((p.smem_bytes - 1024u - x_region) / kTcABytes);
   SA = SA > kTcMaxA ? kTcMaxA : SA;
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   const uint32_t bar0 = smem_u32(bars);
   // TMEM: one accumulator of G x BN columns per fragment, two alternating
   // between fragments while they fit (always for G = 1)
-  const uint32_t tcols = kSw ? 512u : 2u * (uint32_t)BN;
+  const uint32_t tcols = (kSw || kLm) ? 512u : 2u * (uint32_t)BN;
 #define FULL_A(s) (bar0 + 8u * (uint32_t)(s))
 #define EMPTY_A(s) (bar0 + 8u * (uint32_t)(kTcMaxA + (s)))
 #define FULL_B(s) (bar0 + 8u * (uint32_t)(2 * kTcMaxA + (s)))
@@ -478,7 +480,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
   }
   const int passes = (M + BN - 1) / BN;
   // G token passes per weight tile (a group); the fragment iterators walk groups
-  const int G = kSw ? min(passes, gmax) : 1;
+  const int G = (kSw || kLm) ? min(passes, gmax) : 1;
   const int ngroups = (passes + G - 1) / G, grows = G * BN;
   const bool dbuf = 2u * (uint32_t)grows <= tcols;  // two accumulators alternate
   const uint32_t x_stage = (uint32_t)G * b_stage;
@@ -562,7 +564,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           // the whole token pass in one box: TMA throughput is bound by the number
           // of copies, not their bytes (rows past the packed count are never read
           // by the MMA; rows past the buffer are zero-filled)
-          if (!kSw || G == 1) {
+          if ((!kSw && !kLm) || G == 1) {
             mbar_expect_tx(FULL_B(stage), b_bytes);
             tma_load_2d(STAGE_B(stage), &p.ph[ph].b, cb.kb * 64, cb.m0, FULL_B(stage), pol_x);
           } else {  // one box per token pass of the group
@@ -597,7 +599,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         while (ok && next_frag<false>(p, ngroups, it, f)) {
           const int mrows = min(BN, M - it.pass * grows);  // rows of the group's first pass
           const uint32_t idesc = idesc_bf16(128, (mrows + 15) & ~15);
-          const int lm_halves = mrows > 128 ? 2 : 1;
           const int npg = min(G, passes - it.pass * G);
           const uint32_t acc = dbuf ? (nfrag & 1u) : 0u, use = dbuf ? nfrag >> 1 : nfrag;
           const uint32_t dtm = tmem + acc * (uint32_t)grows;
@@ -617,13 +618,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
             const uint64_t bd = sw128_desc(STAGE_B(sb));
             if (kLm) {
               // LM head: tokens are the MMA M dimension (one or two 128-row halves of
-              // the activation box), the tile's 128 vocabulary rows are N
-              for (int mt = 0; mt < lm_halves; ++mt) {
-                const uint64_t xd = sw128_desc(STAGE_B(sb) + (uint32_t)mt * 16384u);
+              // each pass's activation box), the tile's 128 vocabulary rows are N;
+              // pass q of the group accumulates at columns q * BN
+              for (int q = 0; q < npg; ++q) {
+                const int mq = min(BN, M - it.pass * grows - q * BN);
+                for (int mt = 0; mt < (mq > 128 ? 2 : 1); ++mt) {
+                  const uint64_t xd = sw128_desc(STAGE_B(sb) + (uint32_t)q * b_stage + (uint32_t)mt * 16384u);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                  tc_mma(dtm + (uint32_t)(mt * 128), xd + (uint64_t)(2 * k), ad + (uint64_t)(2 * k), idesc_lm,
-                         (kb > f.kb0 || k > 0) ? 1u : 0u);
+                  for (int k = 0; k < 4; ++k)
+                    tc_mma(dtm + (uint32_t)(q * BN + mt * 128), xd + (uint64_t)(2 * k), ad + (uint64_t)(2 * k),
+                           idesc_lm, (kb > f.kb0 || k > 0) ? 1u : 0u);
+                }
               }
             } else {
 #pragma unroll
@@ -667,22 +672,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
     const int q4 = warp & 3;  // TMEM lane quarter this warp may access
     const int ew = warp - 2, t128 = threadIdx.x - 64;
     uint32_t nfrag = 0;
-    float lm_max[2] = {-INFINITY, -INFINITY};
-    double lm_sum[2] = {0.0, 0.0};  // fp64 running sums: ~1000 terms per CTA
-    int lm_arg[2] = {0x7fffffff, 0x7fffffff};
-    int lm_pass = 0;
-    // LM head: this CTA's statistics of the pass's tokens over its vocabulary range
-    auto lm_flush = [&](int pass) {
-      for (int mt = 0; mt < 2; ++mt) {
-        const int m = pass * BN + mt * 128 + q4 * 32 + lane;
-        if (m < M) {
+    // LM head: per (pass of the group, 128-token half) running statistics
+    constexpr int kLmSlots = kLm ? 4 : 1;  // a group holds at most 2 passes of the 256-row box
+    float lm_max[kLmSlots];
+    double lm_sum[kLmSlots];  // fp64 running sums: ~1000 terms per CTA
+    int lm_arg[kLmSlots];
+#pragma unroll
+    for (int i = 0; i < kLmSlots; ++i) {
+      lm_max[i] = -INFINITY;
+      lm_sum[i] = 0.0;
+      lm_arg[i] = 0x7fffffff;
+    }
+    int lm_group = 0;
+    // LM head: this CTA's statistics of the group's tokens over its vocabulary range
+    auto lm_flush = [&](int group) {
+#pragma unroll
+      for (int i = 0; i < kLmSlots; ++i) {
+        const int m = (group * G + (i >> 1)) * BN + (i & 1) * 128 + q4 * 32 + lane;
+        if ((i >> 1) < G && m < M) {
           const size_t o = (size_t)blockIdx.x * p.ldm + (size_t)m;
-          p.smx[o] = make_float2(lm_max[mt], (float)lm_sum[mt]);
-          p.smx_arg[o] = lm_arg[mt];
+          p.smx[o] = make_float2(lm_max[i], (float)lm_sum[i]);
+          p.smx_arg[o] = lm_arg[i];
         }
-        lm_max[mt] = -INFINITY;
-        lm_sum[mt] = 0.0;
-        lm_arg[mt] = 0x7fffffff;
+        lm_max[i] = -INFINITY;
+        lm_sum[i] = 0.0;
+        lm_arg[i] = 0x7fffffff;
       }
     };
     bool alive = true;
@@ -716,17 +730,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
           // tiles arrive in increasing vocabulary order, so on equal maxima the
           // earlier (lower) id is kept
           const int vbase = f.tile * 128;
-          if (it.pass != lm_pass) {
-            lm_flush(lm_pass);
-            lm_pass = it.pass;
+          if (it.pass != lm_group) {
+            lm_flush(lm_group);
+            lm_group = it.pass;
           }
-          const int mrows = min(BN, M - mg);
-          for (int mt = 0; mt < (mrows > 128 ? 2 : 1); ++mt) {
-            const uint32_t tm = tmem + acc * (uint32_t)grows + (uint32_t)(mt * 128) + ((uint32_t)(q4 * 32) << 16);
-            float &RM = lm_max[mt];
-            double &RS = lm_sum[mt];
-            int &RI = lm_arg[mt];
-            const int tok = it.pass * BN + mt * 128 + q4 * 32 + lane;
+#pragma unroll
+          for (int i = 0; i < kLmSlots; ++i) {  // (pass q = i / 2 of the group, half mt = i % 2)
+            const int q = i >> 1, mt = i & 1;
+            const int mq = min(BN, M - mg - q * BN);  // rows of pass q (<= 0 past the group's passes)
+            if (q >= G || mt * 128 >= mq) continue;   // warp-uniform
+            const uint32_t tm =
+                tmem + acc * (uint32_t)grows + (uint32_t)(q * BN + mt * 128) + ((uint32_t)(q4 * 32) << 16);
+            float &RM = lm_max[i];
+            double &RS = lm_sum[i];
+            int &RI = lm_arg[i];
+            const int tok = mg + q * BN + mt * 128 + q4 * 32 + lane;
             float *zdst = (p.zout && tok < M) ? p.zout + (int64_t)p.zrow[tok] * p.ldz + vbase : nullptr;
             for (int c = 0; c < 128; c += 16) {
               float v[16];
@@ -801,7 +819,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_gemm_tc(const __grid_constant
         break;
       }
     }
-    if (kLm) lm_flush(lm_pass);
+    if (kLm) lm_flush(lm_group);
   }
 #undef FULL_A
 #undef EMPTY_A
@@ -901,7 +919,7 @@ cudaError_t launch_gemm_tc(TcParams p, int bn, cudaStream_t s) {
     if (p.smem_bytes < need) p.smem_bytes = need;
     // pass sweep: G passes' accumulators in 512 TMEM columns, and two stages of
     // G activation boxes beside at least 4 weight tiles in shared memory
-    int g = (p.chain || p.epi_mode == EPI_LMHEAD) ? 0 : p.sweep;
+    int g = p.chain ? 0 : p.sweep;
     if (g > 512 / bn) g = 512 / bn;
     while (g > 1 && 1024u + 2u * (uint32_t)g * b_stage + 4u * kTcABytes > p.smem_bytes) --g;
     p.sweep = g > 1 ? g : 0;

@@ -169,10 +169,11 @@ int dcu_step(dcu_ctx *ctx, const int32_t *token_ids, const int32_t *key_position
 #define DCU_OPT_GEMM_SMEM_KB 4
 /*   DCU_OPT_GEMM_PASS_SWEEP (0 or 1, default 1): a layer GEMM multiplies its
  *     rows in token passes of 128 rows (small expected recompute sets) or 256
- *     (larger ones, and the dense forward).  With 256-row passes and more than
- *     one pass, 1 multiplies each weight tile held in shared memory by two
- *     passes of activations, each into its own tensor-memory accumulator, so
- *     the weights stream from HBM once per two passes; 0 streams them once per
+ *     (larger ones, and the dense forward); the LM head of a commit takes the
+ *     masked rows 256 at a time.  With 256-row passes and more than one pass,
+ *     1 multiplies each weight tile held in shared memory by two passes of
+ *     activations, each into its own tensor-memory accumulator, so the
+ *     weights stream from HBM once per two passes; 0 streams them once per
  *     pass.  Results are bit-identical either way. */
 #define DCU_OPT_GEMM_PASS_SWEEP 5
 #define DCU_ATTN_TCGEN05 0

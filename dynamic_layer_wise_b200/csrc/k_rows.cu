@@ -264,6 +264,34 @@ __device__ __forceinline__ float4 csum4(const float *c, const SlotGeo &geo, size
 // written two or more launches earlier (final once this launch has started),
 // so they are loaded before the wait and only the slot loads follow it.
 
+// Two such sums (columns ja and jb of one packed row) with their loads
+// interleaved: each column summed in slot order as csum4 does, two loads in
+// flight instead of one.
+__device__ __forceinline__ void csum4x2(const float *c, const SlotGeo &geo, size_t ja, size_t jb, float4 &va,
+                                        float4 &vb) {
+  va = *reinterpret_cast<const float4 *>(c + ja);
+  vb = *reinterpret_cast<const float4 *>(c + jb);
+  const int na = slot_count(geo, ja), nb = slot_count(geo, jb);
+  const int n = na > nb ? na : nb;
+  for (int sp = 1; sp < n; ++sp) {
+    const float *cs = c + (size_t)sp * (size_t)geo.slot_stride;
+    if (sp < na) {
+      const float4 w = *reinterpret_cast<const float4 *>(cs + ja);
+      va.x += w.x;
+      va.y += w.y;
+      va.z += w.z;
+      va.w += w.w;
+    }
+    if (sp < nb) {
+      const float4 w = *reinterpret_cast<const float4 *>(cs + jb);
+      vb.x += w.x;
+      vb.y += w.y;
+      vb.z += w.z;
+      vb.w += w.w;
+    }
+  }
+}
+
 template <class T>
 __device__ __forceinline__ void store4(T *p, float a, float b, float c, float d);
 template <>
@@ -328,7 +356,8 @@ __global__ void k_epi_qkv(const float *__restrict__ C, int ldc, const SlotGeo ge
       const int t = u * 4;
       const int head = t / half, j = t - head * half;
       const int base = head * hd;  // q heads first, then k heads (contiguous in C)
-      const float4 a = csum4(c, geo, base + j), bb = csum4(c, geo, base + j + half);
+      float4 a, bb;
+      csum4x2(c, geo, base + j, base + j + half, a, bb);
       float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
       if (use_rope) {
 #pragma unroll
@@ -463,7 +492,8 @@ __global__ void k_epi_swiglu(const float *__restrict__ C, int ldc, const SlotGeo
        it += (long long)gridDim.x * blockDim.x) {
     const int r = (int)(it / per_row), j = (int)(it - (long long)r * per_row) * 4;
     const float *c = C + (size_t)r * ldc;
-    const float4 gt = csum4(c, geo, j), up = csum4(c, geo, (size_t)F + j);
+    float4 gt, up;
+    csum4x2(c, geo, j, (size_t)F + j, gt, up);
     store4<T>(act + (size_t)r * F + j, gt.x / (1.0f + expf(-gt.x)) * up.x, gt.y / (1.0f + expf(-gt.y)) * up.y,
               gt.z / (1.0f + expf(-gt.z)) * up.z, gt.w / (1.0f + expf(-gt.w)) * up.w);
   }
